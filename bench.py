@@ -1,0 +1,374 @@
+#!/usr/bin/env python
+"""PQ-HSA decode benchmark: µs per decode step and achieved HBM GB/s on B200.
+
+Workload (default): one Llama-3.1-8B-shaped attention layer at 128K context,
+32 query / 8 KV heads, head dim 128, paged bf16 K/V (page 16, shuffled pool),
+IVF-PQ index with 1024 clusters and 16 x 8-dim subspaces of 256 codes per KV
+head, sink 16 + recent 1024 exact, top-k = 1 % of the indexed tokens.
+Synthetic seeded data (see synth/). One JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn µs/step & achieved HBM GB/s (% peak) at 128K ctx, 1% budget"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b_128k")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what one step must move at minimum)
+# ---------------------------------------------------------------------------
+
+def step_bytes(w, n_idx: int, k: int):
+    """Per-step algorithmic HBM bytes of PQ-HSA, of dense decode and of the scan kernel."""
+    G, C, D = w.G, w.C, w.D
+    R = w.T - w.n_sink - n_idx
+    per_unit = (16 * n_idx                       # PQ codes
+                + 4 * C * D                      # centroids (q . centroid)
+                + 4 * 16 * 256 * 8               # codebook
+                + 4 * G * 16 * 256               # LUT written once
+                + 4 * C * D + 4 * C              # cluster mean values + counts
+                + 512 * (w.n_sink + R + k)       # exact K+V rows (bf16)
+                + 8 * G * D)                     # q in, out
+    ids = 2 * n_idx
+    dense = 512 * w.T + 8 * G * D
+    scan = n_idx * (16 + 2 + 4)                  # codes + cluster id read, selection score written
+    U = w.B * w.Hkv
+    return U * per_unit, U * ids, U * dense, U * scan
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (reported baseline, never the target)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(bt, w, budget, seconds: float):
+    """Run the float64 oracle on units of the workload until `seconds` elapse; µs per whole step."""
+    from threadpoolctl import threadpool_limits
+    import oracle as O
+    scale = float(np.float32(1.0 / math.sqrt(w.D)))
+    done, t0 = 0, time.perf_counter()
+    units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    with threadpool_limits(limits=1):
+        while True:
+            u = units[done % len(units)]
+            O.oracle_decode(bt.q, bt.k_cache, bt.v_cache, bt.block_table, bt.seq_lens, bt.centroids,
+                            bt.codebooks, bt.codes_rec, bt.ids_rec, bt.n_indexed, w.n_sink, scale,
+                            budget=budget, page_size=w.page_size, units=[u])
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds or done >= 4 * len(units):
+                break
+    us_per_step = el / done * len(units) * 1e6
+    return us_per_step, done, el
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_long_context_pq_b200 as P
+    from synth import make_batch, workload
+    from synth.device import index_tensors, kv_tensors
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    w = workload(args.workload)
+    budget = w.budget
+    bt = make_batch(w)
+    kv = P.PagedKV(**kv_tensors(bt, dev))
+    ix = P.PQIndex(**index_tensors(bt, dev, n_indexed=np.zeros(w.B, dtype=np.int32)))
+    stream = torch.cuda.current_stream()
+
+    # ---- index build after prefill: encode every indexed key on the GPU ----
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ws_idx = P.workspace(P.hsa_index_workspace_bytes(), dev)
+    e0.record()
+    P.hsa_append_encode(kv, ix, w.n_indexed, workspace_buf=ws_idx)
+    e1.record()
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    assert P.hsa_read_error(ws_idx) == 0
+
+    scale = float(np.float32(1.0 / math.sqrt(w.D)))
+    q = torch.from_numpy(bt.q).to(dev)
+    out = torch.empty_like(q)
+    out_dense = torch.empty_like(q)
+    ws = P.workspace(P.hsa_decode_workspace_bytes(kv, ix), dev)
+    ws_dense = P.workspace(P.dense_decode_workspace_bytes(kv), dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(P.NUM_STAGES + 1)]
+    for e in stage_ev:
+        e.record()
+    torch.cuda.synchronize()
+
+    def hsa_step():
+        P.hsa_decode(kv, ix, q, out, scale=scale, budget=budget, workspace_buf=ws, stage_events=stage_ev)
+
+    def dense_step():
+        P.dense_decode(kv, q, out_dense, scale=scale, workspace_buf=ws_dense)
+
+    # warm once outside capture, then capture each step into a CUDA graph
+    hsa_step()
+    dense_step()
+    torch.cuda.synchronize()
+    g_hsa, g_dense = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_hsa):
+        hsa_step()
+    with torch.cuda.graph(g_dense):
+        dense_step()
+    torch.cuda.synchronize()
+
+    def timed(graph, steps, stage=False, e2e=None):
+        t, st = [], []
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(steps):
+            flush.zero_()
+            a.record()
+            if e2e is not None:
+                e2e[1].copy_(e2e[0], non_blocking=True)
+            graph.replay()
+            if e2e is not None:
+                e2e[3].copy_(e2e[2], non_blocking=True)
+            b.record()
+            torch.cuda.synchronize()
+            t.append(a.elapsed_time(b))
+            if stage:
+                st.append([stage_ev[i].elapsed_time(stage_ev[i + 1]) for i in range(P.NUM_STAGES)])
+        return t, st
+
+    for _ in range(args.warmup):
+        timed(g_hsa, 1)
+        timed(g_dense, 1)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_hsa, t_stage = timed(g_hsa, args.steps, stage=True)
+        t_dense, _ = timed(g_dense, args.steps)
+        q_h = torch.from_numpy(bt.q).pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        t_e2e, _ = timed(g_hsa, args.steps, e2e=(q_h, q, out, out_h))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    err = P.hsa_read_error(ws)
+    assert err == 0, f"device error word {err}"
+
+    ms_hsa = sum(t_hsa) / len(t_hsa)
+    ms_dense = sum(t_dense) / len(t_dense)
+    ms_e2e = sum(t_e2e) / len(t_e2e)
+    if world > 1:
+        tt = torch.tensor([ms_hsa, ms_dense, ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_hsa, ms_dense, ms_e2e = tt.tolist()
+
+    stage_ms = [sum(s[i] for s in t_stage) / len(t_stage) for i in range(P.NUM_STAGES)]
+    n_idx = int(w.n_indexed)
+    k = P.decode_k(budget, n_idx)
+    hsa_b, ids_b, dense_b, scan_b = step_bytes(w, n_idx, k)
+    peak, peak_kind = measured_peaks()
+    dom = int(np.argmax(stage_ms))
+    dom_name = P.STAGE_NAMES[dom]
+    U = w.B * w.Hkv
+    if dom_name == "scan":
+        dom_bytes = scan_b
+    elif dom_name == "attend":
+        dom_bytes = U * (512 * (w.n_sink + (w.T - w.n_sink - n_idx) + k) + 4 * w.C * w.D)
+    else:
+        dom_bytes = hsa_b
+    dom_gbs = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
+    step_gbs = hsa_b / (ms_hsa * 1e-3) / 1e9
+    dense_gbs = dense_b / (ms_dense * 1e-3) / 1e9
+
+    res = {
+        "metric": METRIC,
+        "value": round(ms_hsa * 1e3, 3),
+        "unit": "us/step",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_hsa, 6),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 KV, fp32 math",
+        "data": "synthetic (seeded; no dataset or weights)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.D, "ctx": w.T,
+                   "clusters": w.C, "pq": "16x8/256", "sink": w.n_sink, "recent": w.n_recent,
+                   "budget": budget, "k": k, "page_size": w.page_size,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MB write) before every timed step",
+                   "timing": "CUDA events per step around a CUDA-graph replay"},
+        "hbm_gbs": round(step_gbs, 1),
+        "hbm_pct_peak": round(100 * step_gbs / peak, 2),
+        "bytes_per_step": hsa_b,
+        "ids_bytes_per_step": ids_b,
+        "dense": {"us_per_step": round(ms_dense * 1e3, 3), "bytes_per_step": dense_b,
+                  "hbm_gbs": round(dense_gbs, 1), "pct_peak": round(100 * dense_gbs / peak, 2),
+                  "speedup_of_pqhsa": round(ms_dense / ms_hsa, 3)},
+        "stages_us": {n: round(v * 1e3, 3) for n, v in zip(P.STAGE_NAMES, stage_ms)},
+        "index_build_ms": round(build_ms, 3),
+        "roofline": {"kernel": dom_name, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
+                     "traffic": None, "algorithmic_bytes": dom_bytes},
+        "e2e": {"value": round(ms_e2e * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": q.numel() * 4,
+                "d2h_bytes_per_step": out.numel() * 4},
+        "gpu_launches": args.steps * 3 * P.NUM_STAGES,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        us, units, el = oracle_sample(bt, w, budget, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": round(us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+                               "sample": f"{units} (sequence, KV head) units of the same workload, "
+                                         f"{el:.1f} s of float64 numpy, scaled to a full step"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from synth import make_batch, workload
+    w = workload(args.workload)
+    bt = make_batch(w)
+    per_step_seconds = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(bt, w, w.budget, per_step_seconds / 4)
+    t = []
+    units_total = 0
+    for _ in range(args.steps):
+        us, units, el = oracle_sample(bt, w, w.budget, per_step_seconds)
+        t.append(us)
+        units_total += units
+    us = sum(t) / len(t)
+    res = {
+        "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us/step",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.T, "budget": w.budget},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: whole (sequence, KV head) units of the workload for "
+                                   f"~{per_step_seconds:.1f} s, scaled to a full step ({units_total} units)"},
+        "e2e": {"value": round(us, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+/*
+ * pqhsa.h - C ABI of a B200 (sm_100a) library for one decode step of PQ-HSA
+ * sparse attention over a paged bf16 KV cache.
+ *
+ * Method: the rit.work article "pq-hsa-long-context-attention" (PQ-HSA),
+ * section "Как приблизительные оценки возвращают отброшенный контекст":
+ * an IVF-PQ index over the keys yields an approximate logit for every indexed
+ * token; the top tokens under a read budget, plus the first tokens and a
+ * recent window, are attended exactly from the KV cache; every other indexed
+ * token stays in the softmax normalisation through its approximate logit, and
+ * its value contribution is its cluster's summed weight times the cluster's
+ * mean value. The index is built after prefill and new tokens are added to it
+ * in batches. At full budget the same machinery is plain dense split-K GQA
+ * decode (dense_decode), the in-library baseline.
+ *
+ * Conventions shared by every entry point
+ * - Pointers are DEVICE pointers unless their name ends in _host. The caller
+ *   owns all memory; the library allocates nothing, keeps no state between
+ *   calls, and touches only the buffers it is given.
+ * - Every call validates its arguments on the host (from the *_host arrays)
+ *   before any launch and returns a status; on an error nothing is launched.
+ *   HSA_ERR_CUDA means a launch failed (the CUDA error is left pending).
+ * - Work is enqueued on `stream` only; calls are asynchronous with respect to
+ *   the host. The *_host arrays are read during the call (and, for
+ *   hsa_append_encode, n_indexed_host is advanced by the call).
+ * - Device-side faults never trap: an out-of-range block-table entry, cluster
+ *   id or a timed-out wait is recorded in the workspace error word (see
+ *   hsa_read_error) and the offending access is skipped.
+ * - Workspaces must be 256-byte aligned and at least as large as the
+ *   matching *_workspace_bytes() says; their contents need no initialisation
+ *   and are clobbered.
+ *
+ * KV cache layout (bf16): [num_pages][Hkv][page_size][D], so one head-page is
+ * page_size contiguous 256-byte rows. Token t of sequence b lives in page
+ * block_table[b * max_pages + t / page_size], slot t % page_size.
+ *
+ * Token sets of sequence b (T = seq_lens[b], s0 = n_sink, N = n_indexed[b]):
+ *   sink S = [0, s0), indexed I = [s0, s0 + N), exact tail R = [s0 + N, T).
+ * Index slot i of a (sequence, KV head) holds the code of position s0 + i.
+ */
+#ifndef PQHSA_H
+#define PQHSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSA_OK = 0,
+  HSA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent shapes */
+  HSA_ERR_UNSUPPORTED = 2,   /* D != 128, M * dsub != D, dsub != 8, ncode != 256, G not in {1,2,4,8},
+                                page_size not a power of two in [1, 128], C too large for shared memory */
+  HSA_ERR_CAPACITY = 3,      /* index capacity or sequence length exceeded */
+  HSA_ERR_ALIGNMENT = 4,     /* a pointer is not aligned as documented */
+  HSA_ERR_WORKSPACE = 5,     /* workspace missing or smaller than required */
+  HSA_ERR_CUDA = 6           /* a CUDA launch or query failed */
+} hsa_status;
+
+/* Paged KV cache view (read only). */
+typedef struct {
+  const void* k_cache;             /* bf16 [num_pages][Hkv][page_size][D], 256-B aligned */
+  const void* v_cache;             /* same layout as k_cache */
+  const int32_t* block_table;      /* [B][max_pages] page ids, each in [0, num_pages) */
+  const int32_t* seq_lens;         /* [B] tokens in each sequence */
+  const int32_t* seq_lens_host;    /* [B] host copy of seq_lens (used for planning/validation) */
+  int32_t B, Hq, Hkv, D, page_size, max_pages, num_pages;
+} hsa_kv_cache;
+
+/* IVF-PQ index storage, one index per (sequence, KV head) "unit" u = b * Hkv + h. */
+typedef struct {
+  float* centroids;                /* fp32 [B][Hkv][C][D]            (caller fills) */
+  float* codebooks;                /* fp32 [B][Hkv][M][ncode][dsub]  (caller fills) */
+  uint8_t* codes;                  /* u8  [B][Hkv][cap][M]  residual PQ code of slot i */
+  uint16_t* ids;                   /* u16 [B][Hkv][cap]     cluster of slot i, < C */
+  float* sum_v;                    /* fp32 [B][Hkv][C][D]   sum of member values */
+  float* mean_v;                   /* fp32 [B][Hkv][C][D]   mean member value (0 if empty) */
+  int32_t* count;                  /* [B][Hkv][C]           members per cluster */
+  int32_t* n_indexed;              /* [B] indexed tokens per sequence (device) */
+  int32_t* n_indexed_host;         /* [B] host copy of n_indexed */
+  int32_t C, M, dsub, ncode, cap, n_sink;
+} hsa_index;
+
+typedef struct {
+  float scale;                     /* logit scale, e.g. 1/sqrt(D) */
+  double budget;                   /* k = floor(budget * N) selected tokens per unit */
+  int32_t k_override;              /* >= 0: use min(k_override, N) instead of the budget */
+  int32_t background;              /* 1: PQ-HSA (unselected tokens enter through the
+                                      cluster background); 0: plain top-k sparse attention */
+} hsa_decode_params;
+
+/* Optional debug outputs of hsa_decode (any member may be NULL). */
+typedef struct {
+  float* approx_logits;            /* fp32 [B][Hq][cap]: approximate logit of slot i (scaled) */
+  int32_t* selected;               /* [B][Hkv][cap]: selected token positions, ascending */
+  int32_t* n_selected;             /* [B][Hkv]: number of selected tokens */
+  cudaEvent_t* stage_events;       /* NULL, or HSA_STAGE_EVENTS events recorded on `stream`
+                                      before each stage and after the last one */
+} hsa_debug;
+
+/* Stages of hsa_decode, in launch order: tables, scan, filter, finalize,
+   exact+background attention, merge. stage_events[i] precedes stage i. */
+#define HSA_NUM_STAGES 6
+#define HSA_STAGE_EVENTS (HSA_NUM_STAGES + 1)
+
+/* ---- decode -------------------------------------------------------------- */
+
+/* Workspace bytes hsa_decode needs for these shapes (0 on invalid arguments). */
+size_t hsa_decode_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* index);
+
+/*
+ * One PQ-HSA decode step (rit.work "pq-hsa-long-context-attention", section
+ * "Как приблизительные оценки возвращают отброшенный контекст").
+ * q: fp32 [B][Hq][D]; out: fp32 [B][Hq][D]; both 16-B aligned. For every unit:
+ *   shat_gj = scale * (q_g . centroid_{a_j} + sum_s q_g,s . codeword_s[code_js]) for j in I;
+ *   K = the k slots of largest max_g shat_gj (ties to the smaller position),
+ *       k = floor(budget * N) computed in double;
+ *   out_g = (sum_{j in S+K+R} e^{s_gj} v_j + sum_c W_gc mean_v_c)
+ *           / (sum_{j in S+K+R} e^{s_gj} + sum_{j in I\K} e^{shat_gj}),
+ *   s_gj = scale * q_g . k_j,  W_gc = sum_{j in I\K, a_j = c} e^{shat_gj}.
+ * Needs mean_v consistent with the index (hsa_build_from_codes / hsa_append_encode).
+ * A unit with N = 0 is dense attention over [0, T).
+ */
+hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* index, const float* q, float* out,
+                      const hsa_decode_params* params, const hsa_debug* debug,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes dense_decode needs. */
+size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv);
+
+/*
+ * Dense split-K GQA decode: out_g = softmax(scale * q_g K^T) V over all T tokens of
+ * each sequence (the in-library baseline; same split-K attention engine as the
+ * exact part of hsa_decode). q, out: fp32 [B][Hq][D].
+ */
+hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, float scale,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---- index maintenance --------------------------------------------------- */
+
+/* Workspace bytes of hsa_build_from_codes / hsa_append_encode (error word only). */
+size_t hsa_index_workspace_bytes(void);
+
+/*
+ * Index build after prefill from caller-provided codes (same article, section
+ * above: "after the prompt is filled the index is built"). The caller fills
+ * centroids, codebooks, codes and ids for slots [0, n_indexed[b]); this call
+ * computes count, sum_v and mean_v of every cluster from the value rows of the
+ * indexed tokens.
+ */
+hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* index,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Batched encoding of new tokens into the index (same article: new tokens are
+ * kept outside the index and added in batches). For every sequence b and KV
+ * head, positions [s0 + N_b, s0 + N_b + n_new) are encoded:
+ *   a = argmin_c sum_d (k_d - centroid_c,d)^2 (fp32, ties to the lower c),
+ *   code_s = argmin_m sum_{d<dsub} (k - centroid_a)_{s*dsub+d} - codeword_s,m,d)^2,
+ * written to slots [N_b, N_b + n_new); the members' values are added to sum_v
+ * and count, mean_v is recomputed, and n_indexed (device and host) grows by
+ * n_new. Requires s0 + N_b + n_new <= seq_lens_host[b] and N_b + n_new <= cap.
+ * With n_indexed = 0 this is the whole index build from raw keys.
+ */
+hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* index, int32_t n_new,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---- diagnostics --------------------------------------------------------- */
+
+/* Human-readable name of a status. */
+const char* hsa_strerror(hsa_status status);
+
+/*
+ * Copies the workspace error word (0 = none; otherwise a HSA_DEVERR_* bit set)
+ * to *error_host and clears it. Synchronises `stream`.
+ */
+hsa_status hsa_read_error(void* workspace, int32_t* error_host, cudaStream_t stream);
+
+#define HSA_DEVERR_PAGE 1          /* block-table entry outside [0, num_pages) */
+#define HSA_DEVERR_CLUSTER 2       /* cluster id >= C */
+#define HSA_DEVERR_TIMEOUT 4       /* a bounded wait gave up */
+#define HSA_DEVERR_SELECT 8        /* top-k bookkeeping inconsistent */
+
+/* ABI self-description: sizeof of the public structs, for bindings to check. */
+void hsa_abi_sizes(int64_t* kv_cache, int64_t* index, int64_t* decode_params, int64_t* debug);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PQHSA_H */

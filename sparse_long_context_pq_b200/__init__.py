@@ -1,0 +1,314 @@
+"""PQ-HSA sparse decode attention for B200 (sm_100a): Python binding of libpqhsa.so.
+
+Every step of the decode path runs in the library's CUDA kernels; this module only
+marshals torch tensors (device memory) and the current CUDA stream into the C ABI
+declared in include/pqhsa.h. There is no CPU fallback: importing works without a
+GPU, but every compute call needs the built library and a CUDA device.
+
+Method: rit.work "pq-hsa-long-context-attention" (PQ-HSA).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "PagedKV", "PQIndex", "HSAError", "load_library", "hsa_decode", "dense_decode",
+    "hsa_build_from_codes", "hsa_append_encode", "hsa_decode_workspace_bytes",
+    "dense_decode_workspace_bytes", "hsa_index_workspace_bytes", "hsa_read_error", "hsa_strerror",
+    "decode_k", "HSA_DEVERR_PAGE", "HSA_DEVERR_CLUSTER", "HSA_DEVERR_TIMEOUT", "HSA_DEVERR_SELECT",
+]
+
+HSA_DEVERR_PAGE, HSA_DEVERR_CLUSTER, HSA_DEVERR_TIMEOUT, HSA_DEVERR_SELECT = 1, 2, 4, 8
+M_SUB, DSUB, NCODE, HEAD_DIM = 16, 8, 256, 128
+
+
+class _KV(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("seq_lens_host", ctypes.c_void_p),
+                ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("page_size", ctypes.c_int32), ("max_pages", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32)]
+
+
+class _Index(ctypes.Structure):
+    _fields_ = [("centroids", ctypes.c_void_p), ("codebooks", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("ids", ctypes.c_void_p), ("sum_v", ctypes.c_void_p), ("mean_v", ctypes.c_void_p),
+                ("count", ctypes.c_void_p), ("n_indexed", ctypes.c_void_p), ("n_indexed_host", ctypes.c_void_p),
+                ("C", ctypes.c_int32), ("M", ctypes.c_int32), ("dsub", ctypes.c_int32),
+                ("ncode", ctypes.c_int32), ("cap", ctypes.c_int32), ("n_sink", ctypes.c_int32)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("scale", ctypes.c_float), ("budget", ctypes.c_double), ("k_override", ctypes.c_int32),
+                ("background", ctypes.c_int32)]
+
+
+class _Debug(ctypes.Structure):
+    _fields_ = [("approx_logits", ctypes.c_void_p), ("selected", ctypes.c_void_p),
+                ("n_selected", ctypes.c_void_p), ("stage_events", ctypes.c_void_p)]
+
+
+NUM_STAGES = 6
+STAGE_NAMES = ("tables", "scan", "filter", "finalize", "attend", "merge")
+
+
+EXPORTS = ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode",
+           "hsa_decode_workspace_bytes", "dense_decode_workspace_bytes", "hsa_index_workspace_bytes",
+           "hsa_read_error", "hsa_strerror", "hsa_abi_sizes")
+
+_lib = None
+
+
+class HSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {hsa_strerror(status)} (status {status})")
+        self.status = status
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libpqhsa.so (built in-tree by sparse_long_context_pq_b200.build). Raises if missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    path = path or os.environ.get("PQHSA_LIB", _build.LIB_PATH)
+    if not os.path.exists(path):
+        raise RuntimeError(f"libpqhsa.so not found at {path}; build it with "
+                           f"`python -m sparse_long_context_pq_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.hsa_decode.argtypes = [P(_KV), P(_Index), vp, vp, P(_Params), P(_Debug), vp, sz, vp]
+    lib.dense_decode.argtypes = [P(_KV), vp, vp, ctypes.c_float, vp, sz, vp]
+    lib.hsa_build_from_codes.argtypes = [P(_KV), P(_Index), vp, sz, vp]
+    lib.hsa_append_encode.argtypes = [P(_KV), P(_Index), i32, vp, sz, vp]
+    lib.hsa_decode_workspace_bytes.argtypes = [P(_KV), P(_Index)]
+    lib.dense_decode_workspace_bytes.argtypes = [P(_KV)]
+    lib.hsa_index_workspace_bytes.argtypes = []
+    lib.hsa_read_error.argtypes = [vp, P(i32), vp]
+    lib.hsa_strerror.argtypes = [ctypes.c_int]
+    lib.hsa_abi_sizes.argtypes = [P(ctypes.c_int64)] * 4
+    for f in ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode", "hsa_read_error"):
+        getattr(lib, f).restype = ctypes.c_int
+    for f in ("hsa_decode_workspace_bytes", "dense_decode_workspace_bytes", "hsa_index_workspace_bytes"):
+        getattr(lib, f).restype = sz
+    lib.hsa_strerror.restype = ctypes.c_char_p
+    lib.hsa_abi_sizes.restype = None
+    sizes = [ctypes.c_int64() for _ in range(4)]
+    lib.hsa_abi_sizes(*[ctypes.byref(s) for s in sizes])
+    mine = [ctypes.sizeof(t) for t in (_KV, _Index, _Params, _Debug)]
+    if [s.value for s in sizes] != mine:
+        raise RuntimeError(f"ABI struct size mismatch: library {[s.value for s in sizes]} vs binding {mine}")
+    if path == _build.LIB_PATH or "PQHSA_LIB" in os.environ:
+        _lib = lib
+    return lib
+
+
+def hsa_strerror(status: int) -> str:
+    return load_library().hsa_strerror(int(status)).decode()
+
+
+def decode_k(budget: float, n_indexed: int, k_override: int = -1) -> int:
+    """Selected tokens per unit, as the library computes it: floor(budget * N) in double."""
+    if n_indexed <= 0:
+        return 0
+    if k_override >= 0:
+        return min(k_override, n_indexed)
+    f = float(budget) * float(n_indexed)
+    return min(n_indexed, int(f) if f > 0 else 0)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise HSAError(fn, status)
+
+
+@dataclass
+class PagedKV:
+    """Paged bf16 KV cache [num_pages][Hkv][page_size][D] plus the block table and lengths."""
+
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_table: torch.Tensor      # int32 [B, max_pages] (device)
+    seq_lens: torch.Tensor         # int32 [B] (device)
+    seq_lens_host: torch.Tensor    # int32 [B] (cpu)
+    Hq: int
+
+    def struct(self) -> _KV:
+        P, Hkv, ps, D = self.k_cache.shape
+        B, maxp = self.block_table.shape
+        assert self.k_cache.dtype == torch.bfloat16 and self.v_cache.dtype == torch.bfloat16
+        assert self.block_table.dtype == torch.int32 and self.seq_lens.dtype == torch.int32
+        assert self.seq_lens_host.dtype == torch.int32 and self.seq_lens_host.device.type == "cpu"
+        assert self.k_cache.is_contiguous() and self.v_cache.is_contiguous() and self.block_table.is_contiguous()
+        return _KV(_ptr(self.k_cache), _ptr(self.v_cache), _ptr(self.block_table), _ptr(self.seq_lens),
+                   _ptr(self.seq_lens_host), B, self.Hq, Hkv, D, ps, maxp, P)
+
+    @property
+    def B(self) -> int:
+        return self.block_table.shape[0]
+
+    @property
+    def Hkv(self) -> int:
+        return self.k_cache.shape[1]
+
+
+@dataclass
+class PQIndex:
+    """Per-(sequence, KV head) IVF-PQ index storage (caller-owned device tensors)."""
+
+    centroids: torch.Tensor        # fp32 [B, Hkv, C, D]
+    codebooks: torch.Tensor        # fp32 [B, Hkv, M, 256, 8]
+    codes: torch.Tensor            # uint8 [B, Hkv, cap, M]
+    ids: torch.Tensor              # int16 storage of u16 cluster ids [B, Hkv, cap]
+    sum_v: torch.Tensor            # fp32 [B, Hkv, C, D]
+    mean_v: torch.Tensor           # fp32 [B, Hkv, C, D]
+    count: torch.Tensor            # int32 [B, Hkv, C]
+    n_indexed: torch.Tensor        # int32 [B] (device)
+    n_indexed_host: torch.Tensor   # int32 [B] (cpu)
+    n_sink: int
+
+    @staticmethod
+    def allocate(B: int, Hkv: int, C: int, cap: int, n_sink: int, device) -> "PQIndex":
+        f = dict(device=device, dtype=torch.float32)
+        return PQIndex(
+            centroids=torch.zeros(B, Hkv, C, HEAD_DIM, **f),
+            codebooks=torch.zeros(B, Hkv, M_SUB, NCODE, DSUB, **f),
+            codes=torch.zeros(B, Hkv, cap, M_SUB, device=device, dtype=torch.uint8),
+            ids=torch.zeros(B, Hkv, cap, device=device, dtype=torch.int16),
+            sum_v=torch.zeros(B, Hkv, C, HEAD_DIM, **f),
+            mean_v=torch.zeros(B, Hkv, C, HEAD_DIM, **f),
+            count=torch.zeros(B, Hkv, C, device=device, dtype=torch.int32),
+            n_indexed=torch.zeros(B, device=device, dtype=torch.int32),
+            n_indexed_host=torch.zeros(B, dtype=torch.int32),
+            n_sink=n_sink,
+        )
+
+    @property
+    def C(self) -> int:
+        return self.centroids.shape[2]
+
+    @property
+    def cap(self) -> int:
+        return self.codes.shape[2]
+
+    def struct(self) -> _Index:
+        for t in (self.centroids, self.codebooks, self.codes, self.ids, self.sum_v, self.mean_v, self.count):
+            assert t.is_contiguous()
+        assert self.n_indexed_host.device.type == "cpu" and self.n_indexed_host.dtype == torch.int32
+        return _Index(_ptr(self.centroids), _ptr(self.codebooks), _ptr(self.codes), _ptr(self.ids),
+                      _ptr(self.sum_v), _ptr(self.mean_v), _ptr(self.count), _ptr(self.n_indexed),
+                      _ptr(self.n_indexed_host), self.C, M_SUB, DSUB, NCODE, self.cap, self.n_sink)
+
+
+def hsa_decode_workspace_bytes(kv: PagedKV, index: PQIndex) -> int:
+    kvs, ixs = kv.struct(), index.struct()
+    n = load_library().hsa_decode_workspace_bytes(ctypes.byref(kvs), ctypes.byref(ixs))
+    if n == 0:
+        raise HSAError("hsa_decode_workspace_bytes", 1)
+    return int(n)
+
+
+def dense_decode_workspace_bytes(kv: PagedKV) -> int:
+    kvs = kv.struct()
+    n = load_library().dense_decode_workspace_bytes(ctypes.byref(kvs))
+    if n == 0:
+        raise HSAError("dense_decode_workspace_bytes", 1)
+    return int(n)
+
+
+def hsa_index_workspace_bytes() -> int:
+    return int(load_library().hsa_index_workspace_bytes())
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A zeroed workspace buffer (torch allocations are 256-byte aligned)."""
+    return torch.zeros(max(256, (nbytes + 255) // 256 * 256), dtype=torch.uint8, device=device)
+
+
+def hsa_decode(kv: PagedKV, index: PQIndex, q: torch.Tensor, out: Optional[torch.Tensor] = None, *,
+               scale: float, budget: float = 0.01, k_override: int = -1, background: bool = True,
+               approx_logits: Optional[torch.Tensor] = None, selected: Optional[torch.Tensor] = None,
+               n_selected: Optional[torch.Tensor] = None, workspace_buf: Optional[torch.Tensor] = None,
+               stage_events=None, stream=None) -> torch.Tensor:
+    """One PQ-HSA decode step (see hsa_decode in include/pqhsa.h). q, out: fp32 [B, Hq, D]."""
+    assert q.dtype == torch.float32 and q.is_contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    kvs, ixs = kv.struct(), index.struct()
+    lib = load_library()
+    if workspace_buf is None:
+        workspace_buf = workspace(hsa_decode_workspace_bytes(kv, index), q.device)
+    prm = _Params(float(scale), float(budget), int(k_override), 1 if background else 0)
+    ev_arr = None
+    if stage_events is not None:
+        assert len(stage_events) == NUM_STAGES + 1
+        ev_arr = (ctypes.c_void_p * (NUM_STAGES + 1))(*[e.cuda_event for e in stage_events])
+    dbg = _Debug(_ptr(approx_logits), _ptr(selected), _ptr(n_selected),
+                 ctypes.cast(ev_arr, ctypes.c_void_p) if ev_arr is not None else None)
+    st = lib.hsa_decode(ctypes.byref(kvs), ctypes.byref(ixs), q.data_ptr(), out.data_ptr(), ctypes.byref(prm),
+                        ctypes.byref(dbg), workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
+    _check("hsa_decode", st)
+    return out
+
+
+def dense_decode(kv: PagedKV, q: torch.Tensor, out: Optional[torch.Tensor] = None, *, scale: float,
+                 workspace_buf: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense split-K GQA decode over every token (see dense_decode in include/pqhsa.h)."""
+    assert q.dtype == torch.float32 and q.is_contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    kvs = kv.struct()
+    if workspace_buf is None:
+        workspace_buf = workspace(dense_decode_workspace_bytes(kv), q.device)
+    st = load_library().dense_decode(ctypes.byref(kvs), q.data_ptr(), out.data_ptr(), ctypes.c_float(scale),
+                                     workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
+    _check("dense_decode", st)
+    return out
+
+
+def hsa_build_from_codes(kv: PagedKV, index: PQIndex, workspace_buf: Optional[torch.Tensor] = None,
+                         stream=None) -> None:
+    """count / sum_v / mean_v of every cluster from the caller's codes and ids."""
+    kvs, ixs = kv.struct(), index.struct()
+    if workspace_buf is None:
+        workspace_buf = workspace(hsa_index_workspace_bytes(), index.centroids.device)
+    st = load_library().hsa_build_from_codes(ctypes.byref(kvs), ctypes.byref(ixs), workspace_buf.data_ptr(),
+                                             workspace_buf.numel(), _stream(stream))
+    _check("hsa_build_from_codes", st)
+
+
+def hsa_append_encode(kv: PagedKV, index: PQIndex, n_new: int, workspace_buf: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+    """Encode the next n_new tokens of every sequence into the index (advances n_indexed)."""
+    kvs, ixs = kv.struct(), index.struct()
+    if workspace_buf is None:
+        workspace_buf = workspace(hsa_index_workspace_bytes(), index.centroids.device)
+    st = load_library().hsa_append_encode(ctypes.byref(kvs), ctypes.byref(ixs), int(n_new),
+                                          workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
+    _check("hsa_append_encode", st)
+
+
+def hsa_read_error(workspace_buf: torch.Tensor, stream=None) -> int:
+    """Read and clear the device error word of a workspace (synchronises the stream)."""
+    v = ctypes.c_int32(0)
+    st = load_library().hsa_read_error(workspace_buf.data_ptr(), ctypes.byref(v), _stream(stream))
+    _check("hsa_read_error", st)
+    return int(v.value)

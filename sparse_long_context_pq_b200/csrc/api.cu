@@ -1,0 +1,511 @@
+// Host side of the C ABI declared in include/pqhsa.h: argument validation,
+// workspace layout, split planning and kernel launches. No allocation, no
+// state across calls beyond a per-device cache of immutable properties.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include "../../include/pqhsa.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace pqhsa;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 148;
+  int scan_ctas_per_sm[9] = {0};
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+bool g_encode_tried = false;
+
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+    d.sms = sms;
+    d.ready = true;
+  }
+  return &d;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode_tried) {
+    g_encode_tried = true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return g_encode;
+}
+
+// Tensor map over a paged cache viewed as rows of D bf16: [num_pages*Hkv*page_size][128],
+// box = 64 columns x box_rows rows, 128-byte swizzle.
+bool make_kv_tmap(CUtensorMap* map, const void* base, const hsa_kv_cache* kv, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD),
+                        static_cast<cuuint64_t>(kv->num_pages) * kv->Hkv * kv->page_size};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+hsa_status check_kv(const hsa_kv_cache* kv) {
+  if (!kv || !kv->k_cache || !kv->v_cache || !kv->block_table || !kv->seq_lens || !kv->seq_lens_host)
+    return HSA_ERR_INVALID_ARG;
+  if (kv->B < 1 || kv->Hkv < 1 || kv->Hq < 1 || kv->max_pages < 1 || kv->num_pages < 1) return HSA_ERR_INVALID_ARG;
+  if (kv->Hq % kv->Hkv) return HSA_ERR_INVALID_ARG;
+  const int G = kv->Hq / kv->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return HSA_ERR_UNSUPPORTED;
+  if (kv->D != kD) return HSA_ERR_UNSUPPORTED;
+  if (!pow2(kv->page_size) || kv->page_size > 128) return HSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(kv->num_pages) * kv->Hkv * kv->page_size >= (1LL << 31)) return HSA_ERR_UNSUPPORTED;
+  if (!aligned(kv->k_cache, 256) || !aligned(kv->v_cache, 256) || !aligned(kv->block_table, 4) ||
+      !aligned(kv->seq_lens, 4))
+    return HSA_ERR_ALIGNMENT;
+  const long long tmax = static_cast<long long>(kv->max_pages) * kv->page_size;
+  for (int b = 0; b < kv->B; ++b)
+    if (kv->seq_lens_host[b] < 0 || kv->seq_lens_host[b] > tmax) return HSA_ERR_CAPACITY;
+  return HSA_OK;
+}
+
+hsa_status check_index(const hsa_kv_cache* kv, const hsa_index* ix, bool need_codes) {
+  if (!ix || !ix->centroids || !ix->codebooks || !ix->ids || !ix->mean_v || !ix->n_indexed || !ix->n_indexed_host)
+    return HSA_ERR_INVALID_ARG;
+  if (need_codes && !ix->codes) return HSA_ERR_INVALID_ARG;
+  if (ix->M != kM || ix->dsub != kDsub || ix->ncode != kNcode || ix->M * ix->dsub != kv->D) return HSA_ERR_UNSUPPORTED;
+  if (ix->C < 1 || ix->C > 65535 || ix->cap < 1 || ix->n_sink < 0) return HSA_ERR_INVALID_ARG;
+  if (!aligned(ix->centroids, 16) || !aligned(ix->codebooks, 16) || !aligned(ix->mean_v, 16) ||
+      (ix->codes && !aligned(ix->codes, 16)) || !aligned(ix->ids, 2))
+    return HSA_ERR_ALIGNMENT;
+  for (int b = 0; b < kv->B; ++b) {
+    const int T = kv->seq_lens_host[b];
+    const int n = ix->n_indexed_host[b];
+    if (n < 0) return HSA_ERR_INVALID_ARG;
+    if (n > ix->cap) return HSA_ERR_CAPACITY;
+    if (n > 0 && ix->n_sink + n > T) return HSA_ERR_CAPACITY;
+  }
+  return HSA_OK;
+}
+
+int host_unit_n(const hsa_kv_cache* kv, const hsa_index* ix, int b) {
+  const int T = std::max(0, kv->seq_lens_host[b]);
+  const int s0 = std::min(ix->n_sink, T);
+  const int N = std::max(0, std::min(ix->n_indexed_host[b], T - s0));
+  return std::min(N, ix->cap);
+}
+
+struct Split {
+  int nsplit;
+  int chunk;
+};
+
+// Choose the split-K chunking of E_max rows per unit: minimise (waves of CTAs) x (rows per CTA).
+Split plan_splits(long long E_max, int U, int nbg, int slots) {
+  Split best{1, static_cast<int>(std::max<long long>(kTile, (E_max + kTile - 1) / kTile * kTile))};
+  if (E_max <= 0) return Split{1, kTile};
+  double best_cost = 1e300;
+  for (int ns = 1; ns <= kMaxSplits; ++ns) {
+    long long chunk = (E_max + ns - 1) / ns;
+    chunk = (chunk + kTile - 1) / kTile * kTile;
+    const int ns_eff = static_cast<int>((E_max + chunk - 1) / chunk);
+    const long long ctas = static_cast<long long>(U) * (ns_eff + nbg);
+    const long long waves = (ctas + slots - 1) / slots;
+    const double per_cta = std::max<double>(static_cast<double>(chunk), nbg ? kBgClusters : 0.0) + 96.0;
+    const double cost = static_cast<double>(waves) * per_cta + 2.0 * ns_eff;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = Split{ns_eff, static_cast<int>(chunk)};
+    }
+  }
+  return best;
+}
+
+size_t dense_layout_bytes(int U, int G) {
+  const size_t parts = static_cast<size_t>(U) * kMaxSplits * G;
+  size_t o = align_up(sizeof(WsHeader), 256);
+  o += align_up(parts * sizeof(float), 256) * 2;
+  o += align_up(parts * kD * sizeof(float), 256);
+  return o;
+}
+
+#define RET_CUDA(x)                         \
+  do {                                      \
+    if ((x) != cudaSuccess) return HSA_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* hsa_strerror(hsa_status s) {
+  switch (s) {
+    case HSA_OK: return "ok";
+    case HSA_ERR_INVALID_ARG: return "invalid argument";
+    case HSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case HSA_ERR_CAPACITY: return "capacity exceeded";
+    case HSA_ERR_ALIGNMENT: return "misaligned pointer";
+    case HSA_ERR_WORKSPACE: return "workspace too small";
+    case HSA_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+void hsa_abi_sizes(int64_t* a, int64_t* b, int64_t* c, int64_t* d) {
+  if (a) *a = sizeof(hsa_kv_cache);
+  if (b) *b = sizeof(hsa_index);
+  if (c) *c = sizeof(hsa_decode_params);
+  if (d) *d = sizeof(hsa_debug);
+}
+
+size_t hsa_decode_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix) {
+  if (check_kv(kv) != HSA_OK || !ix || ix->C < 1 || ix->cap < 1) return 0;
+  const DecodeLayout L = make_decode_layout(kv->B * kv->Hkv, kv->Hq / kv->Hkv, ix->C, ix->cap, kMaxSplits);
+  return L.total;
+}
+
+size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv) {
+  if (check_kv(kv) != HSA_OK) return 0;
+  return dense_layout_bytes(kv->B * kv->Hkv, kv->Hq / kv->Hkv);
+}
+
+size_t hsa_index_workspace_bytes(void) { return sizeof(WsHeader); }
+
+hsa_status hsa_read_error(void* ws, int32_t* error_host, cudaStream_t stream) {
+  if (!ws || !error_host) return HSA_ERR_INVALID_ARG;
+  RET_CUDA(cudaMemcpyAsync(error_host, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
+  RET_CUDA(cudaMemsetAsync(ws, 0, sizeof(int32_t), stream));
+  RET_CUDA(cudaStreamSynchronize(stream));
+  return HSA_OK;
+}
+
+hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, float scale, void* ws, size_t ws_bytes,
+                        cudaStream_t stream) {
+  hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  if (!q || !out) return HSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16)) return HSA_ERR_ALIGNMENT;
+  const int U = kv->B * kv->Hkv, G = kv->Hq / kv->Hkv;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dense_layout_bytes(U, G)) return HSA_ERR_WORKSPACE;
+  const DeviceInfo* dev = device_info();
+  if (!dev) return HSA_ERR_CUDA;
+  long long Tmax = 0;
+  for (int b = 0; b < kv->B; ++b) Tmax = std::max<long long>(Tmax, kv->seq_lens_host[b]);
+  const Split sp = plan_splits(Tmax, U, 0, dev->sms * attend_slots_per_sm());
+  // Page tiles by tensor TMA need boxes of >= 8 rows (1024-byte aligned in shared memory).
+  const bool rows = kv->page_size < 8;
+  CUtensorMap tk = {}, tv = {};
+  const int box_rows = std::min(kv->page_size, kTile);
+  if (!rows && (!make_kv_tmap(&tk, kv->k_cache, kv, box_rows) || !make_kv_tmap(&tv, kv->v_cache, kv, box_rows)))
+    return HSA_ERR_CUDA;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t parts = static_cast<size_t>(U) * kMaxSplits * G;
+  size_t o = align_up(sizeof(WsHeader), 256);
+  float* pm = reinterpret_cast<float*>(base + o);
+  o += align_up(parts * sizeof(float), 256);
+  float* pl = reinterpret_cast<float*>(base + o);
+  o += align_up(parts * sizeof(float), 256);
+  float* pacc = reinterpret_cast<float*>(base + o);
+
+  AttendParams p = {};
+  p.k_cache = static_cast<const uint8_t*>(kv->k_cache);
+  p.v_cache = static_cast<const uint8_t*>(kv->v_cache);
+  p.q = q;
+  p.block_table = kv->block_table;
+  p.seq_lens = kv->seq_lens;
+  p.err = reinterpret_cast<int32_t*>(base);
+  p.pm = pm;
+  p.pl = pl;
+  p.pacc = pacc;
+  p.U = U;
+  p.B = kv->B;
+  p.Hq = kv->Hq;
+  p.Hkv = kv->Hkv;
+  p.page_size = kv->page_size;
+  p.max_pages = kv->max_pages;
+  p.num_pages = kv->num_pages;
+  p.nsplit = sp.nsplit;
+  p.chunk = sp.chunk;
+  p.S_tot = sp.nsplit;
+  p.qscale = scale * kLog2e;
+  p.k_override = -1;
+  RET_CUDA(launch_attend(G, false, rows, tk, tv, p, U * sp.nsplit, stream, false));
+  MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, sp.nsplit};
+  RET_CUDA(launch_merge(G, mp, stream, false));
+  return HSA_OK;
+}
+
+hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* q, float* out,
+                      const hsa_decode_params* prm, const hsa_debug* dbg, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  st = check_index(kv, ix, true);
+  if (st != HSA_OK) return st;
+  if (!q || !out || !prm) return HSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16)) return HSA_ERR_ALIGNMENT;
+  if (!(prm->budget >= 0.0) || !std::isfinite(prm->scale)) return HSA_ERR_INVALID_ARG;
+  const int U = kv->B * kv->Hkv, G = kv->Hq / kv->Hkv;
+  const size_t scan_smem = scan_smem_bytes(G, ix->C);
+  if (scan_smem > 227 * 1024) return HSA_ERR_UNSUPPORTED;
+  const DecodeLayout L = make_decode_layout(U, G, ix->C, ix->cap, kMaxSplits);
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HSA_ERR_WORKSPACE;
+  const DeviceInfo* dev = device_info();
+  if (!dev) return HSA_ERR_CUDA;
+
+  // ---- plan the exact split-K over sink + selected + tail rows ----
+  long long Emax = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    const int T = std::max(0, kv->seq_lens_host[b]);
+    const int s0 = std::min(ix->n_sink, T);
+    const int N = host_unit_n(kv, ix, b);
+    const int k = decode_k(prm->budget, prm->k_override, N);
+    Emax = std::max<long long>(Emax, static_cast<long long>(s0) + k + (T - s0 - N));
+  }
+  const Split sp = plan_splits(Emax, U, L.nbg, dev->sms * attend_slots_per_sm());
+  CUtensorMap tk = {}, tv = {};   // unused: gathered rows are bulk copies
+  cudaEvent_t* ev = dbg ? dbg->stage_events : nullptr;
+  auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], stream) : cudaSuccess; };
+
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* err = reinterpret_cast<int32_t*>(base);
+  UnitState* units = reinterpret_cast<UnitState*>(base + L.off_units);
+  float* bounds = reinterpret_cast<float*>(base + L.off_bounds);
+  float* lut = reinterpret_cast<float*>(base + L.off_lut);
+  float* qc = reinterpret_cast<float*>(base + L.off_qc);
+  float* W = reinterpret_cast<float*>(base + L.off_w);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.off_hist);
+  float* sigma = reinterpret_cast<float*>(base + L.off_sigma);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(base + L.off_bitmap);
+  unsigned long long* cand = reinterpret_cast<unsigned long long*>(base + L.off_cand);
+  int32_t* sel = reinterpret_cast<int32_t*>(base + L.off_sel);
+  float* pm = reinterpret_cast<float*>(base + L.off_pm);
+  float* pl = reinterpret_cast<float*>(base + L.off_pl);
+  float* pacc = reinterpret_cast<float*>(base + L.off_pacc);
+  const int S_tot = sp.nsplit + L.nbg;
+  if (S_tot > kMaxSplits + L.nbg) return HSA_ERR_WORKSPACE;
+
+  TablesParams tp = {};
+  tp.q = q;
+  tp.centroids = ix->centroids;
+  tp.codebooks = ix->codebooks;
+  tp.lut = lut;
+  tp.qc = qc;
+  tp.bounds = bounds;
+  tp.W = W;
+  tp.hist = hist;
+  tp.bitmap = bitmap;
+  tp.units = units;
+  tp.B = kv->B;
+  tp.Hq = kv->Hq;
+  tp.Hkv = kv->Hkv;
+  tp.C = ix->C;
+  tp.nq = L.nq;
+  tp.bitmap_words = L.bitmap_words;
+  tp.scale = prm->scale;
+  RET_CUDA(mark(0));
+  RET_CUDA(launch_tables(G, tp, stream, false));
+
+  ScanParams sc = {};
+  sc.codes = ix->codes;
+  sc.ids = ix->ids;
+  sc.seq_lens = kv->seq_lens;
+  sc.n_indexed = ix->n_indexed;
+  sc.lut = lut;
+  sc.qc = qc;
+  sc.bounds = bounds;
+  sc.W = W;
+  sc.hist = hist;
+  sc.sigma = sigma;
+  sc.approx_logits = dbg ? dbg->approx_logits : nullptr;
+  sc.err = err;
+  sc.B = kv->B;
+  sc.Hq = kv->Hq;
+  sc.Hkv = kv->Hkv;
+  sc.cap = ix->cap;
+  sc.C = ix->C;
+  sc.nq = L.nq;
+  sc.n_sink = ix->n_sink;
+  const int scan_per_sm = (scan_smem <= 110 * 1024) ? 2 : 1;
+  RET_CUDA(mark(1));
+  RET_CUDA(launch_scan(G, sc, dev->sms * scan_per_sm, stream, false));
+
+  SelectParams se = {};
+  se.seq_lens = kv->seq_lens;
+  se.n_indexed = ix->n_indexed;
+  se.codes = ix->codes;
+  se.ids = ix->ids;
+  se.lut = lut;
+  se.qc = qc;
+  se.bounds = bounds;
+  se.sigma = sigma;
+  se.hist = hist;
+  se.bitmap = bitmap;
+  se.cand = cand;
+  se.units = units;
+  se.sel = sel;
+  se.W = W;
+  se.dbg_selected = dbg ? dbg->selected : nullptr;
+  se.dbg_nselected = dbg ? dbg->n_selected : nullptr;
+  se.err = err;
+  se.B = kv->B;
+  se.Hkv = kv->Hkv;
+  se.cap = ix->cap;
+  se.C = ix->C;
+  se.nq = L.nq;
+  se.n_sink = ix->n_sink;
+  se.bitmap_words = L.bitmap_words;
+  se.k_override = prm->k_override;
+  se.background = prm->background ? 1 : 0;
+  se.budget = prm->budget;
+  RET_CUDA(mark(2));
+  RET_CUDA(launch_filter(G, se, dev->sms * 2, stream, false));
+  RET_CUDA(mark(3));
+  RET_CUDA(launch_finalize(G, se, stream, false));
+
+  AttendParams p = {};
+  p.k_cache = static_cast<const uint8_t*>(kv->k_cache);
+  p.v_cache = static_cast<const uint8_t*>(kv->v_cache);
+  p.q = q;
+  p.block_table = kv->block_table;
+  p.seq_lens = kv->seq_lens;
+  p.n_indexed = ix->n_indexed;
+  p.sel = sel;
+  p.err = err;
+  p.pm = pm;
+  p.pl = pl;
+  p.pacc = pacc;
+  p.W = W;
+  p.mean_v = ix->mean_v;
+  p.bounds = bounds;
+  p.U = U;
+  p.B = kv->B;
+  p.Hq = kv->Hq;
+  p.Hkv = kv->Hkv;
+  p.page_size = kv->page_size;
+  p.max_pages = kv->max_pages;
+  p.num_pages = kv->num_pages;
+  p.cap = ix->cap;
+  p.n_sink = ix->n_sink;
+  p.nsplit = sp.nsplit;
+  p.chunk = sp.chunk;
+  p.S_tot = S_tot;
+  p.C = ix->C;
+  p.nbg = L.nbg;
+  p.nq = L.nq;
+  p.bg_enabled = prm->background ? 1 : 0;
+  p.k_override = prm->k_override;
+  p.budget = prm->budget;
+  p.qscale = prm->scale * kLog2e;
+  RET_CUDA(mark(4));
+  RET_CUDA(launch_attend(G, true, true, tk, tv, p, U * (sp.nsplit + L.nbg), stream, false));
+  MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, S_tot};
+  RET_CUDA(mark(5));
+  RET_CUDA(launch_merge(G, mp, stream, false));
+  RET_CUDA(mark(6));
+  return HSA_OK;
+}
+
+static IndexParams index_params(const hsa_kv_cache* kv, hsa_index* ix, void* ws) {
+  IndexParams p = {};
+  p.k_cache = static_cast<const uint16_t*>(kv->k_cache);
+  p.v_cache = static_cast<const uint16_t*>(kv->v_cache);
+  p.block_table = kv->block_table;
+  p.seq_lens = kv->seq_lens;
+  p.centroids = ix->centroids;
+  p.codebooks = ix->codebooks;
+  p.codes = ix->codes;
+  p.ids = ix->ids;
+  p.sum_v = ix->sum_v;
+  p.mean_v = ix->mean_v;
+  p.count = ix->count;
+  p.n_indexed = ix->n_indexed;
+  p.err = static_cast<int32_t*>(ws);
+  p.B = kv->B;
+  p.Hkv = kv->Hkv;
+  p.page_size = kv->page_size;
+  p.max_pages = kv->max_pages;
+  p.num_pages = kv->num_pages;
+  p.C = ix->C;
+  p.cap = ix->cap;
+  p.n_sink = ix->n_sink;
+  return p;
+}
+
+hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* ix, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+  hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  st = check_index(kv, ix, false);
+  if (st != HSA_OK) return st;
+  if (!ix->sum_v || !ix->count) return HSA_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < hsa_index_workspace_bytes()) return HSA_ERR_WORKSPACE;
+  int nmax = 0;
+  for (int b = 0; b < kv->B; ++b) nmax = std::max(nmax, ix->n_indexed_host[b]);
+  IndexParams p = index_params(kv, ix, ws);
+  p.slot_lo_from_indexed = 0;
+  p.n_slots = -1;
+  p.bump_indexed = 0;
+  p.zero_if_empty = 0;
+  RET_CUDA(launch_zero_stats(p, stream));
+  RET_CUDA(launch_accumulate(p, nmax, stream));
+  RET_CUDA(launch_means(p, stream));
+  return HSA_OK;
+}
+
+hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_new, void* ws, size_t ws_bytes,
+                             cudaStream_t stream) {
+  hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  st = check_index(kv, ix, true);
+  if (st != HSA_OK) return st;
+  if (!ix->sum_v || !ix->count) return HSA_ERR_INVALID_ARG;
+  if (n_new < 0) return HSA_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < hsa_index_workspace_bytes()) return HSA_ERR_WORKSPACE;
+  for (int b = 0; b < kv->B; ++b) {
+    const long long N = ix->n_indexed_host[b];
+    if (N + n_new > ix->cap) return HSA_ERR_CAPACITY;
+    if (ix->n_sink + N + n_new > kv->seq_lens_host[b]) return HSA_ERR_CAPACITY;
+  }
+  if (n_new == 0) return HSA_OK;
+  IndexParams p = index_params(kv, ix, ws);
+  p.slot_lo_from_indexed = 1;
+  p.n_slots = n_new;
+  p.bump_indexed = 1;
+  p.zero_if_empty = 1;
+  RET_CUDA(launch_zero_stats(p, stream));
+  RET_CUDA(launch_encode(p, n_new, stream));
+  RET_CUDA(launch_accumulate(p, n_new, stream));
+  RET_CUDA(launch_means(p, stream));
+  for (int b = 0; b < kv->B; ++b) ix->n_indexed_host[b] += n_new;
+  return HSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,246 @@
+// IVF-PQ index maintenance for PQ-HSA: cluster statistics of the indexed
+// tokens' values (count, sum, mean) and batched encoding of new tokens.
+//
+// Source: rit.work "pq-hsa-long-context-attention", section
+// "Как приблизительные оценки возвращают отброшенный контекст": the index is
+// built after prefill, new tokens are kept outside it and added in batches,
+// and an unread token's value is represented by its index group's mean value.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pqhsa {
+
+namespace {
+
+__device__ __forceinline__ int slot_base(const IndexParams& p, int b) {
+  return p.slot_lo_from_indexed ? max(0, p.n_indexed[b]) : 0;
+}
+__device__ __forceinline__ int slot_count(const IndexParams& p, int b) {
+  return p.n_slots >= 0 ? p.n_slots : max(0, p.n_indexed[b]);
+}
+
+// Row address of (position pos, KV head h) of sequence b, or null for an invalid page.
+__device__ __forceinline__ const uint16_t* kv_row(const IndexParams& p, const uint16_t* cache, int b, int h, int pos) {
+  const int lp = pos / p.page_size;
+  const int page = (pos >= 0 && lp < p.max_pages) ? p.block_table[static_cast<size_t>(b) * p.max_pages + lp] : -1;
+  if (page < 0 || page >= p.num_pages) {
+    record_error(p.err, HSA_DEVERR_PAGE);
+    return nullptr;
+  }
+  return cache + ((static_cast<size_t>(page) * p.Hkv + h) * p.page_size + (pos % p.page_size)) * kD;
+}
+
+__global__ void zero_stats_kernel(IndexParams p) {
+  const size_t per_unit = static_cast<size_t>(p.C) * kD;
+  const size_t U = static_cast<size_t>(p.B) * p.Hkv;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < U * per_unit;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int u = static_cast<int>(i / per_unit);
+    if (p.zero_if_empty && p.n_indexed[u / p.Hkv] != 0) continue;
+    p.sum_v[i] = 0.f;
+    if (i % kD == 0) p.count[i / kD] = 0;
+  }
+}
+
+// Warp per token: add the token's value row to its cluster's sum and count.
+__global__ void __launch_bounds__(256) accumulate_kernel(IndexParams p) {
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv, h = u % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = p.seq_lens[b];
+  const int lo = slot_base(p, b);
+  const int n = slot_count(p, b);
+  for (int t = blockIdx.y * 64 + warp; t < min(n, (static_cast<int>(blockIdx.y) + 1) * 64); t += 8) {
+    const int slot = lo + t;
+    const int pos = p.n_sink + slot;
+    if (slot >= p.cap || pos >= T) continue;
+    uint32_t id = p.ids[static_cast<size_t>(u) * p.cap + slot];
+    if (id >= static_cast<uint32_t>(p.C)) {
+      if (lane == 0) record_error(p.err, HSA_DEVERR_CLUSTER);
+      continue;
+    }
+    const uint16_t* row = kv_row(p, p.v_cache, b, h, pos);
+    if (!row) continue;
+    const uint2 raw = *reinterpret_cast<const uint2*>(row + lane * 4);
+    const float4 v = make_float4(bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y));
+    float* dst = p.sum_v + (static_cast<size_t>(u) * p.C + id) * kD + lane * 4;
+    atomicAdd(reinterpret_cast<float4*>(dst), v);
+    if (lane == 0) atomicAdd(p.count + static_cast<size_t>(u) * p.C + id, 1);
+  }
+}
+
+// mean_v = sum_v / count (0 for an empty cluster); optionally advance n_indexed.
+__global__ void means_kernel(IndexParams p) {
+  const size_t total = static_cast<size_t>(p.B) * p.Hkv * p.C * kD;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int c = p.count[i / kD];
+    p.mean_v[i] = c > 0 ? __fdiv_rn(p.sum_v[i], static_cast<float>(c)) : 0.f;
+  }
+  if (p.bump_indexed && blockIdx.x == 0 && threadIdx.x == 0) {
+    for (int b = 0; b < p.B; ++b) p.n_indexed[b] = min(p.cap, p.n_indexed[b] + p.n_slots);
+  }
+}
+
+// Encode 32 new tokens of one unit: lane t of every warp holds token t's key in
+// registers; warp w scans centroids w, w+8, ...; then warp w finds the nearest
+// codeword of subspaces 2w and 2w+1 for all 32 residuals.
+constexpr int kEncTok = 32;
+
+__global__ void __launch_bounds__(256, 1) encode_kernel(IndexParams p) {
+  __shared__ float bd[8][kEncTok];
+  __shared__ int bc[8][kEncTok];
+  __shared__ int assign[kEncTok];
+  __shared__ float rs[kEncTok][kD + 1];
+  __shared__ uint8_t cs[kEncTok][kM];
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv, h = u % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = p.seq_lens[b];
+  const int base = slot_base(p, b);
+  const int n = slot_count(p, b);
+  const int t_idx = blockIdx.y * kEncTok + lane;
+  const int slot = base + t_idx;
+  const int pos = p.n_sink + slot;
+  const bool valid = t_idx < n && slot < p.cap && pos < T;
+
+  float kf[kD];
+  const uint16_t* row = valid ? kv_row(p, p.k_cache, b, h, pos) : nullptr;
+#pragma unroll
+  for (int c = 0; c < kD / 8; ++c) {
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (row) raw = *reinterpret_cast<const uint4*>(row + c * 8);
+    kf[c * 8 + 0] = bf16lo(raw.x);
+    kf[c * 8 + 1] = bf16hi(raw.x);
+    kf[c * 8 + 2] = bf16lo(raw.y);
+    kf[c * 8 + 3] = bf16hi(raw.y);
+    kf[c * 8 + 4] = bf16lo(raw.z);
+    kf[c * 8 + 5] = bf16hi(raw.z);
+    kf[c * 8 + 6] = bf16lo(raw.w);
+    kf[c * 8 + 7] = bf16hi(raw.w);
+  }
+
+  // nearest centroid: direct sum of squared differences, ties to the lower index
+  const float* cent = p.centroids + static_cast<size_t>(u) * p.C * kD;
+  float best = INFINITY;
+  int besti = 0x7fffffff;
+  for (int c = warp; c < p.C; c += 8) {
+    const float4* cr = reinterpret_cast<const float4*>(cent + static_cast<size_t>(c) * kD);
+    float dist = 0.f;
+#pragma unroll
+    for (int q4 = 0; q4 < kD / 4; ++q4) {
+      const float4 cv = __ldg(cr + q4);
+      float t0 = __fsub_rn(kf[q4 * 4 + 0], cv.x);
+      dist = fmaf(t0, t0, dist);
+      t0 = __fsub_rn(kf[q4 * 4 + 1], cv.y);
+      dist = fmaf(t0, t0, dist);
+      t0 = __fsub_rn(kf[q4 * 4 + 2], cv.z);
+      dist = fmaf(t0, t0, dist);
+      t0 = __fsub_rn(kf[q4 * 4 + 3], cv.w);
+      dist = fmaf(t0, t0, dist);
+    }
+    if (dist < best) {
+      best = dist;
+      besti = c;
+    }
+  }
+  bd[warp][lane] = best;
+  bc[warp][lane] = besti;
+  __syncthreads();
+  if (warp == 0) {
+    float bb = bd[0][lane];
+    int bi = bc[0][lane];
+    for (int w = 1; w < 8; ++w) {
+      const float d = bd[w][lane];
+      const int ci = bc[w][lane];
+      if (d < bb || (d == bb && ci < bi)) {
+        bb = d;
+        bi = ci;
+      }
+    }
+    if (bi >= p.C || bi < 0) bi = 0;   // only for an empty centroid set / NaN keys
+    assign[lane] = bi;
+    const float* ca = cent + static_cast<size_t>(bi) * kD;
+#pragma unroll
+    for (int d = 0; d < kD; ++d) rs[lane][d] = __fsub_rn(kf[d], __ldg(ca + d));
+  }
+  __syncthreads();
+
+  // nearest codeword per subspace of the residual
+  const float* cb = p.codebooks + static_cast<size_t>(u) * kM * kNcode * kDsub;
+  for (int si = 0; si < 2; ++si) {
+    const int s = warp * 2 + si;
+    float r[kDsub];
+#pragma unroll
+    for (int d = 0; d < kDsub; ++d) r[d] = rs[lane][s * kDsub + d];
+    float bb = INFINITY;
+    int bm = 0;
+    const float4* cw = reinterpret_cast<const float4*>(cb + static_cast<size_t>(s) * kNcode * kDsub);
+    for (int m = 0; m < kNcode; ++m) {
+      const float4 a = __ldg(cw + 2 * m), c2 = __ldg(cw + 2 * m + 1);
+      const float w8[8] = {a.x, a.y, a.z, a.w, c2.x, c2.y, c2.z, c2.w};
+      float dist = 0.f;
+#pragma unroll
+      for (int d = 0; d < kDsub; ++d) {
+        const float t0 = __fsub_rn(r[d], w8[d]);
+        dist = fmaf(t0, t0, dist);
+      }
+      if (dist < bb) {
+        bb = dist;
+        bm = m;
+      }
+    }
+    cs[lane][s] = static_cast<uint8_t>(bm);
+  }
+  __syncthreads();
+  if (warp == 0 && valid) {
+    p.ids[static_cast<size_t>(u) * p.cap + slot] = static_cast<uint16_t>(assign[lane]);
+    uint4 packed;
+    const uint8_t* c8 = cs[lane];
+    packed.x = c8[0] | (c8[1] << 8) | (c8[2] << 16) | (static_cast<uint32_t>(c8[3]) << 24);
+    packed.y = c8[4] | (c8[5] << 8) | (c8[6] << 16) | (static_cast<uint32_t>(c8[7]) << 24);
+    packed.z = c8[8] | (c8[9] << 8) | (c8[10] << 16) | (static_cast<uint32_t>(c8[11]) << 24);
+    packed.w = c8[12] | (c8[13] << 8) | (c8[14] << 16) | (static_cast<uint32_t>(c8[15]) << 24);
+    *reinterpret_cast<uint4*>(p.codes + (static_cast<size_t>(u) * p.cap + slot) * kM) = packed;
+  }
+}
+
+int grid_for(size_t work, int threads) {
+  size_t g = (work + threads - 1) / threads;
+  if (g > 148 * 16) g = 148 * 16;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+}  // namespace
+
+cudaError_t launch_zero_stats(const IndexParams& p, cudaStream_t stream) {
+  const size_t work = static_cast<size_t>(p.B) * p.Hkv * p.C * kD;
+  zero_stats_kernel<<<grid_for(work, 256), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode(const IndexParams& p, int max_new, cudaStream_t stream) {
+  if (max_new <= 0) return cudaSuccess;
+  const dim3 grid(p.B * p.Hkv, (max_new + kEncTok - 1) / kEncTok);
+  encode_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_accumulate(const IndexParams& p, int max_slots, cudaStream_t stream) {
+  if (max_slots <= 0) return cudaSuccess;
+  const dim3 grid(p.B * p.Hkv, (max_slots + 63) / 64);
+  accumulate_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_means(const IndexParams& p, cudaStream_t stream) {
+  const size_t work = static_cast<size_t>(p.B) * p.Hkv * p.C * kD;
+  means_kernel<<<grid_for(work, 256), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace pqhsa

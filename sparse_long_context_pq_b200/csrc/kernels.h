@@ -1,0 +1,166 @@
+// Internal launch interfaces between the C-ABI host code and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace pqhsa {
+
+// Upper/lower bound of the (scaled) approximate logit of every head of unit u:
+//   ub_g = sum_s max_m LUT_s[m][g] + max_c qc[c][g],  lb_g likewise with min.
+// bounds layout: [U][1 + nq][2 (max, min)][4 * GP]; part 0 holds the LUT sums,
+// parts 1..nq the per-slice centroid-term extremes.
+template <int G>
+__device__ __forceinline__ void unit_upper_bounds(const float* bounds, int u, int nq, float* ub) {
+  constexpr int G4 = ((G + 3) / 4) * 4;
+  const float* bu = bounds + static_cast<size_t>(u) * (1 + nq) * 2 * G4;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float qmax = -INFINITY;
+    for (int part = 1; part <= nq; ++part) qmax = fmaxf(qmax, bu[(part * 2 + 0) * G4 + g]);
+    ub[g] = bu[g] + qmax;
+  }
+}
+template <int G>
+__device__ __forceinline__ void unit_lower_bounds(const float* bounds, int u, int nq, float* lb) {
+  constexpr int G4 = ((G + 3) / 4) * 4;
+  const float* bu = bounds + static_cast<size_t>(u) * (1 + nq) * 2 * G4;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float qmin = INFINITY;
+    for (int part = 1; part <= nq; ++part) qmin = fminf(qmin, bu[(part * 2 + 1) * G4 + g]);
+    lb[g] = bu[G4 + g] + qmin;
+  }
+}
+
+struct AttendParams {
+  const uint8_t* k_cache;    // bf16 rows (row-gather modes)
+  const uint8_t* v_cache;
+  const float* q;            // [B][Hq][D]
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const int32_t* n_indexed;  // exact mode
+  const int32_t* sel;        // exact mode: [U][cap] selected positions
+  int32_t* err;
+  float* pm;                 // [U][S_tot][G]
+  float* pl;
+  float* pacc;               // [U][S_tot][G][D]
+  // background (exact mode)
+  const float* W;            // [U][G][C]
+  const float* mean_v;       // [U][C][D]
+  const float* bounds;
+  int U, B, Hq, Hkv, page_size, max_pages, num_pages, cap, n_sink;
+  int nsplit, chunk, S_tot, C, nbg, nq, bg_enabled, k_override;
+  double budget;
+  float qscale;              // scale * log2(e)
+};
+
+struct MergeParams {
+  const float* pm;
+  const float* pl;
+  const float* pacc;
+  float* out;
+  int B, Hq, Hkv, S_tot;
+};
+
+template <int G>
+__device__ void background_block(const AttendParams& p, int j, uint8_t* smem);
+
+int attend_slots_per_sm();
+size_t attend_smem_bytes(int G);
+// Row sources: kExact = sink + selected + tail list of hsa_decode, else every token.
+// Loading: page tiles by tensor TMA (dense, page_size >= 8) or one bulk copy per row.
+cudaError_t launch_attend(int G, bool exact, bool rows, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const AttendParams& p, int grid, cudaStream_t stream, bool pdl);
+cudaError_t launch_merge(int G, const MergeParams& p, cudaStream_t stream, bool pdl);
+
+// ---- PQ tables, scan, top-k ------------------------------------------------
+struct TablesParams {
+  const float* q;            // [B][Hq][D]
+  const float* centroids;    // [U][C][D]
+  const float* codebooks;    // [U][M][256][8]
+  float* lut;                // [U][GP][256][16][4]
+  float* qc;                 // [U][GP][C][4]
+  float* bounds;
+  float* W;                  // [U][G][C] zeroed here
+  uint32_t* hist;            // [U][NB] zeroed here
+  uint32_t* bitmap;          // [U][bitmap_words] zeroed here
+  UnitState* units;          // zeroed here
+  int B, Hq, Hkv, C, nq, bitmap_words;
+  float scale;
+};
+cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, bool pdl);
+
+struct ScanParams {
+  const uint8_t* codes;      // [U][cap][16]
+  const uint16_t* ids;       // [U][cap]
+  const int32_t* seq_lens;
+  const int32_t* n_indexed;
+  const float* lut;
+  const float* qc;
+  const float* bounds;
+  float* W;
+  uint32_t* hist;
+  float* sigma;              // [U][cap]
+  float* approx_logits;      // debug [B][Hq][cap] or null
+  int32_t* err;
+  int B, Hq, Hkv, cap, C, nq, n_sink;
+};
+cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t stream, bool pdl);
+size_t scan_smem_bytes(int G, int C);
+int scan_threads();
+
+struct SelectParams {
+  const int32_t* seq_lens;
+  const int32_t* n_indexed;
+  const uint8_t* codes;
+  const uint16_t* ids;
+  const float* lut;
+  const float* qc;
+  const float* bounds;
+  const float* sigma;
+  const uint32_t* hist;
+  uint32_t* bitmap;
+  unsigned long long* cand;  // [U][cap]
+  UnitState* units;
+  int32_t* sel;              // [U][cap]
+  float* W;
+  int32_t* dbg_selected;     // [U][cap] or null
+  int32_t* dbg_nselected;    // [U] or null
+  int32_t* err;
+  int B, Hkv, cap, C, nq, n_sink, bitmap_words, k_override, background;
+  double budget;
+};
+cudaError_t launch_filter(int G, const SelectParams& p, int grid, cudaStream_t stream, bool pdl);
+cudaError_t launch_finalize(int G, const SelectParams& p, cudaStream_t stream, bool pdl);
+
+// ---- index maintenance -----------------------------------------------------
+struct IndexParams {
+  const uint16_t* k_cache;
+  const uint16_t* v_cache;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const float* centroids;
+  const float* codebooks;
+  uint8_t* codes;
+  uint16_t* ids;
+  float* sum_v;
+  float* mean_v;
+  int32_t* count;
+  int32_t* n_indexed;
+  int32_t* err;
+  int B, Hkv, page_size, max_pages, num_pages, C, cap, n_sink;
+  int slot_lo_from_indexed;  // 1: slots start at n_indexed[b]; 0: slots start at 0
+  int n_slots;               // slots per unit to process (n_new), or -1 = n_indexed[b]
+  int bump_indexed;          // add n_slots to n_indexed[b] in the mean pass
+  int zero_if_empty;         // zero stats of units whose sequence has n_indexed == 0
+};
+cudaError_t launch_zero_stats(const IndexParams& p, cudaStream_t stream);
+cudaError_t launch_encode(const IndexParams& p, int max_new, cudaStream_t stream);
+cudaError_t launch_accumulate(const IndexParams& p, int max_slots, cudaStream_t stream);
+cudaError_t launch_means(const IndexParams& p, cudaStream_t stream);
+
+}  // namespace pqhsa

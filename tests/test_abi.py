@@ -1,0 +1,123 @@
+"""The C-ABI library loads, exports every function include/pqhsa.h declares, and rejects bad
+arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import sparse_long_context_pq_b200 as P
+from sparse_long_context_pq_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pqhsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return P.load_library()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("hsa_build_from_codes", "hsa_append_encode", "hsa_decode", "dense_decode", "hsa_strerror"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_abi_struct_sizes_match_binding(lib):
+    sizes = [ctypes.c_int64() for _ in range(4)]
+    lib.hsa_abi_sizes(*[ctypes.byref(s) for s in sizes])
+    assert [s.value for s in sizes] == [ctypes.sizeof(t) for t in (P._KV, P._Index, P._Params, P._Debug)]
+
+
+def test_strerror(lib):
+    assert P.hsa_strerror(0) == "ok"
+    assert P.hsa_strerror(2) == "unsupported shape"
+
+
+# ---- host-side validation (fake device pointers are never dereferenced on these paths) ----
+
+FAKE = 1 << 20   # 256-byte aligned, never touched
+
+
+def _kv(B=1, Hq=4, Hkv=1, D=128, page_size=16, max_pages=8, num_pages=8, seq=100, aligned=True):
+    lens = np.full(B, seq, dtype=np.int32)
+    base = FAKE if aligned else FAKE + 8
+    kv = P._KV(base, FAKE, FAKE, FAKE, lens.ctypes.data, B, Hq, Hkv, D, page_size, max_pages, num_pages)
+    return kv, lens
+
+
+def _ix(B=1, C=16, cap=128, n_idx=50, n_sink=4, M=16, dsub=8):
+    nh = np.full(B, n_idx, dtype=np.int32)
+    ix = P._Index(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, nh.ctypes.data, C, M, dsub, 256, cap, n_sink)
+    return ix, nh
+
+
+def _decode(lib, kv, ix, ws_bytes=1 << 30, q=FAKE):
+    prm = P._Params(0.088, 0.01, -1, 1)
+    return lib.hsa_decode(ctypes.byref(kv), ctypes.byref(ix), q, FAKE, ctypes.byref(prm), None, FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("mutate,status", [
+    (dict(Hq=6, Hkv=4), 1),            # Hq not a multiple of Hkv
+    (dict(Hq=12, Hkv=1), 2),           # group of 12 heads unsupported
+    (dict(D=64), 2),                   # head dim 64
+    (dict(page_size=24), 2),           # page size not a power of two
+    (dict(seq=1000), 3),               # longer than the block table
+    (dict(aligned=False), 4),          # cache pointer not 256-byte aligned
+])
+def test_decode_rejects_bad_cache(lib, mutate, status):
+    kv, lens = _kv(**mutate)
+    ix, nh = _ix()
+    assert _decode(lib, kv, ix) == status
+
+
+@pytest.mark.parametrize("mutate,status", [
+    (dict(M=8, dsub=16), 2),
+    (dict(C=0), 1),
+    (dict(n_idx=200), 3),              # more than cap
+    (dict(n_idx=99), 3),               # n_sink + N > T
+])
+def test_decode_rejects_bad_index(lib, mutate, status):
+    kv, lens = _kv()
+    ix, nh = _ix(**mutate)
+    assert _decode(lib, kv, ix) == status
+
+
+def test_decode_rejects_small_workspace_and_null_q(lib):
+    kv, lens = _kv()
+    ix, nh = _ix()
+    assert _decode(lib, kv, ix, ws_bytes=16) == 5
+    assert _decode(lib, kv, ix, q=None) == 1
+    need = lib.hsa_decode_workspace_bytes(ctypes.byref(kv), ctypes.byref(ix))
+    assert need > 0 and need % 256 == 0
+
+
+def test_append_checks_capacity(lib):
+    kv, lens = _kv(seq=100)
+    ix, nh = _ix(n_idx=50, n_sink=4, cap=60)
+    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix), 20, FAKE, 256, None) == 3   # cap 60 < 70
+    ix2, nh2 = _ix(n_idx=50, n_sink=4, cap=128)
+    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix2), 50, FAKE, 256, None) == 3  # beyond T
+    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix2), -1, FAKE, 256, None) == 1
+    assert nh2[0] == 50                                                                           # untouched
+
+
+def test_dense_rejects_bad_args(lib):
+    kv, lens = _kv()
+    assert lib.dense_decode(ctypes.byref(kv), FAKE + 4, FAKE, ctypes.c_float(1.0), FAKE, 1 << 30, None) == 4
+    assert lib.dense_decode(ctypes.byref(kv), FAKE, FAKE, ctypes.c_float(1.0), FAKE, 8, None) == 5
