@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <dlfcn.h>
 #include <stdint.h>
 
 #include <algorithm>
@@ -52,8 +53,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess && fn) {
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    } else if (void* h = dlopen("libcuda.so.1", RTLD_NOW | RTLD_LOCAL)) {
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(dlsym(h, "cuTensorMapEncodeTiled"));
+    }
   }
   return g_encode;
 }

@@ -422,7 +422,7 @@ cudaError_t launch_attend_t(const CUtensorMap& tk, const CUtensorMap& tv, const 
                             cudaStream_t stream, bool pdl) {
   auto kern = attend_kernel<G, kExact, kRows>;
   const size_t smem = AttendSmem<G>::total;
-  cudaError_t e = ensure_dyn_smem(kern, smem);
+  cudaError_t e = ensure_dyn_smem<attend_kernel<G, kExact, kRows>>(smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

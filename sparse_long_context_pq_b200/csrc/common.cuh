@@ -146,15 +146,16 @@ __host__ __device__ __forceinline__ int decode_k(double budget, int32_t k_overri
 
 // Raise a kernel's dynamic shared-memory limit once per device (never inside a
 // stream capture after the first call on that device).
-template <typename Kern>
-inline cudaError_t ensure_dyn_smem(Kern kern, size_t bytes) {
+// The cache is per kernel (template on the function itself, not its type).
+template <auto Kern>
+inline cudaError_t ensure_dyn_smem(size_t bytes) {
   static int set_bytes[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (set_bytes[dev] >= static_cast<int>(bytes)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
   if (e == cudaSuccess) set_bytes[dev] = static_cast<int>(bytes);
   return e;
 }

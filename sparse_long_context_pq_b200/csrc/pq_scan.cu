@@ -685,7 +685,7 @@ cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t strea
   const size_t smem = scan_smem_bytes(G, p.C);
 #define CALL(GG)                                                                                         \
   {                                                                                                      \
-    cudaError_t e = ensure_dyn_smem(scan_kernel<GG>, smem);                                             \
+    cudaError_t e = ensure_dyn_smem<scan_kernel<GG>>(smem);                                             \
     if (e != cudaSuccess) return e;                                                                      \
     return launch_ex(scan_kernel<GG>, dim3(grid), dim3(kScanThreads), smem, stream, pdl, p);            \
   }
