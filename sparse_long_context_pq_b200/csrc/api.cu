@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cmath>
 #include <mutex>
 
@@ -76,6 +77,17 @@ bool make_kv_tmap(CUtensorMap* map, const void* base, const hsa_kv_cache* kv, in
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Programmatic dependent launch between the kernels of a call (and with the
+// previous call): every kernel waits on griddepcontrol before touching memory a
+// predecessor writes. PQHSA_NO_PDL=1 turns it off.
+bool use_pdl() {
+  static const bool on = [] {
+    const char* e = getenv("PQHSA_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -260,9 +272,9 @@ hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, floa
   p.S_tot = sp.nsplit;
   p.qscale = scale * kLog2e;
   p.k_override = -1;
-  RET_CUDA(launch_attend(G, false, rows, tk, tv, p, U * sp.nsplit, stream, false));
+  RET_CUDA(launch_attend(G, false, rows, tk, tv, p, U * sp.nsplit, stream, use_pdl()));
   MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, sp.nsplit};
-  RET_CUDA(launch_merge(G, mp, stream, false));
+  RET_CUDA(launch_merge(G, mp, stream, use_pdl()));
   return HSA_OK;
 }
 
@@ -335,7 +347,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   tp.bitmap_words = L.bitmap_words;
   tp.scale = prm->scale;
   RET_CUDA(mark(0));
-  RET_CUDA(launch_tables(G, tp, stream, false));
+  RET_CUDA(launch_tables(G, tp, stream, use_pdl()));
 
   ScanParams sc = {};
   sc.codes = ix->codes;
@@ -359,7 +371,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   sc.n_sink = ix->n_sink;
   const int scan_per_sm = (scan_smem <= 110 * 1024) ? 2 : 1;
   RET_CUDA(mark(1));
-  RET_CUDA(launch_scan(G, sc, dev->sms * scan_per_sm, stream, false));
+  RET_CUDA(launch_scan(G, sc, dev->sms * scan_per_sm, stream, use_pdl()));
 
   SelectParams se = {};
   se.seq_lens = kv->seq_lens;
@@ -390,9 +402,9 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   se.background = prm->background ? 1 : 0;
   se.budget = prm->budget;
   RET_CUDA(mark(2));
-  RET_CUDA(launch_filter(G, se, dev->sms * 2, stream, false));
+  RET_CUDA(launch_filter(G, se, dev->sms * 2, stream, use_pdl()));
   RET_CUDA(mark(3));
-  RET_CUDA(launch_finalize(G, se, stream, false));
+  RET_CUDA(launch_finalize(G, se, stream, use_pdl()));
 
   AttendParams p = {};
   p.k_cache = static_cast<const uint8_t*>(kv->k_cache);
@@ -429,10 +441,10 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   p.budget = prm->budget;
   p.qscale = prm->scale * kLog2e;
   RET_CUDA(mark(4));
-  RET_CUDA(launch_attend(G, true, true, tk, tv, p, U * (sp.nsplit + L.nbg), stream, false));
+  RET_CUDA(launch_attend(G, true, true, tk, tv, p, U * (sp.nsplit + L.nbg), stream, use_pdl()));
   MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, S_tot};
   RET_CUDA(mark(5));
-  RET_CUDA(launch_merge(G, mp, stream, false));
+  RET_CUDA(launch_merge(G, mp, stream, use_pdl()));
   RET_CUDA(mark(6));
   return HSA_OK;
 }

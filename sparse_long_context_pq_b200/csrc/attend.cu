@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int h = u % p.Hkv;
 
   pdl_wait();
+  pdl_launch_dependents();
 
   // ---- row range of this split ------------------------------------------
   const int T = max(0, p.seq_lens[b]);
@@ -327,6 +328,7 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
   const int warp = tid >> 5, lane = tid & 31;
   constexpr int NW = kThreads / 32;
   pdl_wait();
+  pdl_launch_dependents();
   const int T = max(0, p.seq_lens[b]);
   const int s0 = min(p.n_sink, T);
   int N = max(0, min(p.n_indexed[b], T - s0));
@@ -396,6 +398,7 @@ namespace {
 template <int G>
 __global__ void __launch_bounds__(128) merge_kernel(MergeParams p) {
   pdl_wait();
+  pdl_launch_dependents();
   const int bq = blockIdx.x;            // b * Hq + qh
   const int b = bq / p.Hq, qh = bq % p.Hq;
   const int h = qh / G, g = qh % G;

@@ -100,6 +100,7 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
+  pdl_launch_dependents();
   for (int i = tid; i < G4 * kD; i += blockDim.x) {
     const int g = i / kD, d = i % kD;
     qsh[g][d] = (g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.scale : 0.f;
@@ -390,6 +391,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
   }
   const bool swap_words = (l7 >> 2) & 1;
   pdl_wait();
+  pdl_launch_dependents();
   for_each_segment(p.seq_lens, p.n_indexed, p.B, p.Hkv, p.n_sink, p.cap,
                    [&](int u, int j0, int j1) { scan_segment<G>(p, u, j0, j1, smem, ysoff, sel, swap_words); });
 }
@@ -403,6 +405,7 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
   __shared__ int sh_bstar;
   __shared__ uint32_t sh_above;
   pdl_wait();
+  pdl_launch_dependents();
   for_each_segment(p.seq_lens, p.n_indexed, p.B, p.Hkv, p.n_sink, p.cap, [&](int u, int j0, int j1) {
     const int b = u / p.Hkv;
     const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
@@ -488,6 +491,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
   const int b = u / p.Hkv;
   const int tid = threadIdx.x;
   pdl_wait();
+  pdl_launch_dependents();
   const int T = max(0, p.seq_lens[b]);
   const int s0 = min(p.n_sink, T);
   const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
