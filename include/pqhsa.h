@@ -139,6 +139,28 @@ size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv);
 hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, float scale,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * dense_decode_static: dense_decode that allocates nothing and takes no workspace.
+ * The PQ-HSA article has no counterpart to this call. It serves callers that cannot
+ * obtain device memory when they decode: a plain host program with no device
+ * allocator of its own, a serving runtime whose memory pool is fixed before traffic
+ * starts, or a decode loop that must never call cudaMalloc (an allocation there can
+ * stall or fail at the worst moment). Arguments and result are those of dense_decode.
+ * - Scratch: a static 8 MiB device array inside this library, reserved on every GPU
+ *   that loads the library until the process exits.
+ * - The first call on a device looks up that array's device address (once per
+ *   device, with that device current). Make that first call before any stream capture.
+ * - Limit: the split-K partials need B*Hkv*G*520 bytes per chunk; shapes for which
+ *   even one chunk does not fit in 8 MiB (B*Hkv*G above about 16000) return
+ *   HSA_ERR_WORKSPACE; otherwise the number of chunks is capped to fit.
+ * - Every call uses the same array and rewrites what it reads (nothing has to start
+ *   at zero; the array keeps the last call's partials). Calls that overlap on the
+ *   GPU (other streams or threads) race on it: serialise them.
+ * - There is no error word: out-of-range block-table entries are skipped, not reported.
+ */
+hsa_status dense_decode_static(const hsa_kv_cache* kv, const float* q, float* out, float scale,
+                               cudaStream_t stream);
+
 /* ---- index maintenance --------------------------------------------------- */
 
 /* Workspace bytes of hsa_build_from_codes / hsa_append_encode (error word only). */

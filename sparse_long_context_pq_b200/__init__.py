@@ -312,3 +312,20 @@ def hsa_read_error(workspace_buf: torch.Tensor, stream=None) -> int:
     st = load_library().hsa_read_error(workspace_buf.data_ptr(), ctypes.byref(v), _stream(stream))
     _check("hsa_read_error", st)
     return int(v.value)
+
+
+def dense_decode_static(kv: PagedKV, q: torch.Tensor, out: Optional[torch.Tensor] = None, *, scale: float,
+                        stream=None) -> torch.Tensor:
+    """dense_decode with the library's static scratch array: no workspace, no allocation in the
+    library (see dense_decode_static in include/pqhsa.h for its limit and its sharing rules)."""
+    assert q.dtype == torch.float32 and q.is_contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    lib = load_library()
+    fn = lib.dense_decode_static
+    fn.argtypes = [ctypes.POINTER(_KV), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    kvs = kv.struct()
+    _check("dense_decode_static", fn(ctypes.byref(kvs), q.data_ptr(), out.data_ptr(), ctypes.c_float(scale),
+                                     _stream(stream)))
+    return out
