@@ -14,10 +14,10 @@
 // one box per head-page (128-byte swizzle, 1024-byte aligned boxes); gathered
 // rows (sink + selected + tail) use one 1-D bulk copy per 256-byte row into a
 // 272-byte-stride layout. Both layouts are bank-conflict free for the two read
-// patterns below. Four consumer warps each own every fourth 32-token tile:
-// lane t computes token t's G logits, the warp keeps an online softmax, and
-// each lane accumulates 4 output dims for all G heads. Partials are (m, l, acc)
-// in log2 units.
+// patterns below (and for ldmatrix). Four consumer warps each own every fourth
+// 32-token tile and run it on the tensor cores (mma.sync m16n8k16 bf16, with q
+// and P split into bf16 hi + lo so the result keeps fp32-level accuracy), with an
+// online softmax per query head. Partials are (m, l, acc) in log2 units.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -31,7 +31,12 @@ namespace {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 6;
+// Tile t goes to consumer warp t % kConsumerWarps and stage t % kStages. kStages is a
+// multiple of kConsumerWarps, so every stage is always consumed by the same warp and
+// its mbarrier phases are awaited strictly in order: a parity wait can then never
+// alias a phase two steps ahead (which returns immediately on a parity barrier).
+constexpr int kStages = 4;
+static_assert(kStages % kConsumerWarps == 0, "each stage must belong to one consumer warp");
 constexpr int kHalfBytes = kTile * 128;        // swizzled: 32 rows x 128 B (64 bf16)
 constexpr int kRowPitch = 272;                 // padded: 256-byte row + 16
 constexpr int kStageBytes = 2 * kTile * kRowPitch;  // 17408 = 17 KB: K then V (either layout)
@@ -52,7 +57,7 @@ struct AttendSmem {
   static constexpr int GP = (G + 3) / 4;
   static constexpr size_t stages = static_cast<size_t>(kStages) * kStageBytes;
   static constexpr size_t qs = kD * GP * 16;
-  static constexpr size_t pbuf = kConsumerWarps * kTile * GP * 16;
+  static constexpr size_t pbuf = kConsumerWarps * 2 * 8 * kTile * 2;   // P hi/lo bf16 [8 heads][32 tokens]
   static constexpr size_t bars = 2 * kStages * 8;
   static constexpr size_t total = 1024 /*alignment slack*/ + stages + qs + pbuf + bars + 64;
 };
@@ -75,8 +80,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   float4* qs = reinterpret_cast<float4*>(smem + AttendSmem<G>::stages);               // [kD][GP]
-  float4* pbuf = qs + kD * GP;                                                          // [warps][32][GP]
-  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + kConsumerWarps * kTile * GP);
+  uint8_t* pbuf = reinterpret_cast<uint8_t*>(qs + kD * GP);                            // [warps] P buffers
+  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + AttendSmem<G>::pbuf);
   uint64_t* empty = full + kStages;
 
   const int tid = threadIdx.x;
@@ -141,8 +146,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int t = 0; t < ntiles && ok; ++t) {
       const int s = t % kStages;
       if (t >= kStages) {
-        if (lane == 0) ok = mbar_wait(&empty[s], ((t / kStages) - 1) & 1, p.err);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = mbar_wait_warp(&empty[s], ((t / kStages) - 1) & 1, p.err);
         if (!ok) break;
       }
       const int row0 = r0 + t * kTile;
@@ -179,117 +183,153 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
 
-  // ======================= consumer warps =======================
-  float m_run[G], l_lane[G], acc[G][4];
+  // ======================= consumer warps (tensor cores) =======================
+  // QK^T: S[tok][head] = K[tok][:] . q'[head][:] with m16n8k16 bf16 MMAs: A = K tile (ldmatrix),
+  // B = q' split into bf16 hi + lo (the bf16 x bf16 products are exact in fp32, so S carries
+  // ~16 mantissa bits of q'). PV: O^T[dim][head] += V^T[dim][tok] P[tok][head]: A = V^T
+  // (ldmatrix.trans), B = P split into hi + lo and transposed through a per-warp buffer.
+  const int grp = lane >> 2, tig = lane & 3;
+  uint32_t qb[8][2][2];   // [k-step][hi, lo][b0, b1]
+  {
+    const float* qsf = reinterpret_cast<const float*>(qs);   // [kD][GP * 4]
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m_run[g] = -INFINITY;
-    l_lane[g] = 0.f;
+    for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[g][i] = 0.f;
+      for (int r = 0; r < 2; ++r) {
+        const int d0 = 16 * kk + 8 * r + 2 * tig;
+        const float x0 = grp < G ? qsf[d0 * (GP * 4) + grp] : 0.f;
+        const float x1 = grp < G ? qsf[(d0 + 1) * (GP * 4) + grp] : 0.f;
+        uint32_t hi, lo;
+        split_bf16x2(x0, x1, hi, lo);
+        qb[kk][0][r] = hi;
+        qb[kk][1][r] = lo;
+      }
+    }
   }
-  const int vchunk = lane >> 1;          // 16-byte chunk holding dims 4*lane .. 4*lane+3
-  const int vsub = (lane & 1) * 8;
-  float4* pw = pbuf + warp * kTile * GP;
+  float oacc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oacc[i][e] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  uint16_t* pbw = reinterpret_cast<uint16_t*>(pbuf) + warp * (2 * 8 * kTile);   // [hi, lo][8 heads][32 tokens]
 
   for (int t = warp; t < ntiles; t += kConsumerWarps) {
     const int s = t % kStages;
-    if (!mbar_wait(&full[s], (t / kStages) & 1, p.err)) break;
+    if (!mbar_wait_warp(&full[s], (t / kStages) & 1, p.err)) break;   // converged before ldmatrix/mma
     const int nvalid = min(kTile, r1 - (r0 + t * kTile));
-    const uint8_t* st = stage_base + static_cast<size_t>(s) * kStageBytes;
+    uint8_t* st = stage_base + static_cast<size_t>(s) * kStageBytes;
+    const uint32_t sa = smem_addr(st);
+    if (nvalid < kTile) {
+      // stale V rows of a partial tile meet P = 0 in the MMA: make them finite zeros
+      for (int r = nvalid + (lane >> 4); r < kTile; r += 2)
+        *reinterpret_cast<uint4*>(st + v_area<kRows>() + chunk_off<kRows>(r, lane & 15)) = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
 
-    // ---- logits: lane = token row ----
-    float sc[G];
+    // ---- S = K q'^T: two 16-token row blocks x 8 k-steps x (hi, lo) ----
+    float sc[2][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) sc[g] = 0.f;
+    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
+      for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+      const int trow = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(st + chunk_off<kRows>(lane, hf * 8 + c));
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      for (int kk = 0; kk < 8; ++kk) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a0, a1, a2, a3, sa + chunk_off<kRows>(trow, 2 * kk + (lane >> 4)));
+        mma_bf16_16816(sc[mt], a0, a1, a2, a3, qb[kk][0][0], qb[kk][0][1]);
+        mma_bf16_16816(sc[mt], a0, a1, a2, a3, qb[kk][1][0], qb[kk][1][1]);
+      }
+    }
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float kv = e ? bf16hi(w[jj]) : bf16lo(w[jj]);
-            const int d = hf * 64 + c * 8 + jj * 2 + e;
+      for (int e = 0; e < 4; ++e)
+        if (16 * mt + grp + 8 * (e >> 1) >= nvalid) sc[mt][e] = -INFINITY;
+
+    // ---- online softmax, heads 2*tig + j ----
 #pragma unroll
-            for (int gp = 0; gp < GP; ++gp) {
-              const float4 qv = qs[d * GP + gp];
-              if (gp * 4 + 0 < G) sc[gp * 4 + 0] = fmaf(qv.x, kv, sc[gp * 4 + 0]);
-              if (gp * 4 + 1 < G) sc[gp * 4 + 1] = fmaf(qv.y, kv, sc[gp * 4 + 1]);
-              if (gp * 4 + 2 < G) sc[gp * 4 + 2] = fmaf(qv.z, kv, sc[gp * 4 + 2]);
-              if (gp * 4 + 3 < G) sc[gp * 4 + 3] = fmaf(qv.w, kv, sc[gp * 4 + 3]);
-            }
-          }
+    for (int j = 0; j < 2; ++j) {
+      float mx = fmaxf(fmaxf(sc[0][j], sc[0][2 + j]), fmaxf(sc[1][j], sc[1][2 + j]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m_run[j], mx);            // finite: every tile has a valid row
+      const float alpha = fast_exp2(m_run[j] - m_new);    // m_run = -inf -> 0
+      m_run[j] = m_new;
+      l_run[j] *= alpha;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        oacc[i][j] *= alpha;
+        oacc[i][2 + j] *= alpha;
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const float pv = fast_exp2(sc[mt][2 * h2 + j] - m_new);
+          l_run[j] += pv;
+          sc[mt][2 * h2 + j] = pv;
         }
       }
     }
-    const bool valid = lane < nvalid;
-    float pr[G];
+    // ---- P (bf16 hi, lo) to the warp buffer as [head][token] ----
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float sv = valid ? sc[g] : -INFINITY;
-      const float m_new = fmaxf(m_run[g], warp_max(sv));   // finite: at least one valid row
-      const float alpha = fast_exp2(m_run[g] - m_new);     // m_run = -inf -> 0
-      pr[g] = valid ? fast_exp2(sv - m_new) : 0.f;
-      l_lane[g] = l_lane[g] * alpha + pr[g];
+    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[g][i] *= alpha;
-      m_run[g] = m_new;
-    }
-#pragma unroll
-    for (int gp = 0; gp < GP; ++gp) {
-      float4 v;
-      v.x = (gp * 4 + 0 < G) ? pr[gp * 4 + 0] : 0.f;
-      v.y = (gp * 4 + 1 < G) ? pr[gp * 4 + 1] : 0.f;
-      v.z = (gp * 4 + 2 < G) ? pr[gp * 4 + 2] : 0.f;
-      v.w = (gp * 4 + 3 < G) ? pr[gp * 4 + 3] : 0.f;
-      pw[lane * GP + gp] = v;
+      for (int e = 0; e < 4; ++e) {
+        const int tok = 16 * mt + grp + 8 * (e >> 1);
+        const int head = 2 * tig + (e & 1);
+        uint16_t hb, lb;
+        split_bf16(sc[mt][e], hb, lb);
+        pbw[(0 * 8 + head) * kTile + tok] = hb;
+        pbw[(1 * 8 + head) * kTile + tok] = lb;
+      }
     }
     __syncwarp();
 
-    // ---- PV: lane owns dims 4*lane .. 4*lane+3 ----
-    const uint8_t* vbase = st + v_area<kRows>() + vsub;
-    for (int r = 0; r < nvalid; ++r) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(vbase + chunk_off<kRows>(r, vchunk));
-      const float v0 = bf16lo(raw.x), v1 = bf16hi(raw.x), v2 = bf16lo(raw.y), v3 = bf16hi(raw.y);
+    // ---- O^T += V^T P: 8 blocks of 16 dims x 2 k-steps of 16 tokens x (hi, lo) ----
 #pragma unroll
-      for (int gp = 0; gp < GP; ++gp) {
-        const float4 pv = pw[r * GP + gp];
-        const float pp[4] = {pv.x, pv.y, pv.z, pv.w};
+    for (int kk = 0; kk < 2; ++kk) {
+      const uint32_t* ph = reinterpret_cast<const uint32_t*>(pbw + (0 * 8 + grp) * kTile + 16 * kk);
+      const uint32_t* pl = reinterpret_cast<const uint32_t*>(pbw + (1 * 8 + grp) * kTile + 16 * kk);
+      const uint32_t bh0 = ph[tig], bh1 = ph[4 + tig], bl0 = pl[tig], bl1 = pl[4 + tig];
+      const int vrow = 16 * kk + (lane & 7) + 8 * (lane >> 4);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int g = gp * 4 + e;
-          if (g < G) {
-            acc[g][0] = fmaf(pp[e], v0, acc[g][0]);
-            acc[g][1] = fmaf(pp[e], v1, acc[g][1]);
-            acc[g][2] = fmaf(pp[e], v2, acc[g][2]);
-            acc[g][3] = fmaf(pp[e], v3, acc[g][3]);
-          }
-        }
+      for (int i = 0; i < 8; ++i) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(a0, a1, a2, a3, sa + v_area<kRows>() + chunk_off<kRows>(vrow, 2 * i + ((lane >> 3) & 1)));
+        mma_bf16_16816(oacc[i], a0, a1, a2, a3, bh0, bh1);
+        mma_bf16_16816(oacc[i], a0, a1, a2, a3, bl0, bl1);
       }
     }
+    if (nvalid < kTile) fence_proxy_async_smem();   // zero-fill before the stage's next async fill
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 
-  // ---- combine the consumer warps (reuse stage 0 area after the pipeline) ----
+  // ---- combine the consumer warps (reuse the stage area after the pipeline) ----
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-  float* cm = reinterpret_cast<float*>(stage_base);            // [warps][G]
-  float* cl = cm + kConsumerWarps * G;                         // [warps][G]
-  float* cacc = cl + kConsumerWarps * G;                       // [warps][G][kD]
+  float* cm = reinterpret_cast<float*>(stage_base);            // [warps][8]
+  float* cl = cm + kConsumerWarps * 8;                         // [warps][8]
+  float* cacc = cl + kConsumerWarps * 8;                       // [warps][8][kD]
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float lw = warp_sum(l_lane[g]);
-    if (lane == 0) {
-      cm[warp * G + g] = m_run[g];
-      cl[warp * G + g] = lw;
+  for (int j = 0; j < 2; ++j) {
+    float lw = l_run[j];
+    lw += __shfl_xor_sync(0xffffffffu, lw, 4);
+    lw += __shfl_xor_sync(0xffffffffu, lw, 8);
+    lw += __shfl_xor_sync(0xffffffffu, lw, 16);
+    if (grp == 0) {
+      cm[warp * 8 + 2 * tig + j] = m_run[j];
+      cl[warp * 8 + 2 * tig + j] = lw;
     }
-    *reinterpret_cast<float4*>(&cacc[(warp * G + g) * kD + lane * 4]) =
-        make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
   }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      cacc[(warp * 8 + 2 * tig + (e & 1)) * kD + 16 * i + grp + 8 * (e >> 1)] = oacc[i][e];
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
   const size_t slot = static_cast<size_t>(u) * p.S_tot + split;
   const int d = tid;  // 128 consumer threads, one output dim each
@@ -297,14 +337,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int g = 0; g < G; ++g) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * G + g]);
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * 8 + g]);
     float L = 0.f, a = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
-        const float f = fast_exp2(cm[w * G + g] - M);
-        L += f * cl[w * G + g];
-        a += f * cacc[(w * G + g) * kD + d];
+        const float f = fast_exp2(cm[w * 8 + g] - M);
+        L += f * cl[w * 8 + g];
+        a += f * cacc[(w * 8 + g) * kD + d];
       }
     }
     p.pacc[(slot * G + g) * kD + d] = a;
@@ -355,16 +395,30 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[g][i] = 0.f;
   }
-  for (int c = c0 + warp; c < c1; c += NW) {
-    const float4 m4 = *reinterpret_cast<const float4*>(mv + static_cast<size_t>(c) * kD + lane * 4);
+  constexpr int kR = 4;   // clusters whose loads are in flight together, per warp
+  for (int cb0 = c0 + warp; cb0 < c1; cb0 += kR * NW) {
+    float4 m4[kR];
+    float wv[kR][G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float w = fmaxf(W[g * p.C + c], 0.f);
-      lsum[g] += w;
-      acc[g][0] = fmaf(w, m4.x, acc[g][0]);
-      acc[g][1] = fmaf(w, m4.y, acc[g][1]);
-      acc[g][2] = fmaf(w, m4.z, acc[g][2]);
-      acc[g][3] = fmaf(w, m4.w, acc[g][3]);
+    for (int r = 0; r < kR; ++r) {
+      const int c = cb0 + r * NW;
+      const bool ok = c < c1;
+      m4[r] = ok ? *reinterpret_cast<const float4*>(mv + static_cast<size_t>(c) * kD + lane * 4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int g = 0; g < G; ++g) wv[r][g] = ok ? W[g * p.C + c] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float w = fmaxf(wv[r][g], 0.f);
+        lsum[g] += w;
+        acc[g][0] = fmaf(w, m4[r].x, acc[g][0]);
+        acc[g][1] = fmaf(w, m4[r].y, acc[g][1]);
+        acc[g][2] = fmaf(w, m4[r].z, acc[g][2]);
+        acc[g][3] = fmaf(w, m4[r].w, acc[g][3]);
+      }
     }
   }
   float* red = reinterpret_cast<float*>(smem);  // [NW][G][kD] + [NW][G]
@@ -395,29 +449,84 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
 namespace {
 
 // out[b, qh] = sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s over the S_tot partials of its unit.
+// 8 warps: factors e^{m_s - M} computed once, warp w sums splits w, w+8, ..., lane = 4 dims.
+constexpr int kMergeThreads = 256;
 template <int G>
-__global__ void __launch_bounds__(128) merge_kernel(MergeParams p) {
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
+  extern __shared__ float msm[];            // [S_tot] factors, then [8][kD] partial sums
+  __shared__ float sh_red[kMergeThreads / 32];
+  __shared__ float sh_M, sh_L;
   pdl_wait();
   pdl_launch_dependents();
-  const int bq = blockIdx.x;            // b * Hq + qh
+  const int bq = blockIdx.x;               // b * Hq + qh
   const int b = bq / p.Hq, qh = bq % p.Hq;
   const int h = qh / G, g = qh % G;
   const size_t u = static_cast<size_t>(b) * p.Hkv + h;
-  const int d = threadIdx.x;
-  float M = -INFINITY;
-  for (int s = 0; s < p.S_tot; ++s) M = fmaxf(M, p.pm[(u * p.S_tot + s) * G + g]);
-  float L = 0.f, a = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < p.S_tot; ++s) {
-      const size_t sl = (u * p.S_tot + s) * G + g;
-      const float m = p.pm[sl];
-      if (m == -INFINITY) continue;
-      const float f = fast_exp2(m - M);
-      L += f * p.pl[sl];
-      a += f * p.pacc[sl * kD + d];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = p.S_tot;
+  float* fs = msm;
+  float* red = msm + ((S + 3) & ~3);
+  float mloc = -INFINITY;
+  for (int s = tid; s < S; s += kMergeThreads) {
+    const float m = p.pm[(u * S + s) * G + g];
+    fs[s] = m;
+    mloc = fmaxf(mloc, m);
+  }
+  mloc = warp_max(mloc);
+  if (lane == 0) sh_red[warp] = mloc;
+  __syncthreads();
+  if (tid == 0) {
+    float M = sh_red[0];
+    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, sh_red[w]);
+    sh_M = M;
+  }
+  __syncthreads();
+  const float M = sh_M;
+  float lloc = 0.f;
+  for (int s = tid; s < S; s += kMergeThreads) {
+    const float m = fs[s];
+    const float f = (M == -INFINITY || m == -INFINITY) ? 0.f : fast_exp2(m - M);
+    fs[s] = f;
+    if (f != 0.f) lloc += f * p.pl[(u * S + s) * G + g];
+  }
+  lloc = warp_sum(lloc);
+  __syncthreads();
+  if (lane == 0) sh_red[warp] = lloc;
+  __syncthreads();
+  if (tid == 0) {
+    float L = 0.f;
+    for (int w = 0; w < kMergeThreads / 32; ++w) L += sh_red[w];
+    sh_L = L;
+  }
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int kR = 4;
+  for (int s0 = warp; s0 < S; s0 += kR * (kMergeThreads / 32)) {
+    float4 v[kR];
+    float f[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      const int s = s0 + r * (kMergeThreads / 32);
+      f[r] = s < S ? fs[s] : 0.f;
+      v[r] = f[r] != 0.f ? *reinterpret_cast<const float4*>(p.pacc + ((u * S + s) * G + g) * kD + lane * 4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      a.x = fmaf(f[r], v[r].x, a.x);
+      a.y = fmaf(f[r], v[r].y, a.y);
+      a.z = fmaf(f[r], v[r].z, a.z);
+      a.w = fmaf(f[r], v[r].w, a.w);
     }
   }
-  p.out[static_cast<size_t>(bq) * kD + d] = (L > 0.f) ? a / L : 0.f;
+  *reinterpret_cast<float4*>(&red[warp * kD + lane * 4]) = a;
+  __syncthreads();
+  if (tid < kD) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) t += red[w * kD + tid];
+    const float L = sh_L;
+    p.out[static_cast<size_t>(bq) * kD + tid] = (L > 0.f) ? t / L : 0.f;
+  }
 }
 
 template <int G, bool kExact, bool kRows>
@@ -444,8 +553,8 @@ template <int G>
 cudaError_t launch_merge_t(const MergeParams& p, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.B * p.Hq);
-  cfg.blockDim = dim3(kD);
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = (((p.S_tot + 3) & ~3) + (kMergeThreads / 32) * kD) * sizeof(float);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -1,6 +1,7 @@
 // Device-side helpers shared by the PQ-HSA kernels (sm_100a).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,6 +17,7 @@ constexpr int kNB = 2048;      // selection-score histogram bins
 constexpr int kBgClusters = 64;  // clusters per background CTA
 constexpr int kMaxSplits = 64;   // exact/dense split-K chunks per unit (upper bound)
 constexpr int kTile = 32;        // tokens per attention tile (one per lane)
+constexpr int kLutParts = 4;     // table-builder CTAs per unit for the LUT (4 subspaces each)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Workspace error word lives at offset 0 of every workspace.
@@ -68,15 +70,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase. Returns false (and records a timeout) when
-// the phase has not completed after a fixed number of polls.
-constexpr uint32_t kSpinLimit = 1u << 24;
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase: gives up after kWaitLimitNs of wall time,
+// records a timeout and returns false. Lanes may leave at different polls, so a
+// warp must reconverge (e.g. one polling lane + __shfl_sync) before any
+// .aligned warp-collective instruction.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) break;
   }
   record_error(err, HSA_DEVERR_TIMEOUT);
   return false;
+}
+
+// Warp-uniform wait: lane 0 polls, the verdict is broadcast (and the warp reconverged).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int32_t* err) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // 2-D tiled TMA load, completion signalled on `bar` (transaction bytes).
@@ -106,6 +126,44 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core fragments (mma.sync m16n8k16, bf16 in, fp32 accumulate)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                              uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// x = hi + lo with hi, lo bf16 (round to nearest): |x - hi - lo| <= 2^-16 |x| roughly.
+__device__ __forceinline__ void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
+  hi = __bfloat16_as_ushort(h);
+  lo = __bfloat16_as_ushort(l);
+}
+// Two values packed as bf16x2 (x0 in the low half), split into hi and lo parts.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  uint16_t h0, l0, h1, l1;
+  split_bf16(x0, h0, l0);
+  split_bf16(x1, h1, l1);
+  hi = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+  lo = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
 }
 
 // ---------------------------------------------------------------------------
@@ -212,7 +270,7 @@ __host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, 
   };
   const size_t u = static_cast<size_t>(U);
   L.off_units = take(u * sizeof(UnitState));
-  L.off_bounds = take(u * (1 + L.nq) * 2 * 4 * L.GP * sizeof(float));
+  L.off_bounds = take(u * (kLutParts + L.nq) * 2 * 4 * L.GP * sizeof(float));
   L.off_lut = take(u * L.GP * kNcode * kM * 4 * sizeof(float));
   L.off_qc = take(u * L.GP * C * 4 * sizeof(float));
   L.off_w = take(u * G * C * sizeof(float));

@@ -11,29 +11,40 @@ namespace pqhsa {
 
 // Upper/lower bound of the (scaled) approximate logit of every head of unit u:
 //   ub_g = sum_s max_m LUT_s[m][g] + max_c qc[c][g],  lb_g likewise with min.
-// bounds layout: [U][1 + nq][2 (max, min)][4 * GP]; part 0 holds the LUT sums,
-// parts 1..nq the per-slice centroid-term extremes.
+// bounds layout: [U][kLutParts + nq][2 (max, min)][4 * GP]; parts 0..kLutParts-1
+// hold partial sums over their subspaces of the per-subspace extremes, parts
+// kLutParts.. the extremes of one 128-cluster slice of the centroid term.
 template <int G>
-__device__ __forceinline__ void unit_upper_bounds(const float* bounds, int u, int nq, float* ub) {
+__device__ __forceinline__ void unit_bounds(const float* bounds, int u, int nq, float* ub, float* lb) {
   constexpr int G4 = ((G + 3) / 4) * 4;
-  const float* bu = bounds + static_cast<size_t>(u) * (1 + nq) * 2 * G4;
+  const float* bu = bounds + static_cast<size_t>(u) * (kLutParts + nq) * 2 * G4;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    float qmax = -INFINITY;
-    for (int part = 1; part <= nq; ++part) qmax = fmaxf(qmax, bu[(part * 2 + 0) * G4 + g]);
-    ub[g] = bu[g] + qmax;
+    float smax = 0.f, smin = 0.f;
+#pragma unroll
+    for (int part = 0; part < kLutParts; ++part) {
+      smax += bu[(part * 2 + 0) * G4 + g];
+      smin += bu[(part * 2 + 1) * G4 + g];
+    }
+    float qmax = -INFINITY, qmin = INFINITY;
+#pragma unroll 4
+    for (int part = kLutParts; part < kLutParts + nq; ++part) {
+      qmax = fmaxf(qmax, bu[(part * 2 + 0) * G4 + g]);
+      qmin = fminf(qmin, bu[(part * 2 + 1) * G4 + g]);
+    }
+    ub[g] = smax + qmax;
+    lb[g] = smin + qmin;
   }
 }
 template <int G>
+__device__ __forceinline__ void unit_upper_bounds(const float* bounds, int u, int nq, float* ub) {
+  float lb[G];
+  unit_bounds<G>(bounds, u, nq, ub, lb);
+}
+template <int G>
 __device__ __forceinline__ void unit_lower_bounds(const float* bounds, int u, int nq, float* lb) {
-  constexpr int G4 = ((G + 3) / 4) * 4;
-  const float* bu = bounds + static_cast<size_t>(u) * (1 + nq) * 2 * G4;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float qmin = INFINITY;
-    for (int part = 1; part <= nq; ++part) qmin = fminf(qmin, bu[(part * 2 + 1) * G4 + g]);
-    lb[g] = bu[G4 + g] + qmin;
-  }
+  float ub[G];
+  unit_bounds<G>(bounds, u, nq, ub, lb);
 }
 
 struct AttendParams {

@@ -92,65 +92,65 @@ template <int G>
 __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
   constexpr int GP = (G + 3) / 4;
   constexpr int G4 = GP * 4;
+  constexpr int kSubPerPart = kM / kLutParts;   // 4 subspaces per LUT CTA
+  constexpr int kQcPerWarp = 16;                // 128 clusters per slice / 8 warps
   __shared__ float qsh[G4][kD];
-  __shared__ float red[2][kM][G4];
-  __shared__ float wred[2][8][G4];
+  __shared__ float wred[2][8][kSubPerPart][G4];
   const int u = blockIdx.x;
   const int part = blockIdx.y;
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
   pdl_launch_dependents();
-  for (int i = tid; i < G4 * kD; i += blockDim.x) {
-    const int g = i / kD, d = i % kD;
-    qsh[g][d] = (g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.scale : 0.f;
-  }
-  __syncthreads();
+  float* bnd = p.bounds + static_cast<size_t>(u) * (kLutParts + p.nq) * 2 * G4;
 
-  if (part == 0) {
-    for (int i = tid; i < kNB; i += blockDim.x) p.hist[static_cast<size_t>(u) * kNB + i] = 0u;
-    for (int i = tid; i < p.bitmap_words; i += blockDim.x) p.bitmap[static_cast<size_t>(u) * p.bitmap_words + i] = 0u;
-    if (tid < static_cast<int>(sizeof(UnitState) / 4)) reinterpret_cast<int32_t*>(p.units + u)[tid] = 0;
-    // LUT[m][s][g] = sum_d q'_g[8s+d] * codeword[s][m][d]; warp w owns subspaces w and w+8.
-    for (int si = 0; si < 2; ++si) {
-      const int s = warp + 8 * si;
-      float mx[G4], mn[G4];
+  if (part < kLutParts) {
+    // ---- LUT[m][s][g] = sum_d q'_g[8s+d] * codeword[s][m][d] for 4 subspaces; thread = codeword m ----
+    const int m = tid;
+    float4 cw[kSubPerPart][2];
+#pragma unroll
+    for (int i = 0; i < kSubPerPart; ++i) {
+      const float4* src = reinterpret_cast<const float4*>(
+          p.codebooks + ((static_cast<size_t>(u) * kM + part * kSubPerPart + i) * kNcode + m) * kDsub);
+      cw[i][0] = src[0];
+      cw[i][1] = src[1];
+    }
+    for (int i = tid; i < G4 * kD; i += blockDim.x) {
+      const int g = i / kD, d = i % kD;
+      qsh[g][d] = (g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.scale : 0.f;
+    }
+    // zero this unit's selection state (spread over the LUT CTAs)
+    for (int i = part * blockDim.x + tid; i < kNB; i += kLutParts * blockDim.x)
+      p.hist[static_cast<size_t>(u) * kNB + i] = 0u;
+    for (int i = part * blockDim.x + tid; i < p.bitmap_words; i += kLutParts * blockDim.x)
+      p.bitmap[static_cast<size_t>(u) * p.bitmap_words + i] = 0u;
+    if (part == 0 && tid < static_cast<int>(sizeof(UnitState) / 4)) reinterpret_cast<int32_t*>(p.units + u)[tid] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kSubPerPart; ++i) {
+      const int s = part * kSubPerPart + i;
+      const float c8[8] = {cw[i][0].x, cw[i][0].y, cw[i][0].z, cw[i][0].w,
+                           cw[i][1].x, cw[i][1].y, cw[i][1].z, cw[i][1].w};
+      float val[G4];
 #pragma unroll
       for (int g = 0; g < G4; ++g) {
-        mx[g] = -INFINITY;
-        mn[g] = INFINITY;
+        float v = 0.f;
+#pragma unroll
+        for (int d = 0; d < kDsub; ++d) v = fmaf(qsh[g][s * kDsub + d], c8[d], v);
+        val[g] = v;
       }
-      for (int jm = 0; jm < kNcode / 32; ++jm) {
-        const int m = lane + 32 * jm;
-        const float4* cwp =
-            reinterpret_cast<const float4*>(p.codebooks + ((static_cast<size_t>(u) * kM + s) * kNcode + m) * kDsub);
-        const float4 c0 = cwp[0], c1 = cwp[1];
-        const float cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        float val[G4];
 #pragma unroll
-        for (int g = 0; g < G4; ++g) {
-          float v = 0.f;
-#pragma unroll
-          for (int d = 0; d < kDsub; ++d) v = fmaf(qsh[g][s * kDsub + d], cw[d], v);
-          val[g] = v;
-          if (g < G) {
-            mx[g] = fmaxf(mx[g], v);
-            mn[g] = fminf(mn[g], v);
-          }
-        }
-#pragma unroll
-        for (int gp = 0; gp < GP; ++gp) {
-          float4* dst = reinterpret_cast<float4*>(p.lut) + ((static_cast<size_t>(u) * GP + gp) * kNcode + m) * kM + s;
-          *dst = make_float4(val[gp * 4 + 0], val[gp * 4 + 1], val[gp * 4 + 2], val[gp * 4 + 3]);
-        }
+      for (int gp = 0; gp < GP; ++gp) {
+        float4* dst = reinterpret_cast<float4*>(p.lut) + ((static_cast<size_t>(u) * GP + gp) * kNcode + m) * kM + s;
+        *dst = make_float4(val[gp * 4 + 0], val[gp * 4 + 1], val[gp * 4 + 2], val[gp * 4 + 3]);
       }
 #pragma unroll
       for (int g = 0; g < G4; ++g) {
-        const float a = warp_max(mx[g]);
-        const float c = warp_min(mn[g]);
+        const float a = warp_max(val[g]);
+        const float c = warp_min(val[g]);
         if (lane == 0) {
-          red[0][s][g] = (g < G) ? a : 0.f;
-          red[1][s][g] = (g < G) ? c : 0.f;
+          wred[0][warp][i][g] = a;
+          wred[1][warp][i][g] = c;
         }
       }
     }
@@ -158,58 +158,80 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
     if (tid < 2 * G4) {
       const int mm = tid / G4, g = tid % G4;
       float acc = 0.f;
-      for (int s = 0; s < kM; ++s) acc += red[mm][s][g];
-      p.bounds[(static_cast<size_t>(u) * (1 + p.nq) * 2 + mm) * G4 + g] = acc;
+      for (int i = 0; i < kSubPerPart; ++i) {
+        float v = wred[mm][0][i][g];
+        for (int w = 1; w < 8; ++w) v = mm == 0 ? fmaxf(v, wred[0][w][i][g]) : fminf(v, wred[1][w][i][g]);
+        acc += v;
+      }
+      bnd[(part * 2 + mm) * G4 + g] = (g < G) ? acc : 0.f;
     }
   } else {
-    const int c0 = (part - 1) * 128;
-    const int c1 = min(p.C, c0 + 128);
-    const int nc = c1 - c0;
-    for (int i = tid; i < G * nc; i += blockDim.x)
-      p.W[(static_cast<size_t>(u) * G + i / nc) * p.C + c0 + (i % nc)] = 0.f;
+    // ---- qc[c][g] = q'_g . centroid_c for one 128-cluster slice; warp = 16 clusters, lane = 4 dims ----
+    const int slice = part - kLutParts;
+    const int c0 = slice * 128 + warp * kQcPerWarp;
+    float4 cv[kQcPerWarp];
+#pragma unroll
+    for (int i = 0; i < kQcPerWarp; ++i) {
+      const int c = c0 + i;
+      cv[i] = c < p.C ? *reinterpret_cast<const float4*>(p.centroids + (static_cast<size_t>(u) * p.C + c) * kD + lane * 4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int i = tid; i < G4 * kD; i += blockDim.x) {
+      const int g = i / kD, d = i % kD;
+      qsh[g][d] = (g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.scale : 0.f;
+    }
+    {   // zero this slice's cluster weights
+      const int cs = slice * 128, ce = min(p.C, cs + 128), nc = ce - cs;
+      for (int i = tid; i < G * nc; i += blockDim.x)
+        p.W[(static_cast<size_t>(u) * G + i / nc) * p.C + cs + (i % nc)] = 0.f;
+    }
+    __syncthreads();
     float mx[G4], mn[G4];
 #pragma unroll
     for (int g = 0; g < G4; ++g) {
       mx[g] = -INFINITY;
       mn[g] = INFINITY;
     }
-    for (int c = c0 + warp; c < c1; c += 8) {
-      const float4 cv = *reinterpret_cast<const float4*>(p.centroids + (static_cast<size_t>(u) * p.C + c) * kD + lane * 4);
+#pragma unroll
+    for (int i = 0; i < kQcPerWarp; ++i) {
+      const int c = c0 + i;
       float val[G4];
 #pragma unroll
       for (int g = 0; g < G4; ++g) {
-        float v = qsh[g][lane * 4 + 0] * cv.x;
-        v = fmaf(qsh[g][lane * 4 + 1], cv.y, v);
-        v = fmaf(qsh[g][lane * 4 + 2], cv.z, v);
-        v = fmaf(qsh[g][lane * 4 + 3], cv.w, v);
+        float v = qsh[g][lane * 4 + 0] * cv[i].x;
+        v = fmaf(qsh[g][lane * 4 + 1], cv[i].y, v);
+        v = fmaf(qsh[g][lane * 4 + 2], cv[i].z, v);
+        v = fmaf(qsh[g][lane * 4 + 3], cv[i].w, v);
         val[g] = warp_sum(v);
-        if (g < G) {
+      }
+      if (c < p.C) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
           mx[g] = fmaxf(mx[g], val[g]);
           mn[g] = fminf(mn[g], val[g]);
         }
-      }
 #pragma unroll
-      for (int gp = 0; gp < GP; ++gp) {
-        if (lane == gp) {
-          float4* dst = reinterpret_cast<float4*>(p.qc) + (static_cast<size_t>(u) * GP + gp) * p.C + c;
-          *dst = make_float4(val[gp * 4 + 0], val[gp * 4 + 1], val[gp * 4 + 2], val[gp * 4 + 3]);
+        for (int gp = 0; gp < GP; ++gp) {
+          if (lane == gp) {
+            float4* dst = reinterpret_cast<float4*>(p.qc) + (static_cast<size_t>(u) * GP + gp) * p.C + c;
+            *dst = make_float4(val[gp * 4 + 0], val[gp * 4 + 1], val[gp * 4 + 2], val[gp * 4 + 3]);
+          }
         }
       }
     }
     if (lane == 0) {
 #pragma unroll
       for (int g = 0; g < G4; ++g) {
-        wred[0][warp][g] = mx[g];
-        wred[1][warp][g] = mn[g];
+        wred[0][warp][0][g] = mx[g];
+        wred[1][warp][0][g] = mn[g];
       }
     }
     __syncthreads();
     if (tid < 2 * G4) {
       const int mm = tid / G4, g = tid % G4;
-      float v = mm == 0 ? -INFINITY : INFINITY;
-      for (int w = 0; w < 8; ++w) v = mm == 0 ? fmaxf(v, wred[0][w][g]) : fminf(v, wred[1][w][g]);
-      if (g >= G) v = 0.f;
-      p.bounds[((static_cast<size_t>(u) * (1 + p.nq) + part) * 2 + mm) * G4 + g] = v;
+      float v = wred[mm][0][0][g];
+      for (int w = 1; w < 8; ++w) v = mm == 0 ? fmaxf(v, wred[0][w][0][g]) : fminf(v, wred[1][w][0][g]);
+      bnd[(part * 2 + mm) * G4 + g] = (g < G) ? v : 0.f;
     }
   }
 }
@@ -218,108 +240,141 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
 // scan
 // ===========================================================================
 constexpr int kScanThreads = 256;
-constexpr int kScanUnroll = 4;
+constexpr int kScanUnroll = 2;   // tokens per thread per batch; the next batch is loaded while one is scored
 
 template <int G>
 struct ScanSmem {
   static constexpr int GP = (G + 3) / 4;
-  static size_t bytes(int C) {
-    return static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 +
-           static_cast<size_t>(G) * C * 4 + kNB * 4;
+  // tables (LUT, centroid terms), cluster weights, histogram; then the mbarrier
+  __host__ __device__ static size_t tables(int C) {
+    return align_up(static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 +
+                        static_cast<size_t>(G) * C * 4 + kNB * 4, 16);
   }
+  __host__ __device__ static size_t bytes(int C) { return tables(C) + 16; }
 };
 
-// Segment [j0, j1) of unit u: score every slot.
+template <int G>
+__device__ __forceinline__ void score_token(const uint4& code, uint32_t id, const uint8_t* lut_b, const float4* qc_s,
+                                            int C, const uint32_t ysoff[8], const uint32_t sel[4], bool swap_words,
+                                            float* sh) {
+  constexpr int GP = (G + 3) / 4;
+  uint32_t w0 = code.x, w1 = code.y, w2 = code.z, w3 = code.w;
+  if (swap_words) {
+    uint32_t t = w0; w0 = w1; w1 = t;
+    t = w2; w2 = w3; w3 = t;
+  }
+  float4 acc[GP];
+#pragma unroll
+  for (int gp = 0; gp < GP; ++gp) acc[gp] = qc_s[gp * C + id];
+#pragma unroll
+  for (int i = 0; i < kM; ++i) {
+    const uint32_t wd = (i < 4) ? w0 : (i < 8) ? w1 : (i < 12) ? w2 : w3;
+    // offset of LUT entry [code][s] with s = i ^ (lane & 7): code*256 + s*16
+    const uint32_t off = __byte_perm(wd, ysoff[i >> 1], sel[i & 3]);
+#pragma unroll
+    for (int gp = 0; gp < GP; ++gp) {
+      const float4 v = *reinterpret_cast<const float4*>(lut_b + gp * (kNcode * kM * 16) + off);
+      acc[gp].x = __fadd_rn(acc[gp].x, v.x);
+      acc[gp].y = __fadd_rn(acc[gp].y, v.y);
+      acc[gp].z = __fadd_rn(acc[gp].z, v.z);
+      acc[gp].w = __fadd_rn(acc[gp].w, v.w);
+    }
+  }
+#pragma unroll
+  for (int gp = 0; gp < GP; ++gp) {
+    if (gp * 4 + 0 < G) sh[gp * 4 + 0] = acc[gp].x;
+    if (gp * 4 + 1 < G) sh[gp * 4 + 1] = acc[gp].y;
+    if (gp * 4 + 2 < G) sh[gp * 4 + 2] = acc[gp].z;
+    if (gp * 4 + 3 < G) sh[gp * 4 + 3] = acc[gp].w;
+  }
+}
+
+// Segment [j0, j1) of unit u: score every slot. `phase` counts segments (mbarrier parity).
 template <int G>
 __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int j0, int j1, uint8_t* smem,
-                                             const uint32_t ysoff[8], const uint32_t sel[4], bool swap_words) {
+                                             uint64_t* bar, uint32_t phase, const uint32_t ysoff[8],
+                                             const uint32_t sel[4], bool swap_words) {
   constexpr int GP = (G + 3) / 4;
   const int tid = threadIdx.x;
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int C = p.C;
+  const uint32_t lut_bytes = GP * kNcode * kM * 16;
+  const uint32_t qc_bytes = GP * C * 16;
   float4* lut_s = reinterpret_cast<float4*>(smem);                               // [GP][256][16]
   float4* qc_s = lut_s + GP * kNcode * kM;                                       // [GP][C]
   float* w_s = reinterpret_cast<float*>(qc_s + GP * C);                          // [G][C]
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(w_s + G * C);                   // [NB]
 
   __syncthreads();  // previous segment finished with shared memory
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
-    uint4* dst = reinterpret_cast<uint4*>(lut_s);
-    for (int i = tid; i < GP * kNcode * kM; i += blockDim.x) dst[i] = src[i];
-    const uint4* srcq = reinterpret_cast<const uint4*>(p.qc) + static_cast<size_t>(u) * GP * C;
-    uint4* dstq = reinterpret_cast<uint4*>(qc_s);
-    for (int i = tid; i < GP * C; i += blockDim.x) dstq[i] = srcq[i];
-    for (int i = tid; i < G * C; i += blockDim.x) w_s[i] = 0.f;
-    for (int i = tid; i < kNB; i += blockDim.x) hist_s[i] = 0u;
+  if (tid == 0) {
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, lut_bytes + qc_bytes);
+    const uint8_t* lg = reinterpret_cast<const uint8_t*>(p.lut) + static_cast<size_t>(u) * lut_bytes;
+    for (uint32_t o = 0; o < lut_bytes; o += 32768u)
+      bulk_load(reinterpret_cast<uint8_t*>(lut_s) + o, lg + o, min(32768u, lut_bytes - o), bar);
+    const uint8_t* qg = reinterpret_cast<const uint8_t*>(p.qc) + static_cast<size_t>(u) * qc_bytes;
+    for (uint32_t o = 0; o < qc_bytes; o += 32768u)
+      bulk_load(reinterpret_cast<uint8_t*>(qc_s) + o, qg + o, min(32768u, qc_bytes - o), bar);
   }
-  float ub2[G];
+  for (int i = tid; i < G * C; i += blockDim.x) w_s[i] = 0.f;
+  for (int i = tid; i < kNB; i += blockDim.x) hist_s[i] = 0u;
+  float ub2[G], lo, inv;
   {
-    float ub[G];
-    unit_upper_bounds<G>(p.bounds, u, p.nq, ub);
+    float ub[G], lb[G];
+    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
+    float hi = ub[0];
+    lo = lb[0];
 #pragma unroll
-    for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
+    for (int g = 0; g < G; ++g) {
+      ub2[g] = ub[g] * kLog2e;
+      hi = fmaxf(hi, ub[g]);
+      lo = fmaxf(lo, lb[g]);
+    }
+    inv = (hi > lo) ? __fdiv_rn(static_cast<float>(kNB), __fsub_rn(hi, lo)) : 0.f;
   }
-  float lo, inv;
-  hist_range<G>(p.bounds, u, p.nq, lo, inv);
-  __syncthreads();
-
   const uint8_t* codes_u = p.codes + static_cast<size_t>(u) * p.cap * kM;
   const uint16_t* ids_u = p.ids + static_cast<size_t>(u) * p.cap;
   float* sig_u = p.sigma + static_cast<size_t>(u) * p.cap;
   const uint8_t* lut_b = reinterpret_cast<const uint8_t*>(lut_s);
+
+  // first batch of codes is in flight while the tables land
+  uint4 cw[kScanUnroll];
+  uint32_t idv[kScanUnroll];
+#pragma unroll
+  for (int r = 0; r < kScanUnroll; ++r) {
+    const int j = j0 + r * kScanThreads + tid;
+    if (j < j1) {
+      cw[r] = __ldcs(reinterpret_cast<const uint4*>(codes_u) + j);
+      idv[r] = __ldcs(ids_u + j);
+    }
+  }
+  __syncthreads();                       // zeroed W / histogram visible
+  mbar_wait(bar, phase & 1, p.err);      // tables landed
   bool bad_id = false;
 
   for (int base = j0; base < j1; base += kScanUnroll * kScanThreads) {
-    uint4 cw[kScanUnroll];
-    uint32_t idv[kScanUnroll];
+    const int nb = base + kScanUnroll * kScanThreads;
+    uint4 cwn[kScanUnroll];
+    uint32_t idn[kScanUnroll];
 #pragma unroll
     for (int r = 0; r < kScanUnroll; ++r) {
-      const int j = base + r * kScanThreads + tid;
+      const int j = nb + r * kScanThreads + tid;
       if (j < j1) {
-        cw[r] = __ldcs(reinterpret_cast<const uint4*>(codes_u) + j);
-        idv[r] = __ldcs(ids_u + j);
+        cwn[r] = __ldcs(reinterpret_cast<const uint4*>(codes_u) + j);
+        idn[r] = __ldcs(ids_u + j);
       }
     }
 #pragma unroll
     for (int r = 0; r < kScanUnroll; ++r) {
       const int j = base + r * kScanThreads + tid;
       if (j >= j1) continue;
-      uint32_t w0 = cw[r].x, w1 = cw[r].y, w2 = cw[r].z, w3 = cw[r].w;
-      if (swap_words) {
-        uint32_t t = w0; w0 = w1; w1 = t;
-        t = w2; w2 = w3; w3 = t;
-      }
       uint32_t id = idv[r];
       if (id >= static_cast<uint32_t>(C)) {
         bad_id = true;
         id = 0;
       }
-      float4 acc[GP];
-#pragma unroll
-      for (int gp = 0; gp < GP; ++gp) acc[gp] = qc_s[gp * C + id];
-#pragma unroll
-      for (int i = 0; i < kM; ++i) {
-        const uint32_t wd = (i < 4) ? w0 : (i < 8) ? w1 : (i < 12) ? w2 : w3;
-        // offset of LUT entry [code][s] with s = i ^ (lane & 7): code*256 + s*16
-        const uint32_t off = __byte_perm(wd, ysoff[i >> 1], sel[i & 3]);
-#pragma unroll
-        for (int gp = 0; gp < GP; ++gp) {
-          const float4 v = *reinterpret_cast<const float4*>(lut_b + gp * (kNcode * kM * 16) + off);
-          acc[gp].x = __fadd_rn(acc[gp].x, v.x);
-          acc[gp].y = __fadd_rn(acc[gp].y, v.y);
-          acc[gp].z = __fadd_rn(acc[gp].z, v.z);
-          acc[gp].w = __fadd_rn(acc[gp].w, v.w);
-        }
-      }
       float sh[G];
-#pragma unroll
-      for (int gp = 0; gp < GP; ++gp) {
-        if (gp * 4 + 0 < G) sh[gp * 4 + 0] = acc[gp].x;
-        if (gp * 4 + 1 < G) sh[gp * 4 + 1] = acc[gp].y;
-        if (gp * 4 + 2 < G) sh[gp * 4 + 2] = acc[gp].z;
-        if (gp * 4 + 3 < G) sh[gp * 4 + 3] = acc[gp].w;
-      }
+      score_token<G>(cw[r], id, lut_b, qc_s, C, ysoff, sel, swap_words, sh);
       float sg = sh[0];
 #pragma unroll
       for (int g = 1; g < G; ++g) sg = fmaxf(sg, sh[g]);
@@ -332,6 +387,11 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int j0,
 #pragma unroll
       for (int g = 0; g < G; ++g) atomicAdd(&w_s[g * C + id], fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])));
       atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
+    }
+#pragma unroll
+    for (int r = 0; r < kScanUnroll; ++r) {
+      cw[r] = cwn[r];
+      idv[r] = idn[r];
     }
   }
   if (bad_id) record_error(p.err, HSA_DEVERR_CLUSTER);
@@ -390,10 +450,18 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
     sel[i] = (4u + 2u * (i & 1)) | (bi << 4) | (5u << 8) | (5u << 12);
   }
   const bool swap_words = (l7 >> 2) & 1;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ScanSmem<G>::tables(p.C));
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
   pdl_wait();
   pdl_launch_dependents();
-  for_each_segment(p.seq_lens, p.n_indexed, p.B, p.Hkv, p.n_sink, p.cap,
-                   [&](int u, int j0, int j1) { scan_segment<G>(p, u, j0, j1, smem, ysoff, sel, swap_words); });
+  uint32_t phase = 0;
+  for_each_segment(p.seq_lens, p.n_indexed, p.B, p.Hkv, p.n_sink, p.cap, [&](int u, int j0, int j1) {
+    scan_segment<G>(p, u, j0, j1, smem, bar, phase, ysoff, sel, swap_words);
+    ++phase;
+  });
 }
 
 // ===========================================================================
@@ -401,7 +469,8 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
 // ===========================================================================
 template <int G>
 __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
-  __shared__ uint32_t hist_s[kNB];
+  constexpr int kBatch = 8;
+  __shared__ __align__(16) uint32_t hist_s[kNB];
   __shared__ int sh_bstar;
   __shared__ uint32_t sh_above;
   pdl_wait();
@@ -410,8 +479,23 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
     const int b = u / p.Hkv;
     const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
     const int k = decode_k(p.budget, p.k_override, N);
+    const float* sig = p.sigma + static_cast<size_t>(u) * p.cap;
+    // first batch of scores in flight while the threshold is found
+    float sv[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int j = j0 + r * blockDim.x + threadIdx.x;
+      sv[r] = j < j1 ? sig[j] : 0.f;
+    }
     __syncthreads();
-    for (int i = threadIdx.x; i < kNB; i += blockDim.x) hist_s[i] = p.hist[static_cast<size_t>(u) * kNB + i];
+    {
+      const uint4* hg = reinterpret_cast<const uint4*>(p.hist + static_cast<size_t>(u) * kNB);
+      uint4 hv[kNB / 4 / 256];
+#pragma unroll
+      for (int r = 0; r < kNB / 4 / 256; ++r) hv[r] = hg[r * 256 + threadIdx.x];
+#pragma unroll
+      for (int r = 0; r < kNB / 4 / 256; ++r) reinterpret_cast<uint4*>(hist_s)[r * 256 + threadIdx.x] = hv[r];
+    }
     if (threadIdx.x == 0) {
       sh_bstar = kNB;   // k == 0: nothing selected
       sh_above = 0;
@@ -425,21 +509,40 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
       p.units[u].above = static_cast<int32_t>(sh_above);
     }
     if (bstar >= kNB) return;
-    float lo, inv;
-    hist_range<G>(p.bounds, u, p.nq, lo, inv);
-    const float* sig = p.sigma + static_cast<size_t>(u) * p.cap;
+    float ub[G], lb[G];
+    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
+    float hi = ub[0], lo = lb[0];
+#pragma unroll
+    for (int g = 1; g < G; ++g) {
+      hi = fmaxf(hi, ub[g]);
+      lo = fmaxf(lo, lb[g]);
+    }
+    const float inv = (hi > lo) ? __fdiv_rn(static_cast<float>(kNB), __fsub_rn(hi, lo)) : 0.f;
     uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
-    for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-      const float s = __ldcs(sig + j);
-      const int bin = score_bin(s, lo, inv);
-      if (bin > bstar) {
-        atomicOr(bm + (j >> 5), 1u << (j & 31));
-      } else if (bin == bstar) {
-        const int slot = atomicAdd(&p.units[u].ncand, 1);
-        if (slot < p.cap)
-          p.cand[static_cast<size_t>(u) * p.cap + slot] =
-              (static_cast<unsigned long long>(float_key(s)) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+    for (int base = j0; base < j1; base += kBatch * blockDim.x) {
+      float nv[kBatch];
+      const int nb = base + kBatch * blockDim.x;
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int j = nb + r * blockDim.x + threadIdx.x;
+        nv[r] = j < j1 ? sig[j] : 0.f;
       }
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int j = base + r * blockDim.x + threadIdx.x;
+        if (j >= j1) continue;
+        const int bin = score_bin(sv[r], lo, inv);
+        if (bin > bstar) {
+          atomicOr(bm + (j >> 5), 1u << (j & 31));
+        } else if (bin == bstar) {
+          const int slot = atomicAdd(&p.units[u].ncand, 1);
+          if (slot < p.cap)
+            p.cand[static_cast<size_t>(u) * p.cap + slot] =
+                (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) sv[r] = nv[r];
     }
   });
 }
@@ -448,7 +551,9 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
 // finalize (one CTA per unit)
 // ===========================================================================
 constexpr int kFinThreads = 1024;
-constexpr int kFinSmemCand = 4096;
+constexpr int kFinWordsPerThread = 4;
+constexpr int kFinChunkWords = kFinWordsPerThread * kFinThreads;   // 131072 slots per pass
+constexpr int kFinSmemCand = kFinThreads;                          // candidates resolved in shared memory
 
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -479,58 +584,100 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_t
   return r;
 }
 
+// Remove the weight e^{shat_gj - ub_g} of selected slot j from its cluster's sums.
+template <int G>
+__device__ __forceinline__ void unselect_weight(const SelectParams& p, int u, int j, const float* ub2) {
+  constexpr int GP = (G + 3) / 4;
+  uint32_t id = p.ids[static_cast<size_t>(u) * p.cap + j];
+  if (id >= static_cast<uint32_t>(p.C)) id = 0;
+  const uint4 cw = *reinterpret_cast<const uint4*>(p.codes + (static_cast<size_t>(u) * p.cap + j) * kM);
+  const uint32_t cwords[4] = {cw.x, cw.y, cw.z, cw.w};
+  const float4* lut4 = reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
+  const float4* qc4 = reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C;
+  float4 acc[GP];
+#pragma unroll
+  for (int gp = 0; gp < GP; ++gp) acc[gp] = qc4[gp * p.C + id];
+#pragma unroll
+  for (int s = 0; s < kM; ++s) {
+    const int code = (cwords[s >> 2] >> (8 * (s & 3))) & 255;
+#pragma unroll
+    for (int gp = 0; gp < GP; ++gp) {
+      const float4 v = lut4[(gp * kNcode + code) * kM + s];
+      acc[gp].x = __fadd_rn(acc[gp].x, v.x);
+      acc[gp].y = __fadd_rn(acc[gp].y, v.y);
+      acc[gp].z = __fadd_rn(acc[gp].z, v.z);
+      acc[gp].w = __fadd_rn(acc[gp].w, v.w);
+    }
+  }
+  float* Wu = p.W + static_cast<size_t>(u) * G * p.C;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float4 a = acc[g / 4];
+    const float sh = (g % 4 == 0) ? a.x : (g % 4 == 1) ? a.y : (g % 4 == 2) ? a.z : a.w;
+    atomicAdd(&Wu[g * p.C + id], -fast_exp2(fmaf(sh, kLog2e, -ub2[g])));
+  }
+}
+
+// One CTA per unit: resolve the threshold bin's candidates exactly (score desc, position
+// asc), compact the selection bitmap into ascending positions, and take the selected
+// tokens' weights out of the cluster sums. Unit state, candidates and the first bitmap
+// pass are loaded in one round trip.
 template <int G>
 __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
-  constexpr int GP = (G + 3) / 4;
   __shared__ unsigned long long ck[kFinSmemCand];
+  __shared__ uint32_t bmc[kFinChunkWords];
+  __shared__ uint32_t wins[kFinSmemCand];
   __shared__ uint32_t dig[256];
   __shared__ uint32_t warp_tot[33];
   __shared__ int sh_bin;
-  __shared__ uint32_t sh_above;
+  __shared__ uint32_t sh_above, sh_nwin;
   const int u = blockIdx.x;
   const int b = u / p.Hkv;
   const int tid = threadIdx.x;
   pdl_wait();
   pdl_launch_dependents();
-  const int T = max(0, p.seq_lens[b]);
+  // ---- one round trip: lengths, unit state, candidates and the first bitmap pass (speculative) ----
+  const int T_raw = p.seq_lens[b];
+  const int n_raw = p.n_indexed[b];
+  const UnitState st = p.units[u];
+  const unsigned long long* cg = p.cand + static_cast<size_t>(u) * p.cap;
+  const unsigned long long ck_mine = tid < p.cap ? cg[tid] : 0ull;
+  const uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
+  uint32_t words[kFinWordsPerThread];
+#pragma unroll
+  for (int e = 0; e < kFinWordsPerThread; ++e) {
+    const int wi = kFinWordsPerThread * tid + e;
+    words[e] = wi < p.bitmap_words ? bm[wi] : 0u;
+  }
+  const int T = max(0, T_raw);
   const int s0 = min(p.n_sink, T);
-  const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
+  const int N = min(max(0, min(n_raw, T - s0)), p.cap);
   const int k = decode_k(p.budget, p.k_override, N);
   int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
-  uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
   if (k == 0) {
     if (tid == 0 && p.dbg_nselected) p.dbg_nselected[u] = 0;
     return;
   }
-  const UnitState st = p.units[u];
   const int m = min(st.ncand, p.cap);
   const int r = k - st.above;
-  if (r < 1 || r > m) {
-    if (tid == 0) record_error(p.err, HSA_DEVERR_SELECT);
-  }
-  const unsigned long long* cg = p.cand + static_cast<size_t>(u) * p.cap;
+  const bool ok = r >= 1 && r <= m;
+  if (!ok && tid == 0) record_error(p.err, HSA_DEVERR_SELECT);
   const bool in_smem = m <= kFinSmemCand;
-  if (in_smem)
-    for (int i = tid; i < m; i += blockDim.x) ck[i] = cg[i];
+  if (in_smem && tid < m) ck[tid] = ck_mine;
+  if (tid == 0) sh_nwin = 0;
   __syncthreads();
   const unsigned long long* keys = in_smem ? ck : cg;
 
   // ---- threshold key: the r-th largest candidate key (keys are distinct) ----
-  unsigned long long tau = ~0ull;
-  if (r >= 1 && r <= m) {
+  if (ok) {
+    unsigned long long tau;
     if (m <= 256) {
-      // rank selection; slot kFinSmemCand-1 is free because m <= 256
-      if (tid == 0) ck[kFinSmemCand - 1] = ~0ull;
-      __syncthreads();
-      for (int i = tid; i < m; i += blockDim.x) {
-        const unsigned long long key = keys[i];
+      if (tid < m) {
+        const unsigned long long key = keys[tid];
         int rank = 0;
         for (int j = 0; j < m; ++j) rank += keys[j] > key;
-        if (rank == r - 1) ck[kFinSmemCand - 1] = key;   // unique writer: keys are distinct
+        if (rank < r) wins[atomicAdd(&sh_nwin, 1u)] = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
       }
-      __syncthreads();
-      tau = ck[kFinSmemCand - 1];
-      __syncthreads();
     } else {
       unsigned long long prefix = 0, mask = 0;
       uint32_t need = static_cast<uint32_t>(r);
@@ -555,41 +702,75 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
         __syncthreads();
       }
       tau = prefix;
-    }
-    for (int i = tid; i < m; i += blockDim.x) {
-      const unsigned long long key = keys[i];
-      if (key >= tau) {
-        const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
-        atomicOr(bm + (j >> 5), 1u << (j & 31));
+      for (int i = tid; i < m; i += blockDim.x) {
+        const unsigned long long key = keys[i];
+        if (key >= tau) {
+          const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
+          const uint32_t w = atomicAdd(&sh_nwin, 1u);
+          if (w < kFinSmemCand) wins[w] = j;
+          else atomicOr(p.bitmap + static_cast<size_t>(u) * p.bitmap_words + (j >> 5), 1u << (j & 31));
+        }
       }
     }
   }
-  __threadfence_block();
   __syncthreads();
+  const uint32_t nwin = min(sh_nwin, static_cast<uint32_t>(kFinSmemCand));
+  if (nwin < sh_nwin) __threadfence_block();   // overflowed winners went to the global bitmap
+
+  float ub2[G];
+  {
+    float ub[G], lb[G];
+    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
+#pragma unroll
+    for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
+  }
+  const bool fix = p.background && N > k;
 
   // ---- compaction of the selection bitmap into ascending positions ----
   const int nw = (N + 31) / 32;
   uint32_t running = 0;
-  for (int w0 = 0; w0 < nw; w0 += 4 * kFinThreads) {
-    uint32_t words[4];
+  for (int w0 = 0; w0 < nw; w0 += kFinChunkWords) {
+    if (w0 > 0 || sh_nwin > kFinSmemCand) {
+#pragma unroll
+      for (int e = 0; e < kFinWordsPerThread; ++e) {
+        const int wi = w0 + kFinWordsPerThread * tid + e;
+        words[e] = wi < nw ? bm[wi] : 0u;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kFinWordsPerThread; ++e) {
+      const int wi = w0 + kFinWordsPerThread * tid + e;
+      bmc[kFinWordsPerThread * tid + e] = wi < nw ? words[e] : 0u;
+    }
+    __syncthreads();
+    for (uint32_t i = tid; i < nwin; i += blockDim.x) {
+      const uint32_t j = wins[i];
+      const int w = static_cast<int>(j >> 5) - w0;
+      if (w >= 0 && w < kFinChunkWords) atomicOr(&bmc[w], 1u << (j & 31));
+    }
+    __syncthreads();
     uint32_t pc = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int wi = w0 + 4 * tid + e;
-      words[e] = wi < nw ? bm[wi] : 0u;
+    for (int e = 0; e < kFinWordsPerThread; ++e) {
+      words[e] = bmc[kFinWordsPerThread * tid + e];
       pc += __popc(words[e]);
     }
     uint32_t tot;
     uint32_t off = running + block_excl_scan(pc, warp_tot, tot);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < kFinWordsPerThread; ++e) {
       uint32_t wv = words[e];
-      const int wi = w0 + 4 * tid + e;
+      const int wi = w0 + kFinWordsPerThread * tid + e;
       while (wv) {
         const int bit = __ffs(wv) - 1;
         wv &= wv - 1;
-        if (off < static_cast<uint32_t>(p.cap)) sel_u[off] = s0 + wi * 32 + bit;
+        const int j = wi * 32 + bit;
+        if (off < static_cast<uint32_t>(p.cap)) {
+          sel_u[off] = s0 + j;
+          if (p.dbg_selected) p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = s0 + j;
+        }
         ++off;
+        if (fix) unselect_weight<G>(p, u, j, ub2);
       }
     }
     running += tot;
@@ -598,46 +779,6 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     p.units[u].nsel = static_cast<int32_t>(running);
     if (running != static_cast<uint32_t>(k)) record_error(p.err, HSA_DEVERR_SELECT);
     if (p.dbg_nselected) p.dbg_nselected[u] = static_cast<int32_t>(running);
-  }
-  __syncthreads();
-  const int nsel = min(static_cast<int>(running), k);
-  if (p.dbg_selected)
-    for (int i = tid; i < nsel; i += blockDim.x) p.dbg_selected[static_cast<size_t>(u) * p.cap + i] = sel_u[i];
-
-  // ---- remove the selected tokens' weights from the cluster sums ----
-  if (p.background && N > k) {
-    float ub[G];
-    unit_upper_bounds<G>(p.bounds, u, p.nq, ub);
-    const float4* lut4 = reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
-    const float4* qc4 = reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C;
-    float* Wu = p.W + static_cast<size_t>(u) * G * p.C;
-    for (int i = tid; i < nsel; i += blockDim.x) {
-      const int j = sel_u[i] - s0;
-      uint32_t id = p.ids[static_cast<size_t>(u) * p.cap + j];
-      if (id >= static_cast<uint32_t>(p.C)) id = 0;
-      const uint8_t* cj = p.codes + (static_cast<size_t>(u) * p.cap + j) * kM;
-      float4 acc[GP];
-#pragma unroll
-      for (int gp = 0; gp < GP; ++gp) acc[gp] = qc4[gp * p.C + id];
-#pragma unroll
-      for (int s = 0; s < kM; ++s) {
-        const int code = cj[s];
-#pragma unroll
-        for (int gp = 0; gp < GP; ++gp) {
-          const float4 v = lut4[(gp * kNcode + code) * kM + s];
-          acc[gp].x = __fadd_rn(acc[gp].x, v.x);
-          acc[gp].y = __fadd_rn(acc[gp].y, v.y);
-          acc[gp].z = __fadd_rn(acc[gp].z, v.z);
-          acc[gp].w = __fadd_rn(acc[gp].w, v.w);
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float4 a = acc[g / 4];
-        const float sh = (g % 4 == 0) ? a.x : (g % 4 == 1) ? a.y : (g % 4 == 2) ? a.z : a.w;
-        atomicAdd(&Wu[g * p.C + id], -fast_exp2(fmaf(sh, kLog2e, -ub[g] * kLog2e)));
-      }
-    }
   }
 }
 
@@ -679,7 +820,7 @@ size_t scan_smem_bytes(int G, int C) {
   }
 
 cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, bool pdl) {
-  const dim3 grid(p.B * p.Hkv, 1 + p.nq);
+  const dim3 grid(p.B * p.Hkv, kLutParts + p.nq);
 #define CALL(GG) return launch_ex(tables_kernel<GG>, grid, dim3(256), 0, stream, pdl, p)
   PQHSA_G_SWITCH(G, CALL)
 #undef CALL
