@@ -38,7 +38,20 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="llama8b_128k")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", choices=["ctx", "budget"], default=None,
+                    help="extra measurements: context-length crossover, or budget / background ablation")
+    ap.add_argument("--append", action="store_true",
+                    help="index-append cost on the Qwen3-30B-A3B-shaped workload (512-token batches)")
     return ap.parse_args(argv)
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (the job's time is its slowest rank's)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
 
 
 def measured_peaks():
@@ -268,10 +281,7 @@ def run_ours(args):
     ms_hsa = sum(t_hsa) / len(t_hsa)
     ms_dense = sum(t_dense) / len(t_dense)
     ms_e2e = sum(t_e2e) / len(t_e2e)
-    if world > 1:
-        tt = torch.tensor([ms_hsa, ms_dense, ms_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_hsa, ms_dense, ms_e2e = tt.tolist()
+    ms_hsa, ms_dense, ms_e2e = max_over_ranks([ms_hsa, ms_dense, ms_e2e], dist if world > 1 else None, dev)
 
     stage_ms = [sum(s[i] for s in t_stage) / len(t_stage) for i in range(P.NUM_STAGES)]
     n_idx = int(w.n_indexed)
@@ -340,6 +350,158 @@ def run_ours(args):
 
 
 # ---------------------------------------------------------------------------
+# extra measurements (one JSON line each; not the headline line)
+# ---------------------------------------------------------------------------
+
+class _Setup:
+    """One workload on the GPU with its index encoded on the GPU (the build after prefill)."""
+
+    def __init__(self, w, dev):
+        import torch
+        import sparse_long_context_pq_b200 as P
+        from synth import make_batch
+        from synth.device import index_tensors, kv_tensors
+        self.P, self.torch, self.w, self.dev = P, torch, w, dev
+        self.bt = make_batch(w)
+        self.kv = P.PagedKV(**kv_tensors(self.bt, dev))
+        self.ix = P.PQIndex(**index_tensors(self.bt, dev, n_indexed=np.zeros(w.B, dtype=np.int32)))
+        self.ws_idx = P.workspace(P.hsa_index_workspace_bytes(), dev)
+        P.hsa_append_encode(self.kv, self.ix, w.n_indexed, workspace_buf=self.ws_idx)
+        self.scale = float(np.float32(1.0 / math.sqrt(w.D)))
+        self.q = torch.from_numpy(self.bt.q).to(dev)
+        self.out = torch.empty_like(self.q)
+        self.out_dense = torch.empty_like(self.q)
+        self.ws = P.workspace(P.hsa_decode_workspace_bytes(self.kv, self.ix), dev)
+        self.ws_dense = P.workspace(P.dense_decode_workspace_bytes(self.kv), dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+
+    def graph(self, fn):
+        fn()
+        self.torch.cuda.synchronize()
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g):
+            fn()
+        self.torch.cuda.synchronize()
+        return g
+
+    def time_graph(self, g, steps, warmup):
+        torch = self.torch
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t = []
+        for i in range(warmup + steps):
+            self.flush.zero_()
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= warmup:
+                t.append(a.elapsed_time(b))
+        return sum(t) / len(t) * 1e3   # us
+
+    def hsa(self, budget=0.01, background=True):
+        return lambda: self.P.hsa_decode(self.kv, self.ix, self.q, self.out, scale=self.scale, budget=budget,
+                                         background=background, workspace_buf=self.ws)
+
+    def dense(self):
+        return lambda: self.P.dense_decode(self.kv, self.q, self.out_dense, scale=self.scale,
+                                           workspace_buf=self.ws_dense)
+
+
+def run_sweep_ctx(args):
+    import torch
+    from synth import workload
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, _ = measured_peaks()
+    pts = []
+    for name in ("llama8b_8k", "llama8b_32k", "llama8b_sweep_128k", "llama8b_512k"):
+        w = workload(name)
+        S = _Setup(w, dev)
+        k = S.P.decode_k(w.budget, w.n_indexed)
+        hsa_b, ids_b, dense_b, _ = step_bytes(w, w.n_indexed, k)
+        us_h = S.time_graph(S.graph(S.hsa()), args.steps, args.warmup)
+        us_d = S.time_graph(S.graph(S.dense()), args.steps, args.warmup)
+        assert S.P.hsa_read_error(S.ws) == 0
+        print(json.dumps({"sweep": "ctx", "workload": name, "T": w.T, "hsa_us": round(us_h, 3),
+                          "dense_us": round(us_d, 3), "speedup": round(us_d / us_h, 3),
+                          "hsa_bytes": hsa_b, "ids_bytes": ids_b, "dense_bytes": dense_b,
+                          "hsa_gbs": round(hsa_b / us_h / 1e3, 1), "dense_gbs": round(dense_b / us_d / 1e3, 1),
+                          "dense_pct_peak": round(100 * dense_b / us_d / 1e3 / peak, 2)}), flush=True)
+        pts.append((w, hsa_b, dense_b, us_h, us_d))
+        del S
+        torch.cuda.empty_cache()
+    # Overhead-aware model (crossover article): t = fixed + bytes / BW per method, fitted by
+    # least squares; the predicted crossover is the length where the two lines meet.
+    def fit(xs, ys):
+        xs, ys = np.asarray(xs, float), np.asarray(ys, float)
+        A = np.stack([np.ones_like(xs), xs], axis=1)
+        (a, b), *_ = np.linalg.lstsq(A, ys, rcond=None)
+        return float(a), float(b)
+    fh = fit([p_[1] for p_ in pts], [p_[3] for p_ in pts])
+    fd = fit([p_[2] for p_ in pts], [p_[4] for p_ in pts])
+    w0 = pts[0][0]
+    cross = None
+    for T in range(2048, 1 << 21, 256):
+        wt = w0.scaled(T=T)
+        hb, _, db, _ = step_bytes(wt, wt.n_indexed, int(math.floor(wt.budget * wt.n_indexed)))
+        if fh[0] + fh[1] * hb <= fd[0] + fd[1] * db:
+            cross = T
+            break
+    print(json.dumps({"sweep": "ctx-model", "hsa_fixed_us": round(fh[0], 2), "hsa_gbs": round(1e-3 / fh[1], 1),
+                      "dense_fixed_us": round(fd[0], 2), "dense_gbs": round(1e-3 / fd[1], 1),
+                      "predicted_crossover_T": cross}), flush=True)
+
+
+def run_sweep_budget(args):
+    import torch
+    from synth import workload
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload(args.workload)
+    S = _Setup(w, dev)
+    S.dense()()
+    torch.cuda.synchronize()
+    ref = S.out_dense.clone()
+    vmax = float(S.kv.v_cache.float().abs().max())
+    for budget in (0.005, 0.01, 0.02, 0.05):
+        for bg in (True, False):
+            us = S.time_graph(S.graph(S.hsa(budget, bg)), args.steps, args.warmup)
+            S.hsa(budget, bg)()
+            torch.cuda.synchronize()
+            err = float((S.out - ref).abs().max()) / vmax
+            rel = float(((S.out - ref).norm(dim=-1) / ref.norm(dim=-1)).mean())
+            print(json.dumps({"sweep": "budget", "workload": w.name, "budget": budget, "background": bg,
+                              "hsa_us": round(us, 3), "max_abs_err_vs_dense_over_max_v": round(err, 6),
+                              "mean_rel_l2_err_vs_dense": round(rel, 6)}), flush=True)
+
+
+def run_append(args):
+    import torch
+    from synth import workload
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload("qwen30b_128k_append")
+    S = _Setup(w, dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    T = w.T
+    for step in range(w.extra_tokens // w.append_batch):
+        us_dec = S.time_graph(S.graph(S.hsa()), args.steps, args.warmup)
+        T += w.append_batch                      # 512 generated tokens later, the oldest tail tokens move in
+        S.kv.seq_lens.fill_(T)
+        S.kv.seq_lens_host.fill_(T)
+        S.flush.zero_()
+        a.record()
+        S.P.hsa_append_encode(S.kv, S.ix, w.append_batch, workspace_buf=S.ws_idx)
+        b.record()
+        torch.cuda.synchronize()
+        assert S.P.hsa_read_error(S.ws_idx) == 0
+        print(json.dumps({"append": step, "workload": w.name, "T_before": T - w.append_batch,
+                          "decode_us": round(us_dec, 3), "append_512_us": round(a.elapsed_time(b) * 1e3, 3),
+                          "n_indexed": int(S.ix.n_indexed_host[0])}), flush=True)
+
+
+# ---------------------------------------------------------------------------
 # reference arm: the float64 oracle on the host cores
 # ---------------------------------------------------------------------------
 
@@ -376,7 +538,13 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
-    if args.impl == "reference":
+    if args.sweep == "ctx":
+        run_sweep_ctx(args)
+    elif args.sweep == "budget":
+        run_sweep_budget(args)
+    elif args.append:
+        run_append(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -81,8 +81,21 @@ typedef struct {
   int32_t* count;                  /* [B][Hkv][C]           members per cluster */
   int32_t* n_indexed;              /* [B] indexed tokens per sequence (device) */
   int32_t* n_indexed_host;         /* [B] host copy of n_indexed */
+  /* Cluster-ordered copy of the codes, kept by hsa_build_from_codes / hsa_append_encode
+     and read by hsa_decode: the list slots of a unit form 32-slot chunks, each chunk
+     holding members of one cluster (its last chunk may be partly empty). */
+  uint8_t* list_codes;             /* u8  [B][Hkv][list_slots][M] */
+  int32_t* list_slot;              /* [B][Hkv][list_slots]  index slot of the member, -1 = empty */
+  uint16_t* chunk_cluster;         /* [B][Hkv][list_slots / 32] cluster of each chunk */
+  int32_t* list_meta;              /* [B][Hkv][2 + 2*C]: chunks in use, unused, then per cluster
+                                      (its open chunk or -1, members in that chunk) */
   int32_t C, M, dsub, ncode, cap, n_sink;
+  int32_t list_slots;              /* >= hsa_index_list_slots(cap, C) */
 } hsa_index;
+
+/* List capacity (slots per unit) an index of `cap` tokens and C clusters needs:
+   32 * (ceil(cap / 32) + C). */
+int64_t hsa_index_list_slots(int32_t cap, int32_t C);
 
 typedef struct {
   float scale;                     /* logit scale, e.g. 1/sqrt(D) */
@@ -171,7 +184,7 @@ size_t hsa_index_workspace_bytes(void);
  * above: "after the prompt is filled the index is built"). The caller fills
  * centroids, codebooks, codes and ids for slots [0, n_indexed[b]); this call
  * computes count, sum_v and mean_v of every cluster from the value rows of the
- * indexed tokens.
+ * indexed tokens, and builds the cluster-ordered lists read by hsa_decode.
  */
 hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* index,
                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -183,8 +196,10 @@ hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* index,
  *   a = argmin_c sum_d (k_d - centroid_c,d)^2 (fp32, ties to the lower c),
  *   code_s = argmin_m sum_{d<dsub} (k - centroid_a)_{s*dsub+d} - codeword_s,m,d)^2,
  * written to slots [N_b, N_b + n_new); the members' values are added to sum_v
- * and count, mean_v is recomputed, and n_indexed (device and host) grows by
- * n_new. Requires s0 + N_b + n_new <= seq_lens_host[b] and N_b + n_new <= cap.
+ * and count, mean_v is recomputed, the new members join their clusters' lists
+ * (list_codes / list_slot), and n_indexed (device and host) grows by n_new.
+ * Requires s0 + N_b + n_new <= seq_lens_host[b] and N_b + n_new <= cap, and
+ * lists built by earlier calls (a unit with n_indexed = 0 starts them afresh).
  * With n_indexed = 0 this is the whole index build from raw keys.
  */
 hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* index, int32_t n_new,

@@ -42,8 +42,16 @@ class _Index(ctypes.Structure):
     _fields_ = [("centroids", ctypes.c_void_p), ("codebooks", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("ids", ctypes.c_void_p), ("sum_v", ctypes.c_void_p), ("mean_v", ctypes.c_void_p),
                 ("count", ctypes.c_void_p), ("n_indexed", ctypes.c_void_p), ("n_indexed_host", ctypes.c_void_p),
+                ("list_codes", ctypes.c_void_p), ("list_slot", ctypes.c_void_p),
+                ("chunk_cluster", ctypes.c_void_p), ("list_meta", ctypes.c_void_p),
                 ("C", ctypes.c_int32), ("M", ctypes.c_int32), ("dsub", ctypes.c_int32),
-                ("ncode", ctypes.c_int32), ("cap", ctypes.c_int32), ("n_sink", ctypes.c_int32)]
+                ("ncode", ctypes.c_int32), ("cap", ctypes.c_int32), ("n_sink", ctypes.c_int32),
+                ("list_slots", ctypes.c_int32)]
+
+
+def index_list_slots(cap: int, C: int) -> int:
+    """List slots per unit the cluster-ordered code lists need: 32 * (ceil(cap / 32) + C)."""
+    return 32 * ((cap + 31) // 32 + C)
 
 
 class _Params(ctypes.Structure):
@@ -60,7 +68,7 @@ NUM_STAGES = 6
 STAGE_NAMES = ("tables", "scan", "filter", "finalize", "attend", "merge")
 
 
-EXPORTS = ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode",
+EXPORTS = ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode", "hsa_index_list_slots",
            "hsa_decode_workspace_bytes", "dense_decode_workspace_bytes", "hsa_index_workspace_bytes",
            "hsa_read_error", "hsa_strerror", "hsa_abi_sizes")
 
@@ -184,6 +192,21 @@ class PQIndex:
     n_indexed: torch.Tensor        # int32 [B] (device)
     n_indexed_host: torch.Tensor   # int32 [B] (cpu)
     n_sink: int
+    list_codes: Optional[torch.Tensor] = None     # uint8 [B, Hkv, list_slots, M]  (library-maintained)
+    list_slot: Optional[torch.Tensor] = None      # int32 [B, Hkv, list_slots]
+    chunk_cluster: Optional[torch.Tensor] = None  # int16 storage of u16 [B, Hkv, list_slots / 32]
+    list_meta: Optional[torch.Tensor] = None      # int32 [B, Hkv, 2 + 2C]
+
+    def __post_init__(self):
+        if self.list_codes is None:
+            B, Hkv, cap, _ = self.codes.shape
+            C = self.centroids.shape[2]
+            ls = index_list_slots(cap, C)
+            dev = self.codes.device
+            self.list_codes = torch.zeros(B, Hkv, ls, M_SUB, device=dev, dtype=torch.uint8)
+            self.list_slot = torch.full((B, Hkv, ls), -1, device=dev, dtype=torch.int32)
+            self.chunk_cluster = torch.zeros(B, Hkv, ls // 32, device=dev, dtype=torch.int16)
+            self.list_meta = torch.zeros(B, Hkv, 2 + 2 * C, device=dev, dtype=torch.int32)
 
     @staticmethod
     def allocate(B: int, Hkv: int, C: int, cap: int, n_sink: int, device) -> "PQIndex":
@@ -210,12 +233,15 @@ class PQIndex:
         return self.codes.shape[2]
 
     def struct(self) -> _Index:
-        for t in (self.centroids, self.codebooks, self.codes, self.ids, self.sum_v, self.mean_v, self.count):
+        for t in (self.centroids, self.codebooks, self.codes, self.ids, self.sum_v, self.mean_v, self.count,
+                  self.list_codes, self.list_slot, self.chunk_cluster, self.list_meta):
             assert t.is_contiguous()
         assert self.n_indexed_host.device.type == "cpu" and self.n_indexed_host.dtype == torch.int32
         return _Index(_ptr(self.centroids), _ptr(self.codebooks), _ptr(self.codes), _ptr(self.ids),
                       _ptr(self.sum_v), _ptr(self.mean_v), _ptr(self.count), _ptr(self.n_indexed),
-                      _ptr(self.n_indexed_host), self.C, M_SUB, DSUB, NCODE, self.cap, self.n_sink)
+                      _ptr(self.n_indexed_host), _ptr(self.list_codes), _ptr(self.list_slot),
+                      _ptr(self.chunk_cluster), _ptr(self.list_meta), self.C, M_SUB, DSUB, NCODE, self.cap,
+                      self.n_sink, self.list_codes.shape[2])
 
 
 def hsa_decode_workspace_bytes(kv: PagedKV, index: PQIndex) -> int:

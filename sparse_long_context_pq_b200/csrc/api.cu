@@ -121,6 +121,13 @@ hsa_status check_index(const hsa_kv_cache* kv, const hsa_index* ix, bool need_co
   if (!aligned(ix->centroids, 16) || !aligned(ix->codebooks, 16) || !aligned(ix->mean_v, 16) ||
       (ix->codes && !aligned(ix->codes, 16)) || !aligned(ix->ids, 2))
     return HSA_ERR_ALIGNMENT;
+  // cluster-ordered lists
+  if (!ix->list_codes || !ix->list_slot || !ix->chunk_cluster || !ix->list_meta) return HSA_ERR_INVALID_ARG;
+  if (ix->C > 4096) return HSA_ERR_UNSUPPORTED;
+  if (ix->list_slots < list_slots_needed(ix->cap, ix->C) || ix->list_slots % 32) return HSA_ERR_CAPACITY;
+  if (!aligned(ix->list_codes, 16) || !aligned(ix->list_slot, 4) || !aligned(ix->list_meta, 4) ||
+      !aligned(ix->chunk_cluster, 2))
+    return HSA_ERR_ALIGNMENT;
   for (int b = 0; b < kv->B; ++b) {
     const int T = kv->seq_lens_host[b];
     const int n = ix->n_indexed_host[b];
@@ -203,7 +210,9 @@ void hsa_abi_sizes(int64_t* a, int64_t* b, int64_t* c, int64_t* d) {
 
 size_t hsa_decode_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix) {
   if (check_kv(kv) != HSA_OK || !ix || ix->C < 1 || ix->cap < 1) return 0;
-  const DecodeLayout L = make_decode_layout(kv->B * kv->Hkv, kv->Hq / kv->Hkv, ix->C, ix->cap, kMaxSplits);
+  if (ix->list_slots < 32) return 0;
+  const DecodeLayout L =
+      make_decode_layout(kv->B * kv->Hkv, kv->Hq / kv->Hkv, ix->C, ix->cap, ix->list_slots, kMaxSplits);
   return L.total;
 }
 
@@ -213,6 +222,11 @@ size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv) {
 }
 
 size_t hsa_index_workspace_bytes(void) { return sizeof(WsHeader); }
+
+int64_t hsa_index_list_slots(int32_t cap, int32_t C) {
+  if (cap < 1 || C < 1) return 0;
+  return list_slots_needed(cap, C);
+}
 
 hsa_status hsa_read_error(void* ws, int32_t* error_host, cudaStream_t stream) {
   if (!ws || !error_host) return HSA_ERR_INVALID_ARG;
@@ -291,7 +305,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   const int U = kv->B * kv->Hkv, G = kv->Hq / kv->Hkv;
   const size_t scan_smem = scan_smem_bytes(G, ix->C);
   if (scan_smem > 227 * 1024) return HSA_ERR_UNSUPPORTED;
-  const DecodeLayout L = make_decode_layout(U, G, ix->C, ix->cap, kMaxSplits);
+  const DecodeLayout L = make_decode_layout(U, G, ix->C, ix->cap, ix->list_slots, kMaxSplits);
   if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HSA_ERR_WORKSPACE;
   const DeviceInfo* dev = device_info();
   if (!dev) return HSA_ERR_CUDA;
@@ -350,8 +364,11 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   RET_CUDA(launch_tables(G, tp, stream, use_pdl()));
 
   ScanParams sc = {};
-  sc.codes = ix->codes;
-  sc.ids = ix->ids;
+  sc.list_codes = ix->list_codes;
+  sc.list_slot = ix->list_slot;
+  sc.chunk_cluster = ix->chunk_cluster;
+  sc.list_meta = ix->list_meta;
+  sc.list_slots = ix->list_slots;
   sc.seq_lens = kv->seq_lens;
   sc.n_indexed = ix->n_indexed;
   sc.lut = lut;
@@ -374,6 +391,11 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   RET_CUDA(launch_scan(G, sc, dev->sms * scan_per_sm, stream, use_pdl()));
 
   SelectParams se = {};
+  se.list_codes = ix->list_codes;
+  se.chunk_cluster = ix->chunk_cluster;
+  se.list_slot = ix->list_slot;
+  se.list_meta = ix->list_meta;
+  se.list_slots = ix->list_slots;
   se.seq_lens = kv->seq_lens;
   se.n_indexed = ix->n_indexed;
   se.codes = ix->codes;
@@ -440,11 +462,12 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   p.k_override = prm->k_override;
   p.budget = prm->budget;
   p.qscale = prm->scale * kLog2e;
+  p.units = units;
+  p.out = out;
   RET_CUDA(mark(4));
   RET_CUDA(launch_attend(G, true, true, tk, tv, p, U * (sp.nsplit + L.nbg), stream, use_pdl()));
-  MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, S_tot};
+  // the last CTA of each unit merges it inside the attention launch
   RET_CUDA(mark(5));
-  RET_CUDA(launch_merge(G, mp, stream, use_pdl()));
   RET_CUDA(mark(6));
   return HSA_OK;
 }
@@ -464,6 +487,10 @@ static IndexParams index_params(const hsa_kv_cache* kv, hsa_index* ix, void* ws)
   p.count = ix->count;
   p.n_indexed = ix->n_indexed;
   p.err = static_cast<int32_t*>(ws);
+  p.list_codes = ix->list_codes;
+  p.list_slot = ix->list_slot;
+  p.chunk_cluster = ix->chunk_cluster;
+  p.list_meta = ix->list_meta;
   p.B = kv->B;
   p.Hkv = kv->Hkv;
   p.page_size = kv->page_size;
@@ -472,6 +499,7 @@ static IndexParams index_params(const hsa_kv_cache* kv, hsa_index* ix, void* ws)
   p.C = ix->C;
   p.cap = ix->cap;
   p.n_sink = ix->n_sink;
+  p.list_slots = ix->list_slots;
   return p;
 }
 
@@ -479,7 +507,7 @@ hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* ix, void* ws,
                                 cudaStream_t stream) {
   hsa_status st = check_kv(kv);
   if (st != HSA_OK) return st;
-  st = check_index(kv, ix, false);
+  st = check_index(kv, ix, true);
   if (st != HSA_OK) return st;
   if (!ix->sum_v || !ix->count) return HSA_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < hsa_index_workspace_bytes()) return HSA_ERR_WORKSPACE;
@@ -492,6 +520,8 @@ hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* ix, void* ws,
   p.zero_if_empty = 0;
   RET_CUDA(launch_zero_stats(p, stream));
   RET_CUDA(launch_accumulate(p, nmax, stream));
+  RET_CUDA(launch_list_reset(p, stream));
+  RET_CUDA(launch_list_append(p, stream));
   RET_CUDA(launch_means(p, stream));
   return HSA_OK;
 }
@@ -519,6 +549,8 @@ hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_ne
   RET_CUDA(launch_zero_stats(p, stream));
   RET_CUDA(launch_encode(p, n_new, stream));
   RET_CUDA(launch_accumulate(p, n_new, stream));
+  RET_CUDA(launch_list_reset(p, stream));
+  RET_CUDA(launch_list_append(p, stream));
   RET_CUDA(launch_means(p, stream));
   for (int b = 0; b < kv->B; ++b) ix->n_indexed_host[b] += n_new;
   return HSA_OK;

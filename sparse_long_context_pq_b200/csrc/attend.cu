@@ -29,19 +29,36 @@ namespace pqhsa {
 
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-// Tile t goes to consumer warp t % kConsumerWarps and stage t % kStages. kStages is a
-// multiple of kConsumerWarps, so every stage is always consumed by the same warp and
-// its mbarrier phases are awaited strictly in order: a parity wait can then never
-// alias a phase two steps ahead (which returns immediately on a parity barrier).
-constexpr int kStages = 4;
-static_assert(kStages % kConsumerWarps == 0, "each stage must belong to one consumer warp");
 constexpr int kHalfBytes = kTile * 128;        // swizzled: 32 rows x 128 B (64 bf16)
 constexpr int kRowPitch = 272;                 // padded: 256-byte row + 16
-constexpr int kStageBytes = 2 * kTile * kRowPitch;  // 17408 = 17 KB: K then V (either layout)
-static_assert(kStageBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
-static_assert(4 * kHalfBytes <= kStageBytes, "swizzled tiles fit a stage");
+
+// Pipeline shape per loading mode. Tile t goes to consumer warp t % CW and stage
+// t % S. S is a multiple of CW, so every stage is always consumed by the same warp
+// and its mbarrier phases are awaited strictly in order: a parity wait can then
+// never alias a phase two steps ahead (which returns immediately on a parity barrier).
+// Dense page tiles use tensor TMA into 16 KB stages, gathered rows bulk copies into
+// 272-byte-pitch rows (17 KB stages); both run 4 consumer warps over 4 stages (a deeper
+// 2-warp x 6-stage ring for dense reads measured no faster).
+template <bool kRows>
+struct Pipe {
+  static constexpr int CW = 4;
+  static constexpr int S = 4;
+  static constexpr int threads = (CW + 1) * 32;
+  static constexpr int stage_bytes = kRows ? 2 * kTile * kRowPitch : 4 * kHalfBytes;
+  static_assert(S % CW == 0, "each stage must belong to one consumer warp");
+  static_assert(stage_bytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
+};
+constexpr int kThreads = Pipe<true>::threads;   // the exact+background launch (background CTAs use it)
+
+template <int G, bool kRows>
+struct AttendSmem {
+  static constexpr int GP = (G + 3) / 4;
+  static constexpr size_t stages = static_cast<size_t>(Pipe<kRows>::S) * Pipe<kRows>::stage_bytes;
+  static constexpr size_t qs = kD * GP * 16;
+  static constexpr size_t pbuf = Pipe<kRows>::CW * 2 * 8 * kTile * 2;   // P hi/lo bf16 [8 heads][32 tokens]
+  static constexpr size_t bars = 2 * Pipe<kRows>::S * 8;
+  static constexpr size_t total = 1024 /*alignment slack*/ + stages + qs + pbuf + bars + 64;
+};
 
 // Byte offset of 16-byte chunk c (0..15) of row r inside the K (or V) area of a stage.
 template <bool kRows>
@@ -52,15 +69,6 @@ __device__ __forceinline__ uint32_t chunk_off(int r, int c) {
 template <bool kRows>
 __device__ __forceinline__ uint32_t v_area() { return kRows ? kTile * kRowPitch : 2 * kHalfBytes; }
 
-template <int G>
-struct AttendSmem {
-  static constexpr int GP = (G + 3) / 4;
-  static constexpr size_t stages = static_cast<size_t>(kStages) * kStageBytes;
-  static constexpr size_t qs = kD * GP * 16;
-  static constexpr size_t pbuf = kConsumerWarps * 2 * 8 * kTile * 2;   // P hi/lo bf16 [8 heads][32 tokens]
-  static constexpr size_t bars = 2 * kStages * 8;
-  static constexpr size_t total = 1024 /*alignment slack*/ + stages + qs + pbuf + bars + 64;
-};
 
 // Position of row v of a unit's exact list: sink [0,s0), then the k selected
 // positions (ascending), then the tail [s0+N, T).
@@ -70,18 +78,77 @@ __device__ __forceinline__ int exact_row_pos(int v, int s0, int k, int N, const 
   return s0 + N + (v - s0 - k);
 }
 
+// The CTA that completes a unit's last partial merges the unit: every CTA writes its
+// partial, fences, and takes a ticket; the holder of the last ticket (no waiting)
+// computes out_g = sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s for the unit's heads.
+// `nt` threads (ids 0..nt-1) take part; `scratch` holds 2 * G * S_tot floats.
+template <int G>
+__device__ void merge_unit_if_last(const AttendParams& p, int u, int nt, int t, float* scratch, int* flag,
+                                   bool named_barrier) {
+  auto sync = [&]() {
+    if (named_barrier) asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");
+    else __syncthreads();
+  };
+  sync();                                   // this CTA's partial is fully written
+  if (t == 0) {
+    __threadfence();
+    const int done = atomicAdd(&p.units[u].pad[0], 1);
+    *flag = (done == p.S_tot - 1);
+  }
+  sync();
+  if (!*flag) return;
+  __threadfence();
+  const int S = p.S_tot;
+  const int b = u / p.Hkv, h = u % p.Hkv;
+  float* fs = scratch;                      // [G][S] weights e^{m - M}
+  float* ls = scratch + G * S;              // [G][S] l of each partial
+  for (int i = t; i < G * S; i += nt) {
+    const int g = i / S, sp = i % S;
+    const size_t sl = (static_cast<size_t>(u) * S + sp) * G + g;
+    fs[i] = p.pm[sl];
+    ls[i] = p.pl[sl];
+  }
+  sync();
+  if (t < G) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, fs[t * S + sp]);
+    float L = 0.f;
+    for (int sp = 0; sp < S; ++sp) {
+      const float m = fs[t * S + sp];
+      const float f = (M == -INFINITY || m == -INFINITY) ? 0.f : fast_exp2(m - M);
+      fs[t * S + sp] = f;
+      L += f * ls[t * S + sp];
+    }
+    ls[t * S] = L;                          // L_g kept in the first l slot of head g
+  }
+  sync();
+  for (int i = t; i < G * kD; i += nt) {
+    const int g = i / kD, d = i % kD;
+    float a = 0.f;
+#pragma unroll 4
+    for (int sp = 0; sp < S; ++sp)
+      a = fmaf(fs[g * S + sp], p.pacc[((static_cast<size_t>(u) * S + sp) * G + g) * kD + d], a);
+    const float L = ls[g * S];
+    p.out[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] = L > 0.f ? a / L : 0.f;
+  }
+  if (t == 0) p.units[u].pad[0] = 0;        // ready for the next call
+}
+
 template <int G, bool kExact, bool kRows>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
     attend_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                   AttendParams p) {
   static_assert(kRows || !kExact, "gathered rows use bulk row copies");
+  constexpr int kConsumerWarps = Pipe<kRows>::CW;
+  constexpr int kStages = Pipe<kRows>::S;
+  constexpr int kStageBytes = Pipe<kRows>::stage_bytes;
   constexpr int GP = (G + 3) / 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  float4* qs = reinterpret_cast<float4*>(smem + AttendSmem<G>::stages);               // [kD][GP]
+  float4* qs = reinterpret_cast<float4*>(smem + AttendSmem<G, kRows>::stages);               // [kD][GP]
   uint8_t* pbuf = reinterpret_cast<uint8_t*>(qs + kD * GP);                            // [warps] P buffers
-  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + AttendSmem<G>::pbuf);
+  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + AttendSmem<G, kRows>::pbuf);
   uint64_t* empty = full + kStages;
 
   const int tid = threadIdx.x;
@@ -143,36 +210,57 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     bool ok = true;
     const int box_rows = kRows ? 1 : min(p.page_size, kTile);
-    for (int t = 0; t < ntiles && ok; ++t) {
-      const int s = t % kStages;
-      if (t >= kStages) {
-        ok = mbar_wait_warp(&empty[s], ((t / kStages) - 1) & 1, p.err);
-        if (!ok) break;
-      }
-      const int row0 = r0 + t * kTile;
-      const int nvalid = min(kTile, r1 - row0);
-      uint8_t* st = stage_base + static_cast<size_t>(s) * kStageBytes;
-      const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox) * 2u * box_rows * 256u);
-      __syncwarp();
-      for (int i = lane; i < nbox; i += 32) {
-        const int pos = kExact ? exact_row_pos(row0 + i, s0, k, N, sel_u) : row0 + i * box_rows;
-        int page = (pos >= 0 && pos < T && pos / p.page_size < p.max_pages) ? bt[pos / p.page_size] : -1;
-        if (page < 0 || page >= p.num_pages) {
-          record_error(p.err, HSA_DEVERR_PAGE);
-          page = 0;
+    // Tiles go in groups of kStages: each lane first resolves its box of every tile of the
+    // group (selected-position and block-table loads of the group in flight together),
+    // then the copies are issued tile by tile as stages are released.
+    for (int t0 = 0; t0 < ntiles && ok; t0 += kStages) {
+      int ys[kStages];
+#pragma unroll
+      for (int i = 0; i < kStages; ++i) {
+        ys[i] = -1;
+        const int t = t0 + i;
+        if (t >= ntiles) continue;
+        const int row0 = r0 + t * kTile;
+        const int nvalid = min(kTile, r1 - row0);
+        const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
+        if (lane < nbox) {
+          const int pos = kExact ? exact_row_pos(row0 + lane, s0, k, N, sel_u) : row0 + lane * box_rows;
+          int page = (pos >= 0 && pos < T && pos / p.page_size < p.max_pages) ? bt[pos / p.page_size] : -1;
+          if (page < 0 || page >= p.num_pages) {
+            record_error(p.err, HSA_DEVERR_PAGE);
+            page = 0;
+          }
+          ys[i] = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
         }
-        const int y = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
-        if (kRows) {
-          const size_t src = static_cast<size_t>(y) * (kD * 2);
-          bulk_load(st + i * kRowPitch, p.k_cache + src, 256u, &full[s]);
-          bulk_load(st + v_area<kRows>() + i * kRowPitch, p.v_cache + src, 256u, &full[s]);
-        } else {
-          const int off = i * box_rows * 128;
-          tma_load_2d(st + 0 * kHalfBytes + off, &tmap_k, &full[s], 0, y);
-          tma_load_2d(st + 1 * kHalfBytes + off, &tmap_k, &full[s], 64, y);
-          tma_load_2d(st + 2 * kHalfBytes + off, &tmap_v, &full[s], 0, y);
-          tma_load_2d(st + 3 * kHalfBytes + off, &tmap_v, &full[s], 64, y);
+      }
+#pragma unroll
+      for (int i = 0; i < kStages; ++i) {
+        const int t = t0 + i;
+        if (t >= ntiles) break;
+        const int s = t % kStages;
+        if (t >= kStages) {
+          ok = mbar_wait_warp(&empty[s], ((t / kStages) - 1) & 1, p.err);
+          if (!ok) break;
+        }
+        const int row0 = r0 + t * kTile;
+        const int nvalid = min(kTile, r1 - row0);
+        uint8_t* st = stage_base + static_cast<size_t>(s) * kStageBytes;
+        const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox) * 2u * box_rows * 256u);
+        __syncwarp();
+        if (lane < nbox) {
+          const int y = ys[i];
+          if (kRows) {
+            const size_t src = static_cast<size_t>(y) * (kD * 2);
+            bulk_load(st + lane * kRowPitch, p.k_cache + src, 256u, &full[s]);
+            bulk_load(st + v_area<kRows>() + lane * kRowPitch, p.v_cache + src, 256u, &full[s]);
+          } else {
+            const int off = lane * box_rows * 128;
+            tma_load_2d(st + 0 * kHalfBytes + off, &tmap_k, &full[s], 0, y);
+            tma_load_2d(st + 1 * kHalfBytes + off, &tmap_k, &full[s], 64, y);
+            tma_load_2d(st + 2 * kHalfBytes + off, &tmap_v, &full[s], 0, y);
+            tma_load_2d(st + 3 * kHalfBytes + off, &tmap_v, &full[s], 64, y);
+          }
         }
       }
     }
@@ -332,26 +420,32 @@ __global__ void __launch_bounds__(kThreads, 2)
       cacc[(warp * 8 + 2 * tig + (e & 1)) * kD + 16 * i + grp + 8 * (e >> 1)] = oacc[i][e];
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
   const size_t slot = static_cast<size_t>(u) * p.S_tot + split;
-  const int d = tid;  // 128 consumer threads, one output dim each
+  for (int d = tid; d < kD; d += kConsumerWarps * 32) {   // the consumer threads cover the output dims
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float M = -INFINITY;
+    for (int g = 0; g < G; ++g) {
+      float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * 8 + g]);
-    float L = 0.f, a = 0.f;
-    if (M != -INFINITY) {
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, cm[w * 8 + g]);
+      float L = 0.f, a = 0.f;
+      if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float f = fast_exp2(cm[w * 8 + g] - M);
-        L += f * cl[w * 8 + g];
-        a += f * cacc[(w * 8 + g) * kD + d];
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float f = fast_exp2(cm[w * 8 + g] - M);
+          L += f * cl[w * 8 + g];
+          a += f * cacc[(w * 8 + g) * kD + d];
+        }
+      }
+      p.pacc[(slot * G + g) * kD + d] = a;
+      if (d == 0) {
+        p.pm[slot * G + g] = M;
+        p.pl[slot * G + g] = L;
       }
     }
-    p.pacc[(slot * G + g) * kD + d] = a;
-    if (d == 0) {
-      p.pm[slot * G + g] = M;
-      p.pl[slot * G + g] = L;
-    }
+  }
+  if (kExact) {
+    // the pipeline has drained: the stage area is free for the merge scratch
+    merge_unit_if_last<G>(p, u, kConsumerWarps * 32, tid, reinterpret_cast<float*>(stage_base) + 8192,
+                          reinterpret_cast<int*>(stage_base) + 8191, true);
   }
 }
 
@@ -382,6 +476,8 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
       p.pm[slot * G + tid] = -INFINITY;
       p.pl[slot * G + tid] = 0.f;
     }
+    merge_unit_if_last<G>(p, u, blockDim.x, tid, reinterpret_cast<float*>(smem) + 8192,
+                          reinterpret_cast<int*>(smem) + 8191, false);
     return;
   }
   const int c0 = cb * kBgClusters;
@@ -444,6 +540,8 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
     p.pm[slot * G + tid] = ub[tid] * kLog2e;
     p.pl[slot * G + tid] = l;
   }
+  merge_unit_if_last<G>(p, u, blockDim.x, tid, reinterpret_cast<float*>(smem) + 8192,
+                        reinterpret_cast<int*>(smem) + 8191, false);
 }
 
 namespace {
@@ -466,9 +564,11 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
   const int S = p.S_tot;
   float* fs = msm;
   float* red = msm + ((S + 3) & ~3);
+  float* ls = red;                          // l of each split, until the partial sums need the space
   float mloc = -INFINITY;
   for (int s = tid; s < S; s += kMergeThreads) {
     const float m = p.pm[(u * S + s) * G + g];
+    ls[s] = p.pl[(u * S + s) * G + g];
     fs[s] = m;
     mloc = fmaxf(mloc, m);
   }
@@ -487,7 +587,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
     const float m = fs[s];
     const float f = (M == -INFINITY || m == -INFINITY) ? 0.f : fast_exp2(m - M);
     fs[s] = f;
-    if (f != 0.f) lloc += f * p.pl[(u * S + s) * G + g];
+    lloc += f * ls[s];
   }
   lloc = warp_sum(lloc);
   __syncthreads();
@@ -507,8 +607,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
     for (int r = 0; r < kR; ++r) {
       const int s = s0 + r * (kMergeThreads / 32);
       f[r] = s < S ? fs[s] : 0.f;
-      v[r] = f[r] != 0.f ? *reinterpret_cast<const float4*>(p.pacc + ((u * S + s) * G + g) * kD + lane * 4)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[r] = s < S ? *reinterpret_cast<const float4*>(p.pacc + ((u * S + s) * G + g) * kD + lane * 4)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int r = 0; r < kR; ++r) {
@@ -533,12 +633,12 @@ template <int G, bool kExact, bool kRows>
 cudaError_t launch_attend_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttendParams& p, int grid,
                             cudaStream_t stream, bool pdl) {
   auto kern = attend_kernel<G, kExact, kRows>;
-  const size_t smem = AttendSmem<G>::total;
+  const size_t smem = AttendSmem<G, kRows>::total;
   cudaError_t e = ensure_dyn_smem<attend_kernel<G, kExact, kRows>>(smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(Pipe<kRows>::threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -554,7 +654,8 @@ cudaError_t launch_merge_t(const MergeParams& p, cudaStream_t stream, bool pdl) 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.B * p.Hq);
   cfg.blockDim = dim3(kMergeThreads);
-  cfg.dynamicSmemBytes = (((p.S_tot + 3) & ~3) + (kMergeThreads / 32) * kD) * sizeof(float);
+  const int s4 = (p.S_tot + 3) & ~3;
+  cfg.dynamicSmemBytes = (s4 + (s4 > (kMergeThreads / 32) * kD ? s4 : (kMergeThreads / 32) * kD)) * sizeof(float);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -569,10 +670,10 @@ cudaError_t launch_merge_t(const MergeParams& p, cudaStream_t stream, bool pdl) 
 int attend_slots_per_sm() { return 2; }
 size_t attend_smem_bytes(int G) {
   switch (G) {
-    case 1: return AttendSmem<1>::total;
-    case 2: return AttendSmem<2>::total;
-    case 4: return AttendSmem<4>::total;
-    default: return AttendSmem<8>::total;
+    case 1: return AttendSmem<1, true>::total;
+    case 2: return AttendSmem<2, true>::total;
+    case 4: return AttendSmem<4, true>::total;
+    default: return AttendSmem<8, true>::total;
   }
 }
 

@@ -230,6 +230,12 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ---------------------------------------------------------------------------
+// List slots an index of cap tokens and C clusters needs: every cluster's last chunk
+// of 32 slots may be partly empty.
+__host__ __device__ inline long long list_slots_needed(int cap, int C) {
+  return 32LL * ((static_cast<long long>(cap) + 31) / 32 + C);
+}
+
 // Workspace layout of hsa_decode (computed identically on host and device).
 // ---------------------------------------------------------------------------
 struct UnitState {          // per unit bookkeeping written by the top-k kernels
@@ -250,7 +256,8 @@ struct DecodeLayout {
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, int cap, int nsplit_max) {
+__host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, int cap, int list_slots,
+                                                           int nsplit_max) {
   DecodeLayout L;
   L.U = U;
   L.G = G;
@@ -275,7 +282,7 @@ __host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, 
   L.off_qc = take(u * L.GP * C * 4 * sizeof(float));
   L.off_w = take(u * G * C * sizeof(float));
   L.off_hist = take(u * kNB * sizeof(uint32_t));
-  L.off_sigma = take(u * cap * sizeof(float));
+  L.off_sigma = take(u * list_slots * sizeof(float));   // one score per list slot
   L.off_bitmap = take(u * L.bitmap_words * sizeof(uint32_t));
   L.off_cand = take(u * cap * sizeof(uint64_t));
   L.off_sel = take(u * cap * sizeof(int32_t));

@@ -208,6 +208,117 @@ __global__ void __launch_bounds__(256, 1) encode_kernel(IndexParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Cluster-ordered lists. A unit's list slots form 32-slot chunks; every chunk holds
+// members of one cluster, so the scan sees one cluster per warp-sized chunk. Meta per
+// unit: [0] chunks in use, [1] unused, then per cluster c: [2+2c] its open (last)
+// chunk or -1, [3+2c] members in that chunk.
+// ---------------------------------------------------------------------------
+__global__ void list_reset_kernel(IndexParams p) {
+  const size_t per_unit = 2 + 2 * static_cast<size_t>(p.C);
+  const size_t total = static_cast<size_t>(p.B) * p.Hkv * per_unit;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int u = static_cast<int>(i / per_unit);
+    if (p.zero_if_empty && p.n_indexed[u / p.Hkv] != 0) continue;
+    const size_t r = i % per_unit;
+    p.list_meta[i] = r < 2 ? 0 : ((r & 1) == 0 ? -1 : 32);   // no open chunk: treat as full
+  }
+}
+
+// One CTA per unit: add index slots [lo, lo + n) to their clusters' lists. Count the
+// new members per cluster, give each cluster the room left in its open chunk plus
+// fresh chunks, then place every member (any order inside a cluster).
+constexpr int kListThreads = 1024;
+__global__ void __launch_bounds__(kListThreads) list_append_kernel(IndexParams p) {
+  extern __shared__ int32_t lsm[];
+  const int C = p.C;
+  int32_t* cnt = lsm;
+  int32_t* put = cnt + C;
+  int32_t* base = put + C;
+  int32_t* room = base + C;
+  int32_t* open0 = room + C;
+  int32_t* fill0 = open0 + C;
+  __shared__ int32_t nch_s;
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv;
+  const int tid = threadIdx.x;
+  const int lo = slot_base(p, b);
+  const int n = slot_count(p, b);
+  const int max_chunks = p.list_slots / 32;
+  int32_t* meta = p.list_meta + static_cast<size_t>(u) * (2 + 2 * static_cast<size_t>(C));
+  const uint16_t* ids_u = p.ids + static_cast<size_t>(u) * p.cap;
+  int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
+  uint4* lcodes = reinterpret_cast<uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
+  const uint4* codes_u = reinterpret_cast<const uint4*>(p.codes) + static_cast<size_t>(u) * p.cap;
+  uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * max_chunks;
+  for (int c = tid; c < C; c += blockDim.x) {
+    cnt[c] = 0;
+    put[c] = 0;
+  }
+  if (tid == 0) nch_s = min(max(meta[0], 0), max_chunks);   // garbage metadata cannot index out of range
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) {
+    const int slot = lo + i;
+    if (slot >= p.cap) continue;
+    const uint32_t id = ids_u[slot];
+    if (id < static_cast<uint32_t>(C)) atomicAdd(&cnt[id], 1);
+  }
+  __syncthreads();
+  for (int c = tid; c < C; c += blockDim.x) {
+    const int k = cnt[c];
+    if (k == 0) continue;
+    int op = meta[2 + 2 * c], fl = meta[3 + 2 * c];
+    if (op < 0 || op >= max_chunks || fl < 0 || fl > 32) {   // no (valid) open chunk
+      op = -1;
+      fl = 32;
+    }
+    const int free = op >= 0 ? 32 - fl : 0;
+    const int extra = max(0, k - free);
+    const int nn = (extra + 31) / 32;
+    int bs = nn ? atomicAdd(&nch_s, nn) : 0;
+    if (bs + nn > max_chunks) {   // cannot happen with list_slots >= 32*(ceil(cap/32)+C)
+      record_error(p.err, HSA_DEVERR_SELECT);
+      bs = -1;
+    }
+    base[c] = bs;
+    room[c] = free;
+    open0[c] = op;
+    fill0[c] = fl;
+    if (bs >= 0) {
+      for (int q = 0; q < nn; ++q) ccl[bs + q] = static_cast<uint16_t>(c);
+      if (nn > 0) {
+        const int used = extra - 32 * (nn - 1);
+        for (int r = used; r < 32; ++r) lslot[(bs + nn - 1) * 32 + r] = -1;
+        meta[2 + 2 * c] = bs + nn - 1;
+        meta[3 + 2 * c] = used;
+      } else {
+        meta[3 + 2 * c] = fl + k;
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) {
+    const int slot = lo + i;
+    if (slot >= p.cap) continue;
+    const uint32_t id = ids_u[slot];
+    if (id >= static_cast<uint32_t>(C)) continue;
+    const int r = atomicAdd(&put[id], 1);
+    int ls;
+    if (r < room[id]) {
+      ls = open0[id] * 32 + fill0[id] + r;
+    } else {
+      if (base[id] < 0) continue;
+      const int e = r - room[id];
+      ls = (base[id] + e / 32) * 32 + (e % 32);
+    }
+    lcodes[ls] = codes_u[slot];
+    lslot[ls] = slot;
+  }
+  __syncthreads();
+  if (tid == 0) meta[0] = min(nch_s, max_chunks);
+}
+
 int grid_for(size_t work, int threads) {
   size_t g = (work + threads - 1) / threads;
   if (g > 148 * 16) g = 148 * 16;
@@ -234,6 +345,20 @@ cudaError_t launch_accumulate(const IndexParams& p, int max_slots, cudaStream_t 
   if (max_slots <= 0) return cudaSuccess;
   const dim3 grid(p.B * p.Hkv, (max_slots + 63) / 64);
   accumulate_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_list_reset(const IndexParams& p, cudaStream_t stream) {
+  const size_t work = static_cast<size_t>(p.B) * p.Hkv * (2 + 2 * static_cast<size_t>(p.C));
+  list_reset_kernel<<<grid_for(work, 256), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_list_append(const IndexParams& p, cudaStream_t stream) {
+  const size_t smem = 6 * static_cast<size_t>(p.C) * sizeof(int32_t);
+  cudaError_t e = ensure_dyn_smem<list_append_kernel>(smem);
+  if (e != cudaSuccess) return e;
+  list_append_kernel<<<p.B * p.Hkv, kListThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -63,6 +63,8 @@ struct AttendParams {
   const float* W;            // [U][G][C]
   const float* mean_v;       // [U][C][D]
   const float* bounds;
+  UnitState* units;          // exact mode: per-unit partial counter (pad[0]), zeroed by the table builder
+  float* out;                // exact mode: [B][Hq][D], written by the last CTA of each unit
   int U, B, Hq, Hkv, page_size, max_pages, num_pages, cap, n_sink;
   int nsplit, chunk, S_tot, C, nbg, nq, bg_enabled, k_override;
   double budget;
@@ -106,8 +108,11 @@ struct TablesParams {
 cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, bool pdl);
 
 struct ScanParams {
-  const uint8_t* codes;      // [U][cap][16]
-  const uint16_t* ids;       // [U][cap]
+  const uint8_t* list_codes;     // [U][list_slots][16] cluster-ordered codes
+  const int32_t* list_slot;      // [U][list_slots] index slot of each list slot (-1 empty)
+  const uint16_t* chunk_cluster; // [U][list_slots / 32]
+  const int32_t* list_meta;      // [U][2 + 2C]; [0] = chunks in use
+  int list_slots;
   const int32_t* seq_lens;
   const int32_t* n_indexed;
   const float* lut;
@@ -125,6 +130,11 @@ size_t scan_smem_bytes(int G, int C);
 int scan_threads();
 
 struct SelectParams {
+  const uint8_t* list_codes;     // [U][list_slots][16]
+  const uint16_t* chunk_cluster; // [U][list_slots / 32]
+  const int32_t* list_slot;      // [U][list_slots]
+  const int32_t* list_meta;      // [U][2 + 2C]
+  int list_slots;
   const int32_t* seq_lens;
   const int32_t* n_indexed;
   const uint8_t* codes;
@@ -163,7 +173,12 @@ struct IndexParams {
   int32_t* count;
   int32_t* n_indexed;
   int32_t* err;
-  int B, Hkv, page_size, max_pages, num_pages, C, cap, n_sink;
+  // cluster-ordered lists
+  uint8_t* list_codes;       // [U][list_slots][16]
+  int32_t* list_slot;        // [U][list_slots]
+  uint16_t* chunk_cluster;   // [U][list_slots / 32]
+  int32_t* list_meta;        // [U][2 + 2C]
+  int B, Hkv, page_size, max_pages, num_pages, C, cap, n_sink, list_slots;
   int slot_lo_from_indexed;  // 1: slots start at n_indexed[b]; 0: slots start at 0
   int n_slots;               // slots per unit to process (n_new), or -1 = n_indexed[b]
   int bump_indexed;          // add n_slots to n_indexed[b] in the mean pass
@@ -173,5 +188,7 @@ cudaError_t launch_zero_stats(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_encode(const IndexParams& p, int max_new, cudaStream_t stream);
 cudaError_t launch_accumulate(const IndexParams& p, int max_slots, cudaStream_t stream);
 cudaError_t launch_means(const IndexParams& p, cudaStream_t stream);
+cudaError_t launch_list_reset(const IndexParams& p, cudaStream_t stream);
+cudaError_t launch_list_append(const IndexParams& p, cudaStream_t stream);
 
 }  // namespace pqhsa

@@ -85,6 +85,35 @@ __device__ void find_threshold_desc(const uint32_t* cnt, int nbins, uint32_t nee
   }
 }
 
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t x = lane < nw ? warp_tot[lane] : 0u;
+    uint32_t xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += t;
+    }
+    if (lane < nw) warp_tot[lane] = xi - x;   // exclusive prefix of warp totals
+    if (lane == nw - 1) warp_tot[32] = xi;
+  }
+  __syncthreads();
+  const uint32_t r = warp_tot[warp] + incl - v;
+  total = warp_tot[32];
+  __syncthreads();
+  return r;
+}
+
 // ===========================================================================
 // tables
 // ===========================================================================
@@ -245,10 +274,9 @@ constexpr int kScanUnroll = 2;   // tokens per thread per batch; the next batch 
 template <int G>
 struct ScanSmem {
   static constexpr int GP = (G + 3) / 4;
-  // tables (LUT, centroid terms), cluster weights, histogram; then the mbarrier
+  // tables (LUT, centroid terms) and the score histogram; then the mbarrier
   __host__ __device__ static size_t tables(int C) {
-    return align_up(static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 +
-                        static_cast<size_t>(G) * C * 4 + kNB * 4, 16);
+    return align_up(static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 + kNB * 4, 16);
   }
   __host__ __device__ static size_t bytes(int C) { return tables(C) + 16; }
 };
@@ -289,21 +317,24 @@ __device__ __forceinline__ void score_token(const uint4& code, uint32_t id, cons
   }
 }
 
-// Segment [j0, j1) of unit u: score every slot. `phase` counts segments (mbarrier parity).
+// Chunks [ch0, ch1) of unit u's cluster-ordered list: one warp scores one 32-slot
+// chunk (all members of one cluster), so the centroid term is warp-uniform and the
+// chunk's cluster weights are one warp reduction. `phase` counts segments (mbarrier parity).
 template <int G>
-__device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int j0, int j1, uint8_t* smem,
+__device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0, int ch1, uint8_t* smem,
                                              uint64_t* bar, uint32_t phase, const uint32_t ysoff[8],
                                              const uint32_t sel[4], bool swap_words) {
   constexpr int GP = (G + 3) / 4;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nwarps = blockDim.x >> 5;
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int C = p.C;
+  const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
   const uint32_t lut_bytes = GP * kNcode * kM * 16;
   const uint32_t qc_bytes = GP * C * 16;
   float4* lut_s = reinterpret_cast<float4*>(smem);                               // [GP][256][16]
   float4* qc_s = lut_s + GP * kNcode * kM;                                       // [GP][C]
-  float* w_s = reinterpret_cast<float*>(qc_s + GP * C);                          // [G][C]
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(w_s + G * C);                   // [NB]
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(qc_s + GP * C);                 // [NB]
 
   __syncthreads();  // previous segment finished with shared memory
   if (tid == 0) {
@@ -316,7 +347,6 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int j0,
     for (uint32_t o = 0; o < qc_bytes; o += 32768u)
       bulk_load(reinterpret_cast<uint8_t*>(qc_s) + o, qg + o, min(32768u, qc_bytes - o), bar);
   }
-  for (int i = tid; i < G * C; i += blockDim.x) w_s[i] = 0.f;
   for (int i = tid; i < kNB; i += blockDim.x) hist_s[i] = 0u;
   float ub2[G], lo, inv;
   {
@@ -332,75 +362,65 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int j0,
     }
     inv = (hi > lo) ? __fdiv_rn(static_cast<float>(kNB), __fsub_rn(hi, lo)) : 0.f;
   }
-  const uint8_t* codes_u = p.codes + static_cast<size_t>(u) * p.cap * kM;
-  const uint16_t* ids_u = p.ids + static_cast<size_t>(u) * p.cap;
-  float* sig_u = p.sigma + static_cast<size_t>(u) * p.cap;
+  const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
+  const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
+  const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * (p.list_slots / 32);
+  float* sig_u = p.sigma + static_cast<size_t>(u) * p.list_slots;
+  float* Wu = p.W + static_cast<size_t>(u) * G * C;
   const uint8_t* lut_b = reinterpret_cast<const uint8_t*>(lut_s);
 
-  // first batch of codes is in flight while the tables land
-  uint4 cw[kScanUnroll];
-  uint32_t idv[kScanUnroll];
-#pragma unroll
-  for (int r = 0; r < kScanUnroll; ++r) {
-    const int j = j0 + r * kScanThreads + tid;
-    if (j < j1) {
-      cw[r] = __ldcs(reinterpret_cast<const uint4*>(codes_u) + j);
-      idv[r] = __ldcs(ids_u + j);
-    }
+  // this warp's first chunk is in flight while the tables land
+  int ch = ch0 + warp;
+  uint4 code = make_uint4(0, 0, 0, 0);
+  int32_t js = -1;
+  uint32_t cl = 0;
+  if (ch < ch1) {
+    code = __ldcs(lcodes + ch * 32 + lane);
+    js = __ldcs(lslot + ch * 32 + lane);
+    cl = ccl[ch];
   }
-  __syncthreads();                       // zeroed W / histogram visible
+  __syncthreads();                       // zeroed histogram visible
   mbar_wait(bar, phase & 1, p.err);      // tables landed
   bool bad_id = false;
 
-  for (int base = j0; base < j1; base += kScanUnroll * kScanThreads) {
-    const int nb = base + kScanUnroll * kScanThreads;
-    uint4 cwn[kScanUnroll];
-    uint32_t idn[kScanUnroll];
+  for (; ch < ch1; ch += nwarps) {
+    const int nx = ch + nwarps;
+    uint4 ncode = make_uint4(0, 0, 0, 0);
+    int32_t njs = -1;
+    uint32_t ncl = 0;
+    if (nx < ch1) {
+      ncode = __ldcs(lcodes + nx * 32 + lane);
+      njs = __ldcs(lslot + nx * 32 + lane);
+      ncl = ccl[nx];
+    }
+    uint32_t id = cl;
+    if (id >= static_cast<uint32_t>(C)) {
+      bad_id = true;
+      id = 0;
+    }
+    const bool valid = js >= 0 && js < N;
+    float sh[G];
+    score_token<G>(code, id, lut_b, qc_s, C, ysoff, sel, swap_words, sh);
+    float sg = sh[0];
 #pragma unroll
-    for (int r = 0; r < kScanUnroll; ++r) {
-      const int j = nb + r * kScanThreads + tid;
-      if (j < j1) {
-        cwn[r] = __ldcs(reinterpret_cast<const uint4*>(codes_u) + j);
-        idn[r] = __ldcs(ids_u + j);
-      }
+    for (int g = 1; g < G; ++g) sg = fmaxf(sg, sh[g]);
+    __stcs(sig_u + ch * 32 + lane, valid ? sg : -INFINITY);
+    if (p.approx_logits && valid) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) p.approx_logits[(static_cast<size_t>(b) * p.Hq + h * G + g) * p.cap + js] = sh[g];
     }
 #pragma unroll
-    for (int r = 0; r < kScanUnroll; ++r) {
-      const int j = base + r * kScanThreads + tid;
-      if (j >= j1) continue;
-      uint32_t id = idv[r];
-      if (id >= static_cast<uint32_t>(C)) {
-        bad_id = true;
-        id = 0;
-      }
-      float sh[G];
-      score_token<G>(cw[r], id, lut_b, qc_s, C, ysoff, sel, swap_words, sh);
-      float sg = sh[0];
-#pragma unroll
-      for (int g = 1; g < G; ++g) sg = fmaxf(sg, sh[g]);
-      __stcs(sig_u + j, sg);
-      if (p.approx_logits) {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-          p.approx_logits[(static_cast<size_t>(b) * p.Hq + h * G + g) * p.cap + j] = sh[g];
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) atomicAdd(&w_s[g * C + id], fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])));
-      atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
+    for (int g = 0; g < G; ++g) {
+      const float e = warp_sum(valid ? fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])) : 0.f);
+      if (lane == g) atomicAdd(Wu + g * C + id, e);
     }
-#pragma unroll
-    for (int r = 0; r < kScanUnroll; ++r) {
-      cw[r] = cwn[r];
-      idv[r] = idn[r];
-    }
+    if (valid) atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
+    code = ncode;
+    js = njs;
+    cl = ncl;
   }
   if (bad_id) record_error(p.err, HSA_DEVERR_CLUSTER);
   __syncthreads();
-  float* Wg = p.W + static_cast<size_t>(u) * G * C;
-  for (int i = tid; i < G * C; i += blockDim.x) {
-    const float v = w_s[i];
-    if (v != 0.f) atomicAdd(Wg + i, v);
-  }
   uint32_t* hg = p.hist + static_cast<size_t>(u) * kNB;
   for (int i = tid; i < kNB; i += blockDim.x) {
     const uint32_t v = hist_s[i];
@@ -408,19 +428,20 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int j0,
   }
 }
 
-// Walk the balanced global slot range of this CTA over the units.
-template <typename F>
-__device__ __forceinline__ void for_each_segment(const int32_t* seq_lens, const int32_t* n_indexed, int B, int Hkv,
-                                                 int n_sink, int cap, F&& f) {
+// Walk the balanced global item range of this CTA over the units; count(b, h) gives
+// the items of unit (b, h). f(u, i0, i1) is called for every overlapped unit range.
+template <typename Count, typename F>
+__device__ __forceinline__ void for_each_range(int B, int Hkv, Count&& count, F&& f) {
   long long total = 0;
-  for (int b = 0; b < B; ++b) total += static_cast<long long>(Hkv) * unit_n(seq_lens, n_indexed, b, n_sink, cap);
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hkv; ++h) total += count(b, h);
   const long long start = total * blockIdx.x / gridDim.x;
   const long long end = total * (blockIdx.x + 1) / gridDim.x;
   if (start >= end) return;
   long long acc = 0;
   for (int b = 0; b < B && acc < end; ++b) {
-    const int n = unit_n(seq_lens, n_indexed, b, n_sink, cap);
     for (int h = 0; h < Hkv && acc < end; ++h) {
+      const int n = count(b, h);
       if (start < acc + n && end > acc) {
         const int j0 = static_cast<int>(max(start - acc, 0LL));
         const int j1 = static_cast<int>(min(end - acc, static_cast<long long>(n)));
@@ -429,6 +450,11 @@ __device__ __forceinline__ void for_each_segment(const int32_t* seq_lens, const 
       acc += n;
     }
   }
+}
+
+__device__ __forceinline__ int unit_chunks(const int32_t* list_meta, int u, int C, int max_chunks) {
+  const int n = list_meta[static_cast<size_t>(u) * (2 + 2 * static_cast<size_t>(C))];
+  return max(0, min(n, max_chunks));
 }
 
 template <int G>
@@ -458,139 +484,25 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
   pdl_wait();
   pdl_launch_dependents();
   uint32_t phase = 0;
-  for_each_segment(p.seq_lens, p.n_indexed, p.B, p.Hkv, p.n_sink, p.cap, [&](int u, int j0, int j1) {
-    scan_segment<G>(p, u, j0, j1, smem, bar, phase, ysoff, sel, swap_words);
-    ++phase;
-  });
+  const int max_chunks = p.list_slots / 32;
+  for_each_range(
+      p.B, p.Hkv, [&](int b, int h) { return unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
+      [&](int u, int c0, int c1) {
+        scan_segment<G>(p, u, c0, c1, smem, bar, phase, ysoff, sel, swap_words);
+        ++phase;
+      });
 }
 
 // ===========================================================================
 // filter: tokens above the threshold bin are selected, the bin's tokens are candidates
 // ===========================================================================
+// Remove the weight e^{shat_g - ub_g} of a selected token (cluster id, code words cw)
+// from its cluster's sums.
 template <int G>
-__global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
-  constexpr int kBatch = 8;
-  __shared__ __align__(16) uint32_t hist_s[kNB];
-  __shared__ int sh_bstar;
-  __shared__ uint32_t sh_above;
-  pdl_wait();
-  pdl_launch_dependents();
-  for_each_segment(p.seq_lens, p.n_indexed, p.B, p.Hkv, p.n_sink, p.cap, [&](int u, int j0, int j1) {
-    const int b = u / p.Hkv;
-    const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
-    const int k = decode_k(p.budget, p.k_override, N);
-    const float* sig = p.sigma + static_cast<size_t>(u) * p.cap;
-    // first batch of scores in flight while the threshold is found
-    float sv[kBatch];
-#pragma unroll
-    for (int r = 0; r < kBatch; ++r) {
-      const int j = j0 + r * blockDim.x + threadIdx.x;
-      sv[r] = j < j1 ? sig[j] : 0.f;
-    }
-    __syncthreads();
-    {
-      const uint4* hg = reinterpret_cast<const uint4*>(p.hist + static_cast<size_t>(u) * kNB);
-      uint4 hv[kNB / 4 / 256];
-#pragma unroll
-      for (int r = 0; r < kNB / 4 / 256; ++r) hv[r] = hg[r * 256 + threadIdx.x];
-#pragma unroll
-      for (int r = 0; r < kNB / 4 / 256; ++r) reinterpret_cast<uint4*>(hist_s)[r * 256 + threadIdx.x] = hv[r];
-    }
-    if (threadIdx.x == 0) {
-      sh_bstar = kNB;   // k == 0: nothing selected
-      sh_above = 0;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) find_threshold_desc(hist_s, kNB, static_cast<uint32_t>(k), &sh_bstar, &sh_above);
-    __syncthreads();
-    const int bstar = sh_bstar;
-    if (threadIdx.x == 0) {
-      p.units[u].bstar = bstar;
-      p.units[u].above = static_cast<int32_t>(sh_above);
-    }
-    if (bstar >= kNB) return;
-    float ub[G], lb[G];
-    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
-    float hi = ub[0], lo = lb[0];
-#pragma unroll
-    for (int g = 1; g < G; ++g) {
-      hi = fmaxf(hi, ub[g]);
-      lo = fmaxf(lo, lb[g]);
-    }
-    const float inv = (hi > lo) ? __fdiv_rn(static_cast<float>(kNB), __fsub_rn(hi, lo)) : 0.f;
-    uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
-    for (int base = j0; base < j1; base += kBatch * blockDim.x) {
-      float nv[kBatch];
-      const int nb = base + kBatch * blockDim.x;
-#pragma unroll
-      for (int r = 0; r < kBatch; ++r) {
-        const int j = nb + r * blockDim.x + threadIdx.x;
-        nv[r] = j < j1 ? sig[j] : 0.f;
-      }
-#pragma unroll
-      for (int r = 0; r < kBatch; ++r) {
-        const int j = base + r * blockDim.x + threadIdx.x;
-        if (j >= j1) continue;
-        const int bin = score_bin(sv[r], lo, inv);
-        if (bin > bstar) {
-          atomicOr(bm + (j >> 5), 1u << (j & 31));
-        } else if (bin == bstar) {
-          const int slot = atomicAdd(&p.units[u].ncand, 1);
-          if (slot < p.cap)
-            p.cand[static_cast<size_t>(u) * p.cap + slot] =
-                (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < kBatch; ++r) sv[r] = nv[r];
-    }
-  });
-}
-
-// ===========================================================================
-// finalize (one CTA per unit)
-// ===========================================================================
-constexpr int kFinThreads = 1024;
-constexpr int kFinWordsPerThread = 4;
-constexpr int kFinChunkWords = kFinWordsPerThread * kFinThreads;   // 131072 slots per pass
-constexpr int kFinSmemCand = kFinThreads;                          // candidates resolved in shared memory
-
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = blockDim.x >> 5;
-  uint32_t incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t x = lane < nw ? warp_tot[lane] : 0u;
-    uint32_t xi = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, xi, o);
-      if (lane >= o) xi += t;
-    }
-    if (lane < nw) warp_tot[lane] = xi - x;   // exclusive prefix of warp totals
-    if (lane == nw - 1) warp_tot[32] = xi;
-  }
-  __syncthreads();
-  const uint32_t r = warp_tot[warp] + incl - v;
-  total = warp_tot[32];
-  __syncthreads();
-  return r;
-}
-
-// Remove the weight e^{shat_gj - ub_g} of selected slot j from its cluster's sums.
-template <int G>
-__device__ __forceinline__ void unselect_weight(const SelectParams& p, int u, int j, const float* ub2) {
+__device__ __forceinline__ void unselect_weight(const SelectParams& p, int u, uint32_t id, const uint4 cw,
+                                                const float* ub2) {
   constexpr int GP = (G + 3) / 4;
-  uint32_t id = p.ids[static_cast<size_t>(u) * p.cap + j];
   if (id >= static_cast<uint32_t>(p.C)) id = 0;
-  const uint4 cw = *reinterpret_cast<const uint4*>(p.codes + (static_cast<size_t>(u) * p.cap + j) * kM);
   const uint32_t cwords[4] = {cw.x, cw.y, cw.z, cw.w};
   const float4* lut4 = reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
   const float4* qc4 = reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C;
@@ -617,6 +529,140 @@ __device__ __forceinline__ void unselect_weight(const SelectParams& p, int u, in
     atomicAdd(&Wu[g * p.C + id], -fast_exp2(fmaf(sh, kLog2e, -ub2[g])));
   }
 }
+
+template <int G>
+__global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
+  constexpr int kBatch = 8;
+  __shared__ __align__(16) uint32_t hist_s[kNB];
+  __shared__ uint32_t scan_tot[33];
+  __shared__ int sh_bstar;
+  __shared__ uint32_t sh_above;
+  static_assert(kNB == 8 * 256, "filter threshold search: 256 threads x 8 bins");
+  pdl_wait();
+  pdl_launch_dependents();
+  const int max_chunks = p.list_slots / 32;
+  for_each_range(
+      p.B, p.Hkv, [&](int b, int h) { return 32 * unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
+      [&](int u, int j0, int j1) {
+    const int b = u / p.Hkv;
+    const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
+    const int k = decode_k(p.budget, p.k_override, N);
+    const float* sig = p.sigma + static_cast<size_t>(u) * p.list_slots;
+    const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
+    // first batch of scores in flight while the threshold is found
+    float sv[kBatch];
+    int32_t jv[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int j = j0 + r * blockDim.x + threadIdx.x;
+      sv[r] = j < j1 ? sig[j] : 0.f;
+      jv[r] = j < j1 ? lslot[j] : -1;
+    }
+    __syncthreads();
+    {
+      const uint4* hg = reinterpret_cast<const uint4*>(p.hist + static_cast<size_t>(u) * kNB);
+      uint4 hv[kNB / 4 / 256];
+#pragma unroll
+      for (int r = 0; r < kNB / 4 / 256; ++r) hv[r] = hg[r * 256 + threadIdx.x];
+#pragma unroll
+      for (int r = 0; r < kNB / 4 / 256; ++r) reinterpret_cast<uint4*>(hist_s)[r * 256 + threadIdx.x] = hv[r];
+    }
+    if (threadIdx.x == 0) {
+      sh_bstar = kNB;   // k == 0: nothing selected
+      sh_above = 0;
+    }
+    __syncthreads();
+    {
+      // thread t owns the 8 bins [kNB-8(t+1), kNB-8t): block scan of counts from the top
+      const int hi = kNB - 8 * static_cast<int>(threadIdx.x);
+      uint32_t c8[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c8[i] = hist_s[hi - 1 - i];
+        local += c8[i];
+      }
+      uint32_t tot;
+      const uint32_t excl = block_excl_scan(local, scan_tot, tot);
+      const uint32_t need = static_cast<uint32_t>(k);
+      if (need > 0 && excl < need && excl + local >= need) {
+        uint32_t cum = excl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (cum < need && cum + c8[i] >= need) {
+            sh_bstar = hi - 1 - i;
+            sh_above = cum;
+          }
+          cum += c8[i];
+        }
+      }
+    }
+    __syncthreads();
+    const int bstar = sh_bstar;
+    if (threadIdx.x == 0) {
+      p.units[u].bstar = bstar;
+      p.units[u].above = static_cast<int32_t>(sh_above);
+    }
+    if (bstar >= kNB) return;
+    float ub[G], lb[G];
+    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
+    float hi = ub[0], lo = lb[0];
+#pragma unroll
+    for (int g = 1; g < G; ++g) {
+      hi = fmaxf(hi, ub[g]);
+      lo = fmaxf(lo, lb[g]);
+    }
+    const float inv = (hi > lo) ? __fdiv_rn(static_cast<float>(kNB), __fsub_rn(hi, lo)) : 0.f;
+    float ub2[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
+    const bool fix = p.background && N > k;
+    const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
+    const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * (p.list_slots / 32);
+    uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
+    for (int base = j0; base < j1; base += kBatch * blockDim.x) {
+      float nv[kBatch];
+      int32_t njv[kBatch];
+      const int nb = base + kBatch * blockDim.x;
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int j = nb + r * blockDim.x + threadIdx.x;
+        nv[r] = j < j1 ? sig[j] : 0.f;
+        njv[r] = j < j1 ? lslot[j] : -1;
+      }
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int j = jv[r];            // index slot of this list slot
+        if (j < 0 || j >= N) continue;
+        const int bin = score_bin(sv[r], lo, inv);
+        if (bin > bstar) {
+          atomicOr(bm + (j >> 5), 1u << (j & 31));
+          if (fix) {   // selected for sure: take its weight out of its cluster's sums now
+            const int ls = base + r * blockDim.x + threadIdx.x;
+            unselect_weight<G>(p, u, ccl[ls >> 5], lcodes[ls], ub2);
+          }
+        } else if (bin == bstar) {
+          const int slot = atomicAdd(&p.units[u].ncand, 1);
+          if (slot < p.cap)
+            p.cand[static_cast<size_t>(u) * p.cap + slot] =
+                (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        sv[r] = nv[r];
+        jv[r] = njv[r];
+      }
+    }
+  });
+}
+
+// ===========================================================================
+// finalize (one CTA per unit)
+// ===========================================================================
+constexpr int kFinThreads = 1024;
+constexpr int kFinWordsPerThread = 4;
+constexpr int kFinChunkWords = kFinWordsPerThread * kFinThreads;   // 131072 slots per pass
+constexpr int kFinSmemCand = kFinThreads;                          // candidates resolved in shared memory
 
 // One CTA per unit: resolve the threshold bin's candidates exactly (score desc, position
 // asc), compact the selection bitmap into ascending positions, and take the selected
@@ -770,7 +816,6 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
           if (p.dbg_selected) p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = s0 + j;
         }
         ++off;
-        if (fix) unselect_weight<G>(p, u, j, ub2);
       }
     }
     running += tot;
@@ -779,6 +824,16 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     p.units[u].nsel = static_cast<int32_t>(running);
     if (running != static_cast<uint32_t>(k)) record_error(p.err, HSA_DEVERR_SELECT);
     if (p.dbg_nselected) p.dbg_nselected[u] = static_cast<int32_t>(running);
+  }
+  if (fix) {
+    // the filter already removed the tokens above the threshold bin; here only the
+    // winners taken from the threshold bin, one per thread
+    for (uint32_t i = tid; i < nwin; i += blockDim.x) {
+      const int j = static_cast<int>(wins[i]);
+      const uint32_t id = p.ids[static_cast<size_t>(u) * p.cap + j];
+      const uint4 cw = *reinterpret_cast<const uint4*>(p.codes + (static_cast<size_t>(u) * p.cap + j) * kM);
+      unselect_weight<G>(p, u, id, cw, ub2);
+    }
   }
 }
 

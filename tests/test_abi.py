@@ -44,6 +44,13 @@ def test_abi_struct_sizes_match_binding(lib):
     assert [s.value for s in sizes] == [ctypes.sizeof(t) for t in (P._KV, P._Index, P._Params, P._Debug)]
 
 
+def test_list_capacity(lib):
+    lib.hsa_index_list_slots.restype = ctypes.c_int64
+    lib.hsa_index_list_slots.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    assert lib.hsa_index_list_slots(130032, 1024) == 32 * (4064 + 1024) == P.index_list_slots(130032, 1024)
+    assert lib.hsa_index_list_slots(0, 4) == 0
+
+
 def test_strerror(lib):
     assert P.hsa_strerror(0) == "ok"
     assert P.hsa_strerror(2) == "unsupported shape"
@@ -61,9 +68,13 @@ def _kv(B=1, Hq=4, Hkv=1, D=128, page_size=16, max_pages=8, num_pages=8, seq=100
     return kv, lens
 
 
-def _ix(B=1, C=16, cap=128, n_idx=50, n_sink=4, M=16, dsub=8):
+def _ix(B=1, C=16, cap=128, n_idx=50, n_sink=4, M=16, dsub=8, list_slots=None):
     nh = np.full(B, n_idx, dtype=np.int32)
-    ix = P._Index(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, nh.ctypes.data, C, M, dsub, 256, cap, n_sink)
+    ls = P.index_list_slots(cap, max(C, 1)) if list_slots is None else list_slots
+    ix = P._Index(centroids=FAKE, codebooks=FAKE, codes=FAKE, ids=FAKE, sum_v=FAKE, mean_v=FAKE, count=FAKE,
+                  n_indexed=FAKE, n_indexed_host=nh.ctypes.data, list_codes=FAKE, list_slot=FAKE,
+                  chunk_cluster=FAKE, list_meta=FAKE, C=C, M=M, dsub=dsub, ncode=256, cap=cap, n_sink=n_sink,
+                  list_slots=ls)
     return ix, nh
 
 
@@ -91,6 +102,8 @@ def test_decode_rejects_bad_cache(lib, mutate, status):
     (dict(C=0), 1),
     (dict(n_idx=200), 3),              # more than cap
     (dict(n_idx=99), 3),               # n_sink + N > T
+    (dict(list_slots=32 * 4), 3),      # cluster lists too small
+    (dict(C=5000), 2),                 # too many clusters for the list builder
 ])
 def test_decode_rejects_bad_index(lib, mutate, status):
     kv, lens = _kv()
