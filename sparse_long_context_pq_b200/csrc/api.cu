@@ -462,12 +462,11 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   p.k_override = prm->k_override;
   p.budget = prm->budget;
   p.qscale = prm->scale * kLog2e;
-  p.units = units;
-  p.out = out;
   RET_CUDA(mark(4));
   RET_CUDA(launch_attend(G, true, true, tk, tv, p, U * (sp.nsplit + L.nbg), stream, use_pdl()));
-  // the last CTA of each unit merges it inside the attention launch
+  MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, S_tot};
   RET_CUDA(mark(5));
+  RET_CUDA(launch_merge(G, mp, stream, use_pdl()));
   RET_CUDA(mark(6));
   return HSA_OK;
 }

@@ -78,62 +78,6 @@ __device__ __forceinline__ int exact_row_pos(int v, int s0, int k, int N, const 
   return s0 + N + (v - s0 - k);
 }
 
-// The CTA that completes a unit's last partial merges the unit: every CTA writes its
-// partial, fences, and takes a ticket; the holder of the last ticket (no waiting)
-// computes out_g = sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s for the unit's heads.
-// `nt` threads (ids 0..nt-1) take part; `scratch` holds 2 * G * S_tot floats.
-template <int G>
-__device__ void merge_unit_if_last(const AttendParams& p, int u, int nt, int t, float* scratch, int* flag,
-                                   bool named_barrier) {
-  auto sync = [&]() {
-    if (named_barrier) asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");
-    else __syncthreads();
-  };
-  sync();                                   // this CTA's partial is fully written
-  if (t == 0) {
-    __threadfence();
-    const int done = atomicAdd(&p.units[u].pad[0], 1);
-    *flag = (done == p.S_tot - 1);
-  }
-  sync();
-  if (!*flag) return;
-  __threadfence();
-  const int S = p.S_tot;
-  const int b = u / p.Hkv, h = u % p.Hkv;
-  float* fs = scratch;                      // [G][S] weights e^{m - M}
-  float* ls = scratch + G * S;              // [G][S] l of each partial
-  for (int i = t; i < G * S; i += nt) {
-    const int g = i / S, sp = i % S;
-    const size_t sl = (static_cast<size_t>(u) * S + sp) * G + g;
-    fs[i] = p.pm[sl];
-    ls[i] = p.pl[sl];
-  }
-  sync();
-  if (t < G) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, fs[t * S + sp]);
-    float L = 0.f;
-    for (int sp = 0; sp < S; ++sp) {
-      const float m = fs[t * S + sp];
-      const float f = (M == -INFINITY || m == -INFINITY) ? 0.f : fast_exp2(m - M);
-      fs[t * S + sp] = f;
-      L += f * ls[t * S + sp];
-    }
-    ls[t * S] = L;                          // L_g kept in the first l slot of head g
-  }
-  sync();
-  for (int i = t; i < G * kD; i += nt) {
-    const int g = i / kD, d = i % kD;
-    float a = 0.f;
-#pragma unroll 4
-    for (int sp = 0; sp < S; ++sp)
-      a = fmaf(fs[g * S + sp], p.pacc[((static_cast<size_t>(u) * S + sp) * G + g) * kD + d], a);
-    const float L = ls[g * S];
-    p.out[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] = L > 0.f ? a / L : 0.f;
-  }
-  if (t == 0) p.units[u].pad[0] = 0;        // ready for the next call
-}
-
 template <int G, bool kExact, bool kRows>
 __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
     attend_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -442,11 +386,6 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
       }
     }
   }
-  if (kExact) {
-    // the pipeline has drained: the stage area is free for the merge scratch
-    merge_unit_if_last<G>(p, u, kConsumerWarps * 32, tid, reinterpret_cast<float*>(stage_base) + 8192,
-                          reinterpret_cast<int*>(stage_base) + 8191, true);
-  }
 }
 
 }  // namespace
@@ -476,8 +415,6 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
       p.pm[slot * G + tid] = -INFINITY;
       p.pl[slot * G + tid] = 0.f;
     }
-    merge_unit_if_last<G>(p, u, blockDim.x, tid, reinterpret_cast<float*>(smem) + 8192,
-                          reinterpret_cast<int*>(smem) + 8191, false);
     return;
   }
   const int c0 = cb * kBgClusters;
@@ -540,8 +477,6 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
     p.pm[slot * G + tid] = ub[tid] * kLog2e;
     p.pl[slot * G + tid] = l;
   }
-  merge_unit_if_last<G>(p, u, blockDim.x, tid, reinterpret_cast<float*>(smem) + 8192,
-                        reinterpret_cast<int*>(smem) + 8191, false);
 }
 
 namespace {

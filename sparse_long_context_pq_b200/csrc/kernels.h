@@ -63,8 +63,6 @@ struct AttendParams {
   const float* W;            // [U][G][C]
   const float* mean_v;       // [U][C][D]
   const float* bounds;
-  UnitState* units;          // exact mode: per-unit partial counter (pad[0]), zeroed by the table builder
-  float* out;                // exact mode: [B][Hq][D], written by the last CTA of each unit
   int U, B, Hq, Hkv, page_size, max_pages, num_pages, cap, n_sink;
   int nsplit, chunk, S_tot, C, nbg, nq, bg_enabled, k_override;
   double budget;

@@ -291,9 +291,13 @@ __device__ __forceinline__ void score_token(const uint4& code, uint32_t id, cons
     uint32_t t = w0; w0 = w1; w1 = t;
     t = w2; w2 = w3; w3 = t;
   }
-  float4 acc[GP];
+  // two independent partial sums per head (even / odd lookups) halve the dependent add chain
+  float4 acc[2][GP];
 #pragma unroll
-  for (int gp = 0; gp < GP; ++gp) acc[gp] = qc_s[gp * C + id];
+  for (int gp = 0; gp < GP; ++gp) {
+    acc[0][gp] = qc_s[gp * C + id];
+    acc[1][gp] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
   for (int i = 0; i < kM; ++i) {
     const uint32_t wd = (i < 4) ? w0 : (i < 8) ? w1 : (i < 12) ? w2 : w3;
@@ -302,19 +306,48 @@ __device__ __forceinline__ void score_token(const uint4& code, uint32_t id, cons
 #pragma unroll
     for (int gp = 0; gp < GP; ++gp) {
       const float4 v = *reinterpret_cast<const float4*>(lut_b + gp * (kNcode * kM * 16) + off);
-      acc[gp].x = __fadd_rn(acc[gp].x, v.x);
-      acc[gp].y = __fadd_rn(acc[gp].y, v.y);
-      acc[gp].z = __fadd_rn(acc[gp].z, v.z);
-      acc[gp].w = __fadd_rn(acc[gp].w, v.w);
+      float4& a = acc[i & 1][gp];
+      a.x = __fadd_rn(a.x, v.x);
+      a.y = __fadd_rn(a.y, v.y);
+      a.z = __fadd_rn(a.z, v.z);
+      a.w = __fadd_rn(a.w, v.w);
     }
   }
 #pragma unroll
   for (int gp = 0; gp < GP; ++gp) {
-    if (gp * 4 + 0 < G) sh[gp * 4 + 0] = acc[gp].x;
-    if (gp * 4 + 1 < G) sh[gp * 4 + 1] = acc[gp].y;
-    if (gp * 4 + 2 < G) sh[gp * 4 + 2] = acc[gp].z;
-    if (gp * 4 + 3 < G) sh[gp * 4 + 3] = acc[gp].w;
+    if (gp * 4 + 0 < G) sh[gp * 4 + 0] = __fadd_rn(acc[0][gp].x, acc[1][gp].x);
+    if (gp * 4 + 1 < G) sh[gp * 4 + 1] = __fadd_rn(acc[0][gp].y, acc[1][gp].y);
+    if (gp * 4 + 2 < G) sh[gp * 4 + 2] = __fadd_rn(acc[0][gp].z, acc[1][gp].z);
+    if (gp * 4 + 3 < G) sh[gp * 4 + 3] = __fadd_rn(acc[0][gp].w, acc[1][gp].w);
   }
+}
+
+// Warp sum of G per-lane values, scattered: after log2(G) halving exchanges each lane
+// holds a partial of one value, then plain butterflies finish it. Returns the total of
+// value (lane >> (5 - log2 G)) in every lane of that group (lane (32/G)*g holds head g).
+template <int G>
+__device__ __forceinline__ float warp_sum_scatter(float* v) {
+  const int lane = threadIdx.x & 31;
+  int n = G;
+  int o = 16;
+#pragma unroll
+  for (int step = 0; (1 << step) < G; ++step) {
+    const bool up = (lane & o) != 0;
+    const int half = n >> 1;
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) {
+      if (i < half) {
+        const float send = up ? v[i] : v[i + half];
+        const float keep = up ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    n = half;
+    o >>= 1;
+  }
+  float t = v[0];
+  for (; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  return t;
 }
 
 // Chunks [ch0, ch1) of unit u's cluster-ordered list: one warp scores one 32-slot
@@ -409,10 +442,13 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
 #pragma unroll
       for (int g = 0; g < G; ++g) p.approx_logits[(static_cast<size_t>(b) * p.Hq + h * G + g) * p.cap + js] = sh[g];
     }
+    {
+      float ev[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float e = warp_sum(valid ? fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])) : 0.f);
-      if (lane == g) atomicAdd(Wu + g * C + id, e);
+      for (int g = 0; g < G; ++g) ev[g] = valid ? fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])) : 0.f;
+      const float e = warp_sum_scatter<G>(ev);
+      constexpr int kGroup = 32 / G;
+      if ((lane & (kGroup - 1)) == 0) atomicAdd(Wu + (lane / kGroup) * C + id, e);
     }
     if (valid) atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
     code = ncode;
