@@ -530,7 +530,8 @@ def run_reference(args):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.T, "budget": w.budget},
         "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
                          "sample": f"each step: whole (sequence, KV head) units of the workload for "
-                                   f"~{per_step_seconds:.1f} s, scaled to a full step ({units_total} units)"},
+                                   f"~{per_step_seconds:.1f} s, scaled to a full step of {w.B * w.Hkv} units "
+                                   f"({units_total} units timed over {args.steps} steps)"},
         "e2e": {"value": round(us, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(res), flush=True)

@@ -72,20 +72,21 @@ typedef struct {
 
 /* IVF-PQ index storage, one index per (sequence, KV head) "unit" u = b * Hkv + h. */
 typedef struct {
-  float* centroids;                /* fp32 [B][Hkv][C][D]            (caller fills) */
-  float* codebooks;                /* fp32 [B][Hkv][M][ncode][dsub]  (caller fills) */
+  float* centroids;                /* fp32 [B][Hkv][C][D]            (caller fills; 16-B aligned) */
+  float* codebooks;                /* fp32 [B][Hkv][M][ncode][dsub]  (caller fills; 16-B aligned) */
   uint8_t* codes;                  /* u8  [B][Hkv][cap][M]  residual PQ code of slot i */
   uint16_t* ids;                   /* u16 [B][Hkv][cap]     cluster of slot i, < C */
   float* sum_v;                    /* fp32 [B][Hkv][C][D]   sum of member values */
-  float* mean_v;                   /* fp32 [B][Hkv][C][D]   mean member value (0 if empty) */
+  float* mean_v;                   /* fp32 [B][Hkv][C][D]   mean member value (0 if empty); 16-B aligned */
   int32_t* count;                  /* [B][Hkv][C]           members per cluster */
   int32_t* n_indexed;              /* [B] indexed tokens per sequence (device) */
   int32_t* n_indexed_host;         /* [B] host copy of n_indexed */
   /* Cluster-ordered copy of the codes, kept by hsa_build_from_codes / hsa_append_encode
      and read by hsa_decode: the list slots of a unit form 32-slot chunks, each chunk
      holding members of one cluster (its last chunk may be partly empty). */
-  uint8_t* list_codes;             /* u8  [B][Hkv][list_slots][M] */
-  int32_t* list_slot;              /* [B][Hkv][list_slots]  index slot of the member, -1 = empty */
+  uint8_t* list_codes;             /* u8  [B][Hkv][list_slots][M], 16-B aligned */
+  int32_t* list_slot;              /* [B][Hkv][list_slots]  index slot of the member, -1 = empty;
+                                      16-B aligned (both are streamed by bulk copies) */
   uint16_t* chunk_cluster;         /* [B][Hkv][list_slots / 32] cluster of each chunk */
   int32_t* list_meta;              /* [B][Hkv][2 + 2*C]: chunks in use, unused, then per cluster
                                       (its open chunk or -1, members in that chunk) */

@@ -123,9 +123,9 @@ hsa_status check_index(const hsa_kv_cache* kv, const hsa_index* ix, bool need_co
     return HSA_ERR_ALIGNMENT;
   // cluster-ordered lists
   if (!ix->list_codes || !ix->list_slot || !ix->chunk_cluster || !ix->list_meta) return HSA_ERR_INVALID_ARG;
-  if (ix->C > 4096) return HSA_ERR_UNSUPPORTED;
+  if (ix->C > kMaxClusters) return HSA_ERR_UNSUPPORTED;
   if (ix->list_slots < list_slots_needed(ix->cap, ix->C) || ix->list_slots % 32) return HSA_ERR_CAPACITY;
-  if (!aligned(ix->list_codes, 16) || !aligned(ix->list_slot, 4) || !aligned(ix->list_meta, 4) ||
+  if (!aligned(ix->list_codes, 16) || !aligned(ix->list_slot, 16) || !aligned(ix->list_meta, 4) ||
       !aligned(ix->chunk_cluster, 2))
     return HSA_ERR_ALIGNMENT;
   for (int b = 0; b < kv->B; ++b) {
@@ -303,8 +303,8 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   if (!aligned(q, 16) || !aligned(out, 16)) return HSA_ERR_ALIGNMENT;
   if (!(prm->budget >= 0.0) || !std::isfinite(prm->scale)) return HSA_ERR_INVALID_ARG;
   const int U = kv->B * kv->Hkv, G = kv->Hq / kv->Hkv;
-  const size_t scan_smem = scan_smem_bytes(G, ix->C);
-  if (scan_smem > 227 * 1024) return HSA_ERR_UNSUPPORTED;
+  const int ring_depth = scan_ring_depth(G, ix->C);
+  if (ring_depth < 2) return HSA_ERR_UNSUPPORTED;   // LUT + centroid terms too large for shared memory
   const DecodeLayout L = make_decode_layout(U, G, ix->C, ix->cap, ix->list_slots, kMaxSplits);
   if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HSA_ERR_WORKSPACE;
   const DeviceInfo* dev = device_info();
@@ -328,6 +328,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   int32_t* err = reinterpret_cast<int32_t*>(base);
   UnitState* units = reinterpret_cast<UnitState*>(base + L.off_units);
   float* bounds = reinterpret_cast<float*>(base + L.off_bounds);
+  float* fbounds = reinterpret_cast<float*>(base + L.off_fbounds);
   float* lut = reinterpret_cast<float*>(base + L.off_lut);
   float* qc = reinterpret_cast<float*>(base + L.off_qc);
   float* W = reinterpret_cast<float*>(base + L.off_w);
@@ -335,6 +336,8 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   float* sigma = reinterpret_cast<float*>(base + L.off_sigma);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(base + L.off_bitmap);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(base + L.off_cand);
+  float* cand_w = reinterpret_cast<float*>(base + L.off_candw);
+  int32_t* cand_c = reinterpret_cast<int32_t*>(base + L.off_candc);
   int32_t* sel = reinterpret_cast<int32_t*>(base + L.off_sel);
   float* pm = reinterpret_cast<float*>(base + L.off_pm);
   float* pl = reinterpret_cast<float*>(base + L.off_pl);
@@ -385,10 +388,11 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   sc.cap = ix->cap;
   sc.C = ix->C;
   sc.nq = L.nq;
+  sc.fbounds = fbounds;
   sc.n_sink = ix->n_sink;
-  const int scan_per_sm = (scan_smem <= 110 * 1024) ? 2 : 1;
+  sc.ring_depth = ring_depth;
   RET_CUDA(mark(1));
-  RET_CUDA(launch_scan(G, sc, dev->sms * scan_per_sm, stream, use_pdl()));
+  RET_CUDA(launch_scan(G, sc, dev->sms, stream, use_pdl()));
 
   SelectParams se = {};
   se.list_codes = ix->list_codes;
@@ -407,6 +411,8 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   se.hist = hist;
   se.bitmap = bitmap;
   se.cand = cand;
+  se.cand_w = cand_w;
+  se.cand_c = cand_c;
   se.units = units;
   se.sel = sel;
   se.W = W;
@@ -418,6 +424,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   se.cap = ix->cap;
   se.C = ix->C;
   se.nq = L.nq;
+  se.fbounds = fbounds;
   se.n_sink = ix->n_sink;
   se.bitmap_words = L.bitmap_words;
   se.k_override = prm->k_override;
@@ -458,6 +465,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   p.C = ix->C;
   p.nbg = L.nbg;
   p.nq = L.nq;
+  p.fbounds = fbounds;
   p.bg_enabled = prm->background ? 1 : 0;
   p.k_override = prm->k_override;
   p.budget = prm->budget;

@@ -70,12 +70,14 @@ template <bool kRows>
 __device__ __forceinline__ uint32_t v_area() { return kRows ? kTile * kRowPitch : 2 * kHalfBytes; }
 
 
-// Position of row v of a unit's exact list: sink [0,s0), then the k selected
-// positions (ascending), then the tail [s0+N, T).
-__device__ __forceinline__ int exact_row_pos(int v, int s0, int k, int N, const int32_t* sel_u) {
+// Position of row v of a unit's exact list: the sink [0, s0), then the R tail rows
+// [s0+N, T), then the k selected positions (ascending). Sink and tail rows come first
+// because they do not depend on the selection: their copies and math can run while
+// the selection kernels are still finishing.
+__device__ __forceinline__ int exact_row_pos(int v, int s0, int N, int R, const int32_t* sel_u) {
   if (v < s0) return v;
-  if (v < s0 + k) return sel_u[v - s0];
-  return s0 + N + (v - s0 - k);
+  if (v < s0 + R) return s0 + N + (v - s0);
+  return sel_u[v - s0 - R];
 }
 
 template <int G, bool kExact, bool kRows>
@@ -110,22 +112,29 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
   const int b = u / p.Hkv;
   const int h = u % p.Hkv;
 
-  pdl_wait();
+  // Dense decode waits for the previous kernel at once (its partials may still be read by
+  // the previous merge). The exact part reads only data that predate the step until it
+  // needs the selection: sink and tail rows are copied and attended while the selection
+  // kernels finish; the producer waits before the first selected position, every thread
+  // before writing its partials.
+  if (!kExact) pdl_wait();
   pdl_launch_dependents();
 
   // ---- row range of this split ------------------------------------------
   const int T = max(0, p.seq_lens[b]);
-  int s0 = 0, N = 0, k = 0, E = T;
+  int s0 = 0, N = 0, R = 0, E = T;
   if (kExact) {
     s0 = min(p.n_sink, T);
     N = max(0, min(p.n_indexed[b], T - s0));
     N = min(N, p.cap);
-    k = decode_k(p.budget, p.k_override, N);
-    E = s0 + k + (T - s0 - N);
+    R = T - s0 - N;
+    E = s0 + R + decode_k(p.budget, p.k_override, N);
   }
   const int r0 = split * p.chunk;
   const int r1 = min(E, r0 + p.chunk);
   const int ntiles = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
+  // first tile holding a selected row (rows >= s0 + R); ntiles or more if none
+  const int first_sel_tile = kExact ? max(0, s0 + R - r0) / kTile : 0;
   const int32_t* sel_u = kExact ? p.sel + static_cast<size_t>(u) * p.cap : nullptr;
   const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
 
@@ -139,7 +148,7 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], kRows ? 32 : 1);   // rows: one cp.async arrival per producer lane
       mbar_init(&empty[s], 1);
     }
     fence_mbar_init();
@@ -152,23 +161,30 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
     }
-    bool ok = true;
+    bool ok = true, waited = !kExact;
     const int box_rows = kRows ? 1 : min(p.page_size, kTile);
-    // Tiles go in groups of kStages: each lane first resolves its box of every tile of the
-    // group (selected-position and block-table loads of the group in flight together),
-    // then the copies are issued tile by tile as stages are released.
-    for (int t0 = 0; t0 < ntiles && ok; t0 += kStages) {
+    // Tiles go in groups of up to kStages: each lane first resolves its box of every tile of
+    // the group (selected-position and block-table loads of the group in flight together),
+    // then the copies are issued tile by tile as stages are released. A group never mixes
+    // tiles before and after first_sel_tile, so selection-free tiles never wait.
+    for (int t0 = 0, t1; t0 < ntiles && ok; t0 = t1) {
+      t1 = min(ntiles, t0 + kStages);
+      if (t0 < first_sel_tile) t1 = min(t1, first_sel_tile);
+      if (!waited && t0 >= first_sel_tile) {
+        pdl_wait();
+        waited = true;
+      }
       int ys[kStages];
 #pragma unroll
       for (int i = 0; i < kStages; ++i) {
         ys[i] = -1;
         const int t = t0 + i;
-        if (t >= ntiles) continue;
+        if (t >= t1) continue;
         const int row0 = r0 + t * kTile;
         const int nvalid = min(kTile, r1 - row0);
         const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
         if (lane < nbox) {
-          const int pos = kExact ? exact_row_pos(row0 + lane, s0, k, N, sel_u) : row0 + lane * box_rows;
+          const int pos = kExact ? exact_row_pos(row0 + lane, s0, N, R, sel_u) : row0 + lane * box_rows;
           int page = (pos >= 0 && pos < T && pos / p.page_size < p.max_pages) ? bt[pos / p.page_size] : -1;
           if (page < 0 || page >= p.num_pages) {
             record_error(p.err, HSA_DEVERR_PAGE);
@@ -180,7 +196,7 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
 #pragma unroll
       for (int i = 0; i < kStages; ++i) {
         const int t = t0 + i;
-        if (t >= ntiles) break;
+        if (t >= t1) break;
         const int s = t % kStages;
         if (t >= kStages) {
           ok = mbar_wait_warp(&empty[s], ((t / kStages) - 1) & 1, p.err);
@@ -190,15 +206,27 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
         const int nvalid = min(kTile, r1 - row0);
         uint8_t* st = stage_base + static_cast<size_t>(s) * kStageBytes;
         const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox) * 2u * box_rows * 256u);
-        __syncwarp();
-        if (lane < nbox) {
-          const int y = ys[i];
-          if (kRows) {
-            const size_t src = static_cast<size_t>(y) * (kD * 2);
-            bulk_load(st + lane * kRowPitch, p.k_cache + src, 256u, &full[s]);
-            bulk_load(st + v_area<kRows>() + lane * kRowPitch, p.v_cache + src, 256u, &full[s]);
-          } else {
+        if (kRows) {
+          // Gathered rows: 16 lanes copy one 256-byte row in 16-byte pieces (LSU async
+          // copies; a bulk copy per row would be bound by the copy engine's per-copy
+          // cost), two rows per step; each lane then arrives once its copies have landed.
+          const int c16 = lane & 15, half = lane >> 4;
+#pragma unroll 4
+          for (int rr = 0; rr < kTile / 2; ++rr) {
+            const int r = 2 * rr + half;
+            const int y = __shfl_sync(0xffffffffu, ys[i], r);
+            if (r < nvalid) {
+              const size_t src = static_cast<size_t>(y) * (kD * 2) + c16 * 16;
+              cp_async_16(st + r * kRowPitch + c16 * 16, p.k_cache + src);
+              cp_async_16(st + v_area<kRows>() + r * kRowPitch + c16 * 16, p.v_cache + src);
+            }
+          }
+          cp_async_arrive(&full[s]);
+        } else {
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox) * 2u * box_rows * 256u);
+          __syncwarp();
+          if (lane < nbox) {
+            const int y = ys[i];
             const int off = lane * box_rows * 128;
             tma_load_2d(st + 0 * kHalfBytes + off, &tmap_k, &full[s], 0, y);
             tma_load_2d(st + 1 * kHalfBytes + off, &tmap_k, &full[s], 64, y);
@@ -209,6 +237,7 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
       }
     }
     // Drain: make sure every issued copy has landed before the CTA can exit.
+    if (kRows) cp_async_wait<0>();
     if (lane == 0) {
       for (int t = max(0, ntiles - kStages); t < ntiles; ++t) mbar_wait(&full[t % kStages], (t / kStages) & 1, p.err);
     }
@@ -363,6 +392,7 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
     for (int e = 0; e < 4; ++e)
       cacc[(warp * 8 + 2 * tig + (e & 1)) * kD + 16 * i + grp + 8 * (e >> 1)] = oacc[i][e];
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  if (kExact) pdl_wait();
   const size_t slot = static_cast<size_t>(u) * p.S_tot + split;
   for (int d = tid; d < kD; d += kConsumerWarps * 32) {   // the consumer threads cover the output dims
 #pragma unroll
@@ -394,13 +424,13 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
 // relative to the reference ub_g (W was accumulated as e^{shat - ub}).
 template <int G>
 __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
+  constexpr int NW = kThreads / 32;
+  constexpr int kPerWarp = (kBgClusters + NW - 1) / NW;   // clusters per warp: c0 + warp + r * NW
   const int u = j / p.nbg;
   const int cb = j % p.nbg;
   const int b = u / p.Hkv;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  constexpr int NW = kThreads / 32;
-  pdl_wait();
   pdl_launch_dependents();
   const int T = max(0, p.seq_lens[b]);
   const int s0 = min(p.n_sink, T);
@@ -408,6 +438,18 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
   N = min(N, p.cap);
   const int k = decode_k(p.budget, p.k_override, N);
   const bool active = p.bg_enabled && N > k;
+  const int c0 = cb * kBgClusters;
+  const int c1 = active ? min(p.C, c0 + kBgClusters) : c0;
+  // The cluster means predate the step: their loads go out before waiting for the selection.
+  const float* mv = p.mean_v + static_cast<size_t>(u) * p.C * kD;
+  float4 m4[kPerWarp];
+#pragma unroll
+  for (int r = 0; r < kPerWarp; ++r) {
+    const int c = c0 + warp + r * NW;
+    m4[r] = c < c1 ? *reinterpret_cast<const float4*>(mv + static_cast<size_t>(c) * kD + lane * 4)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  pdl_wait();   // W (final after the selection's fix-up), bounds; partial slots free
   const size_t slot = static_cast<size_t>(u) * p.S_tot + p.nsplit + cb;
   if (!active) {
     for (int i = tid; i < G * kD; i += blockDim.x) p.pacc[slot * G * kD + i] = 0.f;
@@ -417,10 +459,26 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
     }
     return;
   }
-  const int c0 = cb * kBgClusters;
-  const int c1 = min(p.C, c0 + kBgClusters);
-  const float* W = p.W + static_cast<size_t>(u) * G * p.C;
-  const float* mv = p.mean_v + static_cast<size_t>(u) * p.C * kD;
+  float* ws = reinterpret_cast<float*>(smem);          // [G][kBgClusters] cluster weights
+  float* red = ws + G * kBgClusters;                   // [NW][G][kD]
+  float* redl = red + NW * G * kD;                     // [NW][G]
+  {
+    const float* W = p.W + static_cast<size_t>(u) * G * p.C;
+    constexpr int kLoads = (G * kBgClusters + kThreads - 1) / kThreads;
+    float wv[kLoads];
+#pragma unroll
+    for (int r = 0; r < kLoads; ++r) {
+      const int i = tid + r * kThreads;
+      const int g = i / kBgClusters, c = c0 + i % kBgClusters;
+      wv[r] = (i < G * kBgClusters && c < c1) ? fmaxf(W[static_cast<size_t>(g) * p.C + c], 0.f) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < kLoads; ++r) {
+      const int i = tid + r * kThreads;
+      if (i < G * kBgClusters) ws[i] = wv[r];
+    }
+  }
+  __syncthreads();
   float acc[G][4], lsum[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -428,34 +486,20 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[g][i] = 0.f;
   }
-  constexpr int kR = 4;   // clusters whose loads are in flight together, per warp
-  for (int cb0 = c0 + warp; cb0 < c1; cb0 += kR * NW) {
-    float4 m4[kR];
-    float wv[kR][G];
 #pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      const int c = cb0 + r * NW;
-      const bool ok = c < c1;
-      m4[r] = ok ? *reinterpret_cast<const float4*>(mv + static_cast<size_t>(c) * kD + lane * 4)
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = 0; r < kPerWarp; ++r) {
+    const int cl = warp + r * NW;   // cluster c0 + cl (weight 0 past c1)
+    if (cl >= kBgClusters) break;
 #pragma unroll
-      for (int g = 0; g < G; ++g) wv[r][g] = ok ? W[g * p.C + c] : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < kR; ++r) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float w = fmaxf(wv[r][g], 0.f);
-        lsum[g] += w;
-        acc[g][0] = fmaf(w, m4[r].x, acc[g][0]);
-        acc[g][1] = fmaf(w, m4[r].y, acc[g][1]);
-        acc[g][2] = fmaf(w, m4[r].z, acc[g][2]);
-        acc[g][3] = fmaf(w, m4[r].w, acc[g][3]);
-      }
+    for (int g = 0; g < G; ++g) {
+      const float w = ws[g * kBgClusters + cl];
+      lsum[g] += w;
+      acc[g][0] = fmaf(w, m4[r].x, acc[g][0]);
+      acc[g][1] = fmaf(w, m4[r].y, acc[g][1]);
+      acc[g][2] = fmaf(w, m4[r].z, acc[g][2]);
+      acc[g][3] = fmaf(w, m4[r].w, acc[g][3]);
     }
   }
-  float* red = reinterpret_cast<float*>(smem);  // [NW][G][kD] + [NW][G]
-  float* redl = red + NW * G * kD;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     *reinterpret_cast<float4*>(&red[(warp * G + g) * kD + lane * 4]) =
@@ -463,8 +507,8 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
     if (lane == 0) redl[warp * G + g] = lsum[g];
   }
   __syncthreads();
-  float ub[G];
-  unit_upper_bounds<G>(p.bounds, u, p.nq, ub);
+  float ub[G], lb[G];
+  final_bounds<G>(p.fbounds, u, ub, lb);
   for (int i = tid; i < G * kD; i += blockDim.x) {
     const int g = i / kD;
     float a = 0.f;
@@ -472,9 +516,11 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
     p.pacc[slot * G * kD + i] = a;
   }
   if (tid < G) {
-    float l = 0.f;
+    float l = 0.f, ubt = 0.f;
     for (int w = 0; w < NW; ++w) l += redl[w * G + tid];
-    p.pm[slot * G + tid] = ub[tid] * kLog2e;
+#pragma unroll
+    for (int g = 0; g < G; ++g) ubt = g == tid ? ub[g] : ubt;   // no run-time index into registers
+    p.pm[slot * G + tid] = ubt * kLog2e;
     p.pl[slot * G + tid] = l;
   }
 }
@@ -482,13 +528,16 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
 namespace {
 
 // out[b, qh] = sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s over the S_tot partials of its unit.
-// 8 warps: factors e^{m_s - M} computed once, warp w sums splits w, w+8, ..., lane = 4 dims.
+// 8 warps; warp w owns splits w, w+8, ... (at most kMergePerWarp); lane = 4 dims. Every
+// partial (m, l and the 128-wide acc row) is loaded in one round trip, before any math.
 constexpr int kMergeThreads = 256;
+constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kMergePerWarp = 16;
+static_assert(kMaxSplits + kMaxBgChunks <= kMergeWarps * kMergePerWarp, "merge covers every partial");
 template <int G>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
-  extern __shared__ float msm[];            // [S_tot] factors, then [8][kD] partial sums
-  __shared__ float sh_red[kMergeThreads / 32];
-  __shared__ float sh_M, sh_L;
+  __shared__ float sh_m[kMergeWarps], sh_l[kMergeWarps];
+  __shared__ float4 red[kMergeWarps][32];
   pdl_wait();
   pdl_launch_dependents();
   const int bq = blockIdx.x;               // b * Hq + qh
@@ -496,71 +545,58 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
   const int h = qh / G, g = qh % G;
   const size_t u = static_cast<size_t>(b) * p.Hkv + h;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = p.S_tot;
-  float* fs = msm;
-  float* red = msm + ((S + 3) & ~3);
-  float* ls = red;                          // l of each split, until the partial sums need the space
-  float mloc = -INFINITY;
-  for (int s = tid; s < S; s += kMergeThreads) {
-    const float m = p.pm[(u * S + s) * G + g];
-    ls[s] = p.pl[(u * S + s) * G + g];
-    fs[s] = m;
-    mloc = fmaxf(mloc, m);
+  const int S = min(p.S_tot, kMergeWarps * kMergePerWarp);
+  float4 v[kMergePerWarp];
+  float mv[kMergePerWarp], lv[kMergePerWarp];
+#pragma unroll
+  for (int r = 0; r < kMergePerWarp; ++r) {
+    const int s = warp + r * kMergeWarps;
+    const bool ok = s < S;
+    const size_t row = (u * S + s) * G + g;
+    mv[r] = ok ? p.pm[row] : -INFINITY;
+    lv[r] = ok ? p.pl[row] : 0.f;
+    v[r] = ok ? *reinterpret_cast<const float4*>(p.pacc + row * kD + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  mloc = warp_max(mloc);
-  if (lane == 0) sh_red[warp] = mloc;
+  float mx = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < kMergePerWarp; ++r) mx = fmaxf(mx, mv[r]);
+  if (lane == 0) sh_m[warp] = mx;
   __syncthreads();
-  if (tid == 0) {
-    float M = sh_red[0];
-    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, sh_red[w]);
-    sh_M = M;
-  }
-  __syncthreads();
-  const float M = sh_M;
-  float lloc = 0.f;
-  for (int s = tid; s < S; s += kMergeThreads) {
-    const float m = fs[s];
-    const float f = (M == -INFINITY || m == -INFINITY) ? 0.f : fast_exp2(m - M);
-    fs[s] = f;
-    lloc += f * ls[s];
-  }
-  lloc = warp_sum(lloc);
-  __syncthreads();
-  if (lane == 0) sh_red[warp] = lloc;
-  __syncthreads();
-  if (tid == 0) {
-    float L = 0.f;
-    for (int w = 0; w < kMergeThreads / 32; ++w) L += sh_red[w];
-    sh_L = L;
-  }
+  float M = sh_m[0];
+#pragma unroll
+  for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, sh_m[w]);
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-  constexpr int kR = 4;
-  for (int s0 = warp; s0 < S; s0 += kR * (kMergeThreads / 32)) {
-    float4 v[kR];
-    float f[kR];
+  float L = 0.f;
 #pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      const int s = s0 + r * (kMergeThreads / 32);
-      f[r] = s < S ? fs[s] : 0.f;
-      v[r] = s < S ? *reinterpret_cast<const float4*>(p.pacc + ((u * S + s) * G + g) * kD + lane * 4)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      a.x = fmaf(f[r], v[r].x, a.x);
-      a.y = fmaf(f[r], v[r].y, a.y);
-      a.z = fmaf(f[r], v[r].z, a.z);
-      a.w = fmaf(f[r], v[r].w, a.w);
-    }
+  for (int r = 0; r < kMergePerWarp; ++r) {
+    const float f = (M == -INFINITY || mv[r] == -INFINITY) ? 0.f : fast_exp2(mv[r] - M);
+    L = fmaf(f, lv[r], L);
+    a.x = fmaf(f, v[r].x, a.x);
+    a.y = fmaf(f, v[r].y, a.y);
+    a.z = fmaf(f, v[r].z, a.z);
+    a.w = fmaf(f, v[r].w, a.w);
   }
-  *reinterpret_cast<float4*>(&red[warp * kD + lane * 4]) = a;
+  red[warp][lane] = a;
+  if (lane == 0) sh_l[warp] = L;
   __syncthreads();
-  if (tid < kD) {
-    float t = 0.f;
+  if (tid < 32) {
+    float4 t = red[0][tid];
+    float Lt = sh_l[0];
 #pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) t += red[w * kD + tid];
-    const float L = sh_L;
-    p.out[static_cast<size_t>(bq) * kD + tid] = (L > 0.f) ? t / L : 0.f;
+    for (int w = 1; w < kMergeWarps; ++w) {
+      const float4 x = red[w][tid];
+      t.x += x.x;
+      t.y += x.y;
+      t.z += x.z;
+      t.w += x.w;
+      Lt += sh_l[w];
+    }
+    float4 o;
+    o.x = Lt > 0.f ? t.x / Lt : 0.f;
+    o.y = Lt > 0.f ? t.y / Lt : 0.f;
+    o.z = Lt > 0.f ? t.z / Lt : 0.f;
+    o.w = Lt > 0.f ? t.w / Lt : 0.f;
+    *reinterpret_cast<float4*>(p.out + static_cast<size_t>(bq) * kD + tid * 4) = o;
   }
 }
 
@@ -589,8 +625,7 @@ cudaError_t launch_merge_t(const MergeParams& p, cudaStream_t stream, bool pdl) 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.B * p.Hq);
   cfg.blockDim = dim3(kMergeThreads);
-  const int s4 = (p.S_tot + 3) & ~3;
-  cfg.dynamicSmemBytes = (s4 + (s4 > (kMergeThreads / 32) * kD ? s4 : (kMergeThreads / 32) * kD)) * sizeof(float);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -15,7 +15,10 @@ constexpr int kDsub = 8;       // dims per subspace
 constexpr int kNcode = 256;    // codewords per subspace
 constexpr int kNB = 2048;      // selection-score histogram bins
 constexpr int kBgClusters = 64;  // clusters per background CTA
+constexpr int kCandWeights = 1024;  // threshold-bin candidates whose head weights the filter precomputes
 constexpr int kMaxSplits = 64;   // exact/dense split-K chunks per unit (upper bound)
+constexpr int kMaxClusters = 4096;                        // IVF clusters per unit (upper bound)
+constexpr int kMaxBgChunks = kMaxClusters / kBgClusters;  // background partials per unit
 constexpr int kTile = 32;        // tokens per attention tile (one per lane)
 constexpr int kLutParts = 4;     // table-builder CTAs per unit for the LUT (4 subspaces each)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -116,6 +119,36 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// Two fp32 additions in one instruction (sm_100 packed f32x2), each rounded to nearest
+// like __fadd_rn; a and b hold (lo, hi) = (first, second) float.
+__device__ __forceinline__ unsigned long long fadd2_rn(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float lo_f(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+
+// LSU asynchronous copies (16 or 4 bytes per thread): for small gathers, where one
+// bulk copy per few hundred bytes would be limited by the copy engine's per-operation
+// cost. Completion is tracked per thread by commit groups, or signalled on an mbarrier.
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed; the
+// arrival counts toward the barrier's expected count (initialise it accordingly).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
@@ -250,8 +283,8 @@ struct DecodeLayout {
   // sizes
   int U, G, GP, C, cap, nq, nsplit_max, nbg, bitmap_words;
   // byte offsets from the workspace base
-  size_t off_units, off_bounds, off_lut, off_qc, off_w, off_hist, off_sigma, off_bitmap, off_cand,
-      off_sel, off_pm, off_pl, off_pacc, total;
+  size_t off_units, off_bounds, off_fbounds, off_lut, off_qc, off_w, off_hist, off_sigma, off_bitmap, off_cand,
+      off_candw, off_candc, off_sel, off_pm, off_pl, off_pacc, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -278,6 +311,7 @@ __host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, 
   const size_t u = static_cast<size_t>(U);
   L.off_units = take(u * sizeof(UnitState));
   L.off_bounds = take(u * (kLutParts + L.nq) * 2 * 4 * L.GP * sizeof(float));
+  L.off_fbounds = take(u * 2 * G * sizeof(float));
   L.off_lut = take(u * L.GP * kNcode * kM * 4 * sizeof(float));
   L.off_qc = take(u * L.GP * C * 4 * sizeof(float));
   L.off_w = take(u * G * C * sizeof(float));
@@ -285,6 +319,8 @@ __host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, 
   L.off_sigma = take(u * list_slots * sizeof(float));   // one score per list slot
   L.off_bitmap = take(u * L.bitmap_words * sizeof(uint32_t));
   L.off_cand = take(u * cap * sizeof(uint64_t));
+  L.off_candw = take(u * kCandWeights * G * sizeof(float));
+  L.off_candc = take(u * kCandWeights * sizeof(int32_t));
   L.off_sel = take(u * cap * sizeof(int32_t));
   const size_t parts = u * (nsplit_max + L.nbg) * G;
   L.off_pm = take(parts * sizeof(float));

@@ -11,40 +11,47 @@ namespace pqhsa {
 
 // Upper/lower bound of the (scaled) approximate logit of every head of unit u:
 //   ub_g = sum_s max_m LUT_s[m][g] + max_c qc[c][g],  lb_g likewise with min.
-// bounds layout: [U][kLutParts + nq][2 (max, min)][4 * GP]; parts 0..kLutParts-1
-// hold partial sums over their subspaces of the per-subspace extremes, parts
-// kLutParts.. the extremes of one 128-cluster slice of the centroid term.
+// The table builder leaves partial extremes in `bounds`, layout
+// [U][kLutParts + nq][2 (max, min)][4 * GP]: parts 0..kLutParts-1 hold partial sums over
+// their subspaces of the per-subspace extremes, parts kLutParts.. the extremes of one
+// 128-cluster slice of the centroid term. The scan reduces them once per unit (one warp)
+// into the final bounds `fbounds` [U][2][G] that every later kernel reads.
+static_assert(kMaxClusters / 128 <= 32, "one lane per centroid slice");
 template <int G>
-__device__ __forceinline__ void unit_bounds(const float* bounds, int u, int nq, float* ub, float* lb) {
+__device__ __forceinline__ void reduce_bounds_warp(const float* bounds, int u, int nq, float* ub, float* lb) {
   constexpr int G4 = ((G + 3) / 4) * 4;
+  const int lane = threadIdx.x & 31;
   const float* bu = bounds + static_cast<size_t>(u) * (kLutParts + nq) * 2 * G4;
-#pragma unroll
+  // one head at a time (few live registers); lane l holds centroid slice l
+#pragma unroll 1
   for (int g = 0; g < G; ++g) {
+    float qmax = lane < nq ? bu[((kLutParts + lane) * 2 + 0) * G4 + g] : -INFINITY;
+    float qmin = lane < nq ? bu[((kLutParts + lane) * 2 + 1) * G4 + g] : INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+      qmin = fminf(qmin, __shfl_xor_sync(0xffffffffu, qmin, o));
+    }
     float smax = 0.f, smin = 0.f;
 #pragma unroll
-    for (int part = 0; part < kLutParts; ++part) {
+    for (int part = 0; part < kLutParts; ++part) {   // fixed order: the same sums in every CTA
       smax += bu[(part * 2 + 0) * G4 + g];
       smin += bu[(part * 2 + 1) * G4 + g];
     }
-    float qmax = -INFINITY, qmin = INFINITY;
-#pragma unroll 4
-    for (int part = kLutParts; part < kLutParts + nq; ++part) {
-      qmax = fmaxf(qmax, bu[(part * 2 + 0) * G4 + g]);
-      qmin = fminf(qmin, bu[(part * 2 + 1) * G4 + g]);
+    if (lane == 0) {
+      ub[g] = smax + qmax;
+      lb[g] = smin + qmin;
     }
-    ub[g] = smax + qmax;
-    lb[g] = smin + qmin;
   }
 }
+// Final bounds of unit u as the scan stored them.
 template <int G>
-__device__ __forceinline__ void unit_upper_bounds(const float* bounds, int u, int nq, float* ub) {
-  float lb[G];
-  unit_bounds<G>(bounds, u, nq, ub, lb);
-}
-template <int G>
-__device__ __forceinline__ void unit_lower_bounds(const float* bounds, int u, int nq, float* lb) {
-  float ub[G];
-  unit_bounds<G>(bounds, u, nq, ub, lb);
+__device__ __forceinline__ void final_bounds(const float* fbounds, int u, float* ub, float* lb) {
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    ub[g] = fbounds[(static_cast<size_t>(u) * 2 + 0) * G + g];
+    lb[g] = fbounds[(static_cast<size_t>(u) * 2 + 1) * G + g];
+  }
 }
 
 struct AttendParams {
@@ -63,6 +70,7 @@ struct AttendParams {
   const float* W;            // [U][G][C]
   const float* mean_v;       // [U][C][D]
   const float* bounds;
+  const float* fbounds;      // [U][2][G] final (ub, lb) from the scan
   int U, B, Hq, Hkv, page_size, max_pages, num_pages, cap, n_sink;
   int nsplit, chunk, S_tot, C, nbg, nq, bg_enabled, k_override;
   double budget;
@@ -116,16 +124,18 @@ struct ScanParams {
   const float* lut;
   const float* qc;
   const float* bounds;
+  float* fbounds;            // [U][2][G] final (ub, lb), written here
   float* W;
   uint32_t* hist;
   float* sigma;              // [U][cap]
   float* approx_logits;      // debug [B][Hq][cap] or null
   int32_t* err;
   int B, Hq, Hkv, cap, C, nq, n_sink;
+  int ring_depth;            // chunk slots per warp (scan_ring_depth)
 };
 cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t stream, bool pdl);
+int scan_ring_depth(int G, int C);   // 0: the tables do not fit in shared memory
 size_t scan_smem_bytes(int G, int C);
-int scan_threads();
 
 struct SelectParams {
   const uint8_t* list_codes;     // [U][list_slots][16]
@@ -140,10 +150,13 @@ struct SelectParams {
   const float* lut;
   const float* qc;
   const float* bounds;
+  const float* fbounds;      // [U][2][G] final (ub, lb) from the scan
   const float* sigma;
   const uint32_t* hist;
   uint32_t* bitmap;
   unsigned long long* cand;  // [U][cap]
+  float* cand_w;             // [U][kCandWeights][G] e^{shat_g - ub_g} of the first candidates
+  int32_t* cand_c;           // [U][kCandWeights] their clusters
   UnitState* units;
   int32_t* sel;              // [U][cap]
   float* W;

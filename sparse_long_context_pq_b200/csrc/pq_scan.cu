@@ -34,20 +34,6 @@ __device__ __forceinline__ int unit_n(const int32_t* seq_lens, const int32_t* n_
   return min(N, cap);
 }
 
-template <int G>
-__device__ __forceinline__ void hist_range(const float* bounds, int u, int nq, float& lo, float& inv) {
-  float ub[G], lb[G];
-  unit_upper_bounds<G>(bounds, u, nq, ub);
-  unit_lower_bounds<G>(bounds, u, nq, lb);
-  float hi = ub[0];
-  lo = lb[0];
-#pragma unroll
-  for (int g = 1; g < G; ++g) {
-    hi = fmaxf(hi, ub[g]);
-    lo = fmaxf(lo, lb[g]);   // sigma = max_g shat_g >= lb_g for every g
-  }
-  inv = (hi > lo) ? __fdiv_rn(static_cast<float>(kNB), __fsub_rn(hi, lo)) : 0.f;
-}
 
 __device__ __forceinline__ float warp_min(float v) {
 #pragma unroll
@@ -268,17 +254,34 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
 // ===========================================================================
 // scan
 // ===========================================================================
-constexpr int kScanThreads = 256;
-constexpr int kScanUnroll = 2;   // tokens per thread per batch; the next batch is loaded while one is scored
+// One CTA per SM: 16 warps share one copy of the tables. Each lane streams the codes
+// (16 B) and index slot (4 B) of its own list slot, for the warp's next D chunks, into a
+// private ring with LSU async copies (one commit group per chunk), so D chunks per warp
+// are in flight while it scores the current one.
+// threads per scan CTA (one CTA per SM; registers bound the warp count)
+template <int G>
+constexpr int scan_threads_of() { return 512; }
+constexpr int kRingCodeBytes = 32 * kM;                     // 512 per chunk
+constexpr int kRingSlotBytes = kRingCodeBytes + 32 * 4;     // + index slots = 640
+constexpr size_t kScanSmemLimit = 226 * 1024;   // dynamic; the rest of 227 KB is static
 
 template <int G>
 struct ScanSmem {
   static constexpr int GP = (G + 3) / 4;
-  // tables (LUT, centroid terms) and the score histogram; then the mbarrier
+  // tables (LUT, centroid terms) and the score histogram; then the warps' rings
+  // ([D][32][16 B] codes, then [D][32] index slots per warp); then the tables mbarrier
   __host__ __device__ static size_t tables(int C) {
-    return align_up(static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 + kNB * 4, 16);
+    return align_up(static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 + kNB * 4, 128);
   }
-  __host__ __device__ static size_t bytes(int C) { return tables(C) + 16; }
+  __host__ __device__ static size_t bytes(int C, int depth) {
+    return tables(C) + static_cast<size_t>(scan_threads_of<G>() / 32) * depth * kRingSlotBytes + 8;
+  }
+  // deepest ring (8, 4 or 2 chunks per warp) that fits; 0 if none does
+  static int depth(int C) {
+    for (int d = 8; d >= 2; d >>= 1)
+      if (bytes(C, d) <= kScanSmemLimit) return d;
+    return 0;
+  }
 };
 
 template <int G>
@@ -291,12 +294,13 @@ __device__ __forceinline__ void score_token(const uint4& code, uint32_t id, cons
     uint32_t t = w0; w0 = w1; w1 = t;
     t = w2; w2 = w3; w3 = t;
   }
-  // two independent partial sums per head (even / odd lookups) halve the dependent add chain
-  float4 acc[2][GP];
+  // Two independent partial sums per head (even / odd lookups) halve the dependent add
+  // chain; each float4 of 4 heads is two packed f32x2 additions.
+  ulonglong2 acc[2][GP];
 #pragma unroll
   for (int gp = 0; gp < GP; ++gp) {
-    acc[0][gp] = qc_s[gp * C + id];
-    acc[1][gp] = make_float4(0.f, 0.f, 0.f, 0.f);
+    acc[0][gp] = reinterpret_cast<const ulonglong2*>(qc_s)[gp * C + id];
+    acc[1][gp] = make_ulonglong2(0ull, 0ull);
   }
 #pragma unroll
   for (int i = 0; i < kM; ++i) {
@@ -305,20 +309,20 @@ __device__ __forceinline__ void score_token(const uint4& code, uint32_t id, cons
     const uint32_t off = __byte_perm(wd, ysoff[i >> 1], sel[i & 3]);
 #pragma unroll
     for (int gp = 0; gp < GP; ++gp) {
-      const float4 v = *reinterpret_cast<const float4*>(lut_b + gp * (kNcode * kM * 16) + off);
-      float4& a = acc[i & 1][gp];
-      a.x = __fadd_rn(a.x, v.x);
-      a.y = __fadd_rn(a.y, v.y);
-      a.z = __fadd_rn(a.z, v.z);
-      a.w = __fadd_rn(a.w, v.w);
+      const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(lut_b + gp * (kNcode * kM * 16) + off);
+      ulonglong2& a = acc[i & 1][gp];
+      a.x = fadd2_rn(a.x, v.x);
+      a.y = fadd2_rn(a.y, v.y);
     }
   }
 #pragma unroll
   for (int gp = 0; gp < GP; ++gp) {
-    if (gp * 4 + 0 < G) sh[gp * 4 + 0] = __fadd_rn(acc[0][gp].x, acc[1][gp].x);
-    if (gp * 4 + 1 < G) sh[gp * 4 + 1] = __fadd_rn(acc[0][gp].y, acc[1][gp].y);
-    if (gp * 4 + 2 < G) sh[gp * 4 + 2] = __fadd_rn(acc[0][gp].z, acc[1][gp].z);
-    if (gp * 4 + 3 < G) sh[gp * 4 + 3] = __fadd_rn(acc[0][gp].w, acc[1][gp].w);
+    const unsigned long long xy = fadd2_rn(acc[0][gp].x, acc[1][gp].x);
+    const unsigned long long zw = fadd2_rn(acc[0][gp].y, acc[1][gp].y);
+    if (gp * 4 + 0 < G) sh[gp * 4 + 0] = lo_f(xy);
+    if (gp * 4 + 1 < G) sh[gp * 4 + 1] = hi_f(xy);
+    if (gp * 4 + 2 < G) sh[gp * 4 + 2] = lo_f(zw);
+    if (gp * 4 + 3 < G) sh[gp * 4 + 3] = hi_f(zw);
   }
 }
 
@@ -352,14 +356,14 @@ __device__ __forceinline__ float warp_sum_scatter(float* v) {
 
 // Chunks [ch0, ch1) of unit u's cluster-ordered list: one warp scores one 32-slot
 // chunk (all members of one cluster), so the centroid term is warp-uniform and the
-// chunk's cluster weights are one warp reduction. `phase` counts segments (mbarrier parity).
-template <int G>
+// chunk's cluster weights are one warp reduction. Warp w takes chunks ch0 + w + 16 i
+// through its D-slot ring; `phase` counts segments (tables mbarrier parity).
+template <int G, int D>
 __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0, int ch1, uint8_t* smem,
-                                             uint64_t* bar, uint32_t phase, const uint32_t ysoff[8],
-                                             const uint32_t sel[4], bool swap_words) {
+                                             uint64_t* bar, uint32_t phase, float* sh_bounds,
+                                             const uint32_t ysoff[8], const uint32_t sel[4], bool swap_words) {
   constexpr int GP = (G + 3) / 4;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nwarps = blockDim.x >> 5;
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int C = p.C;
   const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
@@ -368,6 +372,9 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
   float4* lut_s = reinterpret_cast<float4*>(smem);                               // [GP][256][16]
   float4* qc_s = lut_s + GP * kNcode * kM;                                       // [GP][C]
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(qc_s + GP * C);                 // [NB]
+  uint8_t* wring = smem + ScanSmem<G>::tables(C) + static_cast<size_t>(warp) * D * kRingSlotBytes;
+  uint4* ring_code = reinterpret_cast<uint4*>(wring) + lane;                              // [D][32]
+  int32_t* ring_js = reinterpret_cast<int32_t*>(wring + D * kRingCodeBytes) + lane;       // [D][32]
 
   __syncthreads();  // previous segment finished with shared memory
   if (tid == 0) {
@@ -380,11 +387,47 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
     for (uint32_t o = 0; o < qc_bytes; o += 32768u)
       bulk_load(reinterpret_cast<uint8_t*>(qc_s) + o, qg + o, min(32768u, qc_bytes - o), bar);
   }
+  const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
+  const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
+  const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * (p.list_slots / 32);
+  float* sig_u = p.sigma + static_cast<size_t>(u) * p.list_slots;
+  float* Wu = p.W + static_cast<size_t>(u) * G * C;
+  const uint8_t* lut_b = reinterpret_cast<const uint8_t*>(lut_s);
+
+  // this warp's chunks; the first D go out while the tables land (one commit group per
+  // chunk, empty groups past the end keep the count regular)
+  const int first = ch0 + warp;
+  constexpr int kScanWarps = scan_threads_of<G>() / 32;
+  const int cnt = first < ch1 ? (ch1 - first + kScanWarps - 1) / kScanWarps : 0;
+  uint32_t clreg = 0;   // lane j: cluster of the chunk in ring slot j
+  auto issue = [&](int i) {
+    if (i < cnt) {
+      const int ch = first + kScanWarps * i;
+      const int slot = i % D;
+      cp_async_16(ring_code + slot * 32, lcodes + static_cast<size_t>(ch) * 32 + lane);
+      cp_async_4(ring_js + slot * 32, lslot + static_cast<size_t>(ch) * 32 + lane);
+      if (lane == slot) clreg = ccl[ch];
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int i = 0; i < D; ++i) issue(i);
+
   for (int i = tid; i < kNB; i += blockDim.x) hist_s[i] = 0u;
+  if (warp == 0) {   // final bounds of the unit, once: this CTA's copy and the later kernels'
+    reduce_bounds_warp<G>(p.bounds, u, p.nq, sh_bounds, sh_bounds + G);
+    __syncwarp();
+    if (lane < 2 * G) p.fbounds[static_cast<size_t>(u) * 2 * G + lane] = sh_bounds[lane];
+  }
+  __syncthreads();                       // zeroed histogram and bounds visible
   float ub2[G], lo, inv;
   {
     float ub[G], lb[G];
-    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      ub[g] = sh_bounds[g];
+      lb[g] = sh_bounds[G + g];
+    }
     float hi = ub[0];
     lo = lb[0];
 #pragma unroll
@@ -395,38 +438,16 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
     }
     inv = (hi > lo) ? __fdiv_rn(static_cast<float>(kNB), __fsub_rn(hi, lo)) : 0.f;
   }
-  const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
-  const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
-  const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * (p.list_slots / 32);
-  float* sig_u = p.sigma + static_cast<size_t>(u) * p.list_slots;
-  float* Wu = p.W + static_cast<size_t>(u) * G * C;
-  const uint8_t* lut_b = reinterpret_cast<const uint8_t*>(lut_s);
-
-  // this warp's first chunk is in flight while the tables land
-  int ch = ch0 + warp;
-  uint4 code = make_uint4(0, 0, 0, 0);
-  int32_t js = -1;
-  uint32_t cl = 0;
-  if (ch < ch1) {
-    code = __ldcs(lcodes + ch * 32 + lane);
-    js = __ldcs(lslot + ch * 32 + lane);
-    cl = ccl[ch];
-  }
-  __syncthreads();                       // zeroed histogram visible
   mbar_wait(bar, phase & 1, p.err);      // tables landed
   bool bad_id = false;
 
-  for (; ch < ch1; ch += nwarps) {
-    const int nx = ch + nwarps;
-    uint4 ncode = make_uint4(0, 0, 0, 0);
-    int32_t njs = -1;
-    uint32_t ncl = 0;
-    if (nx < ch1) {
-      ncode = __ldcs(lcodes + nx * 32 + lane);
-      njs = __ldcs(lslot + nx * 32 + lane);
-      ncl = ccl[nx];
-    }
-    uint32_t id = cl;
+  for (int i = 0; i < cnt; ++i) {
+    const int slot = i % D;
+    cp_async_wait<D - 1>();              // this lane's copies of chunk i have landed
+    const uint4 code = ring_code[slot * 32];
+    const int32_t js = ring_js[slot * 32];
+    uint32_t id = __shfl_sync(0xffffffffu, clreg, slot);
+    const int ch = first + kScanWarps * i;
     if (id >= static_cast<uint32_t>(C)) {
       bad_id = true;
       id = 0;
@@ -437,7 +458,7 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
     float sg = sh[0];
 #pragma unroll
     for (int g = 1; g < G; ++g) sg = fmaxf(sg, sh[g]);
-    __stcs(sig_u + ch * 32 + lane, valid ? sg : -INFINITY);
+    __stcs(sig_u + static_cast<size_t>(ch) * 32 + lane, valid ? sg : -INFINITY);
     if (p.approx_logits && valid) {
 #pragma unroll
       for (int g = 0; g < G; ++g) p.approx_logits[(static_cast<size_t>(b) * p.Hq + h * G + g) * p.cap + js] = sh[g];
@@ -451,10 +472,9 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
       if ((lane & (kGroup - 1)) == 0) atomicAdd(Wu + (lane / kGroup) * C + id, e);
     }
     if (valid) atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
-    code = ncode;
-    js = njs;
-    cl = ncl;
+    issue(i + D);                        // refill this slot with the chunk D ahead
   }
+  cp_async_wait<0>();
   if (bad_id) record_error(p.err, HSA_DEVERR_CLUSTER);
   __syncthreads();
   uint32_t* hg = p.hist + static_cast<size_t>(u) * kNB;
@@ -488,14 +508,53 @@ __device__ __forceinline__ void for_each_range(int B, int Hkv, Count&& count, F&
   }
 }
 
+// Work split for kernels whose items are grouped by unit. With at least as many CTAs as
+// units that have work, every CTA takes one part of exactly one unit (1 + a share of the
+// spare CTAs in proportion to the unit's items), so no CTA pays a second unit's set-up;
+// a few CTAs may be left idle. Otherwise the balanced range walk. Calls f(u, i0, i1).
+template <typename Count, typename F>
+__device__ __forceinline__ void for_each_unit_part(int B, int Hkv, Count&& count, F&& f) {
+  long long total = 0;
+  int active = 0;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hkv; ++h) {
+      const int n = count(b, h);
+      total += n;
+      active += n > 0;
+    }
+  const int grid = static_cast<int>(gridDim.x);
+  if (active == 0) return;
+  if (active > grid) {
+    for_each_range(B, Hkv, count, f);
+    return;
+  }
+  const long long spare = grid - active;
+  int base = 0;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hkv; ++h) {
+      const int n = count(b, h);
+      if (n <= 0) continue;
+      const int parts = 1 + static_cast<int>(spare * n / total);
+      const int k = static_cast<int>(blockIdx.x) - base;
+      if (k >= 0 && k < parts) {
+        const int i0 = static_cast<int>(static_cast<long long>(n) * k / parts);
+        const int i1 = static_cast<int>(static_cast<long long>(n) * (k + 1) / parts);
+        if (i1 > i0) f(b * Hkv + h, i0, i1);
+        return;
+      }
+      base += parts;
+    }
+}
+
 __device__ __forceinline__ int unit_chunks(const int32_t* list_meta, int u, int C, int max_chunks) {
   const int n = list_meta[static_cast<size_t>(u) * (2 + 2 * static_cast<size_t>(C))];
   return max(0, min(n, max_chunks));
 }
 
-template <int G>
-__global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
+template <int G, int D>
+__global__ void __launch_bounds__(scan_threads_of<G>(), 1) scan_kernel(ScanParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float sh_bounds[2 * G];
   const int lane = threadIdx.x & 31;
   const uint32_t l7 = lane & 7;
   // Per-lane subspace skew: lookup i reads subspace s = i ^ (lane & 7), so the 8
@@ -512,7 +571,8 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
     sel[i] = (4u + 2u * (i & 1)) | (bi << 4) | (5u << 8) | (5u << 12);
   }
   const bool swap_words = (l7 >> 2) & 1;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ScanSmem<G>::tables(p.C));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ScanSmem<G>::tables(p.C) +
+                                              static_cast<size_t>(scan_threads_of<G>() / 32) * D * kRingSlotBytes);
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
@@ -521,10 +581,10 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
   pdl_launch_dependents();
   uint32_t phase = 0;
   const int max_chunks = p.list_slots / 32;
-  for_each_range(
+  for_each_unit_part(
       p.B, p.Hkv, [&](int b, int h) { return unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
       [&](int u, int c0, int c1) {
-        scan_segment<G>(p, u, c0, c1, smem, bar, phase, ysoff, sel, swap_words);
+        scan_segment<G, D>(p, u, c0, c1, smem, bar, phase, sh_bounds, ysoff, sel, swap_words);
         ++phase;
       });
 }
@@ -532,13 +592,12 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanParams p) {
 // ===========================================================================
 // filter: tokens above the threshold bin are selected, the bin's tokens are candidates
 // ===========================================================================
-// Remove the weight e^{shat_g - ub_g} of a selected token (cluster id, code words cw)
-// from its cluster's sums.
+// Head weights e^{shat_g - ub_g} of one indexed token (cluster id, code words cw), from
+// the decode tables: the same quantities the scan added into its cluster's sums.
 template <int G>
-__device__ __forceinline__ void unselect_weight(const SelectParams& p, int u, uint32_t id, const uint4 cw,
-                                                const float* ub2) {
+__device__ __forceinline__ void token_weights(const SelectParams& p, int u, uint32_t id, const uint4 cw,
+                                              const float* ub2, float* e) {
   constexpr int GP = (G + 3) / 4;
-  if (id >= static_cast<uint32_t>(p.C)) id = 0;
   const uint32_t cwords[4] = {cw.x, cw.y, cw.z, cw.w};
   const float4* lut4 = reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
   const float4* qc4 = reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C;
@@ -557,19 +616,30 @@ __device__ __forceinline__ void unselect_weight(const SelectParams& p, int u, ui
       acc[gp].w = __fadd_rn(acc[gp].w, v.w);
     }
   }
-  float* Wu = p.W + static_cast<size_t>(u) * G * p.C;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const float4 a = acc[g / 4];
     const float sh = (g % 4 == 0) ? a.x : (g % 4 == 1) ? a.y : (g % 4 == 2) ? a.z : a.w;
-    atomicAdd(&Wu[g * p.C + id], -fast_exp2(fmaf(sh, kLog2e, -ub2[g])));
+    e[g] = fast_exp2(fmaf(sh, kLog2e, -ub2[g]));
   }
 }
 
+// Take a selected token's head weights out of its cluster's sums.
 template <int G>
-__global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
+__device__ __forceinline__ void remove_weights(const SelectParams& p, int u, uint32_t id, const float* e) {
+  float* Wu = p.W + static_cast<size_t>(u) * G * p.C;
+#pragma unroll
+  for (int g = 0; g < G; ++g) atomicAdd(&Wu[g * p.C + id], -e[g]);
+}
+
+template <int G>
+__global__ void __launch_bounds__(256, 2) filter_kernel(SelectParams p) {
   constexpr int kBatch = 8;
+  constexpr int kFixCap = kBatch * 256;   // definite selections of one batch, at most one per slot
   __shared__ __align__(16) uint32_t hist_s[kNB];
+  __shared__ uint32_t fix_list[kFixCap];   // list slots
+  __shared__ int32_t fix_cand[kFixCap];     // candidate slot, or -1 for a definite selection
+  __shared__ uint32_t fix_n;
   __shared__ uint32_t scan_tot[33];
   __shared__ int sh_bstar;
   __shared__ uint32_t sh_above;
@@ -577,7 +647,7 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
   pdl_wait();
   pdl_launch_dependents();
   const int max_chunks = p.list_slots / 32;
-  for_each_range(
+  for_each_unit_part(
       p.B, p.Hkv, [&](int b, int h) { return 32 * unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
       [&](int u, int j0, int j1) {
     const int b = u / p.Hkv;
@@ -585,6 +655,9 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
     const int k = decode_k(p.budget, p.k_override, N);
     const float* sig = p.sigma + static_cast<size_t>(u) * p.list_slots;
     const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
+    // bounds (histogram range, weight reference) load with everything else below
+    float ub[G], lb[G];
+    final_bounds<G>(p.fbounds, u, ub, lb);
     // first batch of scores in flight while the threshold is found
     float sv[kBatch];
     int32_t jv[kBatch];
@@ -606,6 +679,7 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
     if (threadIdx.x == 0) {
       sh_bstar = kNB;   // k == 0: nothing selected
       sh_above = 0;
+      fix_n = 0;
     }
     __syncthreads();
     {
@@ -639,8 +713,6 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
       p.units[u].above = static_cast<int32_t>(sh_above);
     }
     if (bstar >= kNB) return;
-    float ub[G], lb[G];
-    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
     float hi = ub[0], lo = lb[0];
 #pragma unroll
     for (int g = 1; g < G; ++g) {
@@ -665,23 +737,63 @@ __global__ void __launch_bounds__(256) filter_kernel(SelectParams p) {
         nv[r] = j < j1 ? sig[j] : 0.f;
         njv[r] = j < j1 ? lslot[j] : -1;
       }
+      const uint32_t lane = threadIdx.x & 31;
 #pragma unroll
       for (int r = 0; r < kBatch; ++r) {
         const int j = jv[r];            // index slot of this list slot
-        if (j < 0 || j >= N) continue;
-        const int bin = score_bin(sv[r], lo, inv);
-        if (bin > bstar) {
-          atomicOr(bm + (j >> 5), 1u << (j & 31));
-          if (fix) {   // selected for sure: take its weight out of its cluster's sums now
-            const int ls = base + r * blockDim.x + threadIdx.x;
-            unselect_weight<G>(p, u, ccl[ls >> 5], lcodes[ls], ub2);
-          }
-        } else if (bin == bstar) {
-          const int slot = atomicAdd(&p.units[u].ncand, 1);
+        const bool valid = j >= 0 && j < N;
+        const int bin = valid ? score_bin(sv[r], lo, inv) : -1;
+        const bool definite = bin > bstar;
+        if (definite) atomicOr(bm + (j >> 5), 1u << (j & 31));
+        int slot = -1;
+        if (bin == bstar) {
+          slot = atomicAdd(&p.units[u].ncand, 1);
           if (slot < p.cap)
             p.cand[static_cast<size_t>(u) * p.cap + slot] =
                 (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
         }
+        if (fix) {
+          // queue the list slot: a definite selection's weight leaves its cluster's sums
+          // below; a candidate's weights are stored for the finalize's winners
+          const bool queued = definite || (slot >= 0 && slot < kCandWeights);
+          const uint32_t m = __ballot_sync(0xffffffffu, queued);
+          if (m) {
+            const uint32_t leader = __ffs(m) - 1;
+            uint32_t at = 0;
+            if (lane == leader) at = atomicAdd(&fix_n, static_cast<uint32_t>(__popc(m)));
+            at = __shfl_sync(0xffffffffu, at, leader);
+            if (queued) {
+              at += __popc(m & ((1u << lane) - 1u));
+              fix_list[at] = base + r * blockDim.x + threadIdx.x;
+              fix_cand[at] = definite ? -1 : slot;
+            }
+          }
+        }
+      }
+      if (fix) {
+        // Queued tokens of this batch: one per thread, every look-up of a token in flight
+        // together.
+        __syncthreads();
+        const uint32_t n = fix_n;
+        for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
+          const uint32_t ls = fix_list[i];
+          const int cs = fix_cand[i];
+          uint32_t id = ccl[ls >> 5];
+          if (id >= static_cast<uint32_t>(p.C)) id = 0;
+          float e[G];
+          token_weights<G>(p, u, id, lcodes[ls], ub2, e);
+          if (cs < 0) {
+            remove_weights<G>(p, u, id, e);
+          } else {
+            float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + cs) * G;
+#pragma unroll
+            for (int g = 0; g < G; ++g) cw[g] = e[g];
+            p.cand_c[static_cast<size_t>(u) * kCandWeights + cs] = static_cast<int32_t>(id);
+          }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) fix_n = 0;
+        __syncthreads();
       }
 #pragma unroll
       for (int r = 0; r < kBatch; ++r) {
@@ -731,10 +843,52 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     const int wi = kFinWordsPerThread * tid + e;
     words[e] = wi < p.bitmap_words ? bm[wi] : 0u;
   }
+  // bounds, and this thread's candidate weights (slot tid) as stored by the filter
+  float ub2[G];
+  {
+    float ub[G], lb[G];
+    final_bounds<G>(p.fbounds, u, ub, lb);
+#pragma unroll
+    for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
+  }
+  static_assert(kCandWeights <= kFinThreads, "one stored candidate per thread");
+  float cwr[G];
+  int32_t ccr = 0;
+  if (p.background) {
+    const float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + tid) * G;
+#pragma unroll
+    for (int g = 0; g < G; ++g) cwr[g] = tid < kCandWeights ? cw[g] : 0.f;
+    ccr = tid < kCandWeights ? p.cand_c[static_cast<size_t>(u) * kCandWeights + tid] : 0;
+  }
   const int T = max(0, T_raw);
   const int s0 = min(p.n_sink, T);
   const int N = min(max(0, min(n_raw, T - s0)), p.cap);
   const int k = decode_k(p.budget, p.k_override, N);
+  const bool fix = p.background && N > k;
+  // A winner's weights leave its cluster's sums: from registers (slot tid), from the
+  // filter's store (slot < kCandWeights), else recomputed from the tables.
+  auto fix_winner = [&](int i, uint32_t j) {
+    if (!fix) return;
+    float e[G];
+    uint32_t id;
+    if (i == tid && i < kCandWeights) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) e[g] = cwr[g];
+      id = static_cast<uint32_t>(ccr);
+    } else if (i < kCandWeights) {
+      const float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + i) * G;
+#pragma unroll
+      for (int g = 0; g < G; ++g) e[g] = cw[g];
+      id = static_cast<uint32_t>(p.cand_c[static_cast<size_t>(u) * kCandWeights + i]);
+    } else {
+      id = p.ids[static_cast<size_t>(u) * p.cap + j];
+      const uint4 cwd = *reinterpret_cast<const uint4*>(p.codes + (static_cast<size_t>(u) * p.cap + j) * kM);
+      if (id >= static_cast<uint32_t>(p.C)) id = 0;
+      token_weights<G>(p, u, id, cwd, ub2, e);
+    }
+    if (id >= static_cast<uint32_t>(p.C)) id = 0;
+    remove_weights<G>(p, u, id, e);
+  };
   int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
   if (k == 0) {
     if (tid == 0 && p.dbg_nselected) p.dbg_nselected[u] = 0;
@@ -758,7 +912,11 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
         const unsigned long long key = keys[tid];
         int rank = 0;
         for (int j = 0; j < m; ++j) rank += keys[j] > key;
-        if (rank < r) wins[atomicAdd(&sh_nwin, 1u)] = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
+        if (rank < r) {
+          const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
+          wins[atomicAdd(&sh_nwin, 1u)] = j;
+          fix_winner(tid, j);
+        }
       }
     } else {
       unsigned long long prefix = 0, mask = 0;
@@ -791,6 +949,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
           const uint32_t w = atomicAdd(&sh_nwin, 1u);
           if (w < kFinSmemCand) wins[w] = j;
           else atomicOr(p.bitmap + static_cast<size_t>(u) * p.bitmap_words + (j >> 5), 1u << (j & 31));
+          fix_winner(i, j);
         }
       }
     }
@@ -799,14 +958,6 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
   const uint32_t nwin = min(sh_nwin, static_cast<uint32_t>(kFinSmemCand));
   if (nwin < sh_nwin) __threadfence_block();   // overflowed winners went to the global bitmap
 
-  float ub2[G];
-  {
-    float ub[G], lb[G];
-    unit_bounds<G>(p.bounds, u, p.nq, ub, lb);
-#pragma unroll
-    for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
-  }
-  const bool fix = p.background && N > k;
 
   // ---- compaction of the selection bitmap into ascending positions ----
   const int nw = (N + 31) / 32;
@@ -861,16 +1012,6 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     if (running != static_cast<uint32_t>(k)) record_error(p.err, HSA_DEVERR_SELECT);
     if (p.dbg_nselected) p.dbg_nselected[u] = static_cast<int32_t>(running);
   }
-  if (fix) {
-    // the filter already removed the tokens above the threshold bin; here only the
-    // winners taken from the threshold bin, one per thread
-    for (uint32_t i = tid; i < nwin; i += blockDim.x) {
-      const int j = static_cast<int>(wins[i]);
-      const uint32_t id = p.ids[static_cast<size_t>(u) * p.cap + j];
-      const uint4 cw = *reinterpret_cast<const uint4*>(p.codes + (static_cast<size_t>(u) * p.cap + j) * kM);
-      unselect_weight<G>(p, u, id, cw, ub2);
-    }
-  }
 }
 
 template <typename Kern, typename P>
@@ -890,14 +1031,23 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
 
 }  // namespace
 
-int scan_threads() { return kScanThreads; }
+
+int scan_ring_depth(int G, int C) {
+  switch (G) {
+    case 1: return ScanSmem<1>::depth(C);
+    case 2: return ScanSmem<2>::depth(C);
+    case 4: return ScanSmem<4>::depth(C);
+    default: return ScanSmem<8>::depth(C);
+  }
+}
 
 size_t scan_smem_bytes(int G, int C) {
+  const int d = scan_ring_depth(G, C);
   switch (G) {
-    case 1: return ScanSmem<1>::bytes(C);
-    case 2: return ScanSmem<2>::bytes(C);
-    case 4: return ScanSmem<4>::bytes(C);
-    default: return ScanSmem<8>::bytes(C);
+    case 1: return ScanSmem<1>::bytes(C, d);
+    case 2: return ScanSmem<2>::bytes(C, d);
+    case 4: return ScanSmem<4>::bytes(C, d);
+    default: return ScanSmem<8>::bytes(C, d);
   }
 }
 
@@ -917,16 +1067,32 @@ cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, boo
 #undef CALL
 }
 
-cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t stream, bool pdl) {
-  const size_t smem = scan_smem_bytes(G, p.C);
-#define CALL(GG)                                                                                         \
-  {                                                                                                      \
-    cudaError_t e = ensure_dyn_smem<scan_kernel<GG>>(smem);                                             \
-    if (e != cudaSuccess) return e;                                                                      \
-    return launch_ex(scan_kernel<GG>, dim3(grid), dim3(kScanThreads), smem, stream, pdl, p);            \
+template <int G, int D>
+cudaError_t launch_scan_t(const ScanParams& p, int grid, cudaStream_t stream, bool pdl) {
+  const size_t smem = ScanSmem<G>::bytes(p.C, D);
+  cudaError_t e = ensure_dyn_smem<scan_kernel<G, D>>(smem);
+  if (e != cudaSuccess) return e;
+  return launch_ex(scan_kernel<G, D>, dim3(grid), dim3(scan_threads_of<G>()), smem, stream, pdl, p);
+}
+
+template <int G>
+cudaError_t launch_scan_g(const ScanParams& p, int grid, cudaStream_t stream, bool pdl) {
+  switch (p.ring_depth) {
+    case 8: return launch_scan_t<G, 8>(p, grid, stream, pdl);
+    case 4: return launch_scan_t<G, 4>(p, grid, stream, pdl);
+    case 2: return launch_scan_t<G, 2>(p, grid, stream, pdl);
+    default: return cudaErrorInvalidValue;
   }
-  PQHSA_G_SWITCH(G, CALL)
-#undef CALL
+}
+
+cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t stream, bool pdl) {
+  switch (G) {
+    case 1: return launch_scan_g<1>(p, grid, stream, pdl);
+    case 2: return launch_scan_g<2>(p, grid, stream, pdl);
+    case 4: return launch_scan_g<4>(p, grid, stream, pdl);
+    case 8: return launch_scan_g<8>(p, grid, stream, pdl);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_filter(int G, const SelectParams& p, int grid, cudaStream_t stream, bool pdl) {
