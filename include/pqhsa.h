@@ -87,7 +87,7 @@ typedef struct {
   uint8_t* list_codes;             /* u8  [B][Hkv][list_slots][M], 16-B aligned */
   int32_t* list_slot;              /* [B][Hkv][list_slots]  index slot of the member, -1 = empty;
                                       16-B aligned (both are streamed by bulk copies) */
-  uint16_t* chunk_cluster;         /* [B][Hkv][list_slots / 32] cluster of each chunk */
+  uint16_t* chunk_cluster;         /* [B][Hkv][list_slots / 32] cluster of each chunk; 4-B aligned */
   int32_t* list_meta;              /* [B][Hkv][2 + 2*C]: chunks in use, unused, then per cluster
                                       (its open chunk or -1, members in that chunk) */
   int32_t C, M, dsub, ncode, cap, n_sink;

@@ -126,7 +126,7 @@ hsa_status check_index(const hsa_kv_cache* kv, const hsa_index* ix, bool need_co
   if (ix->C > kMaxClusters) return HSA_ERR_UNSUPPORTED;
   if (ix->list_slots < list_slots_needed(ix->cap, ix->C) || ix->list_slots % 32) return HSA_ERR_CAPACITY;
   if (!aligned(ix->list_codes, 16) || !aligned(ix->list_slot, 16) || !aligned(ix->list_meta, 4) ||
-      !aligned(ix->chunk_cluster, 2))
+      !aligned(ix->chunk_cluster, 4))
     return HSA_ERR_ALIGNMENT;
   for (int b = 0; b < kv->B; ++b) {
     const int T = kv->seq_lens_host[b];
@@ -334,6 +334,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   float* W = reinterpret_cast<float*>(base + L.off_w);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.off_hist);
   float* sigma = reinterpret_cast<float*>(base + L.off_sigma);
+  float* cmax = reinterpret_cast<float*>(base + L.off_cmax);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(base + L.off_bitmap);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(base + L.off_cand);
   float* cand_w = reinterpret_cast<float*>(base + L.off_candw);
@@ -389,6 +390,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   sc.C = ix->C;
   sc.nq = L.nq;
   sc.fbounds = fbounds;
+  sc.chunk_max = cmax;
   sc.n_sink = ix->n_sink;
   sc.ring_depth = ring_depth;
   RET_CUDA(mark(1));
@@ -415,6 +417,10 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   se.cand_c = cand_c;
   se.units = units;
   se.sel = sel;
+  se.block_table = kv->block_table;
+  se.page_size = kv->page_size;
+  se.max_pages = kv->max_pages;
+  se.num_pages = kv->num_pages;
   se.W = W;
   se.dbg_selected = dbg ? dbg->selected : nullptr;
   se.dbg_nselected = dbg ? dbg->n_selected : nullptr;
@@ -425,6 +431,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   se.C = ix->C;
   se.nq = L.nq;
   se.fbounds = fbounds;
+  se.chunk_max = cmax;
   se.n_sink = ix->n_sink;
   se.bitmap_words = L.bitmap_words;
   se.k_override = prm->k_override;
@@ -466,6 +473,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   p.nbg = L.nbg;
   p.nq = L.nq;
   p.fbounds = fbounds;
+  p.units = units;
   p.bg_enabled = prm->background ? 1 : 0;
   p.k_override = prm->k_override;
   p.budget = prm->budget;

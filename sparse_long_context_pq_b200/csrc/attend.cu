@@ -70,15 +70,11 @@ template <bool kRows>
 __device__ __forceinline__ uint32_t v_area() { return kRows ? kTile * kRowPitch : 2 * kHalfBytes; }
 
 
-// Position of row v of a unit's exact list: the sink [0, s0), then the R tail rows
-// [s0+N, T), then the k selected positions (ascending). Sink and tail rows come first
-// because they do not depend on the selection: their copies and math can run while
-// the selection kernels are still finishing.
-__device__ __forceinline__ int exact_row_pos(int v, int s0, int N, int R, const int32_t* sel_u) {
-  if (v < s0) return v;
-  if (v < s0 + R) return s0 + N + (v - s0);
-  return sel_u[v - s0 - R];
-}
+// Row v of a unit's exact list: the sink [0, s0), then the R tail rows [s0+N, T), then
+// the k selected tokens (ascending position). Sink and tail rows come first because they
+// do not depend on the selection: their copies and math run while the selection kernels
+// are still finishing. The selection stores selected tokens as KV-pool rows.
+__device__ __forceinline__ int exact_tail_pos(int v, int s0, int N) { return v < s0 ? v : s0 + N + (v - s0); }
 
 template <int G, bool kExact, bool kRows>
 __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
@@ -113,10 +109,11 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
   const int h = u % p.Hkv;
 
   // Dense decode waits for the previous kernel at once (its partials may still be read by
-  // the previous merge). The exact part reads only data that predate the step until it
-  // needs the selection: sink and tail rows are copied and attended while the selection
-  // kernels finish; the producer waits before the first selected position, every thread
-  // before writing its partials.
+  // the previous merge). The exact part starts while the selection's last kernel runs
+  // (every kernel before it has completed, the previous step's merge included: each waited
+  // for its predecessor before letting the next one start). Sink and tail rows need
+  // nothing from the selection; the producer waits for its unit's ready flag before the
+  // first selected row.
   if (!kExact) pdl_wait();
   pdl_launch_dependents();
 
@@ -138,13 +135,22 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
   const int32_t* sel_u = kExact ? p.sel + static_cast<size_t>(u) * p.cap : nullptr;
   const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
 
-  // ---- stage q (pre-scaled by scale*log2 e) -------------------------------
-  for (int i = tid; i < kD * GP * 4; i += blockDim.x) {
-    const int d = i / (GP * 4);
-    const int g = i % (GP * 4);
-    float v = 0.f;
-    if (g < G) v = p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.qscale;
-    reinterpret_cast<float*>(qs)[i] = v;
+  // ---- stage q (pre-scaled by scale*log2 e): every load in flight before the stores ----
+  {
+    constexpr int kQ = kD * GP * 4;
+    constexpr int kPer = (kQ + Pipe<kRows>::threads - 1) / Pipe<kRows>::threads;
+    float v[kPer];
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int i = tid + r * Pipe<kRows>::threads;
+      const int d = i / (GP * 4), g = i % (GP * 4);
+      v[r] = (i < kQ && g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.qscale : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int i = tid + r * Pipe<kRows>::threads;
+      if (i < kQ) reinterpret_cast<float*>(qs)[i] = v[r];
+    }
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -171,8 +177,10 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
       t1 = min(ntiles, t0 + kStages);
       if (t0 < first_sel_tile) t1 = min(t1, first_sel_tile);
       if (!waited && t0 >= first_sel_tile) {
-        pdl_wait();
+        ok = __shfl_sync(0xffffffffu, lane == 0 ? (wait_flag(&p.units[u].ready, p.err) ? 1 : 0) : 0, 0) != 0;
+        __syncwarp();   // the other lanes' reads of the selection follow lane 0's acquire
         waited = true;
+        if (!ok) break;
       }
       int ys[kStages];
 #pragma unroll
@@ -184,13 +192,18 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
         const int nvalid = min(kTile, r1 - row0);
         const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
         if (lane < nbox) {
-          const int pos = kExact ? exact_row_pos(row0 + lane, s0, N, R, sel_u) : row0 + lane * box_rows;
-          int page = (pos >= 0 && pos < T && pos / p.page_size < p.max_pages) ? bt[pos / p.page_size] : -1;
-          if (page < 0 || page >= p.num_pages) {
-            record_error(p.err, HSA_DEVERR_PAGE);
-            page = 0;
+          const int v = row0 + lane;
+          if (kExact && v >= s0 + R) {
+            ys[i] = sel_u[v - s0 - R];   // already a KV-pool row (checked by the selection)
+          } else {
+            const int pos = kExact ? exact_tail_pos(v, s0, N) : row0 + lane * box_rows;
+            int page = (pos >= 0 && pos < T && pos / p.page_size < p.max_pages) ? bt[pos / p.page_size] : -1;
+            if (page < 0 || page >= p.num_pages) {
+              record_error(p.err, HSA_DEVERR_PAGE);
+              page = 0;
+            }
+            ys[i] = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
           }
-          ys[i] = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
         }
       }
 #pragma unroll
@@ -392,7 +405,6 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
     for (int e = 0; e < 4; ++e)
       cacc[(warp * 8 + 2 * tig + (e & 1)) * kD + 16 * i + grp + 8 * (e >> 1)] = oacc[i][e];
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-  if (kExact) pdl_wait();
   const size_t slot = static_cast<size_t>(u) * p.S_tot + split;
   for (int d = tid; d < kD; d += kConsumerWarps * 32) {   // the consumer threads cover the output dims
 #pragma unroll
@@ -449,7 +461,6 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
     m4[r] = c < c1 ? *reinterpret_cast<const float4*>(mv + static_cast<size_t>(c) * kD + lane * 4)
                    : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  pdl_wait();   // W (final after the selection's fix-up), bounds; partial slots free
   const size_t slot = static_cast<size_t>(u) * p.S_tot + p.nsplit + cb;
   if (!active) {
     for (int i = tid; i < G * kD; i += blockDim.x) p.pacc[slot * G * kD + i] = 0.f;
@@ -459,6 +470,8 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem) {
     }
     return;
   }
+  if (tid == 0) wait_flag(&p.units[u].ready, p.err);   // W is final once the unit's selection is published
+  __syncthreads();
   float* ws = reinterpret_cast<float*>(smem);          // [G][kBgClusters] cluster weights
   float* red = ws + G * kBgClusters;                   // [NW][G][kD]
   float* redl = red + NW * G * kD;                     // [NW][G]

@@ -20,7 +20,8 @@ constexpr int kMaxSplits = 64;   // exact/dense split-K chunks per unit (upper b
 constexpr int kMaxClusters = 4096;                        // IVF clusters per unit (upper bound)
 constexpr int kMaxBgChunks = kMaxClusters / kBgClusters;  // background partials per unit
 constexpr int kTile = 32;        // tokens per attention tile (one per lane)
-constexpr int kLutParts = 4;     // table-builder CTAs per unit for the LUT (4 subspaces each)
+constexpr int kLutParts = 8;     // table-builder CTAs per unit for the LUT (2 subspaces each)
+constexpr int kQcSlice = 64;     // clusters per table-builder CTA for the centroid terms
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Workspace error word lives at offset 0 of every workspace.
@@ -276,14 +277,44 @@ struct UnitState {          // per unit bookkeeping written by the top-k kernels
   int32_t above;            // tokens in bins above bstar
   int32_t ncand;            // tokens in bin bstar (candidates)
   int32_t nsel;             // selected count written by finalize
-  int32_t pad[4];
+  int32_t ready;            // set (release) once the unit's selection and weight fix-up are final
+  int32_t pad[3];
 };
+
+// Publish a per-unit flag after this CTA's writes: call from every thread of the CTA.
+__device__ __forceinline__ void publish_flag(int32_t* flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+  }
+}
+
+// Bounded wait (acquire) for a flag another running grid publishes; a timeout is
+// recorded and returns false. Callers only wait on CTAs that are already resident.
+// Call it from one thread and share the outcome through a barrier (the flag's line is
+// also written by the publisher: many pollers would slow it down).
+__device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t* err) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  if (v) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    __nanosleep(256);
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v) return true;
+    if (global_ns() - t0 > kWaitLimitNs) break;
+  }
+  record_error(err, HSA_DEVERR_TIMEOUT);
+  return false;
+}
 
 struct DecodeLayout {
   // sizes
   int U, G, GP, C, cap, nq, nsplit_max, nbg, bitmap_words;
   // byte offsets from the workspace base
-  size_t off_units, off_bounds, off_fbounds, off_lut, off_qc, off_w, off_hist, off_sigma, off_bitmap, off_cand,
+  size_t off_units, off_bounds, off_fbounds, off_lut, off_qc, off_w, off_hist, off_sigma, off_cmax, off_bitmap,
+      off_cand,
       off_candw, off_candc, off_sel, off_pm, off_pl, off_pacc, total;
 };
 
@@ -297,7 +328,7 @@ __host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, 
   L.GP = (G + 3) / 4;
   L.C = C;
   L.cap = cap;
-  L.nq = (C + 127) / 128;  // qc slices per unit in the table builder
+  L.nq = (C + kQcSlice - 1) / kQcSlice;  // qc slices per unit in the table builder
   L.nsplit_max = nsplit_max;
   L.nbg = (C + kBgClusters - 1) / kBgClusters;
   L.bitmap_words = static_cast<int>(align_up(static_cast<size_t>((cap + 31) / 32), 8));
@@ -317,6 +348,7 @@ __host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, 
   L.off_w = take(u * G * C * sizeof(float));
   L.off_hist = take(u * kNB * sizeof(uint32_t));
   L.off_sigma = take(u * list_slots * sizeof(float));   // one score per list slot
+  L.off_cmax = take(u * (list_slots / 32) * sizeof(float));   // largest score per chunk
   L.off_bitmap = take(u * L.bitmap_words * sizeof(uint32_t));
   L.off_cand = take(u * cap * sizeof(uint64_t));
   L.off_candw = take(u * kCandWeights * G * sizeof(float));

@@ -14,19 +14,21 @@ namespace pqhsa {
 // The table builder leaves partial extremes in `bounds`, layout
 // [U][kLutParts + nq][2 (max, min)][4 * GP]: parts 0..kLutParts-1 hold partial sums over
 // their subspaces of the per-subspace extremes, parts kLutParts.. the extremes of one
-// 128-cluster slice of the centroid term. The scan reduces them once per unit (one warp)
-// into the final bounds `fbounds` [U][2][G] that every later kernel reads.
-static_assert(kMaxClusters / 128 <= 32, "one lane per centroid slice");
+// kQcSlice-cluster slice of the centroid term. The scan reduces them once per unit (one
+// warp) into the final bounds `fbounds` [U][2][G] that every later kernel reads.
 template <int G>
 __device__ __forceinline__ void reduce_bounds_warp(const float* bounds, int u, int nq, float* ub, float* lb) {
   constexpr int G4 = ((G + 3) / 4) * 4;
   const int lane = threadIdx.x & 31;
   const float* bu = bounds + static_cast<size_t>(u) * (kLutParts + nq) * 2 * G4;
-  // one head at a time (few live registers); lane l holds centroid slice l
+  // one head at a time (few live registers); lane l takes centroid slices l, l + 32, ...
 #pragma unroll 1
   for (int g = 0; g < G; ++g) {
-    float qmax = lane < nq ? bu[((kLutParts + lane) * 2 + 0) * G4 + g] : -INFINITY;
-    float qmin = lane < nq ? bu[((kLutParts + lane) * 2 + 1) * G4 + g] : INFINITY;
+    float qmax = -INFINITY, qmin = INFINITY;
+    for (int sl = lane; sl < nq; sl += 32) {
+      qmax = fmaxf(qmax, bu[((kLutParts + sl) * 2 + 0) * G4 + g]);
+      qmin = fminf(qmin, bu[((kLutParts + sl) * 2 + 1) * G4 + g]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
@@ -61,7 +63,8 @@ struct AttendParams {
   const int32_t* block_table;
   const int32_t* seq_lens;
   const int32_t* n_indexed;  // exact mode
-  const int32_t* sel;        // exact mode: [U][cap] selected positions
+  const int32_t* sel;        // exact mode: [U][cap] KV-pool rows of the selected tokens
+  const UnitState* units;    // exact mode: per-unit ready flags set by the selection
   int32_t* err;
   float* pm;                 // [U][S_tot][G]
   float* pl;
@@ -127,7 +130,8 @@ struct ScanParams {
   float* fbounds;            // [U][2][G] final (ub, lb), written here
   float* W;
   uint32_t* hist;
-  float* sigma;              // [U][cap]
+  float* sigma;              // [U][list_slots]
+  float* chunk_max;          // [U][list_slots / 32] largest sigma of each chunk
   float* approx_logits;      // debug [B][Hq][cap] or null
   int32_t* err;
   int B, Hq, Hkv, cap, C, nq, n_sink;
@@ -152,15 +156,18 @@ struct SelectParams {
   const float* bounds;
   const float* fbounds;      // [U][2][G] final (ub, lb) from the scan
   const float* sigma;
+  const float* chunk_max;        // [U][list_slots / 32]
   const uint32_t* hist;
   uint32_t* bitmap;
   unsigned long long* cand;  // [U][cap]
   float* cand_w;             // [U][kCandWeights][G] e^{shat_g - ub_g} of the first candidates
   int32_t* cand_c;           // [U][kCandWeights] their clusters
   UnitState* units;
-  int32_t* sel;              // [U][cap]
+  int32_t* sel;              // [U][cap] KV-pool row of each selected token, ascending position
   float* W;
-  int32_t* dbg_selected;     // [U][cap] or null
+  const int32_t* block_table;  // [B][max_pages]
+  int page_size, max_pages, num_pages;
+  int32_t* dbg_selected;     // [U][cap] or null (positions)
   int32_t* dbg_nselected;    // [U] or null
   int32_t* err;
   int B, Hkv, cap, C, nq, n_sink, bitmap_words, k_override, background;

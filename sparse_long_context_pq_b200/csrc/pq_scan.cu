@@ -103,12 +103,29 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_t
 // ===========================================================================
 // tables
 // ===========================================================================
+// q'_g = scale * q_g of the unit's heads into shared memory: every load of the thread in
+// flight before the first store (256 threads).
+template <int G4, int G>
+__device__ __forceinline__ void stage_q(const TablesParams& p, int b, int h, int tid, float (*qsh)[kD]) {
+  constexpr int kPer = G4 * kD / 256;
+  float v[kPer];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int i = tid + r * 256, g = i / kD, d = i % kD;
+    v[r] = (g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.scale : 0.f;
+  }
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int i = tid + r * 256;
+    qsh[i / kD][i % kD] = v[r];
+  }
+}
 template <int G>
 __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
   constexpr int GP = (G + 3) / 4;
   constexpr int G4 = GP * 4;
   constexpr int kSubPerPart = kM / kLutParts;   // 4 subspaces per LUT CTA
-  constexpr int kQcPerWarp = 16;                // 128 clusters per slice / 8 warps
+  constexpr int kQcPerWarp = kQcSlice / 8;      // clusters per warp (8 warps per slice)
   __shared__ float qsh[G4][kD];
   __shared__ float wred[2][8][kSubPerPart][G4];
   const int u = blockIdx.x;
@@ -130,10 +147,7 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
       cw[i][0] = src[0];
       cw[i][1] = src[1];
     }
-    for (int i = tid; i < G4 * kD; i += blockDim.x) {
-      const int g = i / kD, d = i % kD;
-      qsh[g][d] = (g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.scale : 0.f;
-    }
+    stage_q<G4, G>(p, b, h, tid, qsh);
     // zero this unit's selection state (spread over the LUT CTAs)
     for (int i = part * blockDim.x + tid; i < kNB; i += kLutParts * blockDim.x)
       p.hist[static_cast<size_t>(u) * kNB + i] = 0u;
@@ -181,9 +195,9 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
       bnd[(part * 2 + mm) * G4 + g] = (g < G) ? acc : 0.f;
     }
   } else {
-    // ---- qc[c][g] = q'_g . centroid_c for one 128-cluster slice; warp = 16 clusters, lane = 4 dims ----
+    // ---- qc[c][g] = q'_g . centroid_c for one kQcSlice-cluster slice; lane = 4 dims ----
     const int slice = part - kLutParts;
-    const int c0 = slice * 128 + warp * kQcPerWarp;
+    const int c0 = slice * kQcSlice + warp * kQcPerWarp;
     float4 cv[kQcPerWarp];
 #pragma unroll
     for (int i = 0; i < kQcPerWarp; ++i) {
@@ -191,12 +205,9 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
       cv[i] = c < p.C ? *reinterpret_cast<const float4*>(p.centroids + (static_cast<size_t>(u) * p.C + c) * kD + lane * 4)
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int i = tid; i < G4 * kD; i += blockDim.x) {
-      const int g = i / kD, d = i % kD;
-      qsh[g][d] = (g < G) ? p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * kD + d] * p.scale : 0.f;
-    }
+    stage_q<G4, G>(p, b, h, tid, qsh);
     {   // zero this slice's cluster weights
-      const int cs = slice * 128, ce = min(p.C, cs + 128), nc = ce - cs;
+      const int cs = slice * kQcSlice, ce = min(p.C, cs + kQcSlice), nc = ce - cs;
       for (int i = tid; i < G * nc; i += blockDim.x)
         p.W[(static_cast<size_t>(u) * G + i / nc) * p.C + cs + (i % nc)] = 0.f;
     }
@@ -260,16 +271,18 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
 // are in flight while it scores the current one.
 // threads per scan CTA (one CTA per SM; registers bound the warp count)
 template <int G>
-constexpr int scan_threads_of() { return 512; }
+__host__ __device__ constexpr int scan_threads_of() { return 512; }
 constexpr int kRingCodeBytes = 32 * kM;                     // 512 per chunk
-constexpr int kRingSlotBytes = kRingCodeBytes + 32 * 4;     // + index slots = 640
+constexpr int kRingJsBytes = 32 * 4;                        // index slots
+constexpr int kRingSlotBytes = kRingCodeBytes + kRingJsBytes + 16;   // + cluster word (16-B cell) = 656
 constexpr size_t kScanSmemLimit = 226 * 1024;   // dynamic; the rest of 227 KB is static
 
 template <int G>
 struct ScanSmem {
   static constexpr int GP = (G + 3) / 4;
   // tables (LUT, centroid terms) and the score histogram; then the warps' rings
-  // ([D][32][16 B] codes, then [D][32] index slots per warp); then the tables mbarrier
+  // ([D][32][16 B] codes, [D][32] index slots, [D] 16-B cells holding the 4-byte word
+  // with the chunk's cluster id, per warp); then the tables mbarrier
   __host__ __device__ static size_t tables(int C) {
     return align_up(static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 + kNB * 4, 128);
   }
@@ -375,6 +388,7 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
   uint8_t* wring = smem + ScanSmem<G>::tables(C) + static_cast<size_t>(warp) * D * kRingSlotBytes;
   uint4* ring_code = reinterpret_cast<uint4*>(wring) + lane;                              // [D][32]
   int32_t* ring_js = reinterpret_cast<int32_t*>(wring + D * kRingCodeBytes) + lane;       // [D][32]
+  uint32_t* ring_cl = reinterpret_cast<uint32_t*>(wring + D * (kRingCodeBytes + kRingJsBytes));   // [D][4]
 
   __syncthreads();  // previous segment finished with shared memory
   if (tid == 0) {
@@ -395,18 +409,20 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
   const uint8_t* lut_b = reinterpret_cast<const uint8_t*>(lut_s);
 
   // this warp's chunks; the first D go out while the tables land (one commit group per
-  // chunk, empty groups past the end keep the count regular)
+  // chunk, empty groups past the end keep the count regular). The chunk's cluster id
+  // (u16) comes with lane 0's group as the aligned 4-byte word that holds it.
   const int first = ch0 + warp;
   constexpr int kScanWarps = scan_threads_of<G>() / 32;
   const int cnt = first < ch1 ? (ch1 - first + kScanWarps - 1) / kScanWarps : 0;
-  uint32_t clreg = 0;   // lane j: cluster of the chunk in ring slot j
   auto issue = [&](int i) {
     if (i < cnt) {
       const int ch = first + kScanWarps * i;
       const int slot = i % D;
       cp_async_16(ring_code + slot * 32, lcodes + static_cast<size_t>(ch) * 32 + lane);
       cp_async_4(ring_js + slot * 32, lslot + static_cast<size_t>(ch) * 32 + lane);
-      if (lane == slot) clreg = ccl[ch];
+      if (lane == 0)
+        cp_async_4(ring_cl + slot * 4,
+                   reinterpret_cast<const void*>(reinterpret_cast<uintptr_t>(ccl + ch) & ~uintptr_t(3)));
     }
     cp_async_commit();
   };
@@ -444,10 +460,12 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
   for (int i = 0; i < cnt; ++i) {
     const int slot = i % D;
     cp_async_wait<D - 1>();              // this lane's copies of chunk i have landed
+    __syncwarp();                        // ... and lane 0's cluster word
     const uint4 code = ring_code[slot * 32];
     const int32_t js = ring_js[slot * 32];
-    uint32_t id = __shfl_sync(0xffffffffu, clreg, slot);
     const int ch = first + kScanWarps * i;
+    const uint32_t cw = ring_cl[slot * 4];
+    uint32_t id = ((reinterpret_cast<uintptr_t>(ccl + ch) >> 1) & 1) ? (cw >> 16) : (cw & 0xffffu);
     if (id >= static_cast<uint32_t>(C)) {
       bad_id = true;
       id = 0;
@@ -459,6 +477,10 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
 #pragma unroll
     for (int g = 1; g < G; ++g) sg = fmaxf(sg, sh[g]);
     __stcs(sig_u + static_cast<size_t>(ch) * 32 + lane, valid ? sg : -INFINITY);
+    {   // the chunk's largest score lets the filter skip chunks below the threshold
+      const float cmx = warp_max(valid ? sg : -INFINITY);
+      if (lane == 0) p.chunk_max[static_cast<size_t>(u) * (p.list_slots / 32) + ch] = cmx;
+    }
     if (p.approx_logits && valid) {
 #pragma unroll
       for (int g = 0; g < G; ++g) p.approx_logits[(static_cast<size_t>(b) * p.Hq + h * G + g) * p.cap + js] = sh[g];
@@ -472,7 +494,8 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
       if ((lane & (kGroup - 1)) == 0) atomicAdd(Wu + (lane / kGroup) * C + id, e);
     }
     if (valid) atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
-    issue(i + D);                        // refill this slot with the chunk D ahead
+    __syncwarp();                        // every lane has read the slot
+    issue(i + D);                        // refill it with the chunk D ahead
   }
   cp_async_wait<0>();
   if (bad_id) record_error(p.err, HSA_DEVERR_CLUSTER);
@@ -632,51 +655,61 @@ __device__ __forceinline__ void remove_weights(const SelectParams& p, int u, uin
   for (int g = 0; g < G; ++g) atomicAdd(&Wu[g * p.C + id], -e[g]);
 }
 
+// Filter over chunks: the scan left each 32-slot chunk's largest score, so a chunk whose
+// maximum falls below the threshold bin holds no selected or candidate token (the bin is
+// monotone in the score) and is skipped; only the few chunks that reach it are read.
+constexpr int kFilterThreads = 256;
+constexpr int kCmPerThread = 4;                                    // chunk maxima per thread per pass
+constexpr int kCmPass = kCmPerThread * kFilterThreads;             // chunks examined per pass
+constexpr int kActPerWarp = 4;                                     // active chunks per warp per round
+constexpr int kFixCap = kActPerWarp * kFilterThreads;              // queued tokens per round (<= one per slot)
+
 template <int G>
-__global__ void __launch_bounds__(256, 2) filter_kernel(SelectParams p) {
-  constexpr int kBatch = 8;
-  constexpr int kFixCap = kBatch * 256;   // definite selections of one batch, at most one per slot
+__global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams p) {
   __shared__ __align__(16) uint32_t hist_s[kNB];
-  __shared__ uint32_t fix_list[kFixCap];   // list slots
-  __shared__ int32_t fix_cand[kFixCap];     // candidate slot, or -1 for a definite selection
-  __shared__ uint32_t fix_n;
   __shared__ uint32_t scan_tot[33];
   __shared__ int sh_bstar;
   __shared__ uint32_t sh_above;
-  static_assert(kNB == 8 * 256, "filter threshold search: 256 threads x 8 bins");
+  __shared__ int32_t act[kCmPass];          // active chunks of the current pass
+  __shared__ int n_act;
+  __shared__ uint32_t fix_list[kFixCap];   // list slots
+  __shared__ int32_t fix_cand[kFixCap];     // candidate slot, or -1 for a definite selection
+  __shared__ uint32_t fix_n;
+  static_assert(kNB == 8 * kFilterThreads, "filter threshold search: 256 threads x 8 bins");
+  constexpr int NW = kFilterThreads / 32;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t lane = tid & 31;
   pdl_wait();
   pdl_launch_dependents();
   const int max_chunks = p.list_slots / 32;
   for_each_unit_part(
-      p.B, p.Hkv, [&](int b, int h) { return 32 * unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
-      [&](int u, int j0, int j1) {
+      p.B, p.Hkv, [&](int b, int h) { return unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
+      [&](int u, int c0, int c1) {
     const int b = u / p.Hkv;
     const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
     const int k = decode_k(p.budget, p.k_override, N);
     const float* sig = p.sigma + static_cast<size_t>(u) * p.list_slots;
     const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
-    // bounds (histogram range, weight reference) load with everything else below
+    const float* cmax = p.chunk_max + static_cast<size_t>(u) * max_chunks;
+    // bounds and the first pass of chunk maxima load with the histogram
     float ub[G], lb[G];
     final_bounds<G>(p.fbounds, u, ub, lb);
-    // first batch of scores in flight while the threshold is found
-    float sv[kBatch];
-    int32_t jv[kBatch];
+    float cm[kCmPerThread];
 #pragma unroll
-    for (int r = 0; r < kBatch; ++r) {
-      const int j = j0 + r * blockDim.x + threadIdx.x;
-      sv[r] = j < j1 ? sig[j] : 0.f;
-      jv[r] = j < j1 ? lslot[j] : -1;
+    for (int e = 0; e < kCmPerThread; ++e) {
+      const int c = c0 + tid + e * kFilterThreads;
+      cm[e] = c < c1 ? cmax[c] : -INFINITY;
     }
-    __syncthreads();
+    __syncthreads();   // shared state of a previous unit range is no longer read
     {
       const uint4* hg = reinterpret_cast<const uint4*>(p.hist + static_cast<size_t>(u) * kNB);
-      uint4 hv[kNB / 4 / 256];
+      uint4 hv[kNB / 4 / kFilterThreads];
 #pragma unroll
-      for (int r = 0; r < kNB / 4 / 256; ++r) hv[r] = hg[r * 256 + threadIdx.x];
+      for (int r = 0; r < kNB / 4 / kFilterThreads; ++r) hv[r] = hg[r * kFilterThreads + tid];
 #pragma unroll
-      for (int r = 0; r < kNB / 4 / 256; ++r) reinterpret_cast<uint4*>(hist_s)[r * 256 + threadIdx.x] = hv[r];
+      for (int r = 0; r < kNB / 4 / kFilterThreads; ++r) reinterpret_cast<uint4*>(hist_s)[r * kFilterThreads + tid] = hv[r];
     }
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
       sh_bstar = kNB;   // k == 0: nothing selected
       sh_above = 0;
       fix_n = 0;
@@ -684,7 +717,7 @@ __global__ void __launch_bounds__(256, 2) filter_kernel(SelectParams p) {
     __syncthreads();
     {
       // thread t owns the 8 bins [kNB-8(t+1), kNB-8t): block scan of counts from the top
-      const int hi = kNB - 8 * static_cast<int>(threadIdx.x);
+      const int hi = kNB - 8 * tid;
       uint32_t c8[8], local = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -708,7 +741,7 @@ __global__ void __launch_bounds__(256, 2) filter_kernel(SelectParams p) {
     }
     __syncthreads();
     const int bstar = sh_bstar;
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
       p.units[u].bstar = bstar;
       p.units[u].above = static_cast<int32_t>(sh_above);
     }
@@ -725,80 +758,104 @@ __global__ void __launch_bounds__(256, 2) filter_kernel(SelectParams p) {
     for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
     const bool fix = p.background && N > k;
     const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
-    const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * (p.list_slots / 32);
+    const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * max_chunks;
     uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
-    for (int base = j0; base < j1; base += kBatch * blockDim.x) {
-      float nv[kBatch];
-      int32_t njv[kBatch];
-      const int nb = base + kBatch * blockDim.x;
+
+    for (int cb = c0; cb < c1; cb += kCmPass) {
+      if (cb != c0) {
 #pragma unroll
-      for (int r = 0; r < kBatch; ++r) {
-        const int j = nb + r * blockDim.x + threadIdx.x;
-        nv[r] = j < j1 ? sig[j] : 0.f;
-        njv[r] = j < j1 ? lslot[j] : -1;
-      }
-      const uint32_t lane = threadIdx.x & 31;
-#pragma unroll
-      for (int r = 0; r < kBatch; ++r) {
-        const int j = jv[r];            // index slot of this list slot
-        const bool valid = j >= 0 && j < N;
-        const int bin = valid ? score_bin(sv[r], lo, inv) : -1;
-        const bool definite = bin > bstar;
-        if (definite) atomicOr(bm + (j >> 5), 1u << (j & 31));
-        int slot = -1;
-        if (bin == bstar) {
-          slot = atomicAdd(&p.units[u].ncand, 1);
-          if (slot < p.cap)
-            p.cand[static_cast<size_t>(u) * p.cap + slot] =
-                (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+        for (int e = 0; e < kCmPerThread; ++e) {
+          const int c = cb + tid + e * kFilterThreads;
+          cm[e] = c < c1 ? cmax[c] : -INFINITY;
         }
-        if (fix) {
-          // queue the list slot: a definite selection's weight leaves its cluster's sums
-          // below; a candidate's weights are stored for the finalize's winners
-          const bool queued = definite || (slot >= 0 && slot < kCandWeights);
-          const uint32_t m = __ballot_sync(0xffffffffu, queued);
-          if (m) {
-            const uint32_t leader = __ffs(m) - 1;
-            uint32_t at = 0;
-            if (lane == leader) at = atomicAdd(&fix_n, static_cast<uint32_t>(__popc(m)));
-            at = __shfl_sync(0xffffffffu, at, leader);
-            if (queued) {
-              at += __popc(m & ((1u << lane) - 1u));
-              fix_list[at] = base + r * blockDim.x + threadIdx.x;
-              fix_cand[at] = definite ? -1 : slot;
+        __syncthreads();   // the previous pass is done with act[]
+      }
+      if (tid == 0) n_act = 0;
+      __syncthreads();
+      // chunks whose maximum reaches the threshold bin, compacted warp by warp
+#pragma unroll
+      for (int e = 0; e < kCmPerThread; ++e) {
+        const int c = cb + tid + e * kFilterThreads;
+        const bool active = c < c1 && score_bin(cm[e], lo, inv) >= bstar;
+        const uint32_t m = __ballot_sync(0xffffffffu, active);
+        if (m) {
+          const uint32_t leader = __ffs(m) - 1;
+          int at = 0;
+          if (lane == leader) at = atomicAdd(&n_act, __popc(m));
+          at = __shfl_sync(0xffffffffu, at, leader);
+          if (active) act[at + __popc(m & ((1u << lane) - 1u))] = c;
+        }
+      }
+      __syncthreads();
+      const int na = n_act;
+      for (int a0 = 0; a0 < na; a0 += NW * kActPerWarp) {
+        // each warp reads up to kActPerWarp active chunks at once; lane = slot of the chunk
+        float sv[kActPerWarp];
+        int32_t jv[kActPerWarp];
+        int chv[kActPerWarp];
+#pragma unroll
+        for (int r = 0; r < kActPerWarp; ++r) {
+          const int a = a0 + warp + NW * r;
+          chv[r] = a < na ? act[a] : -1;
+          sv[r] = chv[r] >= 0 ? sig[static_cast<size_t>(chv[r]) * 32 + lane] : -INFINITY;
+          jv[r] = chv[r] >= 0 ? lslot[static_cast<size_t>(chv[r]) * 32 + lane] : -1;
+        }
+#pragma unroll
+        for (int r = 0; r < kActPerWarp; ++r) {
+          const int j = jv[r];            // index slot of this list slot
+          const bool valid = j >= 0 && j < N;
+          const int bin = valid ? score_bin(sv[r], lo, inv) : -1;
+          const bool definite = bin > bstar;
+          if (definite) atomicOr(bm + (j >> 5), 1u << (j & 31));
+          int slot = -1;
+          if (bin == bstar) {
+            slot = atomicAdd(&p.units[u].ncand, 1);
+            if (slot < p.cap)
+              p.cand[static_cast<size_t>(u) * p.cap + slot] =
+                  (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+          }
+          if (fix) {
+            // queue the list slot: a definite selection's weight leaves its cluster's sums
+            // below; a candidate's weights are stored for the finalize's winners
+            const bool queued = definite || (slot >= 0 && slot < kCandWeights);
+            const uint32_t m = __ballot_sync(0xffffffffu, queued);
+            if (m) {
+              const uint32_t leader = __ffs(m) - 1;
+              uint32_t at = 0;
+              if (lane == leader) at = atomicAdd(&fix_n, static_cast<uint32_t>(__popc(m)));
+              at = __shfl_sync(0xffffffffu, at, leader);
+              if (queued) {
+                at += __popc(m & ((1u << lane) - 1u));
+                fix_list[at] = static_cast<uint32_t>(chv[r]) * 32 + lane;
+                fix_cand[at] = definite ? -1 : slot;
+              }
             }
           }
         }
-      }
-      if (fix) {
-        // Queued tokens of this batch: one per thread, every look-up of a token in flight
-        // together.
-        __syncthreads();
-        const uint32_t n = fix_n;
-        for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
-          const uint32_t ls = fix_list[i];
-          const int cs = fix_cand[i];
-          uint32_t id = ccl[ls >> 5];
-          if (id >= static_cast<uint32_t>(p.C)) id = 0;
-          float e[G];
-          token_weights<G>(p, u, id, lcodes[ls], ub2, e);
-          if (cs < 0) {
-            remove_weights<G>(p, u, id, e);
-          } else {
-            float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + cs) * G;
+        if (fix) {
+          // queued tokens of this round: one per thread, every look-up of a token in flight together
+          __syncthreads();
+          const uint32_t n = fix_n;
+          for (uint32_t i = tid; i < n; i += kFilterThreads) {
+            const uint32_t ls = fix_list[i];
+            const int cs = fix_cand[i];
+            uint32_t id = ccl[ls >> 5];
+            if (id >= static_cast<uint32_t>(p.C)) id = 0;
+            float e[G];
+            token_weights<G>(p, u, id, lcodes[ls], ub2, e);
+            if (cs < 0) {
+              remove_weights<G>(p, u, id, e);
+            } else {
+              float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + cs) * G;
 #pragma unroll
-            for (int g = 0; g < G; ++g) cw[g] = e[g];
-            p.cand_c[static_cast<size_t>(u) * kCandWeights + cs] = static_cast<int32_t>(id);
+              for (int g = 0; g < G; ++g) cw[g] = e[g];
+              p.cand_c[static_cast<size_t>(u) * kCandWeights + cs] = static_cast<int32_t>(id);
+            }
           }
+          __syncthreads();
+          if (tid == 0) fix_n = 0;
+          __syncthreads();
         }
-        __syncthreads();
-        if (threadIdx.x == 0) fix_n = 0;
-        __syncthreads();
-      }
-#pragma unroll
-      for (int r = 0; r < kBatch; ++r) {
-        sv[r] = nv[r];
-        jv[r] = njv[r];
       }
     }
   });
@@ -811,6 +868,9 @@ constexpr int kFinThreads = 1024;
 constexpr int kFinWordsPerThread = 4;
 constexpr int kFinChunkWords = kFinWordsPerThread * kFinThreads;   // 131072 slots per pass
 constexpr int kFinSmemCand = kFinThreads;                          // candidates resolved in shared memory
+constexpr int kFinBtCache = 8192;   // block-table entries cached in shared memory (longer tables: global)
+
+__host__ __device__ inline int fin_bt_cached(int max_pages) { return max_pages <= kFinBtCache ? max_pages : 0; }
 
 // One CTA per unit: resolve the threshold bin's candidates exactly (score desc, position
 // asc), compact the selection bitmap into ascending positions, and take the selected
@@ -825,9 +885,22 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
   __shared__ uint32_t warp_tot[33];
   __shared__ int sh_bin;
   __shared__ uint32_t sh_above, sh_nwin;
+  extern __shared__ int32_t bt_s[];   // the sequence's block table when it fits
   const int u = blockIdx.x;
   const int b = u / p.Hkv;
+  const int h = u % p.Hkv;
   const int tid = threadIdx.x;
+  const int nbt = fin_bt_cached(p.max_pages);
+  const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
+  {   // the block table predates the step: all of this thread's entries in flight at once
+    constexpr int kPer = kFinBtCache / kFinThreads;
+    int32_t v[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) v[e] = tid + e * kFinThreads < nbt ? bt_row[tid + e * kFinThreads] : 0;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e)
+      if (tid + e * kFinThreads < nbt) bt_s[tid + e * kFinThreads] = v[e];
+  }
   pdl_wait();
   pdl_launch_dependents();
   // ---- one round trip: lengths, unit state, candidates and the first bitmap pass (speculative) ----
@@ -892,6 +965,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
   int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
   if (k == 0) {
     if (tid == 0 && p.dbg_nselected) p.dbg_nselected[u] = 0;
+    publish_flag(&p.units[u].ready);
     return;
   }
   const int m = min(st.ncand, p.cap);
@@ -999,8 +1073,16 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
         wv &= wv - 1;
         const int j = wi * 32 + bit;
         if (off < static_cast<uint32_t>(p.cap)) {
-          sel_u[off] = s0 + j;
-          if (p.dbg_selected) p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = s0 + j;
+          // the token's KV-pool row, so the exact attend reads it in one step
+          const int pos = s0 + j;
+          const int pi = pos / p.page_size;
+          int page = pi < p.max_pages ? (pi < nbt ? bt_s[pi] : bt_row[pi]) : -1;
+          if (page < 0 || page >= p.num_pages) {
+            record_error(p.err, HSA_DEVERR_PAGE);
+            page = 0;
+          }
+          sel_u[off] = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
+          if (p.dbg_selected) p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = pos;
         }
         ++off;
       }
@@ -1012,6 +1094,9 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     if (running != static_cast<uint32_t>(k)) record_error(p.err, HSA_DEVERR_SELECT);
     if (p.dbg_nselected) p.dbg_nselected[u] = static_cast<int32_t>(running);
   }
+  // the exact attend and the background of this unit may start (selection rows and
+  // the winners' weight fix-up are written)
+  publish_flag(&p.units[u].ready);
 }
 
 template <typename Kern, typename P>
@@ -1096,13 +1181,19 @@ cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t strea
 }
 
 cudaError_t launch_filter(int G, const SelectParams& p, int grid, cudaStream_t stream, bool pdl) {
-#define CALL(GG) return launch_ex(filter_kernel<GG>, dim3(grid), dim3(256), 0, stream, pdl, p)
+#define CALL(GG) return launch_ex(filter_kernel<GG>, dim3(grid), dim3(kFilterThreads), 0, stream, pdl, p)
   PQHSA_G_SWITCH(G, CALL)
 #undef CALL
 }
 
 cudaError_t launch_finalize(int G, const SelectParams& p, cudaStream_t stream, bool pdl) {
-#define CALL(GG) return launch_ex(finalize_kernel<GG>, dim3(p.B * p.Hkv), dim3(kFinThreads), 0, stream, pdl, p)
+  const size_t smem = static_cast<size_t>(fin_bt_cached(p.max_pages)) * sizeof(int32_t);
+#define CALL(GG)                                                                                     \
+  {                                                                                                  \
+    cudaError_t e = ensure_dyn_smem<finalize_kernel<GG>>(smem);                                      \
+    if (e != cudaSuccess) return e;                                                                  \
+    return launch_ex(finalize_kernel<GG>, dim3(p.B * p.Hkv), dim3(kFinThreads), smem, stream, pdl, p); \
+  }
   PQHSA_G_SWITCH(G, CALL)
 #undef CALL
 }
