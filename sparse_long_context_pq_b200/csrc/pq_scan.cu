@@ -880,6 +880,7 @@ template <int G>
 __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
   __shared__ unsigned long long ck[kFinSmemCand];
   __shared__ uint32_t bmc[kFinChunkWords];
+  __shared__ uint32_t woff[kFinChunkWords];   // exclusive count of selected bits before each word
   __shared__ uint32_t wins[kFinSmemCand];
   __shared__ uint32_t dig[256];
   __shared__ uint32_t warp_tot[33];
@@ -1063,31 +1064,44 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
       pc += __popc(words[e]);
     }
     uint32_t tot;
-    uint32_t off = running + block_excl_scan(pc, warp_tot, tot);
+    {
+      uint32_t o = block_excl_scan(pc, warp_tot, tot);
 #pragma unroll
-    for (int e = 0; e < kFinWordsPerThread; ++e) {
-      uint32_t wv = words[e];
-      const int wi = w0 + kFinWordsPerThread * tid + e;
-      while (wv) {
-        const int bit = __ffs(wv) - 1;
-        wv &= wv - 1;
-        const int j = wi * 32 + bit;
-        if (off < static_cast<uint32_t>(p.cap)) {
-          // the token's KV-pool row, so the exact attend reads it in one step
-          const int pos = s0 + j;
-          const int pi = pos / p.page_size;
-          int page = pi < p.max_pages ? (pi < nbt ? bt_s[pi] : bt_row[pi]) : -1;
-          if (page < 0 || page >= p.num_pages) {
-            record_error(p.err, HSA_DEVERR_PAGE);
-            page = 0;
-          }
-          sel_u[off] = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
-          if (p.dbg_selected) p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = pos;
+      for (int e = 0; e < kFinWordsPerThread; ++e) {
+        woff[kFinWordsPerThread * tid + e] = o;
+        o += __popc(words[e]);
+      }
+    }
+    __syncthreads();
+    // Output entry i of this pass: the word holding it by binary search over the word
+    // offsets, then its bit; every thread writes about tot / 1024 entries whatever the
+    // positions of the selected tokens.
+    for (uint32_t i = tid; i < tot; i += kFinThreads) {
+      int lo_w = 0, hi_w = kFinChunkWords - 1;   // largest word with woff <= i
+      while (lo_w < hi_w) {
+        const int mid = (lo_w + hi_w + 1) >> 1;
+        if (woff[mid] <= i) lo_w = mid;
+        else hi_w = mid - 1;
+      }
+      uint32_t wv = bmc[lo_w];
+      for (uint32_t c = i - woff[lo_w]; c > 0; --c) wv &= wv - 1;
+      const int j = (w0 + lo_w) * 32 + (__ffs(wv) - 1);
+      const uint32_t off = running + i;
+      if (off < static_cast<uint32_t>(p.cap)) {
+        // the token's KV-pool row, so the exact attend reads it in one step
+        const int pos = s0 + j;
+        const int pi = pos / p.page_size;
+        int page = pi < p.max_pages ? (pi < nbt ? bt_s[pi] : bt_row[pi]) : -1;
+        if (page < 0 || page >= p.num_pages) {
+          record_error(p.err, HSA_DEVERR_PAGE);
+          page = 0;
         }
-        ++off;
+        sel_u[off] = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
+        if (p.dbg_selected) p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = pos;
       }
     }
     running += tot;
+    __syncthreads();   // woff / bmc are rewritten by the next pass
   }
   if (tid == 0) {
     p.units[u].nsel = static_cast<int32_t>(running);
