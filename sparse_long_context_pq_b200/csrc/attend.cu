@@ -12,8 +12,8 @@
 // Design (sm_100a): one producer warp streams K/V rows into a ring of
 // shared-memory tiles with mbarrier completion: dense reads use tensor TMA with
 // one box per head-page (128-byte swizzle, 1024-byte aligned boxes); gathered
-// rows (sink + selected + tail) use one 1-D bulk copy per 256-byte row into a
-// 272-byte-stride layout. Both layouts are bank-conflict free for the two read
+// rows (sink + tail + selected) are copied in 16-byte pieces by the producer lanes
+// (LSU async copies, 16 lanes per 256-byte row) into a 272-byte-stride layout. Both layouts are bank-conflict free for the two read
 // patterns below (and for ldmatrix). Four consumer warps each own every fourth
 // 32-token tile and run it on the tensor cores (mma.sync m16n8k16 bf16, with q
 // and P split into bf16 hi + lo so the result keeps fp32-level accuracy), with an

@@ -94,7 +94,7 @@ __device__ void background_block(const AttendParams& p, int j, uint8_t* smem);
 int attend_slots_per_sm();
 size_t attend_smem_bytes(int G);
 // Row sources: kExact = sink + selected + tail list of hsa_decode, else every token.
-// Loading: page tiles by tensor TMA (dense, page_size >= 8) or one bulk copy per row.
+// Loading: page tiles by tensor TMA (dense, page_size >= 8) or 16-byte async copies per row.
 cudaError_t launch_attend(int G, bool exact, bool rows, const CUtensorMap& tk, const CUtensorMap& tv,
                           const AttendParams& p, int grid, cudaStream_t stream, bool pdl);
 cudaError_t launch_merge(int G, const MergeParams& p, cudaStream_t stream, bool pdl);

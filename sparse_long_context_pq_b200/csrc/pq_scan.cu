@@ -3,12 +3,14 @@
 //              plus exact upper/lower bounds of every head's approximate logit;
 //   scan     - one pass over the uint8 codes: approximate logits of every indexed
 //              token, the selection score sigma = max over the group's heads,
-//              per-cluster exp-weight sums and a histogram of sigma;
+//              per-cluster exp-weight sums, a histogram of sigma, each chunk's
+//              largest sigma and the final logit bounds;
 //   filter   - marks tokens above the threshold histogram bin, collects the
-//              tokens in that bin as candidates;
+//              tokens in that bin as candidates (reading only chunks that reach
+//              the bin) and removes the definite selections' weights;
 //   finalize - resolves the candidates exactly (score desc, position asc),
-//              compacts the selected positions in ascending order and removes
-//              the selected tokens' weights from the cluster sums.
+//              writes the selected tokens as KV-pool rows in ascending position
+//              order, removes the winners' weights and publishes the unit.
 //
 // Source: rit.work "pq-hsa-long-context-attention", section
 // "Как приблизительные оценки возвращают отброшенный контекст" (an approximate
