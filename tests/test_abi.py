@@ -68,12 +68,14 @@ def _kv(B=1, Hq=4, Hkv=1, D=128, page_size=16, max_pages=8, num_pages=8, seq=100
     return kv, lens
 
 
-def _ix(B=1, C=16, cap=128, n_idx=50, n_sink=4, M=16, dsub=8, list_slots=None, list_slot=FAKE):
+def _ix(B=1, C=16, cap=128, n_idx=50, n_sink=4, M=16, dsub=8, list_slots=None, list_slot=FAKE,
+        chunk_cluster=FAKE):
     nh = np.full(B, n_idx, dtype=np.int32)
     ls = P.index_list_slots(cap, max(C, 1)) if list_slots is None else list_slots
     ix = P._Index(centroids=FAKE, codebooks=FAKE, codes=FAKE, ids=FAKE, sum_v=FAKE, mean_v=FAKE, count=FAKE,
                   n_indexed=FAKE, n_indexed_host=nh.ctypes.data, list_codes=FAKE, list_slot=list_slot,
-                  chunk_cluster=FAKE, list_meta=FAKE, C=C, M=M, dsub=dsub, ncode=256, cap=cap, n_sink=n_sink,
+                  chunk_cluster=chunk_cluster, list_meta=FAKE, C=C, M=M, dsub=dsub, ncode=256, cap=cap,
+                  n_sink=n_sink,
                   list_slots=ls)
     return ix, nh
 
@@ -104,7 +106,8 @@ def test_decode_rejects_bad_cache(lib, mutate, status):
     (dict(n_idx=99), 3),               # n_sink + N > T
     (dict(list_slots=32 * 4), 3),      # cluster lists too small
     (dict(C=5000), 2),                 # too many clusters for the list builder
-    (dict(list_slot=FAKE + 4), 4),     # list slots are streamed by 16-byte bulk copies
+    (dict(list_slot=FAKE + 4), 4),     # list slots are streamed by 16-byte async copies
+    (dict(chunk_cluster=FAKE + 2), 4), # cluster ids are fetched as aligned 4-byte words
 ])
 def test_decode_rejects_bad_index(lib, mutate, status):
     kv, lens = _kv()

@@ -26,6 +26,10 @@ CASES = {
     "batch_4x4k": dict(name="batch32_32k", B=4, T=4096),
     "qwen_g8_8k": dict(name="qwen30b_128k_append", B=2, T=8192, extra_tokens=0, append_batch=0),
     "ragged_5003": dict(name="tiny_4k", T=5003, n_recent=101, C=32, n_needles=3),
+    "mha_g1_4k": dict(name="tiny_4k", Hq=2, Hkv=2),                   # one query head per KV head
+    "gqa_g2_4k": dict(name="tiny_4k", Hq=4, Hkv=2),
+    "page4_4k": dict(name="tiny_4k", page_size=4),                    # dense path gathers rows
+    "page64_3000": dict(name="tiny_4k", T=3000, page_size=64, n_recent=64, C=48),
 }
 
 
