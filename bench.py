@@ -53,8 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="llama8b_128k")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["ctx", "budget"], default=None,
-                    help="extra measurements: context-length crossover, or budget / background ablation")
+    ap.add_argument("--sweep", choices=["ctx", "budget", "batch"], default=None,
+                    help="extra measurements: context-length crossover, budget / background ablation, "
+                         "or the 32-sequence batch at 32K")
     ap.add_argument("--append", action="store_true",
                     help="index-append cost on the Qwen3-30B-A3B-shaped workload (512-token batches)")
     return ap.parse_args(argv)
@@ -469,6 +470,27 @@ def run_sweep_ctx(args):
                       "predicted_crossover_T": cross}), flush=True)
 
 
+def run_sweep_batch(args):
+    """32 sequences x 32K context (shuffled pages, per-sequence seeds) at 1 %: PQ-HSA vs dense."""
+    import torch
+    from synth import workload
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, _ = measured_peaks()
+    w = workload("batch32_32k")
+    S = _Setup(w, dev)
+    k = S.P.decode_k(w.budget, w.n_indexed)
+    hsa_b, ids_b, dense_b, _ = step_bytes(w, w.n_indexed, k)
+    us_h = S.time_graph(S.graph(S.hsa()), args.steps, args.warmup)
+    us_d = S.time_graph(S.graph(S.dense()), args.steps, args.warmup)
+    assert S.P.hsa_read_error(S.ws) == 0
+    print(json.dumps({"sweep": "batch", "workload": w.name, "B": w.B, "T": w.T, "k": k,
+                      "hsa_us": round(us_h, 3), "dense_us": round(us_d, 3), "speedup": round(us_d / us_h, 3),
+                      "hsa_bytes": hsa_b, "dense_bytes": dense_b,
+                      "hsa_gbs": round(hsa_b / us_h / 1e3, 1), "dense_gbs": round(dense_b / us_d / 1e3, 1),
+                      "dense_pct_peak": round(100 * dense_b / us_d / 1e3 / peak, 2)}), flush=True)
+
+
 def run_sweep_budget(args):
     import torch
     from synth import workload
@@ -559,6 +581,8 @@ def main(argv=None):
         run_sweep_ctx(args)
     elif args.sweep == "budget":
         run_sweep_budget(args)
+    elif args.sweep == "batch":
+        run_sweep_batch(args)
     elif args.append:
         run_append(args)
     elif args.impl == "reference":

@@ -320,7 +320,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
     Emax = std::max<long long>(Emax, static_cast<long long>(s0) + k + (T - s0 - N));
   }
   const Split sp = plan_splits(Emax, U, L.nbg, dev->sms * attend_slots_per_sm());
-  CUtensorMap tk = {}, tv = {};   // unused: gathered rows are bulk copies
+  CUtensorMap tk = {}, tv = {};   // unused: gathered rows are copied by the producer lanes
   cudaEvent_t* ev = dbg ? dbg->stage_events : nullptr;
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], stream) : cudaSuccess; };
 

@@ -36,9 +36,9 @@ constexpr int kRowPitch = 272;                 // padded: 256-byte row + 16
 // t % S. S is a multiple of CW, so every stage is always consumed by the same warp
 // and its mbarrier phases are awaited strictly in order: a parity wait can then
 // never alias a phase two steps ahead (which returns immediately on a parity barrier).
-// Dense page tiles use tensor TMA into 16 KB stages, gathered rows bulk copies into
-// 272-byte-pitch rows (17 KB stages); both run 4 consumer warps over 4 stages (a deeper
-// 2-warp x 6-stage ring for dense reads measured no faster).
+// Dense page tiles use tensor TMA into 16 KB stages, gathered rows 16-byte async copies
+// into 272-byte-pitch rows (17 KB stages); both run 4 consumer warps over 4 stages (a
+// deeper 2-warp x 6-stage ring for dense reads measured no faster).
 template <bool kRows>
 struct Pipe {
   static constexpr int CW = 4;
