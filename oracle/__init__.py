@@ -19,4 +19,9 @@ from .pqhsa_oracle import (  # noqa: F401
     oracle_build_means,
     oracle_append,
     decode_k,
+    lloyd_assign,
+    lloyd_update,
+    kmeans_objective,
+    train_unit,
+    oracle_train,
 )

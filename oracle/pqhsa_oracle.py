@@ -277,6 +277,76 @@ def encode_keys(keys: np.ndarray, centroids: np.ndarray, codebooks: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# Index training (the step before the path: the index is built after prefill)
+# ---------------------------------------------------------------------------
+# The article says the index is built after prefill and groups the keys (IVF) with
+# compressed per-key codes (PQ); it does not say how the centroids and codebooks are
+# found. Reading: the plain Lloyd k-means iteration, for the coarse centroids on the
+# unit's keys and, per subspace, for the codebook on the residuals (key minus its
+# centroid). Initial centres are given rows of the training set (the draw is an input).
+
+def lloyd_assign(X: np.ndarray, centres: np.ndarray, chunk: int = 256) -> np.ndarray:
+    """a[j] = argmin_c sum_d (X_jd - centre_cd)^2: float64 distances compared as float32,
+    ties to the lower index."""
+    X = np.asarray(X, dtype=np.float64)
+    cen = np.asarray(centres, dtype=np.float64)
+    a = np.zeros(X.shape[0], dtype=np.int64)
+    for i in range(0, X.shape[0], chunk):
+        d = ((X[i:i + chunk, None, :] - cen[None, :, :]) ** 2).sum(axis=2)
+        a[i:i + chunk] = np.argmin(d.astype(np.float32), axis=1)   # first minimum = lowest index
+    return a
+
+
+def lloyd_update(X: np.ndarray, a: np.ndarray, centres: np.ndarray) -> np.ndarray:
+    """centre_c = mean of the rows assigned to c (float64, rounded to float32); a centre
+    with no rows keeps its value."""
+    X = np.asarray(X, dtype=np.float64)
+    k = centres.shape[0]
+    sums = np.zeros((k, X.shape[1]))
+    np.add.at(sums, a, X)
+    cnt = np.bincount(a, minlength=k)
+    out = np.asarray(centres, dtype=np.float64).copy()
+    nz = cnt > 0
+    out[nz] = sums[nz] / cnt[nz, None]
+    return out.astype(np.float32)
+
+
+def kmeans_objective(X: np.ndarray, centres: np.ndarray, a: np.ndarray) -> float:
+    """sum_j |X_j - centre_{a_j}|^2 in float64."""
+    X = np.asarray(X, dtype=np.float64)
+    return float(((X - np.asarray(centres, dtype=np.float64)[a]) ** 2).sum())
+
+
+def train_unit(keys: np.ndarray, init_slots: np.ndarray, C: int, coarse_iters: int, pq_iters: int,
+               M: int = 16, ncode: int = 256) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Centroids [C, D] and codebooks [M, ncode, D/M] of one unit from its training keys [n, D]
+    (float32 values of the bf16 keys).
+
+    Coarse: centres start at rows init_slots[:C]; coarse_iters Lloyd iterations (assign,
+    update); then a final assignment gives the residuals r_j = k_j - centroid_{a_j}
+    (float32). Codebook s: centres start at the subspace-s residuals of rows
+    init_slots[C + s*ncode : C + (s+1)*ncode]; pq_iters Lloyd iterations on the residuals'
+    subspace s. Returns (centroids, codebooks, final coarse assignment).
+    """
+    X = np.asarray(keys, dtype=np.float32)
+    init_slots = np.asarray(init_slots, dtype=np.int64)
+    cent = X[init_slots[:C]].copy()
+    for _ in range(coarse_iters):
+        cent = lloyd_update(X, lloyd_assign(X, cent), cent)
+    a = lloyd_assign(X, cent)
+    R = (X.astype(np.float64) - cent[a].astype(np.float64)).astype(np.float32)
+    dsub = X.shape[1] // M
+    books = np.empty((M, ncode, dsub), dtype=np.float32)
+    for s in range(M):
+        Z = R[:, s * dsub:(s + 1) * dsub]
+        W = Z[init_slots[C + s * ncode:C + (s + 1) * ncode]].copy()
+        for _ in range(pq_iters):
+            W = lloyd_update(Z, lloyd_assign(Z, W), W)
+        books[s] = W
+    return cent, books, a
+
+
+# ---------------------------------------------------------------------------
 # Batch-level wrappers over (sequence, KV head) units
 # ---------------------------------------------------------------------------
 
@@ -344,3 +414,16 @@ def oracle_append(k_cache, block_table, centroids, codebooks, n_indexed, n_new: 
         keys = unit_rows(k_cache, block_table[b], h, pos, page_size)
         res[(b, h)] = encode_keys(keys, centroids[b, h], codebooks[b, h])
     return res
+
+
+def oracle_train(k_cache, block_table, n_sink: int, n_train: int, init_slots, C: int, coarse_iters: int,
+                 pq_iters: int, page_size: int = 16, units=None):
+    """train_unit on the keys at positions [n_sink, n_sink + n_train) of every (b, h) unit.
+    init_slots: [B, Hkv, C + M*ncode] int. Returns {(b, h): (centroids, codebooks, assign)}."""
+    B = block_table.shape[0]
+    Hkv = k_cache.shape[1]
+    out = {}
+    for b, h in _units(B, Hkv, units):
+        keys = unit_rows(k_cache, block_table[b], h, n_sink + np.arange(n_train), page_size)
+        out[(b, h)] = train_unit(keys.astype(np.float32), init_slots[b, h], C, coarse_iters, pq_iters)
+    return out
