@@ -58,6 +58,9 @@ def parse_args(argv=None):
                          "or the 32-sequence batch at 32K")
     ap.add_argument("--append", action="store_true",
                     help="index-append cost on the Qwen3-30B-A3B-shaped workload (512-token batches)")
+    ap.add_argument("--train", action="store_true",
+                    help="index build cost: k-means centroids + PQ codebooks from raw keys, then encoding")
+    ap.add_argument("--train-iters", type=int, default=8, help="Lloyd iterations of each kind for --train")
     return ap.parse_args(argv)
 
 
@@ -539,6 +542,66 @@ def run_append(args):
                           "n_indexed": int(S.ix.n_indexed_host[0])}), flush=True)
 
 
+def run_train(args):
+    """Index build cost from raw prefill keys: Lloyd k-means centroids and residual PQ codebooks
+    (hsa_train_index), then encoding every indexed key (hsa_append_encode)."""
+    import torch
+    import sparse_long_context_pq_b200 as P
+    from synth import make_batch, train_init_slots, workload
+    from synth.device import index_tensors, kv_tensors
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    for name in ("llama8b_128k", "qwen30b_128k_append"):
+        w = workload(name)
+        bt = make_batch(w)
+        kv = P.PagedKV(**kv_tensors(bt, dev))
+        ix = P.PQIndex(**index_tensors(bt, dev, n_indexed=np.zeros(w.B, dtype=np.int32)))
+        n_train = w.n_indexed
+        init = torch.from_numpy(train_init_slots(w, n_train)).to(dev)
+        ws = P.workspace(P.hsa_train_workspace_bytes(kv, ix, n_train), dev)
+        ws_idx = P.workspace(P.hsa_index_workspace_bytes(), dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def timed(fn, reps):
+            t = []
+            for i in range(reps + 1):          # the first call is the warm-up
+                flush.zero_()
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                if i:
+                    t.append(a.elapsed_time(b))
+            return sum(t) / len(t)             # ms
+
+        def train(ci, pi):
+            return lambda: P.hsa_train_index(kv, ix, n_train, init, coarse_iters=ci, pq_iters=pi, workspace_buf=ws)
+
+        def encode():
+            ix.n_indexed.zero_()
+            ix.n_indexed_host.zero_()
+            P.hsa_append_encode(kv, ix, n_train, workspace_buf=ws_idx)
+
+        reps = max(1, min(args.steps, 3))
+        t0 = timed(train(0, 0), reps)           # seeding + one assignment + codeword seeding
+        t1 = timed(train(1, 0), reps)
+        tp = timed(train(0, 1), reps)
+        tf = timed(train(args.train_iters, args.train_iters), reps)
+        te = timed(encode, reps)
+        assert P.hsa_read_error(ws) == 0 and P.hsa_read_error(ws_idx) == 0
+        U = w.B * w.Hkv
+        assign_flop = 3.0 * U * n_train * w.C * w.D          # subtract + multiply-add per element
+        print(json.dumps({
+            "train": name, "units": U, "n_train": n_train, "C": w.C, "M": w.M, "ncode": w.ncode,
+            "coarse_iters": args.train_iters, "pq_iters": args.train_iters,
+            "train_ms": round(tf, 3), "coarse_iter_ms": round(t1 - t0, 3), "pq_iter_ms": round(tp - t0, 3),
+            "fixed_ms": round(t0, 3), "encode_ms": round(te, 3), "build_ms": round(tf + te, 3),
+            "assign_fp32_tflops": round(assign_flop / max(t0, 1e-9) / 1e9, 2),
+            "timing": "CUDA events, L2 flushed before every call, mean of %d after one warm-up" % reps,
+        }), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # reference arm: the float64 oracle on the host cores
 # ---------------------------------------------------------------------------
@@ -585,6 +648,8 @@ def main(argv=None):
         run_sweep_batch(args)
     elif args.append:
         run_append(args)
+    elif args.train:
+        run_train(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -206,6 +206,36 @@ hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* index,
 hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* index, int32_t n_new,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * hsa_train_index: trains the index's centroids and codebooks on raw keys, the step
+ * before hsa_append_encode when no trained index exists (rit.work PQ-HSA article,
+ * section "Как приблизительные оценки возвращают отброшенный контекст": the index
+ * is built after prefill; how its groups and codes are found is left open, and this
+ * is the plain Lloyd k-means).
+ *
+ * For every sequence b and KV head the training set is the keys at positions
+ * [s0, s0 + n_train) (training slot j = position s0 + j):
+ *   centroids: start at the keys of slots init_slots[0 .. C); coarse_iters times
+ *     assign every key to its nearest centroid (fp32 sum of squared differences,
+ *     ties to the lower index) and move each centroid to the mean of its keys (a
+ *     centroid with no keys keeps its value); then assign once more;
+ *   codebook s: start at the subspace-s residuals (key - centroid of its final
+ *     assignment) of slots init_slots[C + s*ncode .. C + (s+1)*ncode); pq_iters times
+ *     the same assign/move on the residuals' subspace s.
+ * init_slots: device int32 [B][Hkv][C + M*ncode], each in [0, n_train) (the caller
+ *   draws them; an out-of-range slot is replaced by 0 and flagged HSA_DEVERR_SLOT).
+ * assign_out: NULL, or device int32 [B][Hkv][n_train] receiving the final coarse
+ *   assignment. Writes index->centroids and index->codebooks only.
+ * Requires 1 <= n_train <= 1048560, s0 + n_train <= seq_lens_host[b], M = 16, dsub = 8,
+ * ncode = 256, C <= 4096, 0 <= iterations <= 1000; the workspace as
+ * hsa_train_workspace_bytes says (its error word is read by hsa_read_error).
+ */
+size_t hsa_train_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* index, int32_t n_train);
+hsa_status hsa_train_index(const hsa_kv_cache* kv, hsa_index* index, int32_t n_train,
+                           const int32_t* init_slots, int32_t coarse_iters, int32_t pq_iters,
+                           int32_t* assign_out, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
 /* ---- diagnostics --------------------------------------------------------- */
 
 /* Human-readable name of a status. */
@@ -221,6 +251,7 @@ hsa_status hsa_read_error(void* workspace, int32_t* error_host, cudaStream_t str
 #define HSA_DEVERR_CLUSTER 2       /* cluster id >= C */
 #define HSA_DEVERR_TIMEOUT 4       /* a bounded wait gave up */
 #define HSA_DEVERR_SELECT 8        /* top-k bookkeeping inconsistent */
+#define HSA_DEVERR_SLOT 16         /* a training slot outside [0, n_train) */
 
 /* ABI self-description: sizeof of the public structs, for bindings to check. */
 void hsa_abi_sizes(int64_t* kv_cache, int64_t* index, int64_t* decode_params, int64_t* debug);

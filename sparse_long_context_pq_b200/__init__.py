@@ -97,15 +97,19 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dense_decode.argtypes = [P(_KV), vp, vp, ctypes.c_float, vp, sz, vp]
     lib.hsa_build_from_codes.argtypes = [P(_KV), P(_Index), vp, sz, vp]
     lib.hsa_append_encode.argtypes = [P(_KV), P(_Index), i32, vp, sz, vp]
+    lib.hsa_train_workspace_bytes.argtypes = [P(_KV), P(_Index), i32]
+    lib.hsa_train_index.argtypes = [P(_KV), P(_Index), i32, vp, i32, i32, vp, vp, sz, vp]
     lib.hsa_decode_workspace_bytes.argtypes = [P(_KV), P(_Index)]
     lib.dense_decode_workspace_bytes.argtypes = [P(_KV)]
     lib.hsa_index_workspace_bytes.argtypes = []
     lib.hsa_read_error.argtypes = [vp, P(i32), vp]
     lib.hsa_strerror.argtypes = [ctypes.c_int]
     lib.hsa_abi_sizes.argtypes = [P(ctypes.c_int64)] * 4
-    for f in ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode", "hsa_read_error"):
+    for f in ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode", "hsa_read_error",
+              "hsa_train_index"):
         getattr(lib, f).restype = ctypes.c_int
-    for f in ("hsa_decode_workspace_bytes", "dense_decode_workspace_bytes", "hsa_index_workspace_bytes"):
+    for f in ("hsa_decode_workspace_bytes", "dense_decode_workspace_bytes", "hsa_index_workspace_bytes",
+              "hsa_train_workspace_bytes"):
         getattr(lib, f).restype = sz
     lib.hsa_strerror.restype = ctypes.c_char_p
     lib.hsa_abi_sizes.restype = None
@@ -330,6 +334,32 @@ def hsa_append_encode(kv: PagedKV, index: PQIndex, n_new: int, workspace_buf: Op
     st = load_library().hsa_append_encode(ctypes.byref(kvs), ctypes.byref(ixs), int(n_new),
                                           workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
     _check("hsa_append_encode", st)
+
+
+def hsa_train_workspace_bytes(kv: PagedKV, index: PQIndex, n_train: int) -> int:
+    kvs, ixs = kv.struct(), index.struct()
+    n = load_library().hsa_train_workspace_bytes(ctypes.byref(kvs), ctypes.byref(ixs), int(n_train))
+    if n == 0:
+        raise HSAError("hsa_train_workspace_bytes", 1)
+    return int(n)
+
+
+def hsa_train_index(kv: PagedKV, index: PQIndex, n_train: int, init_slots: torch.Tensor, *,
+                    coarse_iters: int = 8, pq_iters: int = 8, assign_out: Optional[torch.Tensor] = None,
+                    workspace_buf: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Train index.centroids / index.codebooks by Lloyd k-means on the keys at positions
+    [n_sink, n_sink + n_train) (see hsa_train_index in include/pqhsa.h).
+    init_slots: int32 [B, Hkv, C + 16 * 256] training slots seeding the centroids, then the codewords."""
+    assert init_slots.dtype == torch.int32 and init_slots.is_contiguous()
+    if assign_out is not None:
+        assert assign_out.dtype == torch.int32 and assign_out.is_contiguous()
+    kvs, ixs = kv.struct(), index.struct()
+    if workspace_buf is None:
+        workspace_buf = workspace(hsa_train_workspace_bytes(kv, index, n_train), index.centroids.device)
+    st = load_library().hsa_train_index(ctypes.byref(kvs), ctypes.byref(ixs), int(n_train), init_slots.data_ptr(),
+                                        int(coarse_iters), int(pq_iters), _ptr(assign_out),
+                                        workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
+    _check("hsa_train_index", st)
 
 
 def hsa_read_error(workspace_buf: torch.Tensor, stream=None) -> int:

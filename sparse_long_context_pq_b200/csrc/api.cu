@@ -571,4 +571,137 @@ hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_ne
   return HSA_OK;
 }
 
+// Training workspace: error header, assignment [U][n_train], centroid sums [U][C][D] and
+// counts [U][C], codeword sums [U][M][ncode][dsub] and counts [U][M][ncode].
+struct TrainLayout {
+  size_t assign, sums, counts, pq_sums, pq_counts, terms, cnorm, total;
+};
+// Longest training set: the fallback assignment launches one grid row per 32 keys (at most 65535).
+constexpr int32_t kMaxTrain = 65535 * 16;
+constexpr size_t kAssignTileN = 256;   // centroids per tensor-core tile
+
+// Tensor map over row-major [rows][128] bf16 (the centroid terms), box 64 x 256, 128-byte swizzle.
+bool make_rows_tmap(CUtensorMap* map, const void* base, size_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(kAssignTileN)};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static TrainLayout train_layout(int U, int C, int n_train) {
+  TrainLayout L;
+  size_t o = align_up(sizeof(WsHeader), 256);
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + bytes, 256);
+    return r;
+  };
+  L.assign = take(static_cast<size_t>(U) * n_train * sizeof(int32_t));
+  L.sums = take(static_cast<size_t>(U) * C * kD * sizeof(float));
+  L.counts = take(static_cast<size_t>(U) * C * sizeof(int32_t));
+  L.pq_sums = take(static_cast<size_t>(U) * kM * kNcode * kDsub * sizeof(float));
+  L.pq_counts = take(static_cast<size_t>(U) * kM * kNcode * sizeof(int32_t));
+  const size_t cpad = align_up(static_cast<size_t>(C), kAssignTileN);
+  L.terms = take(static_cast<size_t>(U) * 3 * cpad * kD * sizeof(uint16_t));
+  L.cnorm = take(static_cast<size_t>(U) * cpad * sizeof(float));
+  L.total = o;
+  return L;
+}
+
+size_t hsa_train_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix, int32_t n_train) {
+  if (!kv || !ix || n_train < 1 || ix->C < 1 || kv->B < 1 || kv->Hkv < 1) return 0;
+  return train_layout(kv->B * kv->Hkv, ix->C, n_train).total;
+}
+
+hsa_status hsa_train_index(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_train, const int32_t* init_slots,
+                           int32_t coarse_iters, int32_t pq_iters, int32_t* assign_out, void* ws,
+                           size_t ws_bytes, cudaStream_t stream) {
+  hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  if (!ix || !ix->centroids || !ix->codebooks || !init_slots) return HSA_ERR_INVALID_ARG;
+  if (ix->M != kM || ix->dsub != kDsub || ix->ncode != kNcode) return HSA_ERR_UNSUPPORTED;
+  if (ix->C < 1 || ix->n_sink < 0) return HSA_ERR_INVALID_ARG;
+  if (ix->C > kMaxClusters) return HSA_ERR_UNSUPPORTED;
+  if (n_train < 1 || coarse_iters < 0 || pq_iters < 0 || coarse_iters > 1000 || pq_iters > 1000)
+    return HSA_ERR_INVALID_ARG;
+  if (n_train > kMaxTrain) return HSA_ERR_UNSUPPORTED;   // grid rows of the codebook step
+  if (!aligned(ix->centroids, 16) || !aligned(ix->codebooks, 16) || !aligned(init_slots, 4) ||
+      (assign_out && !aligned(assign_out, 4)))
+    return HSA_ERR_ALIGNMENT;
+  for (int b = 0; b < kv->B; ++b)
+    if (static_cast<long long>(ix->n_sink) + n_train > kv->seq_lens_host[b]) return HSA_ERR_CAPACITY;
+  const int U = kv->B * kv->Hkv;
+  const TrainLayout L = train_layout(U, ix->C, n_train);
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HSA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  TrainParams p = {};
+  p.k_cache = static_cast<const uint16_t*>(kv->k_cache);
+  p.block_table = kv->block_table;
+  p.centroids = ix->centroids;
+  p.codebooks = ix->codebooks;
+  p.init_slots = init_slots;
+  p.assign = reinterpret_cast<int32_t*>(base + L.assign);
+  p.sums = reinterpret_cast<float*>(base + L.sums);
+  p.counts = reinterpret_cast<int32_t*>(base + L.counts);
+  p.pq_sums = reinterpret_cast<float*>(base + L.pq_sums);
+  p.pq_counts = reinterpret_cast<int32_t*>(base + L.pq_counts);
+  p.err = reinterpret_cast<int32_t*>(base);
+  p.B = kv->B;
+  p.Hkv = kv->Hkv;
+  p.C = ix->C;
+  p.n_sink = ix->n_sink;
+  p.n_train = n_train;
+  p.page_size = kv->page_size;
+  p.max_pages = kv->max_pages;
+  p.num_pages = kv->num_pages;
+  p.terms = reinterpret_cast<uint16_t*>(base + L.terms);
+  p.cnorm = reinterpret_cast<float*>(base + L.cnorm);
+  p.Cpad = static_cast<int>(align_up(static_cast<size_t>(ix->C), kAssignTileN));
+  p.p0 = ix->n_sink / 8 * 8;
+  p.tiles_per_unit = (ix->n_sink + n_train - p.p0 + 127) / 128;
+  p.items = U * p.tiles_per_unit;
+
+  // Nearest-centroid assignment: on the tensor cores (keys streamed by TMA in 8-row
+  // boxes, so pages of at least 8 rows); 4-row pages use the CUDA-core kernel.
+  const bool mma = kv->page_size >= 8;
+  CUtensorMap tmk = {}, tmb = {};
+  int grid = 0;
+  if (mma) {
+    const DeviceInfo* di = device_info();
+    if (!di) return HSA_ERR_CUDA;
+    if (!make_kv_tmap(&tmk, kv->k_cache, kv, 8) ||
+        !make_rows_tmap(&tmb, p.terms, static_cast<size_t>(U) * 3 * p.Cpad))
+      return HSA_ERR_CUDA;
+    grid = std::min(p.items, di->sms);
+  }
+  auto assign = [&]() -> cudaError_t {
+    if (!mma) return launch_train_assign(p, stream);
+    cudaError_t e = launch_centroid_terms(p, stream);
+    if (e != cudaSuccess) return e;
+    return launch_assign_mma(tmk, tmb, p, grid, stream);
+  };
+
+  // the sums start at zero; every update clears what it used
+  RET_CUDA(cudaMemsetAsync(base + L.sums, 0, L.terms - L.sums, stream));
+  RET_CUDA(launch_train_init(p, stream));
+  for (int it = 0; it < coarse_iters; ++it) {
+    RET_CUDA(assign());
+    RET_CUDA(launch_train_accumulate(p, stream));
+    RET_CUDA(launch_train_update(p, stream));
+  }
+  p.assign_out = assign_out;   // the final assignment is the one returned
+  RET_CUDA(assign());
+  RET_CUDA(launch_train_pq_init(p, stream));
+  for (int it = 0; it < pq_iters; ++it) {
+    RET_CUDA(launch_train_pq_step(p, stream));
+    RET_CUDA(launch_train_pq_update(p, stream));
+  }
+  return HSA_OK;
+}
+
 }  // extern "C"

@@ -326,6 +326,241 @@ int grid_for(size_t work, int threads) {
   return static_cast<int>(g);
 }
 
+// ---------------------------------------------------------------------------
+// Index training. The article builds the index after prefill and leaves the training
+// open; the reading here is the plain Lloyd k-means: coarse centroids on the unit's keys
+// at positions [n_sink, n_sink + n_train), then per subspace a codebook on the residuals
+// (key minus its centroid). Initial centres are the given training rows. Distances are
+// direct sums of squared differences in fp32, ties to the lower index; a centre that
+// gets no rows keeps its value.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ const uint16_t* train_key(const TrainParams& p, int b, int h, int slot) {
+  if (slot < 0 || slot >= p.n_train) {
+    record_error(p.err, HSA_DEVERR_SLOT);
+    slot = 0;
+  }
+  const int pos = p.n_sink + slot;
+  const int lp = pos / p.page_size;
+  const int page = lp < p.max_pages ? p.block_table[static_cast<size_t>(b) * p.max_pages + lp] : -1;
+  if (page < 0 || page >= p.num_pages) {
+    record_error(p.err, HSA_DEVERR_PAGE);
+    return nullptr;
+  }
+  return p.k_cache + ((static_cast<size_t>(page) * p.Hkv + h) * p.page_size + (pos % p.page_size)) * kD;
+}
+
+__device__ __forceinline__ size_t init_stride(const TrainParams& p) {
+  return static_cast<size_t>(p.C) + static_cast<size_t>(kM) * kNcode;
+}
+
+// Warp per centroid: centroid c = the key of training slot init_slots[c].
+__global__ void __launch_bounds__(256) train_init_kernel(TrainParams p) {
+  const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.y * 8 + warp;
+  if (c >= p.C) return;
+  const uint16_t* row = train_key(p, b, h, p.init_slots[u * init_stride(p) + c]);
+  uint2 raw = make_uint2(0, 0);
+  if (row) raw = *reinterpret_cast<const uint2*>(row + lane * 4);
+  *reinterpret_cast<float4*>(p.centroids + (static_cast<size_t>(u) * p.C + c) * kD + lane * 4) =
+      make_float4(bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y));
+}
+
+// Nearest centroid of 32 training keys per CTA: lane t of every warp holds key t in
+// registers; warp w scans centroids w, w + 8, ...; the 8 warps' best are merged.
+__global__ void __launch_bounds__(256, 1) train_assign_kernel(TrainParams p) {
+  __shared__ float bd[8][32];
+  __shared__ int bc[8][32];
+  const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.y * 32 + lane;
+  const bool valid = j < p.n_train;
+  float kf[kD];
+  const uint16_t* row = valid ? train_key(p, b, h, j) : nullptr;
+#pragma unroll
+  for (int c = 0; c < kD / 8; ++c) {
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (row) raw = *reinterpret_cast<const uint4*>(row + c * 8);
+    kf[c * 8 + 0] = bf16lo(raw.x);
+    kf[c * 8 + 1] = bf16hi(raw.x);
+    kf[c * 8 + 2] = bf16lo(raw.y);
+    kf[c * 8 + 3] = bf16hi(raw.y);
+    kf[c * 8 + 4] = bf16lo(raw.z);
+    kf[c * 8 + 5] = bf16hi(raw.z);
+    kf[c * 8 + 6] = bf16lo(raw.w);
+    kf[c * 8 + 7] = bf16hi(raw.w);
+  }
+  const float* cent = p.centroids + static_cast<size_t>(u) * p.C * kD;
+  float best = INFINITY;
+  int besti = 0x7fffffff;
+  for (int c = warp; c < p.C; c += 8) {
+    const float4* cr = reinterpret_cast<const float4*>(cent + static_cast<size_t>(c) * kD);
+    float dist = 0.f;
+#pragma unroll
+    for (int q4 = 0; q4 < kD / 4; ++q4) {
+      const float4 cv = __ldg(cr + q4);
+      float t0 = __fsub_rn(kf[q4 * 4 + 0], cv.x);
+      dist = fmaf(t0, t0, dist);
+      t0 = __fsub_rn(kf[q4 * 4 + 1], cv.y);
+      dist = fmaf(t0, t0, dist);
+      t0 = __fsub_rn(kf[q4 * 4 + 2], cv.z);
+      dist = fmaf(t0, t0, dist);
+      t0 = __fsub_rn(kf[q4 * 4 + 3], cv.w);
+      dist = fmaf(t0, t0, dist);
+    }
+    if (dist < best) {
+      best = dist;
+      besti = c;
+    }
+  }
+  bd[warp][lane] = best;
+  bc[warp][lane] = besti;
+  __syncthreads();
+  if (warp == 0 && valid) {
+    float bb = bd[0][lane];
+    int bi = bc[0][lane];
+    for (int w = 1; w < 8; ++w) {
+      const float d = bd[w][lane];
+      const int ci = bc[w][lane];
+      if (d < bb || (d == bb && ci < bi)) {
+        bb = d;
+        bi = ci;
+      }
+    }
+    if (bi >= p.C || bi < 0) bi = 0;   // NaN keys only
+    p.assign[static_cast<size_t>(u) * p.n_train + j] = bi;
+    if (p.assign_out) p.assign_out[static_cast<size_t>(u) * p.n_train + j] = bi;
+  }
+}
+
+// Warp per training key: add it to its centre's sum and count.
+__global__ void __launch_bounds__(256) train_accumulate_kernel(TrainParams p) {
+  const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = blockIdx.y * 64 + warp; j < min(p.n_train, (static_cast<int>(blockIdx.y) + 1) * 64); j += 8) {
+    const int a = p.assign[static_cast<size_t>(u) * p.n_train + j];
+    const uint16_t* row = train_key(p, b, h, j);
+    if (!row) continue;
+    const uint2 raw = *reinterpret_cast<const uint2*>(row + lane * 4);
+    atomicAdd(reinterpret_cast<float4*>(p.sums + (static_cast<size_t>(u) * p.C + a) * kD + lane * 4),
+              make_float4(bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y)));
+    if (lane == 0) atomicAdd(p.counts + static_cast<size_t>(u) * p.C + a, 1);
+  }
+}
+
+// centre = sum / count where the centre got rows (else unchanged); then clear the sums.
+__global__ void train_update_kernel(float* centres, float* sums, int32_t* counts, size_t n, int dim) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int c = counts[i / dim];
+    if (c > 0) centres[i] = __fdiv_rn(sums[i], static_cast<float>(c));
+    sums[i] = 0.f;
+  }
+}
+__global__ void train_clear_counts_kernel(int32_t* counts, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    counts[i] = 0;
+}
+
+// Thread per codeword m of subspace s: its initial value is the subspace-s residual of
+// training slot init_slots[C + s * ncode + m] under the final coarse assignment.
+__global__ void __launch_bounds__(256) train_pq_init_kernel(TrainParams p) {
+  const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
+  const int s = blockIdx.y, m = threadIdx.x;
+  int slot = p.init_slots[u * init_stride(p) + p.C + s * kNcode + m];
+  const uint16_t* row = train_key(p, b, h, slot);
+  if (slot < 0 || slot >= p.n_train) slot = 0;
+  const int a = p.assign[static_cast<size_t>(u) * p.n_train + slot];
+  uint4 raw = make_uint4(0, 0, 0, 0);
+  if (row) raw = *reinterpret_cast<const uint4*>(row + s * kDsub);
+  const float kv8[8] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y),
+                        bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w)};
+  const float* ca = p.centroids + (static_cast<size_t>(u) * p.C + a) * kD + s * kDsub;
+  float* dst = p.codebooks + ((static_cast<size_t>(u) * kM + s) * kNcode + m) * kDsub;
+#pragma unroll
+  for (int d = 0; d < kDsub; ++d) dst[d] = __fsub_rn(kv8[d], ca[d]);
+}
+
+// One Lloyd assignment of the residual sub-vectors. A CTA takes kPqGroup subspaces of
+// one unit and kPqKeys training keys: the group's codebooks and its partial sums live
+// in shared memory, each warp works on one subspace (so every codeword read is a
+// broadcast), a lane per key finds the nearest codeword and adds the residual
+// sub-vector to the shared sums; the CTA then adds its sums to the global ones.
+constexpr int kPqGroup = 4;
+constexpr int kPqKeys = 4096;
+constexpr int kPqThreads = 256;
+constexpr size_t kPqSmem = static_cast<size_t>(kPqGroup) * kNcode * (2 * kDsub + 1) * sizeof(float);
+
+__global__ void __launch_bounds__(kPqThreads) train_pq_step_kernel(TrainParams p) {
+  extern __shared__ __align__(16) float pq_sh[];
+  float* book = pq_sh;                                   // [kPqGroup][ncode][dsub]
+  float* sums = book + kPqGroup * kNcode * kDsub;        // [kPqGroup][ncode][dsub]
+  int* cnt = reinterpret_cast<int*>(sums + kPqGroup * kNcode * kDsub);   // [kPqGroup][ncode]
+  const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
+  const int s0 = blockIdx.y * kPqGroup;
+  const float* gbook = p.codebooks + (static_cast<size_t>(u) * kM + s0) * kNcode * kDsub;
+  for (int i = threadIdx.x; i < kPqGroup * kNcode * kDsub / 4; i += kPqThreads) {
+    reinterpret_cast<float4*>(book)[i] = reinterpret_cast<const float4*>(gbook)[i];
+    reinterpret_cast<float4*>(sums)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int i = threadIdx.x; i < kPqGroup * kNcode; i += kPqThreads) cnt[i] = 0;
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sl = warp % kPqGroup, s = s0 + sl;
+  const float4* wb = reinterpret_cast<const float4*>(book + sl * kNcode * kDsub);
+  const int j_end = min(p.n_train, static_cast<int>(blockIdx.z + 1) * kPqKeys);
+  for (int j = blockIdx.z * kPqKeys + (warp / kPqGroup) * 32 + lane; j < j_end;
+       j += (kPqThreads / 32 / kPqGroup) * 32) {
+    const uint16_t* row = train_key(p, b, h, j);
+    if (!row) continue;
+    const int a = p.assign[static_cast<size_t>(u) * p.n_train + j];
+    const uint4 raw = *reinterpret_cast<const uint4*>(row + s * kDsub);
+    const float kv8[8] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y),
+                          bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w)};
+    const float4* ca = reinterpret_cast<const float4*>(p.centroids + (static_cast<size_t>(u) * p.C + a) * kD +
+                                                       s * kDsub);
+    const float4 c0 = __ldg(ca), c1 = __ldg(ca + 1);
+    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    float r[kDsub];
+#pragma unroll
+    for (int d = 0; d < kDsub; ++d) r[d] = __fsub_rn(kv8[d], cv[d]);
+    float bb = INFINITY;
+    int bm = 0;
+#pragma unroll 4
+    for (int m = 0; m < kNcode; ++m) {
+      const float4 x = wb[2 * m], y = wb[2 * m + 1];
+      const float w8[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+      float dist = 0.f;
+#pragma unroll
+      for (int d = 0; d < kDsub; ++d) {
+        const float t0 = __fsub_rn(r[d], w8[d]);
+        dist = fmaf(t0, t0, dist);
+      }
+      if (dist < bb) {
+        bb = dist;
+        bm = m;
+      }
+    }
+    float* dst = sums + (sl * kNcode + bm) * kDsub;
+#pragma unroll
+    for (int d = 0; d < kDsub; ++d) atomicAdd(dst + d, r[d]);
+    atomicAdd(cnt + sl * kNcode + bm, 1);
+  }
+  __syncthreads();
+  float* gsum = p.pq_sums + (static_cast<size_t>(u) * kM + s0) * kNcode * kDsub;
+  int* gcnt = p.pq_counts + (static_cast<size_t>(u) * kM + s0) * kNcode;
+  for (int i = threadIdx.x; i < kPqGroup * kNcode; i += kPqThreads) {
+    const int c = cnt[i];
+    if (c == 0) continue;
+    const float4* src = reinterpret_cast<const float4*>(sums + i * kDsub);
+    atomicAdd(reinterpret_cast<float4*>(gsum + i * kDsub), src[0]);
+    atomicAdd(reinterpret_cast<float4*>(gsum + i * kDsub + 4), src[1]);
+    atomicAdd(gcnt + i, c);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_zero_stats(const IndexParams& p, cudaStream_t stream) {
@@ -365,6 +600,53 @@ cudaError_t launch_list_append(const IndexParams& p, cudaStream_t stream) {
 cudaError_t launch_means(const IndexParams& p, cudaStream_t stream) {
   const size_t work = static_cast<size_t>(p.B) * p.Hkv * p.C * kD;
   means_kernel<<<grid_for(work, 256), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_train_init(const TrainParams& p, cudaStream_t stream) {
+  train_init_kernel<<<dim3(p.B * p.Hkv, (p.C + 7) / 8), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_train_assign(const TrainParams& p, cudaStream_t stream) {
+  train_assign_kernel<<<dim3(p.B * p.Hkv, (p.n_train + 31) / 32), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_train_accumulate(const TrainParams& p, cudaStream_t stream) {
+  train_accumulate_kernel<<<dim3(p.B * p.Hkv, (p.n_train + 63) / 64), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+// New centroids from the sums (clears sums and counts for the next iteration).
+cudaError_t launch_train_update(const TrainParams& p, cudaStream_t stream) {
+  const size_t n = static_cast<size_t>(p.B) * p.Hkv * p.C * kD;
+  train_update_kernel<<<grid_for(n, 256), 256, 0, stream>>>(p.centroids, p.sums, p.counts, n, kD);
+  const size_t nc = static_cast<size_t>(p.B) * p.Hkv * p.C;
+  train_clear_counts_kernel<<<grid_for(nc, 256), 256, 0, stream>>>(p.counts, nc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_train_pq_init(const TrainParams& p, cudaStream_t stream) {
+  train_pq_init_kernel<<<dim3(p.B * p.Hkv, kM), kNcode, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_train_pq_step(const TrainParams& p, cudaStream_t stream) {
+  static_assert(kM % kPqGroup == 0, "subspace groups must tile the subspaces");
+  cudaError_t e = ensure_dyn_smem<train_pq_step_kernel>(kPqSmem);
+  if (e != cudaSuccess) return e;
+  train_pq_step_kernel<<<dim3(p.B * p.Hkv, kM / kPqGroup, (p.n_train + kPqKeys - 1) / kPqKeys), kPqThreads, kPqSmem,
+                         stream>>>(p);
+  return cudaGetLastError();
+}
+
+// New codewords from the sums (clears sums and counts for the next iteration).
+cudaError_t launch_train_pq_update(const TrainParams& p, cudaStream_t stream) {
+  const size_t n = static_cast<size_t>(p.B) * p.Hkv * kM * kNcode * kDsub;
+  train_update_kernel<<<grid_for(n, 256), 256, 0, stream>>>(p.codebooks, p.pq_sums, p.pq_counts, n, kDsub);
+  const size_t nc = static_cast<size_t>(p.B) * p.Hkv * kM * kNcode;
+  train_clear_counts_kernel<<<grid_for(nc, 256), 256, 0, stream>>>(p.pq_counts, nc);
   return cudaGetLastError();
 }
 

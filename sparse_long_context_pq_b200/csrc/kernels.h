@@ -209,4 +209,37 @@ cudaError_t launch_means(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_list_reset(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_list_append(const IndexParams& p, cudaStream_t stream);
 
+// ---- index training (k-means centroids, residual PQ codebooks) --------------
+struct TrainParams {
+  const uint16_t* k_cache;
+  const int32_t* block_table;
+  float* centroids;            // [U][C][D] written
+  float* codebooks;            // [U][M][ncode][dsub] written
+  const int32_t* init_slots;   // [U][C + M * ncode] training slots seeding the centres
+  int32_t* assign;             // [U][n_train] coarse assignment (workspace)
+  int32_t* assign_out;         // [U][n_train] final coarse assignment, or null
+  float* sums;                 // [U][C][D]
+  int32_t* counts;             // [U][C]
+  float* pq_sums;              // [U][M][ncode][dsub]
+  int32_t* pq_counts;          // [U][M][ncode]
+  int32_t* err;
+  uint16_t* terms;             // [U][3][Cpad][D] bf16 terms of the centroids (tensor-core assignment)
+  float* cnorm;                // [U][Cpad] |c|^2, +inf for the padding rows
+  int B, Hkv, C, n_sink, n_train, page_size, max_pages, num_pages;
+  int Cpad;                    // C rounded up to the 256-centroid tile
+  int p0;                      // first position of the first key tile (n_sink rounded down to 8)
+  int tiles_per_unit, items;   // 128-key tiles per unit, units x tiles
+};
+cudaError_t launch_train_init(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_train_assign(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_train_accumulate(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_train_update(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_train_pq_init(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_train_pq_step(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_train_pq_update(const TrainParams& p, cudaStream_t stream);
+size_t assign_mma_smem_bytes();
+cudaError_t launch_centroid_terms(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_assign_mma(const CUtensorMap& tmk, const CUtensorMap& tmb, const TrainParams& p, int grid,
+                              cudaStream_t stream);
+
 }  // namespace pqhsa

@@ -14,4 +14,5 @@ from .workloads import (  # noqa: F401
     make_unit,
     f32_to_bf16_bits,
     bf16_bits_to_f32,
+    train_init_slots,
 )

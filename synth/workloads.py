@@ -31,7 +31,7 @@ from typing import Dict, List, Optional
 import numpy as np
 
 # Stream purposes.
-_IDX, _TOK, _VAL, _QRY, _PAGES = 0, 1, 2, 3, 4
+_IDX, _TOK, _VAL, _QRY, _PAGES, _TRAIN = 0, 1, 2, 3, 4, 5
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -131,6 +131,17 @@ WORKLOADS: Dict[str, Workload] = {
                                     n_sink=16, n_recent=1024, n_needles=8,
                                     extra_tokens=2048, append_batch=512),
 }
+
+
+def train_init_slots(w: Workload, n_train: int, seed: int = 0) -> np.ndarray:
+    """Training slots seeding an index's centres, the random draw both sides take as input:
+    int32 [B, Hkv, C + M * ncode] uniform in [0, n_train) (centroids first, then the
+    codewords of every subspace), per-unit seeded."""
+    out = np.empty((w.B, w.Hkv, w.C + w.M * w.ncode), dtype=np.int32)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            out[b, h] = _rng(w, b, h, _TRAIN, seed).integers(0, n_train, size=out.shape[2])
+    return out
 
 
 def workload(name: str, **changes) -> Workload:

@@ -138,3 +138,35 @@ def test_dense_rejects_bad_args(lib):
     kv, lens = _kv()
     assert lib.dense_decode(ctypes.byref(kv), FAKE + 4, FAKE, ctypes.c_float(1.0), FAKE, 1 << 30, None) == 4
     assert lib.dense_decode(ctypes.byref(kv), FAKE, FAKE, ctypes.c_float(1.0), FAKE, 8, None) == 5
+
+
+def _train(lib, kv, ix, n_train=40, coarse=2, pq=2, ws_bytes=1 << 30, init=FAKE, assign_out=None):
+    return lib.hsa_train_index(ctypes.byref(kv), ctypes.byref(ix), n_train, init, coarse, pq, assign_out, FAKE,
+                               ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_train=0), 1),
+    (dict(coarse=-1), 1),
+    (dict(pq=1001), 1),
+    (dict(init=None), 1),
+    (dict(n_train=97), 3),             # n_sink 4 + 97 > T = 100
+    (dict(init=FAKE + 2), 4),          # init slots are 4-byte words
+    (dict(assign_out=FAKE + 2), 4),
+    (dict(ws_bytes=64), 5),
+])
+def test_train_rejects_bad_args(lib, kw, status):
+    kv, lens = _kv()
+    ix, nh = _ix()
+    assert _train(lib, kv, ix, **kw) == status
+
+
+def test_train_rejects_unsupported_index(lib):
+    kv, lens = _kv(seq=2 << 20, max_pages=(2 << 20) // 16, num_pages=(2 << 20) // 16)
+    ix, nh = _ix(cap=2 << 20)
+    assert _train(lib, kv, ix, n_train=65535 * 16 + 1) == 2   # beyond the longest training set
+    ix2, nh2 = _ix(M=8, dsub=16)
+    kv2, lens2 = _kv()
+    assert _train(lib, kv2, ix2) == 2
+    assert lib.hsa_train_workspace_bytes(ctypes.byref(kv2), ctypes.byref(ix), 0) == 0
+    assert lib.hsa_train_workspace_bytes(ctypes.byref(kv2), ctypes.byref(ix), 40) % 256 == 0
