@@ -177,8 +177,12 @@ hsa_status dense_decode_static(const hsa_kv_cache* kv, const float* q, float* ou
 
 /* ---- index maintenance --------------------------------------------------- */
 
-/* Workspace bytes of hsa_build_from_codes / hsa_append_encode (error word only). */
-size_t hsa_index_workspace_bytes(void);
+/* Workspace bytes of hsa_append_encode of n_new tokens (n_new = 0: of
+ * hsa_build_from_codes, the error word only). With pages of at least 8 rows the
+ * encoding's nearest-centroid search runs on the tensor cores and the workspace also
+ * holds the centroids as bf16 terms [B*Hkv][3][C rounded up to 256][128], their squared
+ * norms and the new tokens' assignment [B*Hkv][n_new]. Never 0. */
+size_t hsa_index_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* index, int32_t n_new);
 
 /*
  * Index build after prefill from caller-provided codes (same article, section
@@ -194,14 +198,19 @@ hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* index,
  * Batched encoding of new tokens into the index (same article: new tokens are
  * kept outside the index and added in batches). For every sequence b and KV
  * head, positions [s0 + N_b, s0 + N_b + n_new) are encoded:
- *   a = argmin_c sum_d (k_d - centroid_c,d)^2 (fp32, ties to the lower c),
- *   code_s = argmin_m sum_{d<dsub} (k - centroid_a)_{s*dsub+d} - codeword_s,m,d)^2,
+ *   a = argmin_c sum_d (k_d - centroid_c,d)^2 (ties to the lower c),
+ *   code_s = argmin_m sum_{d<dsub} (k - centroid_a)_{s*dsub+d} - codeword_s,m,d)^2
+ *   (ties to the lower m). The decisions are taken in fp32: with pages of at least 8
+ *   rows as |c|^2 - 2 k.c on the tensor cores (centroids as three bf16 terms, fp32
+ *   accumulation) and |w|^2 - 2 r.w for the codewords; results can differ from an
+ *   exact evaluation only where two candidates' distances nearly tie.
  * written to slots [N_b, N_b + n_new); the members' values are added to sum_v
  * and count, mean_v is recomputed, the new members join their clusters' lists
  * (list_codes / list_slot), and n_indexed (device and host) grows by n_new.
  * Requires s0 + N_b + n_new <= seq_lens_host[b] and N_b + n_new <= cap, and
  * lists built by earlier calls (a unit with n_indexed = 0 starts them afresh).
- * With n_indexed = 0 this is the whole index build from raw keys.
+ * With n_indexed = 0 this is the whole index build from raw keys. The workspace is
+ * hsa_index_workspace_bytes(kv, index, n_new) bytes.
  */
 hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* index, int32_t n_new,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);

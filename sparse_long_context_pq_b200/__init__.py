@@ -101,7 +101,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.hsa_train_index.argtypes = [P(_KV), P(_Index), i32, vp, i32, i32, vp, vp, sz, vp]
     lib.hsa_decode_workspace_bytes.argtypes = [P(_KV), P(_Index)]
     lib.dense_decode_workspace_bytes.argtypes = [P(_KV)]
-    lib.hsa_index_workspace_bytes.argtypes = []
+    lib.hsa_index_workspace_bytes.argtypes = [P(_KV), P(_Index), i32]
     lib.hsa_read_error.argtypes = [vp, P(i32), vp]
     lib.hsa_strerror.argtypes = [ctypes.c_int]
     lib.hsa_abi_sizes.argtypes = [P(ctypes.c_int64)] * 4
@@ -264,8 +264,10 @@ def dense_decode_workspace_bytes(kv: PagedKV) -> int:
     return int(n)
 
 
-def hsa_index_workspace_bytes() -> int:
-    return int(load_library().hsa_index_workspace_bytes())
+def hsa_index_workspace_bytes(kv: PagedKV, index: PQIndex, n_new: int = 0) -> int:
+    """Workspace of hsa_append_encode(kv, index, n_new) (n_new = 0: of hsa_build_from_codes)."""
+    kvs, ixs = kv.struct(), index.struct()
+    return int(load_library().hsa_index_workspace_bytes(ctypes.byref(kvs), ctypes.byref(ixs), int(n_new)))
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
@@ -319,7 +321,7 @@ def hsa_build_from_codes(kv: PagedKV, index: PQIndex, workspace_buf: Optional[to
     """count / sum_v / mean_v of every cluster from the caller's codes and ids."""
     kvs, ixs = kv.struct(), index.struct()
     if workspace_buf is None:
-        workspace_buf = workspace(hsa_index_workspace_bytes(), index.centroids.device)
+        workspace_buf = workspace(hsa_index_workspace_bytes(kv, index), index.centroids.device)
     st = load_library().hsa_build_from_codes(ctypes.byref(kvs), ctypes.byref(ixs), workspace_buf.data_ptr(),
                                              workspace_buf.numel(), _stream(stream))
     _check("hsa_build_from_codes", st)
@@ -330,7 +332,7 @@ def hsa_append_encode(kv: PagedKV, index: PQIndex, n_new: int, workspace_buf: Op
     """Encode the next n_new tokens of every sequence into the index (advances n_indexed)."""
     kvs, ixs = kv.struct(), index.struct()
     if workspace_buf is None:
-        workspace_buf = workspace(hsa_index_workspace_bytes(), index.centroids.device)
+        workspace_buf = workspace(hsa_index_workspace_bytes(kv, index, n_new), index.centroids.device)
     st = load_library().hsa_append_encode(ctypes.byref(kvs), ctypes.byref(ixs), int(n_new),
                                           workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
     _check("hsa_append_encode", st)

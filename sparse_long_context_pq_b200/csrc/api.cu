@@ -221,7 +221,7 @@ size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv) {
   return dense_layout_bytes(kv->B * kv->Hkv, kv->Hq / kv->Hkv);
 }
 
-size_t hsa_index_workspace_bytes(void) { return sizeof(WsHeader); }
+
 
 int64_t hsa_index_list_slots(int32_t cap, int32_t C) {
   if (cap < 1 || C < 1) return 0;
@@ -487,6 +487,77 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   return HSA_OK;
 }
 
+// Longest training set: the fallback assignment launches one grid row per 32 keys (at most 65535).
+constexpr int32_t kMaxTrain = 65535 * 16;
+constexpr size_t kAssignTileN = 256;   // centroids per tensor-core tile
+
+// Tensor map over row-major [rows][128] bf16 (the centroid terms), box 64 x 256, 128-byte swizzle.
+bool make_rows_tmap(CUtensorMap* map, const void* base, size_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(kAssignTileN)};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core nearest-centroid search of keys [0, n) of every unit (key j of sequence b at
+// position n_sink + slot0[b] + j), p.assign receiving the centroid index: tensor maps,
+// tile counts and grid. lead = the largest (n_sink + slot0[b]) mod 8 over the sequences.
+static hsa_status plan_mma_assign(const hsa_kv_cache* kv, TrainParams& p, int lead, CUtensorMap* tmk,
+                                  CUtensorMap* tmb, int* grid) {
+  const DeviceInfo* di = device_info();
+  if (!di) return HSA_ERR_CUDA;
+  const int U = kv->B * kv->Hkv;
+  p.Cpad = static_cast<int>(align_up(static_cast<size_t>(p.C), kAssignTileN));
+  p.tiles_per_unit = (lead + p.n_train + 127) / 128;
+  p.items = U * p.tiles_per_unit;
+  if (!make_kv_tmap(tmk, kv->k_cache, kv, 8) || !make_rows_tmap(tmb, p.terms, static_cast<size_t>(U) * 3 * p.Cpad))
+    return HSA_ERR_CUDA;
+  *grid = std::min(p.items, di->sms);
+  return HSA_OK;
+}
+
+static cudaError_t run_mma_assign(const CUtensorMap& tmk, const CUtensorMap& tmb, const TrainParams& p, int grid,
+                                  cudaStream_t stream) {
+  cudaError_t e = launch_centroid_terms(p, stream);
+  if (e != cudaSuccess) return e;
+  return launch_assign_mma(tmk, tmb, p, grid, stream);
+}
+
+// Encoding workspace (tensor-core path): error header, centroid terms [U][3][Cpad][D]
+// bf16, |c|^2 [U][Cpad], assignment [U][n_new].
+struct EncodeLayout {
+  size_t terms, cnorm, assign, total;
+};
+static EncodeLayout encode_layout(int U, int C, int n_new) {
+  EncodeLayout L;
+  size_t o = align_up(sizeof(WsHeader), 256);
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + bytes, 256);
+    return r;
+  };
+  const size_t cpad = align_up(static_cast<size_t>(C), kAssignTileN);
+  L.terms = take(static_cast<size_t>(U) * 3 * cpad * kD * sizeof(uint16_t));
+  L.cnorm = take(static_cast<size_t>(U) * cpad * sizeof(float));
+  L.assign = take(static_cast<size_t>(U) * n_new * sizeof(int32_t));
+  L.total = o;
+  return L;
+}
+
+// Encoding runs on the tensor cores when the cache has pages of at least 8 rows.
+static bool mma_encode(const hsa_kv_cache* kv, int n_new) { return kv->page_size >= 8 && n_new > 0; }
+
+size_t hsa_index_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix, int32_t n_new) {
+  if (!kv || !ix || kv->B < 1 || kv->Hkv < 1 || ix->C < 1 || n_new < 0) return sizeof(WsHeader);
+  if (!mma_encode(kv, n_new)) return sizeof(WsHeader);
+  return encode_layout(kv->B * kv->Hkv, ix->C, n_new).total;
+}
+
 static IndexParams index_params(const hsa_kv_cache* kv, hsa_index* ix, void* ws) {
   IndexParams p = {};
   p.k_cache = static_cast<const uint16_t*>(kv->k_cache);
@@ -525,7 +596,7 @@ hsa_status hsa_build_from_codes(const hsa_kv_cache* kv, hsa_index* ix, void* ws,
   st = check_index(kv, ix, true);
   if (st != HSA_OK) return st;
   if (!ix->sum_v || !ix->count) return HSA_ERR_INVALID_ARG;
-  if (!ws || !aligned(ws, 256) || ws_bytes < hsa_index_workspace_bytes()) return HSA_ERR_WORKSPACE;
+  if (!ws || !aligned(ws, 256) || ws_bytes < sizeof(WsHeader)) return HSA_ERR_WORKSPACE;
   int nmax = 0;
   for (int b = 0; b < kv->B; ++b) nmax = std::max(nmax, ix->n_indexed_host[b]);
   IndexParams p = index_params(kv, ix, ws);
@@ -549,7 +620,7 @@ hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_ne
   if (st != HSA_OK) return st;
   if (!ix->sum_v || !ix->count) return HSA_ERR_INVALID_ARG;
   if (n_new < 0) return HSA_ERR_INVALID_ARG;
-  if (!ws || !aligned(ws, 256) || ws_bytes < hsa_index_workspace_bytes()) return HSA_ERR_WORKSPACE;
+  if (!ws || !aligned(ws, 256) || ws_bytes < hsa_index_workspace_bytes(kv, ix, n_new)) return HSA_ERR_WORKSPACE;
   for (int b = 0; b < kv->B; ++b) {
     const long long N = ix->n_indexed_host[b];
     if (N + n_new > ix->cap) return HSA_ERR_CAPACITY;
@@ -562,7 +633,39 @@ hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_ne
   p.bump_indexed = 1;
   p.zero_if_empty = 1;
   RET_CUDA(launch_zero_stats(p, stream));
-  RET_CUDA(launch_encode(p, n_new, stream));
+  if (mma_encode(kv, n_new)) {
+    const int U = kv->B * kv->Hkv;
+    const EncodeLayout L = encode_layout(U, ix->C, n_new);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    TrainParams t = {};
+    t.k_cache = static_cast<const uint16_t*>(kv->k_cache);
+    t.block_table = kv->block_table;
+    t.centroids = ix->centroids;
+    t.codebooks = ix->codebooks;
+    t.assign = reinterpret_cast<int32_t*>(base + L.assign);
+    t.err = static_cast<int32_t*>(ws);
+    t.terms = reinterpret_cast<uint16_t*>(base + L.terms);
+    t.cnorm = reinterpret_cast<float*>(base + L.cnorm);
+    t.slot0 = ix->n_indexed;   // read before the mean pass advances it
+    t.B = kv->B;
+    t.Hkv = kv->Hkv;
+    t.C = ix->C;
+    t.n_sink = ix->n_sink;
+    t.n_train = n_new;
+    t.page_size = kv->page_size;
+    t.max_pages = kv->max_pages;
+    t.num_pages = kv->num_pages;
+    int lead = 0;
+    for (int b = 0; b < kv->B; ++b) lead = std::max(lead, (ix->n_sink + ix->n_indexed_host[b]) & 7);
+    CUtensorMap tmk = {}, tmb = {};
+    int grid = 0;
+    st = plan_mma_assign(kv, t, lead, &tmk, &tmb, &grid);
+    if (st != HSA_OK) return st;
+    RET_CUDA(run_mma_assign(tmk, tmb, t, grid, stream));
+    RET_CUDA(launch_encode_codes(t, ix->codes, ix->ids, ix->cap, stream));
+  } else {
+    RET_CUDA(launch_encode(p, n_new, stream));
+  }
   RET_CUDA(launch_accumulate(p, n_new, stream));
   RET_CUDA(launch_list_reset(p, stream));
   RET_CUDA(launch_list_append(p, stream));
@@ -576,23 +679,6 @@ hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_ne
 struct TrainLayout {
   size_t assign, sums, counts, pq_sums, pq_counts, terms, cnorm, total;
 };
-// Longest training set: the fallback assignment launches one grid row per 32 keys (at most 65535).
-constexpr int32_t kMaxTrain = 65535 * 16;
-constexpr size_t kAssignTileN = 256;   // centroids per tensor-core tile
-
-// Tensor map over row-major [rows][128] bf16 (the centroid terms), box 64 x 256, 128-byte swizzle.
-bool make_rows_tmap(CUtensorMap* map, const void* base, size_t rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
-  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(kAssignTileN)};
-  cuuint32_t estr[2] = {1u, 1u};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 static TrainLayout train_layout(int U, int C, int n_train) {
   TrainLayout L;
   size_t o = align_up(sizeof(WsHeader), 256);
@@ -661,10 +747,6 @@ hsa_status hsa_train_index(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_trai
   p.num_pages = kv->num_pages;
   p.terms = reinterpret_cast<uint16_t*>(base + L.terms);
   p.cnorm = reinterpret_cast<float*>(base + L.cnorm);
-  p.Cpad = static_cast<int>(align_up(static_cast<size_t>(ix->C), kAssignTileN));
-  p.p0 = ix->n_sink / 8 * 8;
-  p.tiles_per_unit = (ix->n_sink + n_train - p.p0 + 127) / 128;
-  p.items = U * p.tiles_per_unit;
 
   // Nearest-centroid assignment: on the tensor cores (keys streamed by TMA in 8-row
   // boxes, so pages of at least 8 rows); 4-row pages use the CUDA-core kernel.
@@ -672,18 +754,12 @@ hsa_status hsa_train_index(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_trai
   CUtensorMap tmk = {}, tmb = {};
   int grid = 0;
   if (mma) {
-    const DeviceInfo* di = device_info();
-    if (!di) return HSA_ERR_CUDA;
-    if (!make_kv_tmap(&tmk, kv->k_cache, kv, 8) ||
-        !make_rows_tmap(&tmb, p.terms, static_cast<size_t>(U) * 3 * p.Cpad))
-      return HSA_ERR_CUDA;
-    grid = std::min(p.items, di->sms);
+    st = plan_mma_assign(kv, p, ix->n_sink & 7, &tmk, &tmb, &grid);
+    if (st != HSA_OK) return st;
   }
   auto assign = [&]() -> cudaError_t {
     if (!mma) return launch_train_assign(p, stream);
-    cudaError_t e = launch_centroid_terms(p, stream);
-    if (e != cudaSuccess) return e;
-    return launch_assign_mma(tmk, tmb, p, grid, stream);
+    return run_mma_assign(tmk, tmb, p, grid, stream);
   };
 
   // the sums start at zero; every update clears what it used

@@ -334,12 +334,13 @@ int grid_for(size_t work, int threads) {
 // direct sums of squared differences in fp32, ties to the lower index; a centre that
 // gets no rows keeps its value.
 // ---------------------------------------------------------------------------
+// Key row of training key j of unit (b, h): position n_sink + slot0[b] + j (slot0 null: 0).
 __device__ __forceinline__ const uint16_t* train_key(const TrainParams& p, int b, int h, int slot) {
   if (slot < 0 || slot >= p.n_train) {
     record_error(p.err, HSA_DEVERR_SLOT);
     slot = 0;
   }
-  const int pos = p.n_sink + slot;
+  const int pos = p.n_sink + (p.slot0 ? p.slot0[b] : 0) + slot;
   const int lp = pos / p.page_size;
   const int page = lp < p.max_pages ? p.block_table[static_cast<size_t>(b) * p.max_pages + lp] : -1;
   if (page < 0 || page >= p.num_pages) {
@@ -482,71 +483,126 @@ __global__ void __launch_bounds__(256) train_pq_init_kernel(TrainParams p) {
   for (int d = 0; d < kDsub; ++d) dst[d] = __fsub_rn(kv8[d], ca[d]);
 }
 
-// One Lloyd assignment of the residual sub-vectors. A CTA takes kPqGroup subspaces of
-// one unit and kPqKeys training keys: the group's codebooks and its partial sums live
-// in shared memory, each warp works on one subspace (so every codeword read is a
-// broadcast), a lane per key finds the nearest codeword and adds the residual
-// sub-vector to the shared sums; the CTA then adds its sums to the global ones.
-constexpr int kPqGroup = 4;
-constexpr int kPqKeys = 4096;
+// ---- nearest codeword of residual sub-vectors (training step and encoding) ----------
+// A CTA takes kPqGroup subspaces of one unit: the group's codebooks and, per codeword, the
+// pair (|w|^2 / 2, |w|^2 / 2) sit in shared memory; each warp works on one subspace (every
+// codeword read is a broadcast) and each lane on kPqLane keys, which share the reads. The
+// distance is evaluated as |w|^2 - 2 r.w (|r - w|^2 minus the key's constant |r|^2) with
+// packed fp32x2 fused multiply-adds; ties go to the lower codeword index.
+constexpr int kPqGroup = 2;
+constexpr int kPqLane = 4;                                       // keys per lane
+constexpr int kPqKeys = 2048;                                    // keys per CTA
 constexpr int kPqThreads = 256;
-constexpr size_t kPqSmem = static_cast<size_t>(kPqGroup) * kNcode * (2 * kDsub + 1) * sizeof(float);
+constexpr int kPqWarpKeys = 32 * kPqLane;
+constexpr int kPqKeyStride = (kPqThreads / 32 / kPqGroup) * kPqWarpKeys;   // keys per loop round of a CTA
+constexpr size_t kPqBookFloats = static_cast<size_t>(kPqGroup) * kNcode * kDsub;
+constexpr size_t kPqSmemCodes = (kPqBookFloats + kPqGroup * kNcode * 2) * sizeof(float);
+constexpr size_t kPqSmemStep = kPqSmemCodes + (kPqBookFloats + kPqGroup * kNcode) * sizeof(float);
 
-__global__ void __launch_bounds__(kPqThreads) train_pq_step_kernel(TrainParams p) {
+// Stage the codebooks of subspaces [s0, s0 + kPqGroup) of unit u and their half norms.
+__device__ __forceinline__ void stage_books(const float* codebooks, int u, int s0, float* book, float2* hn) {
+  const float* g = codebooks + (static_cast<size_t>(u) * kM + s0) * kNcode * kDsub;
+  for (int i = threadIdx.x; i < static_cast<int>(kPqBookFloats / 4); i += blockDim.x)
+    reinterpret_cast<float4*>(book)[i] = reinterpret_cast<const float4*>(g)[i];
+  __syncthreads();
+  for (int i = threadIdx.x; i < kPqGroup * kNcode; i += blockDim.x) {
+    const float* w = book + i * kDsub;
+    float n = 0.f;
+#pragma unroll
+    for (int d = 0; d < kDsub; ++d) n = fmaf(w[d], w[d], n);
+    hn[i] = make_float2(0.5f * n, 0.5f * n);
+  }
+  __syncthreads();
+}
+
+// Residual sub-vector s of key j: key - its centroid (fp32); zeros and false for a key
+// outside [0, j_end) or on an invalid page.
+__device__ __forceinline__ bool residual_sub(const TrainParams& p, int u, int b, int h, int j, int j_end, int s,
+                                             float* r) {
+  const uint16_t* row = j < j_end ? train_key(p, b, h, j) : nullptr;
+  if (!row) {
+#pragma unroll
+    for (int d = 0; d < kDsub; ++d) r[d] = 0.f;
+    return false;
+  }
+  const int a = p.assign[static_cast<size_t>(u) * p.n_train + j];
+  const uint4 raw = *reinterpret_cast<const uint4*>(row + s * kDsub);
+  const float kv8[8] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y),
+                        bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w)};
+  const float4* ca = reinterpret_cast<const float4*>(p.centroids + (static_cast<size_t>(u) * p.C + a) * kD +
+                                                     s * kDsub);
+  const float4 c0 = __ldg(ca), c1 = __ldg(ca + 1);
+  const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int d = 0; d < kDsub; ++d) r[d] = __fsub_rn(kv8[d], cv[d]);
+  return true;
+}
+
+// Nearest codewords of kPqLane residual sub-vectors in one subspace's staged codebook.
+__device__ __forceinline__ void nearest_codewords(const float (&r)[kPqLane][kDsub], const float* book,
+                                                  const float2* hn, int (&best_m)[kPqLane]) {
+  unsigned long long pr[kPqLane][4];
+  float best[kPqLane];
+#pragma unroll
+  for (int k = 0; k < kPqLane; ++k) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pr[k][i] = pack_f2(-2.f * r[k][2 * i], -2.f * r[k][2 * i + 1]);
+    best[k] = INFINITY;
+    best_m[k] = 0;
+  }
+  const ulonglong2* w = reinterpret_cast<const ulonglong2*>(book);
+  const unsigned long long* h = reinterpret_cast<const unsigned long long*>(hn);
+#pragma unroll 2
+  for (int m = 0; m < kNcode; ++m) {
+    const ulonglong2 w0 = w[2 * m], w1 = w[2 * m + 1];
+    const unsigned long long hm = h[m];
+#pragma unroll
+    for (int k = 0; k < kPqLane; ++k) {
+      unsigned long long x = ffma2_rn(pr[k][0], w0.x, hm);
+      x = ffma2_rn(pr[k][1], w0.y, x);
+      x = ffma2_rn(pr[k][2], w1.x, x);
+      x = ffma2_rn(pr[k][3], w1.y, x);
+      const float d = lo_f(x) + hi_f(x);
+      if (d < best[k]) {
+        best[k] = d;
+        best_m[k] = m;
+      }
+    }
+  }
+}
+
+// One Lloyd step of the codebooks: nearest codeword of every residual sub-vector, added to
+// the CTA's shared sums, which are then added to the global ones.
+__global__ void __launch_bounds__(kPqThreads, 3) train_pq_step_kernel(TrainParams p) {
   extern __shared__ __align__(16) float pq_sh[];
-  float* book = pq_sh;                                   // [kPqGroup][ncode][dsub]
-  float* sums = book + kPqGroup * kNcode * kDsub;        // [kPqGroup][ncode][dsub]
-  int* cnt = reinterpret_cast<int*>(sums + kPqGroup * kNcode * kDsub);   // [kPqGroup][ncode]
+  float* book = pq_sh;
+  float2* hn = reinterpret_cast<float2*>(book + kPqBookFloats);
+  float* sums = reinterpret_cast<float*>(hn + kPqGroup * kNcode);
+  int* cnt = reinterpret_cast<int*>(sums + kPqBookFloats);
   const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
   const int s0 = blockIdx.y * kPqGroup;
-  const float* gbook = p.codebooks + (static_cast<size_t>(u) * kM + s0) * kNcode * kDsub;
-  for (int i = threadIdx.x; i < kPqGroup * kNcode * kDsub / 4; i += kPqThreads) {
-    reinterpret_cast<float4*>(book)[i] = reinterpret_cast<const float4*>(gbook)[i];
-    reinterpret_cast<float4*>(sums)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+  for (int i = threadIdx.x; i < static_cast<int>(kPqBookFloats); i += kPqThreads) sums[i] = 0.f;
   for (int i = threadIdx.x; i < kPqGroup * kNcode; i += kPqThreads) cnt[i] = 0;
-  __syncthreads();
+  stage_books(p.codebooks, u, s0, book, hn);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sl = warp % kPqGroup, s = s0 + sl;
-  const float4* wb = reinterpret_cast<const float4*>(book + sl * kNcode * kDsub);
   const int j_end = min(p.n_train, static_cast<int>(blockIdx.z + 1) * kPqKeys);
-  for (int j = blockIdx.z * kPqKeys + (warp / kPqGroup) * 32 + lane; j < j_end;
-       j += (kPqThreads / 32 / kPqGroup) * 32) {
-    const uint16_t* row = train_key(p, b, h, j);
-    if (!row) continue;
-    const int a = p.assign[static_cast<size_t>(u) * p.n_train + j];
-    const uint4 raw = *reinterpret_cast<const uint4*>(row + s * kDsub);
-    const float kv8[8] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y),
-                          bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w)};
-    const float4* ca = reinterpret_cast<const float4*>(p.centroids + (static_cast<size_t>(u) * p.C + a) * kD +
-                                                       s * kDsub);
-    const float4 c0 = __ldg(ca), c1 = __ldg(ca + 1);
-    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    float r[kDsub];
+  for (int j = blockIdx.z * kPqKeys + (warp / kPqGroup) * kPqWarpKeys + lane; j < j_end; j += kPqKeyStride) {
+    float r[kPqLane][kDsub];
+    bool v[kPqLane];
 #pragma unroll
-    for (int d = 0; d < kDsub; ++d) r[d] = __fsub_rn(kv8[d], cv[d]);
-    float bb = INFINITY;
-    int bm = 0;
-#pragma unroll 4
-    for (int m = 0; m < kNcode; ++m) {
-      const float4 x = wb[2 * m], y = wb[2 * m + 1];
-      const float w8[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
-      float dist = 0.f;
+    for (int k = 0; k < kPqLane; ++k) v[k] = residual_sub(p, u, b, h, j + 32 * k, j_end, s, r[k]);
+    int m[kPqLane];
+    nearest_codewords(r, book + sl * kNcode * kDsub, hn + sl * kNcode, m);
 #pragma unroll
-      for (int d = 0; d < kDsub; ++d) {
-        const float t0 = __fsub_rn(r[d], w8[d]);
-        dist = fmaf(t0, t0, dist);
-      }
-      if (dist < bb) {
-        bb = dist;
-        bm = m;
-      }
+    for (int k = 0; k < kPqLane; ++k) {
+      if (!v[k]) continue;
+      float* dst = sums + (sl * kNcode + m[k]) * kDsub;
+#pragma unroll
+      for (int d = 0; d < kDsub; ++d) atomicAdd(dst + d, r[k][d]);
+      atomicAdd(cnt + sl * kNcode + m[k], 1);
     }
-    float* dst = sums + (sl * kNcode + bm) * kDsub;
-#pragma unroll
-    for (int d = 0; d < kDsub; ++d) atomicAdd(dst + d, r[d]);
-    atomicAdd(cnt + sl * kNcode + bm, 1);
   }
   __syncthreads();
   float* gsum = p.pq_sums + (static_cast<size_t>(u) * kM + s0) * kNcode * kDsub;
@@ -558,6 +614,38 @@ __global__ void __launch_bounds__(kPqThreads) train_pq_step_kernel(TrainParams p
     atomicAdd(reinterpret_cast<float4*>(gsum + i * kDsub), src[0]);
     atomicAdd(reinterpret_cast<float4*>(gsum + i * kDsub + 4), src[1]);
     atomicAdd(gcnt + i, c);
+  }
+}
+
+// Encoding: ids and codes of keys [0, n_train) of every unit, i.e. index slots
+// slot0[b] + j, from the nearest-centroid assignment in p.assign.
+__global__ void __launch_bounds__(kPqThreads, 3) encode_codes_kernel(TrainParams p, uint8_t* codes, uint16_t* ids,
+                                                                  int cap) {
+  extern __shared__ __align__(16) float pq_sh[];
+  float* book = pq_sh;
+  float2* hn = reinterpret_cast<float2*>(book + kPqBookFloats);
+  const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
+  const int s0 = blockIdx.y * kPqGroup;
+  stage_books(p.codebooks, u, s0, book, hn);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sl = warp % kPqGroup, s = s0 + sl;
+  const int first = p.slot0 ? p.slot0[b] : 0;
+  const int j_end = min(p.n_train, static_cast<int>(blockIdx.z + 1) * kPqKeys);
+  for (int j = blockIdx.z * kPqKeys + (warp / kPqGroup) * kPqWarpKeys + lane; j < j_end; j += kPqKeyStride) {
+    float r[kPqLane][kDsub];
+    bool v[kPqLane];
+#pragma unroll
+    for (int k = 0; k < kPqLane; ++k) v[k] = residual_sub(p, u, b, h, j + 32 * k, j_end, s, r[k]);
+    int m[kPqLane];
+    nearest_codewords(r, book + sl * kNcode * kDsub, hn + sl * kNcode, m);
+#pragma unroll
+    for (int k = 0; k < kPqLane; ++k) {
+      if (!v[k]) continue;
+      const int jk = j + 32 * k;
+      const size_t slot = static_cast<size_t>(u) * cap + first + jk;
+      codes[slot * kM + s] = static_cast<uint8_t>(m[k]);
+      if (s == 0) ids[slot] = static_cast<uint16_t>(p.assign[static_cast<size_t>(u) * p.n_train + jk]);
+    }
   }
 }
 
@@ -634,10 +722,19 @@ cudaError_t launch_train_pq_init(const TrainParams& p, cudaStream_t stream) {
 
 cudaError_t launch_train_pq_step(const TrainParams& p, cudaStream_t stream) {
   static_assert(kM % kPqGroup == 0, "subspace groups must tile the subspaces");
-  cudaError_t e = ensure_dyn_smem<train_pq_step_kernel>(kPqSmem);
+  static_assert(kPqKeys % kPqKeyStride == 0, "a key block is whole loop rounds");
+  cudaError_t e = ensure_dyn_smem<train_pq_step_kernel>(kPqSmemStep);
   if (e != cudaSuccess) return e;
-  train_pq_step_kernel<<<dim3(p.B * p.Hkv, kM / kPqGroup, (p.n_train + kPqKeys - 1) / kPqKeys), kPqThreads, kPqSmem,
-                         stream>>>(p);
+  train_pq_step_kernel<<<dim3(p.B * p.Hkv, kM / kPqGroup, (p.n_train + kPqKeys - 1) / kPqKeys), kPqThreads,
+                         kPqSmemStep, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_codes(const TrainParams& p, uint8_t* codes, uint16_t* ids, int cap, cudaStream_t stream) {
+  cudaError_t e = ensure_dyn_smem<encode_codes_kernel>(kPqSmemCodes);
+  if (e != cudaSuccess) return e;
+  encode_codes_kernel<<<dim3(p.B * p.Hkv, kM / kPqGroup, (p.n_train + kPqKeys - 1) / kPqKeys), kPqThreads,
+                        kPqSmemCodes, stream>>>(p, codes, ids, cap);
   return cudaGetLastError();
 }
 

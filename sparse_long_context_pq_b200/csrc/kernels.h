@@ -226,8 +226,8 @@ struct TrainParams {
   uint16_t* terms;             // [U][3][Cpad][D] bf16 terms of the centroids (tensor-core assignment)
   float* cnorm;                // [U][Cpad] |c|^2, +inf for the padding rows
   int B, Hkv, C, n_sink, n_train, page_size, max_pages, num_pages;
+  const int32_t* slot0;        // [B] first slot of each sequence's keys (null: 0), as for encoding
   int Cpad;                    // C rounded up to the 256-centroid tile
-  int p0;                      // first position of the first key tile (n_sink rounded down to 8)
   int tiles_per_unit, items;   // 128-key tiles per unit, units x tiles
 };
 cudaError_t launch_train_init(const TrainParams& p, cudaStream_t stream);
@@ -239,6 +239,7 @@ cudaError_t launch_train_pq_step(const TrainParams& p, cudaStream_t stream);
 cudaError_t launch_train_pq_update(const TrainParams& p, cudaStream_t stream);
 size_t assign_mma_smem_bytes();
 cudaError_t launch_centroid_terms(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_encode_codes(const TrainParams& p, uint8_t* codes, uint16_t* ids, int cap, cudaStream_t stream);
 cudaError_t launch_assign_mma(const CUtensorMap& tmk, const CUtensorMap& tmb, const TrainParams& p, int grid,
                               cudaStream_t stream);
 

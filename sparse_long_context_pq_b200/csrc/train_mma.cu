@@ -8,8 +8,10 @@
 // fp32 dot product to fp32 accuracy while the tensor cores accumulate in fp32.
 //
 // One persistent CTA per SM, warp-specialised:
-//   warp 0  TMA producer: key tile (128 keys = 16 page-row groups of 8) into one of two
-//           A buffers, then per 256-centroid tile and term a 256 x 128 B operand stage;
+//   warp 0  TMA producer: key tile (128 keys = 16 page-row groups of 8, starting at the
+//           8-aligned position at or before the unit's first key) into one of two
+//           A buffers, then per 256-centroid tile, term and 64-column half a 32 KB operand
+//           stage (four stages in flight);
 //   warp 1  allocates 512 TMEM columns (two 128 x 256 fp32 accumulators) and issues the
 //           tcgen05.mma instructions (one elected lane);
 //   warps 2-5 epilogue: tcgen05.ld of the accumulator rows (TMEM lane = key), running
@@ -35,15 +37,15 @@ constexpr int kAsRows = 8;                // rows per key-tile TMA box (one page
 constexpr uint32_t kAHalf = kAsM * 128;   // one 64-column half of the key tile (16 KB)
 constexpr uint32_t kBHalf = kAsN * 128;   // one 64-column half of a centroid stage (32 KB)
 constexpr uint32_t kATile = 2 * kAHalf;
-constexpr uint32_t kBTile = 2 * kBHalf;
+constexpr int kBStages = 4;               // centroid operand stages (one term, one 64-column half each)
 constexpr int kAsThreads = 192;
 constexpr uint32_t kTmemCols = 2 * kAsN;
 
 struct AsSmem {
-  static constexpr uint32_t a = 0;                    // 2 x 32 KB key tiles
-  static constexpr uint32_t b = 2 * kATile;           // 2 x 64 KB centroid stages
-  static constexpr uint32_t bars = b + 2 * kBTile;    // mbarriers
-  static constexpr uint32_t total = bars + 16 * 8 + 16;
+  static constexpr uint32_t a = 0;                         // 2 x 32 KB key tiles
+  static constexpr uint32_t b = 2 * kATile;                // 4 x 32 KB centroid stages
+  static constexpr uint32_t bars = b + kBStages * kBHalf;  // mbarriers
+  static constexpr uint32_t total = bars + 24 * 8 + 16;
 };
 constexpr size_t kAsSmemBytes = AsSmem::total + 1024;   // + alignment slack (1024-byte swizzle atoms)
 
@@ -77,8 +79,8 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
+// 32 consecutive fp32 columns of this thread's TMEM lane (completion: tmem_wait_ld).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
       "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -87,10 +89,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Split every centroid into three bf16 terms (rows >= C are zero) and write |c|^2
 // (+inf for the padding rows, so they never win). One warp per centroid row.
@@ -133,22 +133,24 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + AsSmem::bars);
   uint64_t* a_full = bars + 0;     // [2]
   uint64_t* a_empty = bars + 2;    // [2]
-  uint64_t* b_full = bars + 4;     // [2]
-  uint64_t* b_empty = bars + 6;    // [2]
-  uint64_t* acc_full = bars + 8;   // [2]
-  uint64_t* acc_empty = bars + 10; // [2]
-  uint64_t* mma_done = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* b_full = bars + 4;     // [kBStages]
+  uint64_t* b_empty = bars + 8;    // [kBStages]
+  uint64_t* acc_full = bars + 12;  // [2]
+  uint64_t* acc_empty = bars + 14; // [2]
+  uint64_t* mma_done = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(a_full + i, 1);
       mbar_init(a_empty + i, 1);
-      mbar_init(b_full + i, 1);
-      mbar_init(b_empty + i, 1);
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, 4);
+    }
+    for (int i = 0; i < kBStages; ++i) {
+      mbar_init(b_full + i, 1);
+      mbar_init(b_empty + i, 1);
     }
     mbar_init(mma_done, 1);
     fence_mbar_init();
@@ -166,52 +168,70 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 
   const int n_tiles = p.Cpad / kAsN;
   if (warp == 0) {
+    // The whole warp produces: lanes 0-15 each load one 8-row group of the key tile (its
+    // page looked up one item ahead, so the block-table reads overlap the previous
+    // item's operand stream); lane 0 arms the barriers and loads the centroid stages.
     if (lane == 0) {
       prefetch_tmap(&tmk);
       prefetch_tmap(&tmb);
-      uint32_t armed[4] = {0, 0, 0, 0};   // arms of a_full[0..1], b_full[0..1]
-      int li = 0, sb = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++li) {
-        const int u = it / p.tiles_per_unit, t = it % p.tiles_per_unit;
-        const int b = u / p.Hkv, h = u % p.Hkv;
-        const int ia = li & 1;
-        if (!mbar_wait(a_empty + ia, ((li >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
+    }
+    auto group_row = [&](int it) -> int {
+      if (it >= p.items || lane >= kAsM / kAsRows) return 0;
+      const int u = it / p.tiles_per_unit, t = it % p.tiles_per_unit;
+      const int b = u / p.Hkv, h = u % p.Hkv;
+      const int first = p.n_sink + (p.slot0 ? p.slot0[b] : 0);   // position of key 0
+      const int pos = (first & ~(kAsRows - 1)) + t * kAsM + lane * kAsRows;
+      const int lp = pos / p.page_size;
+      int page = lp < p.max_pages ? p.block_table[static_cast<size_t>(b) * p.max_pages + lp] : -1;
+      if (page < 0 || page >= p.num_pages) {
+        if (pos + kAsRows > first && pos < first + p.n_train) record_error(p.err, HSA_DEVERR_PAGE);
+        page = 0;   // rows outside the key range are loaded but never assigned
+      }
+      return (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
+    };
+    uint32_t armed[2 + kBStages] = {};   // arms of a_full[], b_full[] (lane 0)
+    int li = 0, sb = 0;
+    bool ok = true;
+    int row = group_row(blockIdx.x);
+    for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++li) {
+      const int u = it / p.tiles_per_unit;
+      const int ia = li & 1;
+      if (!mbar_wait_warp(a_empty + ia, ((li >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
+      if (lane == 0) {
         mbar_arrive_expect_tx(a_full + ia, kATile);
         ++armed[ia];
-        uint8_t* A = sm + AsSmem::a + ia * kATile;
-        for (int g = 0; g < kAsM / kAsRows; ++g) {
-          const int pos = p.p0 + t * kAsM + g * kAsRows;
-          const int lp = pos / p.page_size;
-          int page = lp < p.max_pages ? p.block_table[static_cast<size_t>(b) * p.max_pages + lp] : -1;
-          if (page < 0 || page >= p.num_pages) {
-            if (pos + kAsRows > p.n_sink && pos < p.n_sink + p.n_train) record_error(p.err, HSA_DEVERR_PAGE);
-            page = 0;   // rows outside the training range are loaded but never assigned
-          }
-          const int row = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
-          tma_load_2d(A + g * kAsRows * 128, &tmk, a_full + ia, 0, row);
-          tma_load_2d(A + kAHalf + g * kAsRows * 128, &tmk, a_full + ia, 64, row);
-        }
-        for (int n = 0; ok && n < n_tiles; ++n) {
-          for (int k = 0; k < 3; ++k, ++sb) {
-            const int ib = sb & 1;
-            if (!mbar_wait(b_empty + ib, ((sb >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
-            mbar_arrive_expect_tx(b_full + ib, kBTile);
-            ++armed[2 + ib];
-            uint8_t* B = sm + AsSmem::b + ib * kBTile;
-            const int y = (u * 3 + k) * p.Cpad + n * kAsN;
-            tma_load_2d(B, &tmb, b_full + ib, 0, y);
-            tma_load_2d(B + kBHalf, &tmb, b_full + ib, 64, y);
-          }
-        }
       }
-      // copies still in flight land before the CTA leaves (bounded; immediate when the
-      // MMA warp consumed them all)
-      for (int i = 0; i < 2; ++i) {
-        if (armed[i]) mbar_wait(a_full + i, (armed[i] - 1) & 1, p.err);
-        if (armed[2 + i]) mbar_wait(b_full + i, (armed[2 + i] - 1) & 1, p.err);
+      __syncwarp();
+      uint8_t* A = sm + AsSmem::a + ia * kATile;
+      if (lane < kAsM / kAsRows) {
+        tma_load_2d(A + lane * kAsRows * 128, &tmk, a_full + ia, 0, row);
+        tma_load_2d(A + kAHalf + lane * kAsRows * 128, &tmk, a_full + ia, 64, row);
+      }
+      row = group_row(it + gridDim.x);
+      for (int n = 0; ok && n < n_tiles; ++n) {
+        for (int k = 0; ok && k < 3; ++k) {
+          for (int kh = 0; kh < 2; ++kh, ++sb) {
+            const int ib = sb % kBStages;
+            if (!mbar_wait_warp(b_empty + ib, ((sb / kBStages) & 1) ^ 1, p.err)) { ok = false; break; }
+            if (lane == 0) {
+              mbar_arrive_expect_tx(b_full + ib, kBHalf);
+              ++armed[2 + ib];
+              tma_load_2d(sm + AsSmem::b + ib * kBHalf, &tmb, b_full + ib, kh * 64, (u * 3 + k) * p.Cpad + n * kAsN);
+            }
+            __syncwarp();
+          }
+        }
       }
     }
+    // copies still in flight land before the CTA leaves (bounded; immediate when the
+    // MMA warp consumed them all)
+    if (lane == 0) {
+      for (int i = 0; i < 2; ++i)
+        if (armed[i]) mbar_wait(a_full + i, (armed[i] - 1) & 1, p.err);
+      for (int i = 0; i < kBStages; ++i)
+        if (armed[2 + i]) mbar_wait(b_full + i, (armed[2 + i] - 1) & 1, p.err);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       int li = 0, sb = 0, sa = 0;
@@ -226,19 +246,21 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           if (!mbar_wait(acc_empty + buf, ((sa >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + buf * kAsN;
-          for (int k = 0; k < 3; ++k, ++sb) {
-            const int ib = sb & 1;
-            if (!mbar_wait(b_full + ib, (sb >> 1) & 1, p.err)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t B = smem_addr(sm + AsSmem::b + ib * kBTile);
+          for (int k = 0; ok && k < 3; ++k) {
+            for (int kh = 0; kh < 2; ++kh, ++sb) {
+              const int ib = sb % kBStages;
+              if (!mbar_wait(b_full + ib, (sb / kBStages) & 1, p.err)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t B = smem_addr(sm + AsSmem::b + ib * kBHalf);
 #pragma unroll
-            for (int kk = 0; kk < kD / kAsK; ++kk) {
-              const uint32_t off = (kk & 3) * (kAsK * 2);   // K step inside the 128-byte atom row
-              const uint64_t ad = sw128_desc(A + (kk >> 2) * kAHalf + off);
-              const uint64_t bd = sw128_desc(B + (kk >> 2) * kBHalf + off);
-              tc_mma(d, ad, bd, (k > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 64 / kAsK; ++kk) {
+                const uint32_t off = kk * (kAsK * 2);   // K step inside the 128-byte atom row
+                const uint64_t ad = sw128_desc(A + kh * kAHalf + off);
+                const uint64_t bd = sw128_desc(B + off);
+                tc_mma(d, ad, bd, (k > 0 || kh > 0 || kk > 0) ? 1u : 0u);
+              }
+              tc_commit(b_empty + ib);   // the stage is free once these MMAs have read it
             }
-            tc_commit(b_empty + ib);   // the stage is free once these MMAs have read it
           }
           if (ok) tc_commit(acc_full + buf);
         }
@@ -263,15 +285,19 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         const int buf = sa & 1;
         if (!mbar_wait_warp(acc_full + buf, (sa >> 1) & 1, p.err)) { ok = false; break; }
         tc_fence_after();
-        for (int ch = 0; ch < kAsN / 32; ++ch) {
-          float v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kAsN + ch * 32, v);
-          const int c0 = n * kAsN + ch * 32;
+        for (int ch = 0; ch < kAsN / 64; ++ch) {
+          uint32_t v[64];
+          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kAsN + ch * 64;
+          tmem_ld32(ta, v);
+          tmem_ld32(ta + 32, v + 32);
+          tmem_wait_ld();
+          const int c0 = n * kAsN + ch * 64;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
+          for (int i = 0; i < 64; i += 4) {
             const float4 nn = __ldg(reinterpret_cast<const float4*>(cn + c0 + i));
-            const float e[4] = {fmaf(-2.f, v[i], nn.x), fmaf(-2.f, v[i + 1], nn.y), fmaf(-2.f, v[i + 2], nn.z),
-                                fmaf(-2.f, v[i + 3], nn.w)};
+            const float e[4] = {fmaf(-2.f, __uint_as_float(v[i]), nn.x), fmaf(-2.f, __uint_as_float(v[i + 1]), nn.y),
+                                fmaf(-2.f, __uint_as_float(v[i + 2]), nn.z),
+                                fmaf(-2.f, __uint_as_float(v[i + 3]), nn.w)};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               if (e[j] < best) {
@@ -285,8 +311,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         if (lane == 0) mbar_arrive(acc_empty + buf);
       }
       if (!ok) break;
-      const int pos = p.p0 + t * kAsM + r;
-      const int j = pos - p.n_sink;
+      const int first = p.n_sink + (p.slot0 ? p.slot0[u / p.Hkv] : 0);
+      const int j = (first & ~(kAsRows - 1)) + t * kAsM + r - first;
       if (j >= 0 && j < p.n_train) {
         const int a = besti < p.C ? besti : 0;   // NaN keys only
         p.assign[static_cast<size_t>(u) * p.n_train + j] = a;

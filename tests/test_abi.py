@@ -127,11 +127,24 @@ def test_decode_rejects_small_workspace_and_null_q(lib):
 def test_append_checks_capacity(lib):
     kv, lens = _kv(seq=100)
     ix, nh = _ix(n_idx=50, n_sink=4, cap=60)
-    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix), 20, FAKE, 256, None) == 3   # cap 60 < 70
+    big = 1 << 30
+    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix), 20, FAKE, big, None) == 3   # cap 60 < 70
     ix2, nh2 = _ix(n_idx=50, n_sink=4, cap=128)
-    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix2), 50, FAKE, 256, None) == 3  # beyond T
-    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix2), -1, FAKE, 256, None) == 1
+    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix2), 50, FAKE, big, None) == 3  # beyond T
+    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix2), -1, FAKE, big, None) == 1
     assert nh2[0] == 50                                                                           # untouched
+
+
+def test_append_workspace(lib):
+    kv, lens = _kv(seq=100)
+    ix, nh = _ix(n_idx=40, n_sink=4, cap=128, C=16)
+    q = lambda k, i, n: lib.hsa_index_workspace_bytes(ctypes.byref(k), ctypes.byref(i), n)
+    assert q(kv, ix, 0) == 256                                  # build from codes: the error word
+    need = q(kv, ix, 20)                                        # tensor-core encoding: terms, norms, assignment
+    assert need >= 256 + 3 * 256 * 128 * 2 + 256 * 4 + 20 * 4 and need % 256 == 0
+    assert lib.hsa_append_encode(ctypes.byref(kv), ctypes.byref(ix), 20, FAKE, need - 256, None) == 5
+    kv4, _ = _kv(seq=100, page_size=4, max_pages=32, num_pages=32)
+    assert q(kv4, ix, 20) == 256                                # 4-row pages: CUDA-core encoding
 
 
 def test_dense_rejects_bad_args(lib):

@@ -39,6 +39,8 @@ def _compare_codes(gpu_ids, gpu_codes, orc):
 @pytest.mark.parametrize("case", [
     dict(name="tiny_4k"),
     dict(name="qwen30b_128k_append", B=2, T=4096, extra_tokens=0, append_batch=0, C=256),
+    dict(name="tiny_4k", n_sink=13, page_size=8, C=300),   # key tiles start before the first key; C not a tile multiple
+    dict(name="tiny_4k", page_size=4),                      # CUDA-core encoding
 ])
 def test_build_by_encoding_matches_oracle(cuda_device, case):
     w = workload(**case)
@@ -46,7 +48,7 @@ def test_build_by_encoding_matches_oracle(cuda_device, case):
     dev = torch.device("cuda:0")
     kv = P.PagedKV(**kv_tensors(bt, dev))
     ix = P.PQIndex(**index_tensors(bt, dev, n_indexed=np.zeros(w.B, np.int32)))
-    ws = P.workspace(P.hsa_index_workspace_bytes(), dev)
+    ws = P.workspace(P.hsa_index_workspace_bytes(kv, ix, w.n_indexed), dev)
     P.hsa_append_encode(kv, ix, w.n_indexed, workspace_buf=ws)
     torch.cuda.synchronize()
     assert P.hsa_read_error(ws) == 0
@@ -75,7 +77,7 @@ def test_append_loop_then_decode(cuda_device):
     dev = torch.device("cuda:0")
     kv = P.PagedKV(**kv_tensors(bt, dev))
     ix = P.PQIndex(**index_tensors(bt, dev, n_indexed=np.zeros(w.B, np.int32)))
-    ws = P.workspace(P.hsa_index_workspace_bytes(), dev)
+    ws = P.workspace(P.hsa_index_workspace_bytes(kv, ix, w.n_indexed), dev)
     P.hsa_append_encode(kv, ix, w.n_indexed, workspace_buf=ws)
     scale = scale_for(w.D)
     q = torch.from_numpy(bt.q).to(dev)

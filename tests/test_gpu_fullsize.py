@@ -78,7 +78,7 @@ def test_fullsize_qwen_append(cuda_device):
     T2 = w.T + 512
     kv.seq_lens.fill_(T2)
     kv.seq_lens_host.fill_(T2)
-    ws = P.workspace(P.hsa_index_workspace_bytes(), dev)
+    ws = P.workspace(P.hsa_index_workspace_bytes(kv, ix, 512), dev)
     P.hsa_append_encode(kv, ix, 512, workspace_buf=ws)
     torch.cuda.synchronize()
     assert P.hsa_read_error(ws) == 0

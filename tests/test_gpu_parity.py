@@ -51,7 +51,7 @@ def _setup(case, seq_lens=None, n_indexed=None, n_sink=None):
 
 def _run_hsa(w, bt, codes, ids, kv, ix, dev, budget=0.01, k_override=-1, background=True):
     scale = scale_for(w.D)
-    ws_idx = P.workspace(P.hsa_index_workspace_bytes(), dev)
+    ws_idx = P.workspace(P.hsa_index_workspace_bytes(kv, ix), dev)
     P.hsa_build_from_codes(kv, ix, workspace_buf=ws_idx)
     q = torch.from_numpy(bt.q).to(dev)
     cap = ix.cap

@@ -67,7 +67,9 @@ def _keys(bt, w, b, h, n_train):
     return O.unit_rows(bt.k_cache, bt.block_table[b], h, w.n_sink + np.arange(n_train), w.page_size).astype(np.float32)
 
 
-CASES = [dict(name="tiny_4k"), dict(name="qwen30b_128k_append", B=2, T=4096, extra_tokens=0, append_batch=0, C=128)]
+CASES = [dict(name="tiny_4k"), dict(name="qwen30b_128k_append", B=2, T=4096, extra_tokens=0, append_batch=0, C=128),
+         dict(name="tiny_4k", n_sink=13, page_size=8, C=300),   # unaligned first key; C not a tile multiple
+         dict(name="tiny_4k", page_size=4)]                      # CUDA-core assignment
 
 
 @pytest.mark.parametrize("case", CASES)
@@ -157,7 +159,7 @@ def test_trained_index_encodes_and_decodes(cuda_device):
     n_train = w.n_indexed
     init = train_init_slots(w, n_train, seed=3)
     cen, books, _ = _train(w, dev, kv, ix, n_train, init, coarse=4, pq=4)
-    ws = P.workspace(P.hsa_index_workspace_bytes(), dev)
+    ws = P.workspace(P.hsa_index_workspace_bytes(kv, ix, w.n_indexed), dev)
     P.hsa_append_encode(kv, ix, w.n_indexed, workspace_buf=ws)
     torch.cuda.synchronize()
     assert P.hsa_read_error(ws) == 0
