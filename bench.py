@@ -350,6 +350,7 @@ def run_ours(args):
                    "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MB write) before every timed step",
                    "timing": "CUDA events per step around a CUDA-graph replay; per-kernel times from "
                              "eager steps with stage events on the launching stream"},
+        "percentiles_us": {f"p{q}": round(float(np.percentile(t_hsa, q)) * 1e3, 3) for q in (10, 50, 90)},
         "hbm_gbs": round(step_gbs, 1),
         "hbm_pct_peak": round(100 * step_gbs / peak, 2),
         "bytes_per_step": hsa_b,
