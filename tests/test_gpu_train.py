@@ -29,7 +29,8 @@ def _ties(X, Cn):
     Returns ({row: (winner, runner-up)}, the centres such rows touch)."""
     X64 = X.astype(np.float64)
     C64 = Cn.astype(np.float64)
-    same = (Cn[:, None, :] == Cn[None, :, :]).all(axis=2)
+    inv = np.unique(Cn, axis=0, return_inverse=True)[1].reshape(-1)
+    same = inv[:, None] == inv[None, :]
     rows, centres = {}, set()
     for i in range(0, len(X), 256):
         d = ((X64[i:i + 256, None, :] - C64[None]) ** 2).sum(axis=2)
@@ -45,6 +46,7 @@ def _ties(X, Cn):
 
 
 def _setup(case):
+    case = {k: v for k, v in case.items() if k != "n_train"}
     w = workload(**case)
     bt = make_batch(w)
     dev = torch.device("cuda:0")
@@ -69,13 +71,16 @@ def _keys(bt, w, b, h, n_train):
 
 CASES = [dict(name="tiny_4k"), dict(name="qwen30b_128k_append", B=2, T=4096, extra_tokens=0, append_batch=0, C=128),
          dict(name="tiny_4k", n_sink=13, page_size=8, C=300),   # unaligned first key; C not a tile multiple
-         dict(name="tiny_4k", page_size=4)]                      # CUDA-core assignment
+         dict(name="tiny_4k", page_size=4),                      # CUDA-core assignment
+         dict(name="tiny_4k", C=1),                              # one centroid: the mean of all keys
+         dict(name="tiny_4k", n_sink=0, n_train=200),            # no sink; a partial, ragged training set
+         dict(name="tiny_4k", n_train=1, C=1)]                   # a single training key
 
 
-@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("case", CASES + [dict(name="tiny_4k", C=4096)])   # the largest C: 16 centroid tiles
 def test_one_coarse_step_matches_oracle(cuda_device, case):
     w, bt, dev, kv, ix = _setup(case)
-    n_train = w.n_indexed
+    n_train = case.get("n_train", w.n_indexed)
     init = train_init_slots(w, n_train)
     cen, books, aout = _train(w, dev, kv, ix, n_train, init, coarse=1, pq=0)
     orc = O.oracle_train(bt.k_cache, bt.block_table, w.n_sink, n_train, init, w.C, 1, 0, page_size=w.page_size)
@@ -103,7 +108,7 @@ def test_one_coarse_step_matches_oracle(cuda_device, case):
 @pytest.mark.parametrize("case", CASES)
 def test_one_codebook_step_matches_oracle(cuda_device, case):
     w, bt, dev, kv, ix = _setup(case)
-    n_train = w.n_indexed
+    n_train = case.get("n_train", w.n_indexed)
     init = train_init_slots(w, n_train, seed=1)
     cen, books, aout = _train(w, dev, kv, ix, n_train, init, coarse=0, pq=1)
     orc = O.oracle_train(bt.k_cache, bt.block_table, w.n_sink, n_train, init, w.C, 0, 1, page_size=w.page_size)
