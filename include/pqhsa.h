@@ -225,12 +225,17 @@ hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* index, int32_t n
  * For every sequence b and KV head the training set is the keys at positions
  * [s0, s0 + n_train) (training slot j = position s0 + j):
  *   centroids: start at the keys of slots init_slots[0 .. C); coarse_iters times
- *     assign every key to its nearest centroid (fp32 sum of squared differences,
- *     ties to the lower index) and move each centroid to the mean of its keys (a
- *     centroid with no keys keeps its value); then assign once more;
+ *     assign every key to its nearest centroid (squared Euclidean distance, ties to
+ *     the lower index) and move each centroid to the mean of its keys (a centroid
+ *     with no keys keeps its value); then assign once more;
  *   codebook s: start at the subspace-s residuals (key - centroid of its final
  *     assignment) of slots init_slots[C + s*ncode .. C + (s+1)*ncode); pq_iters times
  *     the same assign/move on the residuals' subspace s.
+ * Decisions are taken in fp32: with pages of at least 8 rows the nearest centroid
+ *   minimises |c|^2 - 2 k.c with k.c on the tensor cores (each centroid as three bf16
+ *   terms, fp32 accumulation; 4-row pages: direct fp32 sums of squared differences),
+ *   the nearest codeword minimises |w|^2 - 2 r.w; the means are fp32 sums (atomics,
+ *   so the last bits depend on the order of addition).
  * init_slots: device int32 [B][Hkv][C + M*ncode], each in [0, n_train) (the caller
  *   draws them; an out-of-range slot is replaced by 0 and flagged HSA_DEVERR_SLOT).
  * assign_out: NULL, or device int32 [B][Hkv][n_train] receiving the final coarse
