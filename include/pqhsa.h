@@ -240,7 +240,7 @@ hsa_status hsa_append_encode(const hsa_kv_cache* kv, hsa_index* index, int32_t n
  *   draws them; an out-of-range slot is replaced by 0 and flagged HSA_DEVERR_SLOT).
  * assign_out: NULL, or device int32 [B][Hkv][n_train] receiving the final coarse
  *   assignment. Writes index->centroids and index->codebooks only.
- * Requires 1 <= n_train <= 1048560, s0 + n_train <= seq_lens_host[b], M = 16, dsub = 8,
+ * Requires 1 <= n_train <= 2097120, s0 + n_train <= seq_lens_host[b], M = 16, dsub = 8,
  * ncode = 256, C <= 4096, 0 <= iterations <= 1000; the workspace as
  * hsa_train_workspace_bytes says (its error word is read by hsa_read_error).
  */

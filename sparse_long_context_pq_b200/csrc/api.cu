@@ -488,7 +488,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
 }
 
 // Longest training set: the fallback assignment launches one grid row per 32 keys (at most 65535).
-constexpr int32_t kMaxTrain = 65535 * 16;
+constexpr int32_t kMaxTrain = 65535 * 32;
 constexpr size_t kAssignTileN = 256;   // centroids per tensor-core tile
 
 // Tensor map over row-major [rows][128] bf16 (the centroid terms), box 64 x 256, 128-byte swizzle.
@@ -715,7 +715,7 @@ hsa_status hsa_train_index(const hsa_kv_cache* kv, hsa_index* ix, int32_t n_trai
   if (ix->C > kMaxClusters) return HSA_ERR_UNSUPPORTED;
   if (n_train < 1 || coarse_iters < 0 || pq_iters < 0 || coarse_iters > 1000 || pq_iters > 1000)
     return HSA_ERR_INVALID_ARG;
-  if (n_train > kMaxTrain) return HSA_ERR_UNSUPPORTED;   // grid rows of the codebook step
+  if (n_train > kMaxTrain) return HSA_ERR_UNSUPPORTED;   // grid rows of the CUDA-core assignment
   if (!aligned(ix->centroids, 16) || !aligned(ix->codebooks, 16) || !aligned(init_slots, 4) ||
       (assign_out && !aligned(assign_out, 4)))
     return HSA_ERR_ALIGNMENT;

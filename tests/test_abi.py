@@ -177,7 +177,7 @@ def test_train_rejects_bad_args(lib, kw, status):
 def test_train_rejects_unsupported_index(lib):
     kv, lens = _kv(seq=2 << 20, max_pages=(2 << 20) // 16, num_pages=(2 << 20) // 16)
     ix, nh = _ix(cap=2 << 20)
-    assert _train(lib, kv, ix, n_train=65535 * 16 + 1) == 2   # beyond the longest training set
+    assert _train(lib, kv, ix, n_train=65535 * 32 + 1) == 2   # beyond the longest training set
     ix2, nh2 = _ix(M=8, dsub=16)
     kv2, lens2 = _kv()
     assert _train(lib, kv2, ix2) == 2
