@@ -102,3 +102,35 @@ def test_train_unit_shapes_and_determinism():
     assert c1.shape == (8, 128) and b1.shape == (16, 16, 8) and a1.shape == (500,)
     np.testing.assert_array_equal(c1, c2)
     np.testing.assert_array_equal(b1, b2)
+
+
+def test_single_centre_is_the_mean_of_all_keys_and_codewords_start_at_seed_residuals():
+    """C = 1: one coarse step puts the centroid at the mean of every key (closed form); with no
+    codebook step, codeword m of subspace s is the subspace-s residual of its seed key."""
+    rng = np.random.default_rng(7)
+    X = (rng.standard_normal((50, 16)) * 3).astype(np.float32)
+    init = rng.integers(0, 50, size=1 + 2 * 4)
+    cen, books, a = O.train_unit(X, init, C=1, coarse_iters=1, pq_iters=0, M=2, ncode=4)
+    np.testing.assert_allclose(cen[0], X.astype(np.float64).mean(0), rtol=0, atol=1e-5)
+    assert (a == 0).all()
+    R = X.astype(np.float64) - cen[0].astype(np.float64)
+    for s in range(2):
+        for m in range(4):
+            np.testing.assert_allclose(books[s, m], R[init[1 + s * 4 + m], 8 * s:8 * s + 8], rtol=0, atol=1e-6)
+
+
+def test_training_does_not_depend_on_key_order():
+    """Lloyd k-means sees a set: permuting the keys (and the seed slots with them) gives the
+    same centroids and codebooks, and the assignment permuted alike."""
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((120, 16)).astype(np.float32)
+    C, M, ncode = 5, 2, 8
+    init = rng.choice(120, size=C + M * ncode, replace=True)
+    perm = rng.permutation(120)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(120)
+    cen1, books1, a1 = O.train_unit(X, init, C, 3, 3, M=M, ncode=ncode)
+    cen2, books2, a2 = O.train_unit(X[perm], inv[init], C, 3, 3, M=M, ncode=ncode)
+    np.testing.assert_allclose(cen1, cen2, rtol=0, atol=1e-6)
+    np.testing.assert_allclose(books1, books2, rtol=0, atol=1e-6)
+    assert np.array_equal(a1[perm], a2)
