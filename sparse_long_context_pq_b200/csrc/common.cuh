@@ -96,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
   return false;
 }
 
-// Warp-uniform wait: lane 0 polls, the verdict is broadcast (and the warp reconverged).
+// Warp-uniform wait: lane 0 polls, the outcome is broadcast (and the warp reconverged).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int32_t* err) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err);
