@@ -141,6 +141,13 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _on_gpu(*ts: Optional[torch.Tensor]) -> None:
+    """The library dereferences these on the device: a host tensor here would be a bad address."""
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("expected a CUDA tensor, got one on " + str(t.device))
+
+
 def _stream(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -170,6 +177,7 @@ class PagedKV:
         assert self.block_table.dtype == torch.int32 and self.seq_lens.dtype == torch.int32
         assert self.seq_lens_host.dtype == torch.int32 and self.seq_lens_host.device.type == "cpu"
         assert self.k_cache.is_contiguous() and self.v_cache.is_contiguous() and self.block_table.is_contiguous()
+        _on_gpu(self.k_cache, self.v_cache, self.block_table, self.seq_lens)
         return _KV(_ptr(self.k_cache), _ptr(self.v_cache), _ptr(self.block_table), _ptr(self.seq_lens),
                    _ptr(self.seq_lens_host), B, self.Hq, Hkv, D, ps, maxp, P)
 
@@ -241,6 +249,8 @@ class PQIndex:
                   self.list_codes, self.list_slot, self.chunk_cluster, self.list_meta):
             assert t.is_contiguous()
         assert self.n_indexed_host.device.type == "cpu" and self.n_indexed_host.dtype == torch.int32
+        _on_gpu(self.centroids, self.codebooks, self.codes, self.ids, self.sum_v, self.mean_v, self.count,
+                self.n_indexed, self.list_codes, self.list_slot, self.chunk_cluster, self.list_meta)
         return _Index(_ptr(self.centroids), _ptr(self.codebooks), _ptr(self.codes), _ptr(self.ids),
                       _ptr(self.sum_v), _ptr(self.mean_v), _ptr(self.count), _ptr(self.n_indexed),
                       _ptr(self.n_indexed_host), _ptr(self.list_codes), _ptr(self.list_slot),
@@ -293,6 +303,7 @@ def hsa_decode(kv: PagedKV, index: PQIndex, q: torch.Tensor, out: Optional[torch
     if stage_events is not None:
         assert len(stage_events) == NUM_STAGES + 1
         ev_arr = (ctypes.c_void_p * (NUM_STAGES + 1))(*[e.cuda_event for e in stage_events])
+    _on_gpu(q, out, approx_logits, selected, n_selected, workspace_buf)
     dbg = _Debug(_ptr(approx_logits), _ptr(selected), _ptr(n_selected),
                  ctypes.cast(ev_arr, ctypes.c_void_p) if ev_arr is not None else None)
     st = lib.hsa_decode(ctypes.byref(kvs), ctypes.byref(ixs), q.data_ptr(), out.data_ptr(), ctypes.byref(prm),
@@ -310,6 +321,7 @@ def dense_decode(kv: PagedKV, q: torch.Tensor, out: Optional[torch.Tensor] = Non
     kvs = kv.struct()
     if workspace_buf is None:
         workspace_buf = workspace(dense_decode_workspace_bytes(kv), q.device)
+    _on_gpu(q, out, workspace_buf)
     st = load_library().dense_decode(ctypes.byref(kvs), q.data_ptr(), out.data_ptr(), ctypes.c_float(scale),
                                      workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
     _check("dense_decode", st)
@@ -322,6 +334,7 @@ def hsa_build_from_codes(kv: PagedKV, index: PQIndex, workspace_buf: Optional[to
     kvs, ixs = kv.struct(), index.struct()
     if workspace_buf is None:
         workspace_buf = workspace(hsa_index_workspace_bytes(kv, index), index.centroids.device)
+    _on_gpu(workspace_buf)
     st = load_library().hsa_build_from_codes(ctypes.byref(kvs), ctypes.byref(ixs), workspace_buf.data_ptr(),
                                              workspace_buf.numel(), _stream(stream))
     _check("hsa_build_from_codes", st)
@@ -333,6 +346,7 @@ def hsa_append_encode(kv: PagedKV, index: PQIndex, n_new: int, workspace_buf: Op
     kvs, ixs = kv.struct(), index.struct()
     if workspace_buf is None:
         workspace_buf = workspace(hsa_index_workspace_bytes(kv, index, n_new), index.centroids.device)
+    _on_gpu(workspace_buf)
     st = load_library().hsa_append_encode(ctypes.byref(kvs), ctypes.byref(ixs), int(n_new),
                                           workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
     _check("hsa_append_encode", st)
@@ -358,6 +372,7 @@ def hsa_train_index(kv: PagedKV, index: PQIndex, n_train: int, init_slots: torch
     kvs, ixs = kv.struct(), index.struct()
     if workspace_buf is None:
         workspace_buf = workspace(hsa_train_workspace_bytes(kv, index, n_train), index.centroids.device)
+    _on_gpu(init_slots, assign_out, workspace_buf)
     st = load_library().hsa_train_index(ctypes.byref(kvs), ctypes.byref(ixs), int(n_train), init_slots.data_ptr(),
                                         int(coarse_iters), int(pq_iters), _ptr(assign_out),
                                         workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
@@ -367,6 +382,7 @@ def hsa_train_index(kv: PagedKV, index: PQIndex, n_train: int, init_slots: torch
 def hsa_read_error(workspace_buf: torch.Tensor, stream=None) -> int:
     """Read and clear the device error word of a workspace (synchronises the stream)."""
     v = ctypes.c_int32(0)
+    _on_gpu(workspace_buf)
     st = load_library().hsa_read_error(workspace_buf.data_ptr(), ctypes.byref(v), _stream(stream))
     _check("hsa_read_error", st)
     return int(v.value)
@@ -384,6 +400,7 @@ def dense_decode_static(kv: PagedKV, q: torch.Tensor, out: Optional[torch.Tensor
     fn.argtypes = [ctypes.POINTER(_KV), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
     fn.restype = ctypes.c_int
     kvs = kv.struct()
+    _on_gpu(q, out)
     _check("dense_decode_static", fn(ctypes.byref(kvs), q.data_ptr(), out.data_ptr(), ctypes.c_float(scale),
                                      _stream(stream)))
     return out

@@ -183,3 +183,18 @@ def test_train_rejects_unsupported_index(lib):
     assert _train(lib, kv2, ix2) == 2
     assert lib.hsa_train_workspace_bytes(ctypes.byref(kv2), ctypes.byref(ix), 0) == 0
     assert lib.hsa_train_workspace_bytes(ctypes.byref(kv2), ctypes.byref(ix), 40) % 256 == 0
+
+
+def test_binding_rejects_host_tensors_for_device_arrays():
+    """A host tensor where the library expects device memory is refused before any call."""
+    import torch
+    B, Hkv, ps, pages = 1, 1, 16, 4
+    kv = P.PagedKV(k_cache=torch.zeros(pages, Hkv, ps, 128, dtype=torch.bfloat16),
+                   v_cache=torch.zeros(pages, Hkv, ps, 128, dtype=torch.bfloat16),
+                   block_table=torch.zeros(B, pages, dtype=torch.int32), seq_lens=torch.zeros(B, dtype=torch.int32),
+                   seq_lens_host=torch.zeros(B, dtype=torch.int32), Hq=4)
+    with pytest.raises(ValueError):
+        kv.struct()
+    ix = P.PQIndex.allocate(B, Hkv, 4, 32, 4, "cpu")
+    with pytest.raises(ValueError):
+        ix.struct()
