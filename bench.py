@@ -47,12 +47,14 @@ def dram_traffic(kernel: str, workload: str):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--master-port", type=int, default=29511, help="rendezvous port when --gpus N spawns replicas")
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama8b_128k")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-train-build", action="store_true", help="skip the index-build-from-keys measurement")
     ap.add_argument("--sweep", choices=["ctx", "budget", "batch"], default=None,
                     help="extra measurements: context-length crossover, budget / background ablation, "
                          "or the 32-sequence batch at 32K")
@@ -96,21 +98,31 @@ def bf16_peak():
 # ---------------------------------------------------------------------------
 
 def step_bytes(w, n_idx: int, k: int):
-    """Per-step algorithmic HBM bytes of PQ-HSA, of dense decode and of the scan kernel."""
+    """Per-step algorithmic HBM bytes (what one step must move at least) of PQ-HSA and of dense
+    decode, the token-major cluster ids (layout overhead, reported apart), and the per-kernel
+    split of the PQ-HSA bytes. Intermediates that stay in L2 (scores, partials, cluster
+    weights) are not counted."""
     G, C, D = w.G, w.C, w.D
     R = w.T - w.n_sink - n_idx
+    lut = 4 * G * 16 * 256                       # PQ look-up table (written once, read once)
+    qc = 4 * G * C                               # q . centroid table (written once, read once)
     per_unit = (16 * n_idx                       # PQ codes
                 + 4 * C * D                      # centroids (q . centroid)
                 + 4 * 16 * 256 * 8               # codebook
-                + 4 * G * 16 * 256               # LUT written once
+                + lut                            # LUT written once
                 + 4 * C * D + 4 * C              # cluster mean values + counts
                 + 512 * (w.n_sink + R + k)       # exact K+V rows (bf16)
                 + 8 * G * D)                     # q in, out
     ids = 2 * n_idx
     dense = 512 * w.T + 8 * G * D
-    scan = n_idx * (16 + 2 + 4)                  # codes + cluster id read, selection score written
     U = w.B * w.Hkv
-    return U * per_unit, U * ids, U * dense, U * scan
+    kernels = {
+        "tables": U * (4 * C * D + 4 * 16 * 256 * 8 + 4 * G * D + lut + qc),   # reads + table writes
+        "scan_select": U * (16 * n_idx + lut + qc),                             # codes + tables
+        "attend": U * (512 * (w.n_sink + R + k) + 4 * C * D + 4 * C + 4 * G * D),
+        "merge": U * 4 * G * D,                                                # out
+    }
+    return U * per_unit, U * ids, U * dense, kernels
 
 
 # ---------------------------------------------------------------------------
@@ -167,28 +179,102 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-# CPU oracle sample (reported baseline, never the target)
+# CPU oracle sample (reported baseline, never the target): a process pool over the
+# (sequence, KV head) units, one single-threaded worker per core up to the unit count
+# and a host-memory bound; the KV pool is shared with the workers, not copied.
 # ---------------------------------------------------------------------------
 
-def oracle_sample(bt, w, budget, seconds: float):
-    """Run the float64 oracle on units of the workload until `seconds` elapse; µs per whole step."""
-    from threadpoolctl import threadpool_limits
+_ORC = {}
+
+
+def _orc_init(shm, small, n_sink, scale, budget, page_size):
+    """Pool worker start: attach the shared K/V pool, keep the small arrays."""
+    from multiprocessing import shared_memory
+    views = {}
+    handles = []
+    for name, (shm_name, shape, dtype) in shm.items():
+        h = shared_memory.SharedMemory(name=shm_name)
+        handles.append(h)
+        views[name] = np.ndarray(shape, dtype=dtype, buffer=h.buf)
+    _ORC.update(views)
+    _ORC.update(small)
+    _ORC.update(handles=handles, n_sink=n_sink, scale=scale, budget=budget, page_size=page_size)
+
+
+def _orc_unit(u):
+    """One (sequence, KV head) unit of the oracle's decode step in this worker."""
     import oracle as O
-    scale = float(np.float32(1.0 / math.sqrt(w.D)))
-    done, t0 = 0, time.perf_counter()
-    units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
-    with threadpool_limits(limits=1):
-        while True:
-            u = units[done % len(units)]
-            O.oracle_decode(bt.q, bt.k_cache, bt.v_cache, bt.block_table, bt.seq_lens, bt.centroids,
-                            bt.codebooks, bt.codes_rec, bt.ids_rec, bt.n_indexed, w.n_sink, scale,
-                            budget=budget, page_size=w.page_size, units=[u])
-            done += 1
-            el = time.perf_counter() - t0
-            if el >= seconds or done >= 4 * len(units):
-                break
-    us_per_step = el / done * len(units) * 1e6
-    return us_per_step, done, el
+    O.oracle_decode(_ORC["q"], _ORC["k_cache"], _ORC["v_cache"], _ORC["block_table"], _ORC["seq_lens"],
+                    _ORC["centroids"], _ORC["codebooks"], _ORC["codes_rec"], _ORC["ids_rec"], _ORC["n_indexed"],
+                    _ORC["n_sink"], _ORC["scale"], budget=_ORC["budget"], page_size=_ORC["page_size"], units=[u])
+    return u
+
+
+class OraclePool:
+    """The float64 oracle on the host cores: whole decode steps, units spread over a pool of
+    spawn-started single-threaded workers (BLAS limited to one thread each)."""
+
+    def __init__(self, bt, w, budget, workers=None):
+        import multiprocessing as mp
+        from multiprocessing import shared_memory
+        import psutil
+        self.units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+        # a worker widens one unit's K and V rows to float64 (plus temporaries)
+        per_worker = 4 * 8 * w.T * w.D * 2 + (64 << 20)
+        mem_cap = max(1, int(0.5 * psutil.virtual_memory().available // per_worker))
+        self.workers = workers or max(1, min(os.cpu_count() or 1, len(self.units), mem_cap))
+        self._shm = []
+        spec = {}
+        for name in ("k_cache", "v_cache"):
+            arr = getattr(bt, name)
+            h = shared_memory.SharedMemory(create=True, size=max(1, arr.nbytes))
+            np.ndarray(arr.shape, dtype=arr.dtype, buffer=h.buf)[...] = arr
+            self._shm.append(h)
+            spec[name] = (h.name, arr.shape, arr.dtype)
+        small = {n: getattr(bt, n) for n in ("q", "block_table", "seq_lens", "centroids", "codebooks", "codes_rec",
+                                             "ids_rec", "n_indexed")}
+        scale = float(np.float32(1.0 / math.sqrt(w.D)))
+        env = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in env:
+            os.environ[k] = "1"            # inherited by the spawned workers at start
+        try:
+            self.pool = mp.get_context("spawn").Pool(
+                self.workers, initializer=_orc_init, initargs=(spec, small, w.n_sink, scale, budget, w.page_size))
+        finally:
+            for k, v in env.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+
+    def step(self):
+        """Wall seconds of one whole decode step (every unit) on the pool."""
+        t0 = time.perf_counter()
+        self.pool.map(_orc_unit, self.units, chunksize=1)
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+        for h in self._shm:
+            h.close()
+            h.unlink()
+
+
+def oracle_sample(bt, w, budget, seconds: float, warmup: int = 1, min_steps: int = 1, max_steps: int = 1000):
+    """Whole oracle steps on the pool until `seconds` elapse (at least min_steps); returns
+    (µs per step, steps timed, worker count, seconds)."""
+    pool = OraclePool(bt, w, budget)
+    try:
+        for _ in range(warmup):
+            pool.step()
+        t, el = [], 0.0
+        while len(t) < max_steps and (len(t) < min_steps or el < seconds):
+            t.append(pool.step())
+            el += t[-1]
+        return sum(t) / len(t) * 1e6, len(t), pool.workers, el
+    finally:
+        pool.close()
 
 
 # ---------------------------------------------------------------------------
@@ -217,7 +303,6 @@ def run_ours(args):
     bt = make_batch(w)
     kv = P.PagedKV(**kv_tensors(bt, dev))
     ix = P.PQIndex(**index_tensors(bt, dev, n_indexed=np.zeros(w.B, dtype=np.int32)))
-    stream = torch.cuda.current_stream()
 
     # ---- index build after prefill: encode every indexed key on the GPU ----
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -240,6 +325,10 @@ def run_ours(args):
     for e in stage_ev:
         e.record()
     torch.cuda.synchronize()
+    # selected tokens per unit as the library counts them (the byte model's k)
+    n_sel = P.selected_counts(kv, ix, q, scale=scale, budget=budget, workspace_buf=ws)
+    k = int(n_sel.max())
+    assert int(n_sel.min()) == k, "every unit of the workload selects the same count"
 
     def hsa_step(events=None):
         P.hsa_decode(kv, ix, q, out, scale=scale, budget=budget, workspace_buf=ws, stage_events=events)
@@ -257,28 +346,21 @@ def run_ours(args):
     with torch.cuda.graph(g_dense):
         dense_step()
     torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def timed(graph, steps, e2e=None, staging=False):
+    def timed(graph, steps, staged=None):
         """Whole steps: one graph replay each, L2 flushed before, CUDA events around. With
-        e2e = (q_host, q, out, out_host) every step also moves q in from pinned host memory
-        and out back to it: by the copy engine, or (staging) by kernels that read and write
-        mapped views of the pinned buffers."""
+        staged = (q_view, out_view) every step also moves q in from and out back to pinned host
+        memory by copy kernels that read and write mapped views of the pinned buffers."""
         t = []
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         for _ in range(steps):
             flush.zero_()
             a.record()
-            if e2e is not None:
-                if staging:
-                    torch.mul(e2e[0], 1.0, out=e2e[1])
-                else:
-                    e2e[1].copy_(e2e[0], non_blocking=True)
+            if staged is not None:
+                torch.mul(staged[0], 1.0, out=q)
             graph.replay()
-            if e2e is not None:
-                if staging:
-                    torch.mul(e2e[2], 1.0, out=e2e[3])
-                else:
-                    e2e[3].copy_(e2e[2], non_blocking=True)
+            if staged is not None:
+                torch.mul(out, 1.0, out=staged[1])
             b.record()
             torch.cuda.synchronize()
             t.append(a.elapsed_time(b))
@@ -293,6 +375,29 @@ def run_ours(args):
         o.__cuda_array_interface__ = {"shape": tuple(t_host.shape), "typestr": "<f4",
                                       "data": (t_host.data_ptr(), False), "version": 3, "strides": None}
         return torch.as_tensor(o, device=dev)
+
+    q_h = torch.from_numpy(bt.q).pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_steps(steps):
+        """End to end through the public API, per step, by the host's wall clock: q copied in from
+        pinned host memory, one hsa_decode call through the binding (argument marshalling, host
+        validation, split planning, the launches), out copied back to pinned host memory, and the
+        wait for it. L2 is flushed, and the flush finished, before each step."""
+        t_wall, t_dev = [], []
+        for _ in range(steps):
+            flush.zero_()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            a.record()
+            q.copy_(q_h, non_blocking=True)
+            P.hsa_decode(kv, ix, q, out, scale=scale, budget=budget, workspace_buf=ws)
+            out_h.copy_(out, non_blocking=True)
+            b.record()
+            b.synchronize()
+            t_wall.append((time.perf_counter() - t0) * 1e3)
+            t_dev.append(a.elapsed_time(b))
+        return t_wall, t_dev
 
     def timed_stages(steps):
         """Per-kernel times: eager steps with the library's stage events on the launching stream."""
@@ -309,6 +414,7 @@ def run_ours(args):
         timed(g_hsa, 1)
         timed(g_dense, 1)
         timed_stages(1)
+        e2e_steps(1)
 
     if world > 1:
         dist.barrier()
@@ -317,76 +423,66 @@ def run_ours(args):
         t_hsa = timed(g_hsa, args.steps)
         t_stage = timed_stages(args.steps)
         t_dense = timed(g_dense, args.steps)
-        q_h = torch.from_numpy(bt.q).pin_memory()
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        t_e2e_ce = timed(g_hsa, args.steps, e2e=(q_h, q, out, out_h))
+        t_e2e, t_e2e_dev = e2e_steps(args.steps)
         try:
-            e2e_views = (mapped_view(q_h), q, out, mapped_view(out_h))
+            views = (mapped_view(q_h), mapped_view(out_h))
         except (RuntimeError, TypeError, ValueError):
-            e2e_views = None
-        t_e2e = t_e2e_ce
-        if e2e_views is not None:
-            timed(g_hsa, 2, e2e=e2e_views, staging=True)
-            t_staged = timed(g_hsa, args.steps, e2e=e2e_views, staging=True)
+            views = None
+        t_staged = None
+        if views is not None:
+            timed(g_hsa, 2, staged=views)
+            t_staged = timed(g_hsa, args.steps, staged=views)
             torch.cuda.synchronize()
-            if torch.equal(out_h, out.cpu()):      # the last step's result did reach host memory
-                t_e2e = t_staged
-            else:
-                e2e_views = None
+            if not torch.equal(out_h, out.cpu()):      # the last step's result did not reach host memory
+                t_staged = None
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     err = P.hsa_read_error(ws)
     assert err == 0, f"device error word {err}"
 
-    # ---- index build from raw keys: k-means centroids + PQ codebooks (8 + 8 Lloyd
-    # iterations), then encoding every indexed key; on a second index, warm, L2 flushed ----
-    from synth import train_init_slots
-    ix_t = P.PQIndex(**index_tensors(bt, dev, n_indexed=np.zeros(w.B, dtype=np.int32)))
-    init_t = torch.from_numpy(train_init_slots(w, w.n_indexed)).to(dev)
-    ws_t = P.workspace(P.hsa_train_workspace_bytes(kv, ix_t, w.n_indexed), dev)
-    ws_e = P.workspace(P.hsa_index_workspace_bytes(kv, ix_t, w.n_indexed), dev)
+    train_build_ms = None
+    if not args.no_train_build:
+        # ---- index build from raw keys: k-means centroids + PQ codebooks (8 + 8 Lloyd
+        # iterations), then encoding every indexed key; on a second index, warm, L2 flushed ----
+        from synth import train_init_slots
+        ix_t = P.PQIndex(**index_tensors(bt, dev, n_indexed=np.zeros(w.B, dtype=np.int32)))
+        init_t = torch.from_numpy(train_init_slots(w, w.n_indexed)).to(dev)
+        ws_t = P.workspace(P.hsa_train_workspace_bytes(kv, ix_t, w.n_indexed), dev)
+        ws_e = P.workspace(P.hsa_index_workspace_bytes(kv, ix_t, w.n_indexed), dev)
 
-    def build_from_keys():
-        P.hsa_train_index(kv, ix_t, w.n_indexed, init_t, workspace_buf=ws_t)
-        ix_t.n_indexed.zero_()
-        ix_t.n_indexed_host.zero_()
-        P.hsa_append_encode(kv, ix_t, w.n_indexed, workspace_buf=ws_e)
+        def build_from_keys():
+            P.hsa_train_index(kv, ix_t, w.n_indexed, init_t, workspace_buf=ws_t)
+            ix_t.n_indexed.zero_()
+            ix_t.n_indexed_host.zero_()
+            P.hsa_append_encode(kv, ix_t, w.n_indexed, workspace_buf=ws_e)
 
-    build_from_keys()
-    flush.zero_()
-    e0.record()
-    build_from_keys()
-    e1.record()
-    torch.cuda.synchronize()
-    train_build_ms = e0.elapsed_time(e1)
-    assert P.hsa_read_error(ws_t) == 0 and P.hsa_read_error(ws_e) == 0
-    del ix_t, ws_t, ws_e
+        build_from_keys()
+        flush.zero_()
+        e0.record()
+        build_from_keys()
+        e1.record()
+        torch.cuda.synchronize()
+        train_build_ms = round(e0.elapsed_time(e1), 3)
+        assert P.hsa_read_error(ws_t) == 0 and P.hsa_read_error(ws_e) == 0
+        del ix_t, ws_t, ws_e
 
-    ms_hsa = sum(t_hsa) / len(t_hsa)
-    ms_dense = sum(t_dense) / len(t_dense)
-    ms_e2e = sum(t_e2e) / len(t_e2e)
-    ms_e2e_ce = sum(t_e2e_ce) / len(t_e2e_ce)
-    ms_hsa, ms_dense, ms_e2e, ms_e2e_ce = max_over_ranks([ms_hsa, ms_dense, ms_e2e, ms_e2e_ce],
-                                                         dist if world > 1 else None, dev)
+    mean = lambda t: sum(t) / len(t)
+    ms_hsa, ms_dense, ms_e2e, ms_e2e_dev = max_over_ranks(
+        [mean(t_hsa), mean(t_dense), mean(t_e2e), mean(t_e2e_dev)], dist if world > 1 else None, dev)
 
-    stage_ms = [sum(s[i] for s in t_stage) / len(t_stage) for i in range(P.NUM_STAGES)]
+    stage_ms = [mean([s_[i] for s_ in t_stage]) for i in range(P.NUM_STAGES)]
     n_idx = int(w.n_indexed)
-    k = P.decode_k(budget, n_idx)
-    hsa_b, ids_b, dense_b, scan_b = step_bytes(w, n_idx, k)
+    hsa_b, ids_b, dense_b, kern_b = step_bytes(w, n_idx, k)
     peak, peak_kind = measured_peaks()
     dom = int(np.argmax(stage_ms))
     dom_name = P.STAGE_NAMES[dom]
-    U = w.B * w.Hkv
-    if dom_name == "scan":
-        dom_bytes = scan_b
-    elif dom_name == "attend":
-        dom_bytes = U * (512 * (w.n_sink + (w.T - w.n_sink - n_idx) + k) + 4 * w.C * w.D)
-    else:
-        dom_bytes = hsa_b
+    dom_bytes = kern_b[dom_name]
     dom_gbs = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
     step_gbs = hsa_b / (ms_hsa * 1e-3) / 1e9
     dense_gbs = dense_b / (ms_dense * 1e-3) / 1e9
+    traffic = dram_traffic(dom_name + "_kernel", w.name)
+    U = w.B * w.Hkv
 
     res = {
         "metric": METRIC,
@@ -408,7 +504,7 @@ def run_ours(args):
                    "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MB write) before every timed step",
                    "timing": "CUDA events per step around a CUDA-graph replay; per-kernel times from "
                              "eager steps with stage events on the launching stream"},
-        "percentiles_us": {f"p{q}": round(float(np.percentile(t_hsa, q)) * 1e3, 3) for q in (10, 50, 90)},
+        "percentiles_us": {f"p{q_}": round(float(np.percentile(t_hsa, q_)) * 1e3, 3) for q_ in (10, 50, 90)},
         "hbm_gbs": round(step_gbs, 1),
         "hbm_pct_peak": round(100 * step_gbs / peak, 2),
         "bytes_per_step": hsa_b,
@@ -417,27 +513,33 @@ def run_ours(args):
                   "hbm_gbs": round(dense_gbs, 1), "pct_peak": round(100 * dense_gbs / peak, 2),
                   "speedup_of_pqhsa": round(ms_dense / ms_hsa, 3)},
         "stages_us": {n: round(v * 1e3, 3) for n, v in zip(P.STAGE_NAMES, stage_ms)},
+        "stage_bytes": kern_b,
         "index_build_ms": round(build_ms, 3),
-        "index_train_and_encode_ms": round(train_build_ms, 3),
+        "index_train_and_encode_ms": train_build_ms,
         "roofline": {"kernel": dom_name, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
-                     "traffic": dram_traffic(dom_name + "_kernel", w.name), "algorithmic_bytes": dom_bytes},
+                     "traffic": traffic, "algorithmic_bytes": dom_bytes,
+                     "traffic_over_algorithmic": round(traffic / dom_bytes, 3) if traffic else None,
+                     "duration_us": round(stage_ms[dom] * 1e3, 3)},
         "e2e": {"value": round(ms_e2e * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": q.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 4,
-                "transfer": ("staging kernels read q from and write out to mapped pinned host memory"
-                             if e2e_views is not None else "copy engine (cudaMemcpyAsync) from/to pinned memory"),
-                "copy_engine_us": round(ms_e2e_ce * 1e3, 3)},
-        # per step: the PQ-HSA graph, the eager stage-timed step, the dense graph (attend +
-        # merge), the copy-engine end-to-end step, and (when used) the staged one plus 2 warm-ups
+                "how": "host wall clock per step: cudaMemcpyAsync of q from pinned host memory, one hsa_decode "
+                       "call through the Python binding (marshalling, validation, planning, launches), "
+                       "cudaMemcpyAsync of out to pinned host memory, wait",
+                "device_us": round(ms_e2e_dev * 1e3, 3),
+                "graph_staged_us": round(mean(t_staged) * 1e3, 3) if t_staged else None},
+        # our kernels in the timed region: graph steps (4 each), eager stage-timed steps (4),
+        # dense graph steps (attend + merge), end-to-end calls (4), staged graph steps (4, + 2 warm)
         "gpu_launches": args.steps * (3 * P.NUM_STAGES + 2) + (
-            (args.steps + 2) * P.NUM_STAGES if e2e_views is not None else 0),
+            (args.steps + 2) * P.NUM_STAGES if t_staged is not None else 0),
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        us, units, el = oracle_sample(bt, w, budget, args.cpu_seconds)
-        res["cpu_baseline"] = {"value": round(us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
-                               "sample": f"{units} (sequence, KV head) units of the same workload, "
-                                         f"{el:.1f} s of float64 numpy, scaled to a full step"}
+        us, steps, workers, el = oracle_sample(bt, w, budget, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": round(us, 1), "unit": "us/step", "cores": workers, "kind": "oracle",
+                               "sample": f"{steps} whole decode steps ({U} (sequence, KV head) units each, "
+                                         f"spread over {workers} single-threaded float64 numpy worker "
+                                         f"processes), {el:.1f} s"}
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -494,6 +596,12 @@ class _Setup:
                 t.append(a.elapsed_time(b))
         return sum(t) / len(t) * 1e3   # us
 
+    def k_selected(self, budget=0.01):
+        """Selected tokens per unit as the library reports them (every unit alike here)."""
+        n = self.P.selected_counts(self.kv, self.ix, self.q, scale=self.scale, budget=budget, workspace_buf=self.ws)
+        assert int(n.min()) == int(n.max())
+        return int(n.max())
+
     def hsa(self, budget=0.01, background=True):
         return lambda: self.P.hsa_decode(self.kv, self.ix, self.q, self.out, scale=self.scale, budget=budget,
                                          background=background, workspace_buf=self.ws)
@@ -503,6 +611,53 @@ class _Setup:
                                            workspace_buf=self.ws_dense)
 
 
+# Overhead-aware crossover model (rit.work "activation-kv-cache-sparsity-crossover", section
+# "Почему один и тот же способ даёт разное ускорение": a byte count gives the direction,
+# and adding each kernel's fixed launch and index cost predicts the measured crossover).
+
+def fit_overhead_model(nbytes, times_us):
+    """Least-squares fit of t = t0 + nbytes / bw to measured points; returns (t0 in µs, bw in
+    bytes per µs)."""
+    x = np.asarray(nbytes, dtype=np.float64)
+    y = np.asarray(times_us, dtype=np.float64)
+    A = np.stack([np.ones_like(x), x], axis=1)
+    (t0, slope), *_ = np.linalg.lstsq(A, y, rcond=None)
+    return float(t0), float(1.0 / slope) if slope > 0 else float("inf")
+
+
+def model_time(fit, nbytes):
+    t0, bw = fit
+    return t0 + nbytes / bw
+
+
+def predicted_crossover(fit_sparse, fit_dense, bytes_at, lengths):
+    """First length (of the increasing `lengths`) where the fitted sparse time is at most the
+    fitted dense time; bytes_at(T) gives (sparse bytes, dense bytes) at length T. None if never."""
+    for T in lengths:
+        hb, db = bytes_at(T)
+        if model_time(fit_sparse, hb) <= model_time(fit_dense, db):
+            return T
+    return None
+
+
+def measured_crossover(points):
+    """Length where the measured sparse and dense times cross, by linear interpolation of
+    (dense - sparse) between the two measured lengths that bracket the sign change;
+    points = [(T, sparse_us, dense_us)]. None if sparse never overtakes; the first length
+    if it already leads there."""
+    pts = sorted(points)
+    if pts and pts[0][2] - pts[0][1] >= 0:
+        return float(pts[0][0])
+    for (t0, h0, d0), (t1, h1, d1) in zip(pts, pts[1:]):
+        g0, g1 = d0 - h0, d1 - h1
+        if g0 < 0 <= g1:
+            return float(t0 + (t1 - t0) * (-g0) / (g1 - g0))
+    return None
+
+
+SWEEP_LENGTHS = (8192, 16384, 32768, 49152, 65536, 98304, 131072, 524288)
+
+
 def run_sweep_ctx(args):
     import torch
     from synth import workload
@@ -510,15 +665,16 @@ def run_sweep_ctx(args):
     torch.cuda.set_device(dev)
     peak, _ = measured_peaks()
     pts = []
-    for name in ("llama8b_8k", "llama8b_32k", "llama8b_sweep_128k", "llama8b_512k"):
-        w = workload(name)
+    base = workload("llama8b_8k")
+    for T in SWEEP_LENGTHS:
+        w = base.scaled(T=T, name=f"llama8b_sweep_{T // 1024}k")
         S = _Setup(w, dev)
-        k = S.P.decode_k(w.budget, w.n_indexed)
+        k = S.k_selected()
         hsa_b, ids_b, dense_b, _ = step_bytes(w, w.n_indexed, k)
         us_h = S.time_graph(S.graph(S.hsa()), args.steps, args.warmup)
         us_d = S.time_graph(S.graph(S.dense()), args.steps, args.warmup)
         assert S.P.hsa_read_error(S.ws) == 0
-        print(json.dumps({"sweep": "ctx", "workload": name, "T": w.T, "hsa_us": round(us_h, 3),
+        print(json.dumps({"sweep": "ctx", "workload": w.name, "T": w.T, "k": k, "hsa_us": round(us_h, 3),
                           "dense_us": round(us_d, 3), "speedup": round(us_d / us_h, 3),
                           "hsa_bytes": hsa_b, "ids_bytes": ids_b, "dense_bytes": dense_b,
                           "hsa_gbs": round(hsa_b / us_h / 1e3, 1), "dense_gbs": round(dense_b / us_d / 1e3, 1),
@@ -526,26 +682,21 @@ def run_sweep_ctx(args):
         pts.append((w, hsa_b, dense_b, us_h, us_d))
         del S
         torch.cuda.empty_cache()
-    # Overhead-aware model (crossover article): t = fixed + bytes / BW per method, fitted by
-    # least squares; the predicted crossover is the length where the two lines meet.
-    def fit(xs, ys):
-        xs, ys = np.asarray(xs, float), np.asarray(ys, float)
-        A = np.stack([np.ones_like(xs), xs], axis=1)
-        (a, b), *_ = np.linalg.lstsq(A, ys, rcond=None)
-        return float(a), float(b)
-    fh = fit([p_[1] for p_ in pts], [p_[3] for p_ in pts])
-    fd = fit([p_[2] for p_ in pts], [p_[4] for p_ in pts])
-    w0 = pts[0][0]
-    cross = None
-    for T in range(2048, 1 << 21, 256):
-        wt = w0.scaled(T=T)
+    fh = fit_overhead_model([p_[1] for p_ in pts], [p_[3] for p_ in pts])
+    fd = fit_overhead_model([p_[2] for p_ in pts], [p_[4] for p_ in pts])
+
+    def bytes_at(T):
+        wt = base.scaled(T=T)
         hb, _, db, _ = step_bytes(wt, wt.n_indexed, int(math.floor(wt.budget * wt.n_indexed)))
-        if fh[0] + fh[1] * hb <= fd[0] + fd[1] * db:
-            cross = T
-            break
-    print(json.dumps({"sweep": "ctx-model", "hsa_fixed_us": round(fh[0], 2), "hsa_gbs": round(1e-3 / fh[1], 1),
-                      "dense_fixed_us": round(fd[0], 2), "dense_gbs": round(1e-3 / fd[1], 1),
-                      "predicted_crossover_T": cross}), flush=True)
+        return hb, db
+
+    pred = predicted_crossover(fh, fd, bytes_at, range(2048, 1 << 21, 256))
+    meas = measured_crossover([(p_[0].T, p_[3], p_[4]) for p_ in pts])
+    print(json.dumps({"sweep": "ctx-model", "hsa_fixed_us": round(fh[0], 2), "hsa_gbs": round(fh[1] / 1e3, 1),
+                      "dense_fixed_us": round(fd[0], 2), "dense_gbs": round(fd[1] / 1e3, 1),
+                      "predicted_crossover_T": pred,
+                      "measured_crossover_T": None if meas is None else round(meas),
+                      "lengths": list(SWEEP_LENGTHS)}), flush=True)
 
 
 def run_sweep_batch(args):
@@ -557,7 +708,7 @@ def run_sweep_batch(args):
     peak, _ = measured_peaks()
     w = workload("batch32_32k")
     S = _Setup(w, dev)
-    k = S.P.decode_k(w.budget, w.n_indexed)
+    k = S.k_selected(w.budget)
     hsa_b, ids_b, dense_b, _ = step_bytes(w, w.n_indexed, k)
     us_h = S.time_graph(S.graph(S.hsa()), args.steps, args.warmup)
     us_d = S.time_graph(S.graph(S.dense()), args.steps, args.warmup)
@@ -696,33 +847,48 @@ def run_reference(args):
     from synth import make_batch, workload
     w = workload(args.workload)
     bt = make_batch(w)
-    per_step_seconds = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
-    for _ in range(args.warmup):
-        oracle_sample(bt, w, w.budget, per_step_seconds / 4)
-    t = []
-    units_total = 0
-    for _ in range(args.steps):
-        us, units, el = oracle_sample(bt, w, w.budget, per_step_seconds)
-        t.append(us)
-        units_total += units
-    us = sum(t) / len(t)
+    pool = OraclePool(bt, w, w.budget)
+    try:
+        for _ in range(args.warmup):
+            pool.step()
+        t = [pool.step() for _ in range(args.steps)]
+    finally:
+        pool.close()
+    us = sum(t) / len(t) * 1e6
+    U = w.B * w.Hkv
     res = {
         "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us/step",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.T, "budget": w.budget},
-        "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: whole (sequence, KV head) units of the workload for "
-                                   f"~{per_step_seconds:.1f} s, scaled to a full step of {w.B * w.Hkv} units "
-                                   f"({units_total} units timed over {args.steps} steps)"},
+        "data": "synthetic (seeded; no dataset or weights)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.D, "ctx": w.T,
+                   "clusters": w.C, "pq": "16x8/256", "sink": w.n_sink, "recent": w.n_recent,
+                   "budget": w.budget, "k": w.k, "page_size": w.page_size, "parallelism": "host cores",
+                   "l2": "n/a (host)", "timing": "host wall clock per whole step"},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": pool.workers, "kind": "oracle",
+                         "sample": f"{args.steps} whole decode steps ({U} (sequence, KV head) units each, "
+                                   f"spread over {pool.workers} single-threaded float64 numpy worker processes)"},
         "e2e": {"value": round(us, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(res), flush=True)
 
 
+def spawn_replicas(args, argv):
+    """`--gpus N` without a launcher: run N replicas, one process per GPU, under torch's launcher
+    (the same command the multi-GPU runs use); returns its exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={args.master_port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world and args.impl == "ours" and not (args.sweep or args.append or args.train):
+        if "WORLD_SIZE" in os.environ:
+            sys.exit(f"--gpus {args.gpus} but the launcher started {world} ranks")
+        sys.exit(spawn_replicas(args, argv))
     if args.sweep == "ctx":
         run_sweep_ctx(args)
     elif args.sweep == "budget":

@@ -27,8 +27,11 @@
  *   id or a timed-out wait is recorded in the workspace error word (see
  *   hsa_read_error) and the offending access is skipped.
  * - Workspaces must be 256-byte aligned and at least as large as the
- *   matching *_workspace_bytes() says; their contents need no initialisation
- *   and are clobbered.
+ *   matching *_workspace_bytes() says. Their first 4 bytes are the device error
+ *   word: it must be zero before the workspace's first use (allocate it zeroed,
+ *   or clear those bytes once); calls only OR bits into it, and hsa_read_error
+ *   reads and clears it. The rest of a workspace needs no initialisation and is
+ *   clobbered by every call.
  *
  * KV cache layout (bf16): [num_pages][Hkv][page_size][D], so one head-page is
  * page_size contiguous 256-byte rows. Token t of sequence b lives in page
@@ -115,9 +118,9 @@ typedef struct {
                                       before each stage and after the last one */
 } hsa_debug;
 
-/* Stages of hsa_decode, in launch order: tables, scan, filter, finalize,
-   exact+background attention, merge. stage_events[i] precedes stage i. */
-#define HSA_NUM_STAGES 6
+/* Stages of hsa_decode, in launch order: tables, scan+selection, exact+background
+   attention, merge. stage_events[i] precedes stage i. */
+#define HSA_NUM_STAGES 4
 #define HSA_STAGE_EVENTS (HSA_NUM_STAGES + 1)
 
 /* ---- decode -------------------------------------------------------------- */
@@ -147,8 +150,14 @@ size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv);
 
 /*
  * Dense split-K GQA decode: out_g = softmax(scale * q_g K^T) V over all T tokens of
- * each sequence (the in-library baseline; same split-K attention engine as the
- * exact part of hsa_decode). q, out: fp32 [B][Hq][D].
+ * each sequence. q, out: fp32 [B][Hq][D] (16-B aligned); the workspace as
+ * dense_decode_workspace_bytes says (its error word as for hsa_decode).
+ * The in-library baseline that PQ-HSA is measured against. The rit.work article
+ * "activation-kv-cache-sparsity-crossover", section "Почему один и тот же способ
+ * даёт разное ускорение", asks that dense and sparse decode read the cache through
+ * the same split-K kernel, so that a measured speed-up reflects the data saved and
+ * not a change of attention kernel: this call runs the same split-K engine (same
+ * tiles, same tensor-core consumers, same merge) as the exact part of hsa_decode.
  */
 hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, float scale,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -170,7 +179,10 @@ hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, floa
  * - Every call uses the same array and rewrites what it reads (nothing has to start
  *   at zero; the array keeps the last call's partials). Calls that overlap on the
  *   GPU (other streams or threads) race on it: serialise them.
- * - There is no error word: out-of-range block-table entries are skipped, not reported.
+ * - There is no error word: out-of-range block-table entries are skipped and a wait
+ *   that gives up (after 2 s) ends the call's copies early; neither is reported, and
+ *   in the second case the output is wrong. Callers that need these reported use
+ *   dense_decode with a workspace.
  */
 hsa_status dense_decode_static(const hsa_kv_cache* kv, const float* q, float* out, float scale,
                                cudaStream_t stream);

@@ -22,7 +22,7 @@ __all__ = [
     "PagedKV", "PQIndex", "HSAError", "load_library", "hsa_decode", "dense_decode",
     "hsa_build_from_codes", "hsa_append_encode", "hsa_decode_workspace_bytes",
     "dense_decode_workspace_bytes", "hsa_index_workspace_bytes", "hsa_read_error", "hsa_strerror",
-    "decode_k", "HSA_DEVERR_PAGE", "HSA_DEVERR_CLUSTER", "HSA_DEVERR_TIMEOUT", "HSA_DEVERR_SELECT",
+    "selected_counts", "HSA_DEVERR_PAGE", "HSA_DEVERR_CLUSTER", "HSA_DEVERR_TIMEOUT", "HSA_DEVERR_SELECT",
 ]
 
 HSA_DEVERR_PAGE, HSA_DEVERR_CLUSTER, HSA_DEVERR_TIMEOUT, HSA_DEVERR_SELECT = 1, 2, 4, 8
@@ -64,8 +64,8 @@ class _Debug(ctypes.Structure):
                 ("n_selected", ctypes.c_void_p), ("stage_events", ctypes.c_void_p)]
 
 
-NUM_STAGES = 6
-STAGE_NAMES = ("tables", "scan", "filter", "finalize", "attend", "merge")
+NUM_STAGES = 4
+STAGE_NAMES = ("tables", "scan_select", "attend", "merge")
 
 
 EXPORTS = ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode", "hsa_index_list_slots",
@@ -125,16 +125,6 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
 
 def hsa_strerror(status: int) -> str:
     return load_library().hsa_strerror(int(status)).decode()
-
-
-def decode_k(budget: float, n_indexed: int, k_override: int = -1) -> int:
-    """Selected tokens per unit, as the library computes it: floor(budget * N) in double."""
-    if n_indexed <= 0:
-        return 0
-    if k_override >= 0:
-        return min(k_override, n_indexed)
-    f = float(budget) * float(n_indexed)
-    return min(n_indexed, int(f) if f > 0 else 0)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -310,6 +300,17 @@ def hsa_decode(kv: PagedKV, index: PQIndex, q: torch.Tensor, out: Optional[torch
                         ctypes.byref(dbg), workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
     _check("hsa_decode", st)
     return out
+
+
+def selected_counts(kv: PagedKV, index: PQIndex, q: torch.Tensor, *, scale: float, budget: float = 0.01,
+                    k_override: int = -1, background: bool = True,
+                    workspace_buf: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Selected tokens per (sequence, KV head) as hsa_decode reports them: int32 [B, Hkv] on the
+    host, from one decode step with the n_selected debug output (synchronises the stream)."""
+    n_sel = torch.full((kv.B, kv.Hkv), -1, dtype=torch.int32, device=q.device)
+    hsa_decode(kv, index, q, scale=scale, budget=budget, k_override=k_override, background=background,
+               n_selected=n_sel, workspace_buf=workspace_buf)
+    return n_sel.cpu()
 
 
 def dense_decode(kv: PagedKV, q: torch.Tensor, out: Optional[torch.Tensor] = None, *, scale: float,

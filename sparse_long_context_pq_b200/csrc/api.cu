@@ -63,6 +63,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return g_encode;
 }
 
+// Programmatic dependent launch between the kernels of a call (and with the
+// previous call): every kernel waits on griddepcontrol before touching memory a
+// predecessor writes. PQHSA_NO_PDL=1 turns it off.
+bool use_pdl() {
+  static const bool on = [] {
+    const char* e = getenv("PQHSA_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+}  // namespace
+
+namespace pqhsa {
+
 // Tensor map over a paged cache viewed as rows of D bf16: [num_pages*Hkv*page_size][128],
 // box = 64 columns x box_rows rows, 128-byte swizzle.
 bool make_kv_tmap(CUtensorMap* map, const void* base, const hsa_kv_cache* kv, int box_rows) {
@@ -79,20 +97,7 @@ bool make_kv_tmap(CUtensorMap* map, const void* base, const hsa_kv_cache* kv, in
   return r == CUDA_SUCCESS;
 }
 
-// Programmatic dependent launch between the kernels of a call (and with the
-// previous call): every kernel waits on griddepcontrol before touching memory a
-// predecessor writes. PQHSA_NO_PDL=1 turns it off.
-bool use_pdl() {
-  static const bool on = [] {
-    const char* e = getenv("PQHSA_NO_PDL");
-    return !(e && e[0] == '1');
-  }();
-  return on;
-}
-
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
-
+// Validation of a KV-cache view shared by every entry point that reads the cache.
 hsa_status check_kv(const hsa_kv_cache* kv) {
   if (!kv || !kv->k_cache || !kv->v_cache || !kv->block_table || !kv->seq_lens || !kv->seq_lens_host)
     return HSA_ERR_INVALID_ARG;
@@ -111,6 +116,10 @@ hsa_status check_kv(const hsa_kv_cache* kv) {
     if (kv->seq_lens_host[b] < 0 || kv->seq_lens_host[b] > tmax) return HSA_ERR_CAPACITY;
   return HSA_OK;
 }
+
+}  // namespace pqhsa
+
+namespace {
 
 hsa_status check_index(const hsa_kv_cache* kv, const hsa_index* ix, bool need_codes) {
   if (!ix || !ix->centroids || !ix->codebooks || !ix->ids || !ix->mean_v || !ix->n_indexed || !ix->n_indexed_host)
@@ -367,7 +376,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   RET_CUDA(mark(0));
   RET_CUDA(launch_tables(G, tp, stream, use_pdl()));
 
-  ScanParams sc = {};
+  StepParams sc = {};
   sc.list_codes = ix->list_codes;
   sc.list_slot = ix->list_slot;
   sc.chunk_cluster = ix->chunk_cluster;
@@ -375,13 +384,29 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   sc.list_slots = ix->list_slots;
   sc.seq_lens = kv->seq_lens;
   sc.n_indexed = ix->n_indexed;
+  sc.codes = ix->codes;
+  sc.ids = ix->ids;
   sc.lut = lut;
   sc.qc = qc;
   sc.bounds = bounds;
+  sc.fbounds = fbounds;
   sc.W = W;
   sc.hist = hist;
   sc.sigma = sigma;
+  sc.chunk_max = cmax;
+  sc.bitmap = bitmap;
+  sc.cand = cand;
+  sc.cand_w = cand_w;
+  sc.cand_c = cand_c;
+  sc.units = units;
+  sc.sel = sel;
+  sc.block_table = kv->block_table;
+  sc.page_size = kv->page_size;
+  sc.max_pages = kv->max_pages;
+  sc.num_pages = kv->num_pages;
   sc.approx_logits = dbg ? dbg->approx_logits : nullptr;
+  sc.dbg_selected = dbg ? dbg->selected : nullptr;
+  sc.dbg_nselected = dbg ? dbg->n_selected : nullptr;
   sc.err = err;
   sc.B = kv->B;
   sc.Hq = kv->Hq;
@@ -389,58 +414,14 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   sc.cap = ix->cap;
   sc.C = ix->C;
   sc.nq = L.nq;
-  sc.fbounds = fbounds;
-  sc.chunk_max = cmax;
   sc.n_sink = ix->n_sink;
+  sc.bitmap_words = L.bitmap_words;
+  sc.k_override = prm->k_override;
+  sc.background = prm->background ? 1 : 0;
   sc.ring_depth = ring_depth;
+  sc.budget = prm->budget;
   RET_CUDA(mark(1));
-  RET_CUDA(launch_scan(G, sc, dev->sms, stream, use_pdl()));
-
-  SelectParams se = {};
-  se.list_codes = ix->list_codes;
-  se.chunk_cluster = ix->chunk_cluster;
-  se.list_slot = ix->list_slot;
-  se.list_meta = ix->list_meta;
-  se.list_slots = ix->list_slots;
-  se.seq_lens = kv->seq_lens;
-  se.n_indexed = ix->n_indexed;
-  se.codes = ix->codes;
-  se.ids = ix->ids;
-  se.lut = lut;
-  se.qc = qc;
-  se.bounds = bounds;
-  se.sigma = sigma;
-  se.hist = hist;
-  se.bitmap = bitmap;
-  se.cand = cand;
-  se.cand_w = cand_w;
-  se.cand_c = cand_c;
-  se.units = units;
-  se.sel = sel;
-  se.block_table = kv->block_table;
-  se.page_size = kv->page_size;
-  se.max_pages = kv->max_pages;
-  se.num_pages = kv->num_pages;
-  se.W = W;
-  se.dbg_selected = dbg ? dbg->selected : nullptr;
-  se.dbg_nselected = dbg ? dbg->n_selected : nullptr;
-  se.err = err;
-  se.B = kv->B;
-  se.Hkv = kv->Hkv;
-  se.cap = ix->cap;
-  se.C = ix->C;
-  se.nq = L.nq;
-  se.fbounds = fbounds;
-  se.chunk_max = cmax;
-  se.n_sink = ix->n_sink;
-  se.bitmap_words = L.bitmap_words;
-  se.k_override = prm->k_override;
-  se.background = prm->background ? 1 : 0;
-  se.budget = prm->budget;
-  RET_CUDA(mark(2));
-  RET_CUDA(launch_filter(G, se, dev->sms * 2, stream, use_pdl()));
-  RET_CUDA(mark(3));
-  RET_CUDA(launch_finalize(G, se, stream, use_pdl()));
+  RET_CUDA(launch_scan_select(G, sc, dev->sms, stream, use_pdl()));
 
   AttendParams p = {};
   p.k_cache = static_cast<const uint8_t*>(kv->k_cache);
@@ -478,12 +459,12 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   p.k_override = prm->k_override;
   p.budget = prm->budget;
   p.qscale = prm->scale * kLog2e;
-  RET_CUDA(mark(4));
+  RET_CUDA(mark(2));
   RET_CUDA(launch_attend(G, true, true, tk, tv, p, U * (sp.nsplit + L.nbg), stream, use_pdl()));
   MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, S_tot};
-  RET_CUDA(mark(5));
+  RET_CUDA(mark(3));
   RET_CUDA(launch_merge(G, mp, stream, use_pdl()));
-  RET_CUDA(mark(6));
+  RET_CUDA(mark(4));
   return HSA_OK;
 }
 

@@ -194,7 +194,14 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
         if (lane < nbox) {
           const int v = row0 + lane;
           if (kExact && v >= s0 + R) {
-            ys[i] = sel_u[v - s0 - R];   // already a KV-pool row (checked by the selection)
+            // already a KV-pool row (checked by the selection); an entry the selection did
+            // not write cannot become an out-of-range read
+            int y = sel_u[v - s0 - R];
+            if (y < 0 || y >= p.num_pages * p.Hkv * p.page_size) {
+              record_error(p.err, HSA_DEVERR_SELECT);
+              y = 0;
+            }
+            ys[i] = y;
           } else {
             const int pos = kExact ? exact_tail_pos(v, s0, N) : row0 + lane * box_rows;
             int page = (pos >= 0 && pos < T && pos / p.page_size < p.max_pages) ? bt[pos / p.page_size] : -1;

@@ -268,6 +268,12 @@ __device__ __forceinline__ float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
+// Largest value over the full warp in one instruction (sm_100a redux of f32).
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -283,14 +289,21 @@ __host__ __device__ inline long long list_slots_needed(int cap, int C) {
 
 // Workspace layout of hsa_decode (computed identically on host and device).
 // ---------------------------------------------------------------------------
-struct UnitState {          // per unit bookkeeping written by the top-k kernels
+// Per unit bookkeeping of the scan and selection (zeroed by the tables). Each unit's state
+// takes its own 128-byte lines, and its ready flag (polled by the attention CTAs while the
+// selection runs) a line of its own, so polling never slows the counters' atomics.
+struct alignas(128) UnitState {
   int32_t bstar;            // threshold bin
   int32_t above;            // tokens in bins above bstar
   int32_t ncand;            // tokens in bin bstar (candidates)
-  int32_t nsel;             // selected count written by finalize
+  int32_t nsel;             // selected count written by the resolution
+  int32_t scan_done;        // chunks of the unit scanned (histogram, weights and scores written)
+  int32_t filt_done;        // chunks of the unit whose selections and candidates are written
+  int32_t pad0[26];
   int32_t ready;            // set (release) once the unit's selection and weight fix-up are final
-  int32_t pad[3];
+  int32_t pad1[31];
 };
+static_assert(sizeof(UnitState) == 256, "two 128-byte lines per unit");
 
 // Publish a per-unit flag after this CTA's writes: call from every thread of the CTA.
 __device__ __forceinline__ void publish_flag(int32_t* flag) {
@@ -314,6 +327,23 @@ __device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t* err) {
     __nanosleep(256);
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
     if (v) return true;
+    if (global_ns() - t0 > kWaitLimitNs) break;
+  }
+  record_error(err, HSA_DEVERR_TIMEOUT);
+  return false;
+}
+
+// Bounded wait (acquire) until a counter that other resident CTAs of this grid advance
+// reaches `target`; a timeout is recorded and returns false. One thread calls it.
+__device__ __forceinline__ bool wait_count(const int32_t* ctr, int32_t target, int32_t* err) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+  if (v >= target) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    __nanosleep(64);
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
     if (global_ns() - t0 > kWaitLimitNs) break;
   }
   record_error(err, HSA_DEVERR_TIMEOUT);

@@ -91,6 +91,11 @@ struct MergeParams {
 template <int G>
 __device__ void background_block(const AttendParams& p, int j, uint8_t* smem);
 
+// Host-side helpers shared by the entry points (api.cu).
+hsa_status check_kv(const hsa_kv_cache* kv);   // shapes, alignment and lengths of a KV-cache view
+// Tensor map over a paged cache viewed as rows of D bf16, box = 64 columns x box_rows rows.
+bool make_kv_tmap(CUtensorMap* map, const void* base, const hsa_kv_cache* kv, int box_rows);
+
 int attend_slots_per_sm();
 size_t attend_smem_bytes(int G);
 // Row sources: kExact = sink + selected + tail list of hsa_decode, else every token.
@@ -116,7 +121,12 @@ struct TablesParams {
 };
 cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, bool pdl);
 
-struct ScanParams {
+// One launch after the tables: the scan of the codes (phase 1), then, per unit, the
+// selection (phase 2: threshold bin from the unit's histogram, definite selections and
+// threshold-bin candidates of this CTA's chunks, weight fix-ups) and its resolution by
+// the unit's last CTA (phase 3: exact order of the candidates, ascending write-out of
+// the selected rows, ready flag).
+struct StepParams {
   const uint8_t* list_codes;     // [U][list_slots][16] cluster-ordered codes
   const int32_t* list_slot;      // [U][list_slots] index slot of each list slot (-1 empty)
   const uint16_t* chunk_cluster; // [U][list_slots / 32]
@@ -124,57 +134,35 @@ struct ScanParams {
   int list_slots;
   const int32_t* seq_lens;
   const int32_t* n_indexed;
+  const uint8_t* codes;          // [U][cap][16] (weights of winners past the stored candidates)
+  const uint16_t* ids;           // [U][cap]
   const float* lut;
   const float* qc;
   const float* bounds;
-  float* fbounds;            // [U][2][G] final (ub, lb), written here
+  float* fbounds;                // [U][2][G] final (ub, lb), written by the scan
   float* W;
   uint32_t* hist;
-  float* sigma;              // [U][list_slots]
-  float* chunk_max;          // [U][list_slots / 32] largest sigma of each chunk
-  float* approx_logits;      // debug [B][Hq][cap] or null
-  int32_t* err;
-  int B, Hq, Hkv, cap, C, nq, n_sink;
-  int ring_depth;            // chunk slots per warp (scan_ring_depth)
-};
-cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t stream, bool pdl);
-int scan_ring_depth(int G, int C);   // 0: the tables do not fit in shared memory
-size_t scan_smem_bytes(int G, int C);
-
-struct SelectParams {
-  const uint8_t* list_codes;     // [U][list_slots][16]
-  const uint16_t* chunk_cluster; // [U][list_slots / 32]
-  const int32_t* list_slot;      // [U][list_slots]
-  const int32_t* list_meta;      // [U][2 + 2C]
-  int list_slots;
-  const int32_t* seq_lens;
-  const int32_t* n_indexed;
-  const uint8_t* codes;
-  const uint16_t* ids;
-  const float* lut;
-  const float* qc;
-  const float* bounds;
-  const float* fbounds;      // [U][2][G] final (ub, lb) from the scan
-  const float* sigma;
-  const float* chunk_max;        // [U][list_slots / 32]
-  const uint32_t* hist;
-  uint32_t* bitmap;
-  unsigned long long* cand;  // [U][cap]
-  float* cand_w;             // [U][kCandWeights][G] e^{shat_g - ub_g} of the first candidates
-  int32_t* cand_c;           // [U][kCandWeights] their clusters
+  float* sigma;                  // [U][list_slots]
+  float* chunk_max;              // [U][list_slots / 32] largest sigma of each chunk
+  uint32_t* bitmap;              // [U][bitmap_words] selected index slots
+  unsigned long long* cand;      // [U][cap] threshold-bin candidates (score key, slot)
+  float* cand_w;                 // [U][kCandWeights][G] e^{shat_g - ub_g} of the first candidates
+  int32_t* cand_c;               // [U][kCandWeights] their clusters
   UnitState* units;
-  int32_t* sel;              // [U][cap] KV-pool row of each selected token, ascending position
-  float* W;
-  const int32_t* block_table;  // [B][max_pages]
+  int32_t* sel;                  // [U][cap] KV-pool row of each selected token, ascending position
+  const int32_t* block_table;    // [B][max_pages]
   int page_size, max_pages, num_pages;
-  int32_t* dbg_selected;     // [U][cap] or null (positions)
-  int32_t* dbg_nselected;    // [U] or null
+  float* approx_logits;          // debug [B][Hq][cap] or null
+  int32_t* dbg_selected;         // [U][cap] or null (positions)
+  int32_t* dbg_nselected;        // [U] or null
   int32_t* err;
-  int B, Hkv, cap, C, nq, n_sink, bitmap_words, k_override, background;
+  int B, Hq, Hkv, cap, C, nq, n_sink, bitmap_words, k_override, background;
+  int ring_depth;                // chunk slots per warp (scan_ring_depth)
   double budget;
 };
-cudaError_t launch_filter(int G, const SelectParams& p, int grid, cudaStream_t stream, bool pdl);
-cudaError_t launch_finalize(int G, const SelectParams& p, cudaStream_t stream, bool pdl);
+cudaError_t launch_scan_select(int G, const StepParams& p, int grid, cudaStream_t stream, bool pdl);
+int scan_ring_depth(int G, int C);   // 0: the tables do not fit in shared memory
+size_t scan_smem_bytes(int G, int C);
 
 // ---- index maintenance -----------------------------------------------------
 struct IndexParams {

@@ -1,16 +1,14 @@
 // PQ-HSA scoring and selection kernels:
-//   tables   - per-query PQ look-up tables and centroid terms (q . codeword, q . centroid),
-//              plus exact upper/lower bounds of every head's approximate logit;
-//   scan     - one pass over the uint8 codes: approximate logits of every indexed
-//              token, the selection score sigma = max over the group's heads,
-//              per-cluster exp-weight sums, a histogram of sigma, each chunk's
-//              largest sigma and the final logit bounds;
-//   filter   - marks tokens above the threshold histogram bin, collects the
-//              tokens in that bin as candidates (reading only chunks that reach
-//              the bin) and removes the definite selections' weights;
-//   finalize - resolves the candidates exactly (score desc, position asc),
-//              writes the selected tokens as KV-pool rows in ascending position
-//              order, removes the winners' weights and publishes the unit.
+//   tables      - per-query PQ look-up tables and centroid terms (q . codeword, q . centroid),
+//                 plus exact upper/lower bounds of every head's approximate logit;
+//   scan+select - one launch: a pass over the uint8 codes (approximate logits of every
+//                 indexed token, the selection score sigma = max over the group's heads,
+//                 per-cluster exp-weight sums, a histogram of sigma, each chunk's largest
+//                 sigma); then, per unit, the tokens above the threshold histogram bin
+//                 (selected) and in it (candidates), the selected tokens' weights taken
+//                 out of the cluster sums; then the unit's last CTA resolves the
+//                 candidates exactly (score desc, position asc), writes the selected
+//                 tokens as KV-pool rows in ascending position order and publishes the unit.
 //
 // Source: rit.work "pq-hsa-long-context-attention", section
 // "Как приблизительные оценки возвращают отброшенный контекст" (an approximate
@@ -41,36 +39,6 @@ __device__ __forceinline__ float warp_min(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
-}
-
-// One full warp: over counts cnt[0..nbins) (nbins a multiple of 32), find the bin
-// b such that sum_{b' > b} cnt < need <= sum_{b' >= b} cnt. Writes *bin/*above
-// only when such a bin exists.
-__device__ void find_threshold_desc(const uint32_t* cnt, int nbins, uint32_t need, int* bin, uint32_t* above) {
-  const int lane = threadIdx.x & 31;
-  const int per = nbins / 32;
-  const int hi = nbins - per * lane;   // lane 0 holds the highest bins
-  const int lo = hi - per;
-  uint32_t local = 0;
-  for (int i = lo; i < hi; ++i) local += cnt[i];
-  uint32_t incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  const uint32_t excl = incl - local;
-  if (need > 0 && excl < need && incl >= need) {
-    uint32_t cum = excl;
-    for (int i = hi - 1; i >= lo; --i) {
-      if (cum + cnt[i] >= need) {
-        *bin = i;
-        *above = cum;
-        break;
-      }
-      cum += cnt[i];
-    }
-  }
 }
 
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
@@ -265,31 +233,41 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
 }
 
 // ===========================================================================
-// scan
+// scan + select: one launch, one 512-thread CTA per SM
 // ===========================================================================
-// One CTA per SM: 16 warps share one copy of the tables. Each lane streams the codes
-// (16 B) and index slot (4 B) of its own list slot, for the warp's next D chunks, into a
-// private ring with LSU async copies (one commit group per chunk), so D chunks per warp
-// are in flight while it scores the current one.
-// threads per scan CTA (one CTA per SM; registers bound the warp count)
-template <int G>
-__host__ __device__ constexpr int scan_threads_of() { return 512; }
-constexpr int kRingCodeBytes = 32 * kM;                     // 512 per chunk
-constexpr int kRingJsBytes = 32 * 4;                        // index slots
-constexpr int kRingSlotBytes = kRingCodeBytes + kRingJsBytes + 16;   // + cluster word (16-B cell) = 656
+// Phase 1 (scan): every CTA streams its chunks of the cluster-ordered code lists and
+// scores them against the unit's tables in shared memory: approximate logits, the
+// selection score sigma, per-cluster exp-weight sums, a histogram of sigma and each
+// chunk's largest sigma. Phase 2 (filter), per unit, once every CTA of the unit has
+// scanned its chunks: the threshold bin from the unit's histogram, the definite
+// selections (bitmap), the threshold-bin candidates and the weight fix-ups of this
+// CTA's chunks. Phase 3 (resolution), by the unit's last CTA to finish phase 2: the
+// exact order of the candidates (score desc, position asc), the selected tokens as
+// KV-pool rows in ascending position order, the winners' weight fix-ups, the ready flag.
+//
+// The per-unit wait of phase 2 only waits on CTAs of the same grid, which are all
+// resident: the grid has one CTA per SM and each CTA needs a whole SM's registers,
+// and a dependent launch starts only after every CTA of this grid has started.
+constexpr int kScanThreads = 512;
+constexpr int kScanWarps = kScanThreads / 32;
+constexpr int kRingCodeBytes = 32 * kM;                    // 512 per chunk
+constexpr int kRingSlotBytes = kRingCodeBytes + 16;        // + a 16-B cell with the cluster word
 constexpr size_t kScanSmemLimit = 226 * 1024;   // dynamic; the rest of 227 KB is static
 
 template <int G>
 struct ScanSmem {
   static constexpr int GP = (G + 3) / 4;
-  // tables (LUT, centroid terms) and the score histogram; then the warps' rings
-  // ([D][32][16 B] codes, [D][32] index slots, [D] 16-B cells holding the 4-byte word
-  // with the chunk's cluster id, per warp); then the tables mbarrier
-  __host__ __device__ static size_t tables(int C) {
-    return align_up(static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16 + kNB * 4, 128);
+  // LUT [GP][256][16] float4, centroid terms [GP][C] float4, the open chunk and fill of
+  // every cluster [C] u32, the score histogram [NB] u32; then the warps' rings ([D][32]
+  // 16-B code rows and [D] 16-B cells holding the 4-byte word with the chunk's cluster id,
+  // per warp); then the tables mbarrier.
+  __host__ __device__ static size_t meta_off(int C) {
+    return static_cast<size_t>(GP) * kNcode * kM * 16 + static_cast<size_t>(GP) * C * 16;
   }
+  __host__ __device__ static size_t hist_off(int C) { return meta_off(C) + align_up(static_cast<size_t>(C) * 4, 16); }
+  __host__ __device__ static size_t tables(int C) { return align_up(hist_off(C) + kNB * 4, 128); }
   __host__ __device__ static size_t bytes(int C, int depth) {
-    return tables(C) + static_cast<size_t>(scan_threads_of<G>() / 32) * depth * kRingSlotBytes + 8;
+    return tables(C) + static_cast<size_t>(kScanWarps) * depth * kRingSlotBytes + 8;
   }
   // deepest ring (8, 4 or 2 chunks per warp) that fits; 0 if none does
   static int depth(int C) {
@@ -298,6 +276,57 @@ struct ScanSmem {
     return 0;
   }
 };
+
+// Phase-2 scratch (after the tables; over the histogram and the rings) and phase-3
+// scratch (from the start of dynamic shared memory, over the tables).
+constexpr int kCmPerThread = 4;                                  // chunk maxima per thread per pass
+constexpr int kCmPass = kCmPerThread * kScanThreads;             // chunks examined per pass
+constexpr int kActPerWarp = 2;                                   // active chunks per warp per round
+constexpr int kFixCap = kActPerWarp * kScanThreads;              // queued tokens per round
+constexpr size_t kFilterScratch = (kCmPass + 2 * kFixCap) * 4;
+constexpr int kFinWordsPerThread = 8;
+constexpr int kFinChunkWords = kFinWordsPerThread * kScanThreads;   // 131072 slots per pass
+constexpr int kFinSmemCand = 1024;                                  // candidates resolved in shared memory
+constexpr int kFinBt = 8192;                                        // block-table entries staged in shared memory
+constexpr size_t kFinScratch =
+    kFinSmemCand * 8 + 2 * kFinChunkWords * 4 + kFinSmemCand * 4 + 256 * 4 + kFinBt * 4;
+static_assert(kFilterScratch <= kNB * 4 + kScanWarps * 2 * kRingSlotBytes, "filter scratch fits");
+// the smallest scan layout (G = 1, C = 1, 8-deep rings) is 141 KB of dynamic shared memory
+static_assert(kFinScratch <= 128 * 1024, "resolution scratch fits in the scan's shared memory");
+static_assert(kCandWeights <= kFinSmemCand, "stored candidate weights are resolved in shared memory");
+
+constexpr int kMaxParts = 24;   // (unit, chunk range) parts one CTA plans in shared memory
+#ifndef PQHSA_SCAN_PAIR
+#define PQHSA_SCAN_PAIR 1
+#endif
+constexpr bool kScanPair = PQHSA_SCAN_PAIR != 0;   // phase 1 scores two chunks per warp step
+
+struct SelShared {
+  uint32_t scan_tot[33];
+  long long red[kScanWarps];
+  int bstar;
+  uint32_t above;
+  int n_act;
+  uint32_t fix_n;
+  int flag;
+  uint32_t nwin;
+  int bin;
+  uint32_t fin_above;
+  int res[kMaxParts];            // units this CTA resolves after its filter parts
+  // this CTA's parts
+  int nparts;                    // -1: more than kMaxParts, walk the units instead
+  int pu[kMaxParts], pc0[kMaxParts], pc1[kMaxParts];
+  long long total;
+  int active;
+};
+
+// Chunks of unit u's lists to scan (0 if nothing is indexed); its three loads go out together.
+__device__ __forceinline__ int unit_chunks(const StepParams& p, int u) {
+  const int b = u / p.Hkv;
+  const int n = p.list_meta[static_cast<size_t>(u) * (2 + 2 * static_cast<size_t>(p.C))];
+  const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
+  return N == 0 ? 0 : max(0, min(n, p.list_slots / 32));
+}
 
 template <int G>
 __device__ __forceinline__ void score_token(const uint4& code, uint32_t id, const uint8_t* lut_b, const float4* qc_s,
@@ -369,12 +398,26 @@ __device__ __forceinline__ float warp_sum_scatter(float* v) {
   return t;
 }
 
-// Chunks [ch0, ch1) of unit u's cluster-ordered list: one warp scores one 32-slot
-// chunk (all members of one cluster), so the centroid term is warp-uniform and the
-// chunk's cluster weights are one warp reduction. Warp w takes chunks ch0 + w + 16 i
-// through its D-slot ring; `phase` counts segments (tables mbarrier parity).
+// Add the warp's per-lane weight sums of one cluster run to the cluster's sums.
+template <int G>
+__device__ __forceinline__ void flush_weights(const float* acc, float* Wu, int C, uint32_t c) {
+  float v[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) v[g] = acc[g];
+  const float e = warp_sum_scatter<G>(v);
+  constexpr int kGroup = 32 / G;
+  const int lane = threadIdx.x & 31;
+  if ((lane & (kGroup - 1)) == 0) atomicAdd(Wu + (lane / kGroup) * C + c, e);
+}
+
+// Phase 1 for chunks [ch0, ch1) of unit u: one warp scores one 32-slot chunk (members of
+// one cluster) at a time, so the centroid term is warp-uniform. Warp w takes a contiguous
+// run of the range through its D-slot ring of async copies (one commit group per chunk);
+// consecutive chunks of one cluster add their weights in registers, and the warp reduces
+// them once per cluster run. A chunk's valid slots are a prefix: all 32, or the cluster's
+// fill count for its open chunk. `phase` counts segments (tables mbarrier parity).
 template <int G, int D>
-__device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0, int ch1, uint8_t* smem,
+__device__ __forceinline__ void scan_segment(const StepParams& p, int u, int ch0, int ch1, uint8_t* smem,
                                              uint64_t* bar, uint32_t phase, float* sh_bounds,
                                              const uint32_t ysoff[8], const uint32_t sel[4], bool swap_words) {
   constexpr int GP = (G + 3) / 4;
@@ -386,13 +429,13 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
   const uint32_t qc_bytes = GP * C * 16;
   float4* lut_s = reinterpret_cast<float4*>(smem);                               // [GP][256][16]
   float4* qc_s = lut_s + GP * kNcode * kM;                                       // [GP][C]
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(qc_s + GP * C);                 // [NB]
+  uint32_t* meta_s = reinterpret_cast<uint32_t*>(smem + ScanSmem<G>::meta_off(C));   // [C]
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + ScanSmem<G>::hist_off(C));   // [NB]
   uint8_t* wring = smem + ScanSmem<G>::tables(C) + static_cast<size_t>(warp) * D * kRingSlotBytes;
   uint4* ring_code = reinterpret_cast<uint4*>(wring) + lane;                              // [D][32]
-  int32_t* ring_js = reinterpret_cast<int32_t*>(wring + D * kRingCodeBytes) + lane;       // [D][32]
-  uint32_t* ring_cl = reinterpret_cast<uint32_t*>(wring + D * (kRingCodeBytes + kRingJsBytes));   // [D][4]
+  uint32_t* ring_cl = reinterpret_cast<uint32_t*>(wring + D * kRingCodeBytes);            // [D][4]
 
-  __syncthreads();  // previous segment finished with shared memory
+  __syncthreads();  // previous segment (or planning) finished with shared memory
   if (tid == 0) {
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(bar, lut_bytes + qc_bytes);
@@ -403,25 +446,26 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
     for (uint32_t o = 0; o < qc_bytes; o += 32768u)
       bulk_load(reinterpret_cast<uint8_t*>(qc_s) + o, qg + o, min(32768u, qc_bytes - o), bar);
   }
+  const int max_chunks = p.list_slots / 32;
   const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
-  const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
-  const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * (p.list_slots / 32);
+  const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * max_chunks;
   float* sig_u = p.sigma + static_cast<size_t>(u) * p.list_slots;
+  float* cmax_u = p.chunk_max + static_cast<size_t>(u) * max_chunks;
   float* Wu = p.W + static_cast<size_t>(u) * G * C;
   const uint8_t* lut_b = reinterpret_cast<const uint8_t*>(lut_s);
 
-  // this warp's chunks; the first D go out while the tables land (one commit group per
-  // chunk, empty groups past the end keep the count regular). The chunk's cluster id
-  // (u16) comes with lane 0's group as the aligned 4-byte word that holds it.
-  const int first = ch0 + warp;
-  constexpr int kScanWarps = scan_threads_of<G>() / 32;
-  const int cnt = first < ch1 ? (ch1 - first + kScanWarps - 1) / kScanWarps : 0;
+  // this warp's contiguous run [wb, we); the first D chunks go out while the tables land
+  const int nch = ch1 - ch0;
+  const int wb = ch0 + static_cast<int>(static_cast<long long>(nch) * warp / kScanWarps);
+  const int we = ch0 + static_cast<int>(static_cast<long long>(nch) * (warp + 1) / kScanWarps);
+  const int cnt = we - wb;
+  // The chunk's cluster id (u16) comes with lane 0's group as the aligned 4-byte word
+  // that holds it; empty commit groups past the end keep the group count regular.
   auto issue = [&](int i) {
     if (i < cnt) {
-      const int ch = first + kScanWarps * i;
+      const int ch = wb + i;
       const int slot = i % D;
       cp_async_16(ring_code + slot * 32, lcodes + static_cast<size_t>(ch) * 32 + lane);
-      cp_async_4(ring_js + slot * 32, lslot + static_cast<size_t>(ch) * 32 + lane);
       if (lane == 0)
         cp_async_4(ring_cl + slot * 4,
                    reinterpret_cast<const void*>(reinterpret_cast<uintptr_t>(ccl + ch) & ~uintptr_t(3)));
@@ -431,13 +475,22 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
 #pragma unroll
   for (int i = 0; i < D; ++i) issue(i);
 
-  for (int i = tid; i < kNB; i += blockDim.x) hist_s[i] = 0u;
-  if (warp == 0) {   // final bounds of the unit, once: this CTA's copy and the later kernels'
+  {   // open chunk (26 bits) and its fill (6 bits) of every cluster; all-ones: no open chunk
+    const int32_t* mg = p.list_meta + static_cast<size_t>(u) * (2 + 2 * static_cast<size_t>(C));
+    for (int c = tid; c < C; c += kScanThreads) {
+      const int op = mg[2 + 2 * c], fl = mg[3 + 2 * c];
+      meta_s[c] = (op >= 0 && op < (1 << 26)) ? ((static_cast<uint32_t>(op) << 6) |
+                                                  static_cast<uint32_t>(min(max(fl, 0), 32)))
+                                              : 0xffffffffu;
+    }
+  }
+  for (int i = tid; i < kNB; i += kScanThreads) hist_s[i] = 0u;
+  if (warp == 0) {   // final bounds of the unit: this CTA's copy and the later phases'
     reduce_bounds_warp<G>(p.bounds, u, p.nq, sh_bounds, sh_bounds + G);
     __syncwarp();
     if (lane < 2 * G) p.fbounds[static_cast<size_t>(u) * 2 * G + lane] = sh_bounds[lane];
   }
-  __syncthreads();                       // zeroed histogram and bounds visible
+  __syncthreads();                       // histogram, cluster fills and bounds visible
   float ub2[G], lo, inv;
   {
     float ub[G], lb[G];
@@ -458,177 +511,123 @@ __device__ __forceinline__ void scan_segment(const ScanParams& p, int u, int ch0
   }
   mbar_wait(bar, phase & 1, p.err);      // tables landed
   bool bad_id = false;
+  uint32_t cur = 0xffffffffu;            // cluster of the current run
+  float wacc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) wacc[g] = 0.f;
 
-  for (int i = 0; i < cnt; ++i) {
+  // Chunk (slot) -> its code row, cluster and fill; then the scores of the chunk's valid
+  // slots are stored, reduced and binned (the weight run is per chunk, in list order).
+  auto chunk_in = [&](int i, uint4& code, uint32_t& id, int& fill) {
     const int slot = i % D;
-    cp_async_wait<D - 1>();              // this lane's copies of chunk i have landed
-    __syncwarp();                        // ... and lane 0's cluster word
-    const uint4 code = ring_code[slot * 32];
-    const int32_t js = ring_js[slot * 32];
-    const int ch = first + kScanWarps * i;
+    const int ch = wb + i;
+    code = ring_code[slot * 32];
     const uint32_t cw = ring_cl[slot * 4];
-    uint32_t id = ((reinterpret_cast<uintptr_t>(ccl + ch) >> 1) & 1) ? (cw >> 16) : (cw & 0xffffu);
+    id = ((reinterpret_cast<uintptr_t>(ccl + ch) >> 1) & 1) ? (cw >> 16) : (cw & 0xffffu);
+    fill = 32;
     if (id >= static_cast<uint32_t>(C)) {
       bad_id = true;
       id = 0;
+      fill = 0;
+    } else {
+      const uint32_t m = meta_s[id];
+      if (m != 0xffffffffu && static_cast<int>(m >> 6) == ch) fill = static_cast<int>(m & 63u);
     }
-    const bool valid = js >= 0 && js < N;
-    float sh[G];
-    score_token<G>(code, id, lut_b, qc_s, C, ysoff, sel, swap_words, sh);
+  };
+  auto chunk_out = [&](int i, uint32_t id, int fill, const float* sh) {
+    const int ch = wb + i;
+    const bool valid = lane < fill;
     float sg = sh[0];
 #pragma unroll
     for (int g = 1; g < G; ++g) sg = fmaxf(sg, sh[g]);
-    __stcs(sig_u + static_cast<size_t>(ch) * 32 + lane, valid ? sg : -INFINITY);
-    {   // the chunk's largest score lets the filter skip chunks below the threshold
-      const float cmx = warp_max(valid ? sg : -INFINITY);
-      if (lane == 0) p.chunk_max[static_cast<size_t>(u) * (p.list_slots / 32) + ch] = cmx;
-    }
+    const float sv = valid ? sg : -INFINITY;
+    sig_u[static_cast<size_t>(ch) * 32 + lane] = sv;
+    const float cmx = warp_max_f32(sv);  // lets the filter skip chunks below the threshold
+    if (lane == 0) cmax_u[ch] = cmx;
     if (p.approx_logits && valid) {
+      const int js = p.list_slot[static_cast<size_t>(u) * p.list_slots + static_cast<size_t>(ch) * 32 + lane];
+      if (js >= 0 && js < N) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) p.approx_logits[(static_cast<size_t>(b) * p.Hq + h * G + g) * p.cap + js] = sh[g];
+        for (int g = 0; g < G; ++g) p.approx_logits[(static_cast<size_t>(b) * p.Hq + h * G + g) * p.cap + js] = sh[g];
+      }
     }
-    {
-      float ev[G];
+    if (id != cur) {                     // warp-uniform: a new cluster run starts
+      if (cur != 0xffffffffu) flush_weights<G>(wacc, Wu, C, cur);
+      cur = id;
 #pragma unroll
-      for (int g = 0; g < G; ++g) ev[g] = valid ? fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])) : 0.f;
-      const float e = warp_sum_scatter<G>(ev);
-      constexpr int kGroup = 32 / G;
-      if ((lane & (kGroup - 1)) == 0) atomicAdd(Wu + (lane / kGroup) * C + id, e);
+      for (int g = 0; g < G; ++g) wacc[g] = 0.f;
     }
+#pragma unroll
+    for (int g = 0; g < G; ++g) wacc[g] += valid ? fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])) : 0.f;
     if (valid) atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
-    __syncwarp();                        // every lane has read the slot
-    issue(i + D);                        // refill it with the chunk D ahead
+  };
+  if (kScanPair) {
+    // two chunks per step: their look-up chains are independent, so each warp keeps twice
+    // as many shared-memory gathers in flight between its synchronisations
+    for (int i = 0; i < cnt; i += 2) {
+      const bool two = i + 1 < cnt;
+      cp_async_wait<D - 2>();            // this lane's copies of chunks i and i + 1 have landed
+      __syncwarp();                      // ... and lane 0's cluster words
+      uint4 code0, code1;
+      uint32_t id0, id1;
+      int fill0, fill1;
+      chunk_in(i, code0, id0, fill0);
+      if (two) chunk_in(i + 1, code1, id1, fill1);
+      else {
+        code1 = code0;
+        id1 = id0;
+        fill1 = 0;
+      }
+      float sh0[G], sh1[G];
+      score_token<G>(code0, id0, lut_b, qc_s, C, ysoff, sel, swap_words, sh0);
+      score_token<G>(code1, id1, lut_b, qc_s, C, ysoff, sel, swap_words, sh1);
+      chunk_out(i, id0, fill0, sh0);
+      if (two) chunk_out(i + 1, id1, fill1, sh1);
+      __syncwarp();                      // every lane has read both slots
+      issue(i + D);                      // refill them with the chunks D ahead
+      issue(i + 1 + D);
+    }
+  } else {
+    for (int i = 0; i < cnt; ++i) {
+      cp_async_wait<D - 1>();            // this lane's copies of chunk i have landed
+      __syncwarp();                      // ... and lane 0's cluster word
+      uint4 code;
+      uint32_t id;
+      int fill;
+      chunk_in(i, code, id, fill);
+      float sh[G];
+      score_token<G>(code, id, lut_b, qc_s, C, ysoff, sel, swap_words, sh);
+      chunk_out(i, id, fill, sh);
+      __syncwarp();                      // every lane has read the slot
+      issue(i + D);                      // refill it with the chunk D ahead
+    }
   }
+  if (cur != 0xffffffffu) flush_weights<G>(wacc, Wu, C, cur);
   cp_async_wait<0>();
   if (bad_id) record_error(p.err, HSA_DEVERR_CLUSTER);
   __syncthreads();
   uint32_t* hg = p.hist + static_cast<size_t>(u) * kNB;
-  for (int i = tid; i < kNB; i += blockDim.x) {
+  for (int i = tid; i < kNB; i += kScanThreads) {
     const uint32_t v = hist_s[i];
     if (v) atomicAdd(hg + i, v);
   }
+  // publish this range: scores, chunk maxima, weights and histogram before the count
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) atomicAdd(&p.units[u].scan_done, nch);
 }
 
-// Walk the balanced global item range of this CTA over the units; count(b, h) gives
-// the items of unit (b, h). f(u, i0, i1) is called for every overlapped unit range.
-template <typename Count, typename F>
-__device__ __forceinline__ void for_each_range(int B, int Hkv, Count&& count, F&& f) {
-  long long total = 0;
-  for (int b = 0; b < B; ++b)
-    for (int h = 0; h < Hkv; ++h) total += count(b, h);
-  const long long start = total * blockIdx.x / gridDim.x;
-  const long long end = total * (blockIdx.x + 1) / gridDim.x;
-  if (start >= end) return;
-  long long acc = 0;
-  for (int b = 0; b < B && acc < end; ++b) {
-    for (int h = 0; h < Hkv && acc < end; ++h) {
-      const int n = count(b, h);
-      if (start < acc + n && end > acc) {
-        const int j0 = static_cast<int>(max(start - acc, 0LL));
-        const int j1 = static_cast<int>(min(end - acc, static_cast<long long>(n)));
-        f(b * Hkv + h, j0, j1);
-      }
-      acc += n;
-    }
-  }
-}
-
-// Work split for kernels whose items are grouped by unit. With at least as many CTAs as
-// units that have work, every CTA takes one part of exactly one unit (1 + a share of the
-// spare CTAs in proportion to the unit's items), so no CTA pays a second unit's set-up;
-// a few CTAs may be left idle. Otherwise the balanced range walk. Calls f(u, i0, i1).
-template <typename Count, typename F>
-__device__ __forceinline__ void for_each_unit_part(int B, int Hkv, Count&& count, F&& f) {
-  long long total = 0;
-  int active = 0;
-  for (int b = 0; b < B; ++b)
-    for (int h = 0; h < Hkv; ++h) {
-      const int n = count(b, h);
-      total += n;
-      active += n > 0;
-    }
-  const int grid = static_cast<int>(gridDim.x);
-  if (active == 0) return;
-  if (active > grid) {
-    for_each_range(B, Hkv, count, f);
-    return;
-  }
-  const long long spare = grid - active;
-  int base = 0;
-  for (int b = 0; b < B; ++b)
-    for (int h = 0; h < Hkv; ++h) {
-      const int n = count(b, h);
-      if (n <= 0) continue;
-      const int parts = 1 + static_cast<int>(spare * n / total);
-      const int k = static_cast<int>(blockIdx.x) - base;
-      if (k >= 0 && k < parts) {
-        const int i0 = static_cast<int>(static_cast<long long>(n) * k / parts);
-        const int i1 = static_cast<int>(static_cast<long long>(n) * (k + 1) / parts);
-        if (i1 > i0) f(b * Hkv + h, i0, i1);
-        return;
-      }
-      base += parts;
-    }
-}
-
-__device__ __forceinline__ int unit_chunks(const int32_t* list_meta, int u, int C, int max_chunks) {
-  const int n = list_meta[static_cast<size_t>(u) * (2 + 2 * static_cast<size_t>(C))];
-  return max(0, min(n, max_chunks));
-}
-
-template <int G, int D>
-__global__ void __launch_bounds__(scan_threads_of<G>(), 1) scan_kernel(ScanParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float sh_bounds[2 * G];
-  const int lane = threadIdx.x & 31;
-  const uint32_t l7 = lane & 7;
-  // Per-lane subspace skew: lookup i reads subspace s = i ^ (lane & 7), so the 8
-  // lanes of a quarter-warp hit 8 different 16-byte bank groups.
-  uint32_t ysoff[8], sel[4];
-#pragma unroll
-  for (int k2 = 0; k2 < 8; ++k2) {
-    const uint32_t s_lo = ((2 * k2) ^ l7) & 15, s_hi = ((2 * k2 + 1) ^ l7) & 15;
-    ysoff[k2] = (s_lo * 16u) | ((s_hi * 16u) << 16);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t bi = (i ^ l7) & 3;              // byte of the (swapped) word holding code s
-    sel[i] = (4u + 2u * (i & 1)) | (bi << 4) | (5u << 8) | (5u << 12);
-  }
-  const bool swap_words = (l7 >> 2) & 1;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ScanSmem<G>::tables(p.C) +
-                                              static_cast<size_t>(scan_threads_of<G>() / 32) * D * kRingSlotBytes);
-  if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-  }
-  pdl_wait();
-  pdl_launch_dependents();
-  uint32_t phase = 0;
-  const int max_chunks = p.list_slots / 32;
-  for_each_unit_part(
-      p.B, p.Hkv, [&](int b, int h) { return unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
-      [&](int u, int c0, int c1) {
-        scan_segment<G, D>(p, u, c0, c1, smem, bar, phase, sh_bounds, ysoff, sel, swap_words);
-        ++phase;
-      });
-}
-
-// ===========================================================================
-// filter: tokens above the threshold bin are selected, the bin's tokens are candidates
-// ===========================================================================
-// Head weights e^{shat_g - ub_g} of one indexed token (cluster id, code words cw), from
-// the decode tables: the same quantities the scan added into its cluster's sums.
+// Head weights e^{shat_g - ub_g} of one indexed token (cluster id, code words cw) from the
+// decode tables (global or shared copies, layout [GP][256][16] and [GP][C] float4): the
+// same quantities the scan added into its cluster's sums.
 template <int G>
-__device__ __forceinline__ void token_weights(const SelectParams& p, int u, uint32_t id, const uint4 cw,
-                                              const float* ub2, float* e) {
+__device__ __forceinline__ void token_weights(const float4* lut4, const float4* qc4, int C, uint32_t id,
+                                              const uint4 cw, const float* ub2, float* e) {
   constexpr int GP = (G + 3) / 4;
   const uint32_t cwords[4] = {cw.x, cw.y, cw.z, cw.w};
-  const float4* lut4 = reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
-  const float4* qc4 = reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C;
   float4 acc[GP];
 #pragma unroll
-  for (int gp = 0; gp < GP; ++gp) acc[gp] = qc4[gp * p.C + id];
+  for (int gp = 0; gp < GP; ++gp) acc[gp] = qc4[gp * C + id];
 #pragma unroll
   for (int s = 0; s < kM; ++s) {
     const int code = (cwords[s >> 2] >> (8 * (s & 3))) & 255;
@@ -651,103 +650,95 @@ __device__ __forceinline__ void token_weights(const SelectParams& p, int u, uint
 
 // Take a selected token's head weights out of its cluster's sums.
 template <int G>
-__device__ __forceinline__ void remove_weights(const SelectParams& p, int u, uint32_t id, const float* e) {
+__device__ __forceinline__ void remove_weights(const StepParams& p, int u, uint32_t id, const float* e) {
   float* Wu = p.W + static_cast<size_t>(u) * G * p.C;
 #pragma unroll
   for (int g = 0; g < G; ++g) atomicAdd(&Wu[g * p.C + id], -e[g]);
 }
 
-// Filter over chunks: the scan left each 32-slot chunk's largest score, so a chunk whose
-// maximum falls below the threshold bin holds no selected or candidate token (the bin is
-// monotone in the score) and is skipped; only the few chunks that reach it are read.
-constexpr int kFilterThreads = 256;
-constexpr int kCmPerThread = 4;                                    // chunk maxima per thread per pass
-constexpr int kCmPass = kCmPerThread * kFilterThreads;             // chunks examined per pass
-constexpr int kActPerWarp = 4;                                     // active chunks per warp per round
-constexpr int kFixCap = kActPerWarp * kFilterThreads;              // queued tokens per round (<= one per slot)
-
 template <int G>
-__global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams p) {
-  __shared__ __align__(16) uint32_t hist_s[kNB];
-  __shared__ uint32_t scan_tot[33];
-  __shared__ int sh_bstar;
-  __shared__ uint32_t sh_above;
-  __shared__ int32_t act[kCmPass];          // active chunks of the current pass
-  __shared__ int n_act;
-  __shared__ uint32_t fix_list[kFixCap];   // list slots
-  __shared__ int32_t fix_cand[kFixCap];     // candidate slot, or -1 for a definite selection
-  __shared__ uint32_t fix_n;
-  static_assert(kNB == 8 * kFilterThreads, "filter threshold search: 256 threads x 8 bins");
-  constexpr int NW = kFilterThreads / 32;
+__device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* fsm, SelShared& ss);
+
+// Phase 2 for chunks [c0, c1) of unit u (after every CTA of the unit has scanned): the
+// threshold bin, then only the chunks whose maximum reaches it (the bin is monotone in the
+// score). Tokens above the bin are selected (bitmap); the bin's tokens are candidates.
+// Definite selections' weights leave their clusters' sums here, from the tables in shared
+// memory when this CTA holds the unit's (`tables`), else from the global copy; the first
+// candidates' weights are stored for the resolution. Returns true if this CTA was the
+// unit's last to finish (it then resolves the unit, after its other filter parts).
+template <int G>
+__device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const uint8_t* tables, uint8_t* smem,
+                            SelShared& ss) {
+  constexpr int GP = (G + 3) / 4;
+  constexpr int NW = kScanWarps;
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane = tid & 31;
-  pdl_wait();
-  pdl_launch_dependents();
+  const int b = u / p.Hkv;
+  const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
+  const int k = decode_k(p.budget, p.k_override, N);
   const int max_chunks = p.list_slots / 32;
-  for_each_unit_part(
-      p.B, p.Hkv, [&](int b, int h) { return unit_chunks(p.list_meta, b * p.Hkv + h, p.C, max_chunks); },
-      [&](int u, int c0, int c1) {
-    const int b = u / p.Hkv;
-    const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
-    const int k = decode_k(p.budget, p.k_override, N);
-    const float* sig = p.sigma + static_cast<size_t>(u) * p.list_slots;
-    const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
-    const float* cmax = p.chunk_max + static_cast<size_t>(u) * max_chunks;
-    // bounds and the first pass of chunk maxima load with the histogram
-    float ub[G], lb[G];
-    final_bounds<G>(p.fbounds, u, ub, lb);
-    float cm[kCmPerThread];
+  const int total = unit_chunks(p, u);
+  uint8_t* scratch = smem + ScanSmem<G>::hist_off(p.C);
+  int32_t* act = reinterpret_cast<int32_t*>(scratch);                    // active chunks of the pass
+  uint32_t* fix_list = reinterpret_cast<uint32_t*>(act + kCmPass);       // list slots
+  int32_t* fix_cand = reinterpret_cast<int32_t*>(fix_list + kFixCap);    // candidate slot, -1 = definite
+  const float4* lut4 = tables ? reinterpret_cast<const float4*>(tables)
+                              : reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
+  const float4* qc4 = tables ? reinterpret_cast<const float4*>(tables) + GP * kNcode * kM
+                             : reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C;
+
+  __syncthreads();   // shared state of the previous part is no longer read
+  if (tid == 0) {
+    wait_count(&p.units[u].scan_done, total, p.err);   // every CTA of the unit has scanned
+    ss.bstar = kNB;   // k == 0: nothing selected
+    ss.above = 0;
+    ss.fix_n = 0;
+  }
+  __syncthreads();
+  // one round trip: this thread's histogram bins, the first pass of chunk maxima, the bounds
+  static_assert(kNB == 4 * kScanThreads, "threshold search: 512 threads x 4 bins");
+  const uint4 hv = __ldcg(reinterpret_cast<const uint4*>(p.hist + static_cast<size_t>(u) * kNB) +
+                          (kNB / 4 - 1 - tid));
+  const float* cmax = p.chunk_max + static_cast<size_t>(u) * max_chunks;
+  float cm[kCmPerThread];
 #pragma unroll
-    for (int e = 0; e < kCmPerThread; ++e) {
-      const int c = c0 + tid + e * kFilterThreads;
-      cm[e] = c < c1 ? cmax[c] : -INFINITY;
-    }
-    __syncthreads();   // shared state of a previous unit range is no longer read
-    {
-      const uint4* hg = reinterpret_cast<const uint4*>(p.hist + static_cast<size_t>(u) * kNB);
-      uint4 hv[kNB / 4 / kFilterThreads];
+  for (int e = 0; e < kCmPerThread; ++e) {
+    const int c = c0 + tid + e * kScanThreads;
+    cm[e] = c < c1 ? __ldcg(cmax + c) : -INFINITY;
+  }
+  float ub[G], lb[G];
 #pragma unroll
-      for (int r = 0; r < kNB / 4 / kFilterThreads; ++r) hv[r] = hg[r * kFilterThreads + tid];
+  for (int g = 0; g < G; ++g) {
+    ub[g] = __ldcg(p.fbounds + (static_cast<size_t>(u) * 2 + 0) * G + g);
+    lb[g] = __ldcg(p.fbounds + (static_cast<size_t>(u) * 2 + 1) * G + g);
+  }
+  {
+    // thread t owns the 4 bins [kNB-4(t+1), kNB-4t): block scan of counts from the top
+    const int hi = kNB - 4 * tid;
+    const uint32_t c4[4] = {hv.w, hv.z, hv.y, hv.x};
+    const uint32_t local = c4[0] + c4[1] + c4[2] + c4[3];
+    uint32_t tot;
+    const uint32_t excl = block_excl_scan(local, ss.scan_tot, tot);
+    const uint32_t need = static_cast<uint32_t>(k);
+    if (need > 0 && excl < need && excl + local >= need) {
+      uint32_t cum = excl;
 #pragma unroll
-      for (int r = 0; r < kNB / 4 / kFilterThreads; ++r) reinterpret_cast<uint4*>(hist_s)[r * kFilterThreads + tid] = hv[r];
-    }
-    if (tid == 0) {
-      sh_bstar = kNB;   // k == 0: nothing selected
-      sh_above = 0;
-      fix_n = 0;
-    }
-    __syncthreads();
-    {
-      // thread t owns the 8 bins [kNB-8(t+1), kNB-8t): block scan of counts from the top
-      const int hi = kNB - 8 * tid;
-      uint32_t c8[8], local = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c8[i] = hist_s[hi - 1 - i];
-        local += c8[i];
-      }
-      uint32_t tot;
-      const uint32_t excl = block_excl_scan(local, scan_tot, tot);
-      const uint32_t need = static_cast<uint32_t>(k);
-      if (need > 0 && excl < need && excl + local >= need) {
-        uint32_t cum = excl;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (cum < need && cum + c8[i] >= need) {
-            sh_bstar = hi - 1 - i;
-            sh_above = cum;
-          }
-          cum += c8[i];
+      for (int i = 0; i < 4; ++i) {
+        if (cum < need && cum + c4[i] >= need) {
+          ss.bstar = hi - 1 - i;
+          ss.above = cum;
         }
+        cum += c4[i];
       }
     }
-    __syncthreads();
-    const int bstar = sh_bstar;
-    if (tid == 0) {
-      p.units[u].bstar = bstar;
-      p.units[u].above = static_cast<int32_t>(sh_above);
-    }
-    if (bstar >= kNB) return;
+  }
+  __syncthreads();
+  const int bstar = ss.bstar;
+  if (tid == 0) {   // every CTA of the unit stores the same values
+    p.units[u].bstar = bstar;
+    p.units[u].above = static_cast<int32_t>(ss.above);
+  }
+  if (bstar < kNB) {
     float hi = ub[0], lo = lb[0];
 #pragma unroll
     for (int g = 1; g < G; ++g) {
@@ -759,6 +750,8 @@ __global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams 
 #pragma unroll
     for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
     const bool fix = p.background && N > k;
+    const float* sig = p.sigma + static_cast<size_t>(u) * p.list_slots;
+    const int32_t* lslot = p.list_slot + static_cast<size_t>(u) * p.list_slots;
     const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
     const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * max_chunks;
     uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
@@ -767,29 +760,28 @@ __global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams 
       if (cb != c0) {
 #pragma unroll
         for (int e = 0; e < kCmPerThread; ++e) {
-          const int c = cb + tid + e * kFilterThreads;
-          cm[e] = c < c1 ? cmax[c] : -INFINITY;
+          const int c = cb + tid + e * kScanThreads;
+          cm[e] = c < c1 ? __ldcg(cmax + c) : -INFINITY;
         }
-        __syncthreads();   // the previous pass is done with act[]
       }
-      if (tid == 0) n_act = 0;
+      if (tid == 0) ss.n_act = 0;
       __syncthreads();
       // chunks whose maximum reaches the threshold bin, compacted warp by warp
 #pragma unroll
       for (int e = 0; e < kCmPerThread; ++e) {
-        const int c = cb + tid + e * kFilterThreads;
+        const int c = cb + tid + e * kScanThreads;
         const bool active = c < c1 && score_bin(cm[e], lo, inv) >= bstar;
         const uint32_t m = __ballot_sync(0xffffffffu, active);
         if (m) {
           const uint32_t leader = __ffs(m) - 1;
           int at = 0;
-          if (lane == leader) at = atomicAdd(&n_act, __popc(m));
+          if (lane == leader) at = atomicAdd(&ss.n_act, __popc(m));
           at = __shfl_sync(0xffffffffu, at, leader);
           if (active) act[at + __popc(m & ((1u << lane) - 1u))] = c;
         }
       }
       __syncthreads();
-      const int na = n_act;
+      const int na = ss.n_act;
       for (int a0 = 0; a0 < na; a0 += NW * kActPerWarp) {
         // each warp reads up to kActPerWarp active chunks at once; lane = slot of the chunk
         float sv[kActPerWarp];
@@ -799,7 +791,7 @@ __global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams 
         for (int r = 0; r < kActPerWarp; ++r) {
           const int a = a0 + warp + NW * r;
           chv[r] = a < na ? act[a] : -1;
-          sv[r] = chv[r] >= 0 ? sig[static_cast<size_t>(chv[r]) * 32 + lane] : -INFINITY;
+          sv[r] = chv[r] >= 0 ? __ldcg(sig + static_cast<size_t>(chv[r]) * 32 + lane) : -INFINITY;
           jv[r] = chv[r] >= 0 ? lslot[static_cast<size_t>(chv[r]) * 32 + lane] : -1;
         }
 #pragma unroll
@@ -818,13 +810,13 @@ __global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams 
           }
           if (fix) {
             // queue the list slot: a definite selection's weight leaves its cluster's sums
-            // below; a candidate's weights are stored for the finalize's winners
+            // below; a candidate's weights are stored for the resolution's winners
             const bool queued = definite || (slot >= 0 && slot < kCandWeights);
             const uint32_t m = __ballot_sync(0xffffffffu, queued);
             if (m) {
               const uint32_t leader = __ffs(m) - 1;
               uint32_t at = 0;
-              if (lane == leader) at = atomicAdd(&fix_n, static_cast<uint32_t>(__popc(m)));
+              if (lane == leader) at = atomicAdd(&ss.fix_n, static_cast<uint32_t>(__popc(m)));
               at = __shfl_sync(0xffffffffu, at, leader);
               if (queued) {
                 at += __popc(m & ((1u << lane) - 1u));
@@ -837,14 +829,14 @@ __global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams 
         if (fix) {
           // queued tokens of this round: one per thread, every look-up of a token in flight together
           __syncthreads();
-          const uint32_t n = fix_n;
-          for (uint32_t i = tid; i < n; i += kFilterThreads) {
+          const uint32_t n = ss.fix_n;
+          for (uint32_t i = tid; i < n; i += kScanThreads) {
             const uint32_t ls = fix_list[i];
             const int cs = fix_cand[i];
             uint32_t id = ccl[ls >> 5];
             if (id >= static_cast<uint32_t>(p.C)) id = 0;
             float e[G];
-            token_weights<G>(p, u, id, lcodes[ls], ub2, e);
+            token_weights<G>(lut4, qc4, p.C, id, lcodes[ls], ub2, e);
             if (cs < 0) {
               remove_weights<G>(p, u, id, e);
             } else {
@@ -855,71 +847,140 @@ __global__ void __launch_bounds__(kFilterThreads, 2) filter_kernel(SelectParams 
             }
           }
           __syncthreads();
-          if (tid == 0) fix_n = 0;
+          if (tid == 0) ss.fix_n = 0;
           __syncthreads();
         }
       }
+      __syncthreads();   // this pass is done with act[] and n_act
     }
-  });
+  }
+  // publish this range's selections, candidates and fix-ups, then count it in
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int n = c1 - c0;
+    const int old = atomicAdd(&p.units[u].filt_done, n);
+    ss.flag = (old < total && old + n >= total) ? 1 : 0;
+  }
+  __syncthreads();
+  return ss.flag != 0;
 }
 
-// ===========================================================================
-// finalize (one CTA per unit)
-// ===========================================================================
-constexpr int kFinThreads = 1024;
-constexpr int kFinWordsPerThread = 4;
-constexpr int kFinChunkWords = kFinWordsPerThread * kFinThreads;   // 131072 slots per pass
-constexpr int kFinSmemCand = kFinThreads;                          // candidates resolved in shared memory
-constexpr int kFinBtCache = 8192;   // block-table entries cached in shared memory (longer tables: global)
+// One full warp: over counts cnt[0..nbins) (nbins a multiple of 32), find the bin b such
+// that sum_{b' > b} cnt < need <= sum_{b' >= b} cnt. Writes *bin/*above only when such a
+// bin exists.
+__device__ void find_threshold_desc(const uint32_t* cnt, int nbins, uint32_t need, int* bin, uint32_t* above) {
+  const int lane = threadIdx.x & 31;
+  const int per = nbins / 32;
+  const int hi = nbins - per * lane;   // lane 0 holds the highest bins
+  const int lo = hi - per;
+  uint32_t local = 0;
+  for (int i = lo; i < hi; ++i) local += cnt[i];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t excl = incl - local;
+  if (need > 0 && excl < need && incl >= need) {
+    uint32_t cum = excl;
+    for (int i = hi - 1; i >= lo; --i) {
+      if (cum + cnt[i] >= need) {
+        *bin = i;
+        *above = cum;
+        break;
+      }
+      cum += cnt[i];
+    }
+  }
+}
 
-__host__ __device__ inline int fin_bt_cached(int max_pages) { return max_pages <= kFinBtCache ? max_pages : 0; }
-
-// One CTA per unit: resolve the threshold bin's candidates exactly (score desc, position
-// asc), compact the selection bitmap into ascending positions, and take the selected
-// tokens' weights out of the cluster sums. Unit state, candidates and the first bitmap
-// pass are loaded in one round trip.
+// Phase 3 for unit u, by the CTA that finished its filter last (or, for a unit with no
+// chunks, by CTA u mod grid): resolve the threshold bin's candidates exactly (score desc,
+// position asc), compact the selection bitmap into ascending positions written as KV-pool
+// rows, take the winners' weights out of the cluster sums, and publish the unit. Every
+// input (lengths, counters, candidate keys and stored weights, the first bitmap pass, the
+// block table) is fetched in one round trip. `fsm` holds kFinScratch bytes (over the
+// tables: the CTA's filter parts are done).
 template <int G>
-__global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
-  __shared__ unsigned long long ck[kFinSmemCand];
-  __shared__ uint32_t bmc[kFinChunkWords];
-  __shared__ uint32_t woff[kFinChunkWords];   // exclusive count of selected bits before each word
-  __shared__ uint32_t wins[kFinSmemCand];
-  __shared__ uint32_t dig[256];
-  __shared__ uint32_t warp_tot[33];
-  __shared__ int sh_bin;
-  __shared__ uint32_t sh_above, sh_nwin;
-  extern __shared__ int32_t bt_s[];   // the sequence's block table when it fits
-  const int u = blockIdx.x;
+__device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* fsm, SelShared& ss) {
+  constexpr int GP = (G + 3) / 4;
+  constexpr int T = kScanThreads;
+  constexpr int kKeysPer = kFinSmemCand / T;   // candidate keys fetched per thread
+  constexpr int kBtPer = kFinBt / T;           // block-table entries fetched per thread
+  unsigned long long* ck = reinterpret_cast<unsigned long long*>(fsm);   // [kFinSmemCand]
+  uint32_t* bmc = reinterpret_cast<uint32_t*>(ck + kFinSmemCand);         // [kFinChunkWords]
+  uint32_t* woff = bmc + kFinChunkWords;                                  // [kFinChunkWords]
+  uint32_t* wins = woff + kFinChunkWords;                                 // [kFinSmemCand]
+  uint32_t* dig = wins + kFinSmemCand;                                    // [256]
+  int32_t* bt_s = reinterpret_cast<int32_t*>(dig + 256);                 // [kFinBt]
   const int b = u / p.Hkv;
   const int h = u % p.Hkv;
   const int tid = threadIdx.x;
-  const int nbt = fin_bt_cached(p.max_pages);
   const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
-  {   // the block table predates the step: all of this thread's entries in flight at once
-    constexpr int kPer = kFinBtCache / kFinThreads;
-    int32_t v[kPer];
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) v[e] = tid + e * kFinThreads < nbt ? bt_row[tid + e * kFinThreads] : 0;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e)
-      if (tid + e * kFinThreads < nbt) bt_s[tid + e * kFinThreads] = v[e];
-  }
-  pdl_wait();
-  pdl_launch_dependents();
-  // ---- one round trip: lengths, unit state, candidates and the first bitmap pass (speculative) ----
+  const unsigned long long* cg = p.cand + static_cast<size_t>(u) * p.cap;
+  const uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
+  const int nbt = min(p.max_pages, kFinBt);
+  __syncthreads();   // the scratch overlays the tables and the filter's queues
+
+  // ---- one round trip: every load below is independent of the others ----
   const int T_raw = p.seq_lens[b];
   const int n_raw = p.n_indexed[b];
-  const UnitState st = p.units[u];
-  const unsigned long long* cg = p.cand + static_cast<size_t>(u) * p.cap;
-  const unsigned long long ck_mine = tid < p.cap ? cg[tid] : 0ull;
-  const uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
-  uint32_t words[kFinWordsPerThread];
+  const int ncand = __ldcg(&p.units[u].ncand);
+  const int above = __ldcg(&p.units[u].above);
+  unsigned long long kr[kKeysPer];   // candidate keys of slots tid + r T (speculative: any count)
+#pragma unroll
+  for (int r = 0; r < kKeysPer; ++r) {
+    const int i = tid + r * T;
+    kr[r] = i < p.cap ? __ldcg(cg + i) : 0ull;
+  }
+  float cwr[G];                      // stored weights of candidate slot tid
+  int32_t ccr = 0;
+  if (p.background) {
+    const float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + tid) * G;
+#pragma unroll
+    for (int g = 0; g < G; ++g) cwr[g] = tid < kCandWeights ? __ldcg(cw + g) : 0.f;
+    ccr = tid < kCandWeights ? __ldcg(p.cand_c + static_cast<size_t>(u) * kCandWeights + tid) : 0;
+  }
+  uint32_t words[kFinWordsPerThread];   // first bitmap pass
 #pragma unroll
   for (int e = 0; e < kFinWordsPerThread; ++e) {
     const int wi = kFinWordsPerThread * tid + e;
-    words[e] = wi < p.bitmap_words ? bm[wi] : 0u;
+    words[e] = wi < p.bitmap_words ? __ldcg(bm + wi) : 0u;
   }
-  // bounds, and this thread's candidate weights (slot tid) as stored by the filter
+  int32_t btv[kBtPer];
+#pragma unroll
+  for (int e = 0; e < kBtPer; ++e) btv[e] = tid + e * T < nbt ? bt_row[tid + e * T] : 0;
+
+  const int T_len = max(0, T_raw);
+  const int s0 = min(p.n_sink, T_len);
+  const int N = min(max(0, min(n_raw, T_len - s0)), p.cap);
+  const int k = decode_k(p.budget, p.k_override, N);
+  const bool fix = p.background && N > k;
+  int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
+  if (k == 0) {
+    if (tid == 0) {
+      p.units[u].nsel = 0;
+      if (p.dbg_nselected) p.dbg_nselected[u] = 0;
+    }
+    publish_flag(&p.units[u].ready);
+    return;
+  }
+  const int m = min(ncand, p.cap);
+  const int r = k - above;
+  const bool ok = r >= 1 && r <= m;
+  if (!ok && tid == 0) record_error(p.err, HSA_DEVERR_SELECT);
+  const bool in_smem = m <= kFinSmemCand;
+#pragma unroll
+  for (int rr = 0; rr < kKeysPer; ++rr)
+    if (tid + rr * T < min(m, kFinSmemCand)) ck[tid + rr * T] = kr[rr];
+#pragma unroll
+  for (int e = 0; e < kBtPer; ++e)
+    if (tid + e * T < nbt) bt_s[tid + e * T] = btv[e];
+  if (tid == 0) ss.nwin = 0;
+  __syncthreads();
+  auto key_at = [&](int i) -> unsigned long long { return in_smem ? ck[i] : __ldcg(cg + i); };
   float ub2[G];
   {
     float ub[G], lb[G];
@@ -927,22 +988,8 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
 #pragma unroll
     for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
   }
-  static_assert(kCandWeights <= kFinThreads, "one stored candidate per thread");
-  float cwr[G];
-  int32_t ccr = 0;
-  if (p.background) {
-    const float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + tid) * G;
-#pragma unroll
-    for (int g = 0; g < G; ++g) cwr[g] = tid < kCandWeights ? cw[g] : 0.f;
-    ccr = tid < kCandWeights ? p.cand_c[static_cast<size_t>(u) * kCandWeights + tid] : 0;
-  }
-  const int T = max(0, T_raw);
-  const int s0 = min(p.n_sink, T);
-  const int N = min(max(0, min(n_raw, T - s0)), p.cap);
-  const int k = decode_k(p.budget, p.k_override, N);
-  const bool fix = p.background && N > k;
-  // A winner's weights leave its cluster's sums: from registers (slot tid), from the
-  // filter's store (slot < kCandWeights), else recomputed from the tables.
+  // A winner's weights leave its cluster's sums: from registers (candidate slot tid), from
+  // the filter's store (slot < kCandWeights), else recomputed from the global tables.
   auto fix_winner = [&](int i, uint32_t j) {
     if (!fix) return;
     float e[G];
@@ -954,44 +1001,30 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     } else if (i < kCandWeights) {
       const float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + i) * G;
 #pragma unroll
-      for (int g = 0; g < G; ++g) e[g] = cw[g];
-      id = static_cast<uint32_t>(p.cand_c[static_cast<size_t>(u) * kCandWeights + i]);
+      for (int g = 0; g < G; ++g) e[g] = __ldcg(cw + g);
+      id = static_cast<uint32_t>(__ldcg(p.cand_c + static_cast<size_t>(u) * kCandWeights + i));
     } else {
       id = p.ids[static_cast<size_t>(u) * p.cap + j];
       const uint4 cwd = *reinterpret_cast<const uint4*>(p.codes + (static_cast<size_t>(u) * p.cap + j) * kM);
       if (id >= static_cast<uint32_t>(p.C)) id = 0;
-      token_weights<G>(p, u, id, cwd, ub2, e);
+      token_weights<G>(reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM,
+                       reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C, p.C, id, cwd,
+                       ub2, e);
     }
     if (id >= static_cast<uint32_t>(p.C)) id = 0;
     remove_weights<G>(p, u, id, e);
   };
-  int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
-  if (k == 0) {
-    if (tid == 0 && p.dbg_nselected) p.dbg_nselected[u] = 0;
-    publish_flag(&p.units[u].ready);
-    return;
-  }
-  const int m = min(st.ncand, p.cap);
-  const int r = k - st.above;
-  const bool ok = r >= 1 && r <= m;
-  if (!ok && tid == 0) record_error(p.err, HSA_DEVERR_SELECT);
-  const bool in_smem = m <= kFinSmemCand;
-  if (in_smem && tid < m) ck[tid] = ck_mine;
-  if (tid == 0) sh_nwin = 0;
-  __syncthreads();
-  const unsigned long long* keys = in_smem ? ck : cg;
 
-  // ---- threshold key: the r-th largest candidate key (keys are distinct) ----
+  // ---- winners: the r largest candidate keys (keys are distinct) ----
   if (ok) {
-    unsigned long long tau;
-    if (m <= 256) {
+    if (m <= T) {
       if (tid < m) {
-        const unsigned long long key = keys[tid];
+        const unsigned long long key = key_at(tid);
         int rank = 0;
-        for (int j = 0; j < m; ++j) rank += keys[j] > key;
+        for (int j = 0; j < m; ++j) rank += key_at(j) > key;
         if (rank < r) {
           const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
-          wins[atomicAdd(&sh_nwin, 1u)] = j;
+          wins[atomicAdd(&ss.nwin, 1u)] = j;
           fix_winner(tid, j);
         }
       }
@@ -999,31 +1032,31 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
       unsigned long long prefix = 0, mask = 0;
       uint32_t need = static_cast<uint32_t>(r);
       for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += blockDim.x) dig[i] = 0u;
+        for (int i = tid; i < 256; i += T) dig[i] = 0u;
         if (tid == 0) {
-          sh_bin = -1;
-          sh_above = 0;
+          ss.bin = -1;
+          ss.fin_above = 0;
         }
         __syncthreads();
-        for (int i = tid; i < m; i += blockDim.x) {
-          const unsigned long long key = keys[i];
+        for (int i = tid; i < m; i += T) {
+          const unsigned long long key = key_at(i);
           if ((key & mask) == prefix) atomicAdd(&dig[(key >> shift) & 255ull], 1u);
         }
         __syncthreads();
-        if (tid < 32) find_threshold_desc(dig, 256, need, &sh_bin, &sh_above);
+        if (tid < 32) find_threshold_desc(dig, 256, need, &ss.bin, &ss.fin_above);
         __syncthreads();
-        const int d = sh_bin < 0 ? 0 : sh_bin;
-        need -= sh_above;
+        const int d = ss.bin < 0 ? 0 : ss.bin;
+        need -= ss.fin_above;
         prefix |= static_cast<unsigned long long>(d) << shift;
         mask |= 255ull << shift;
         __syncthreads();
       }
-      tau = prefix;
-      for (int i = tid; i < m; i += blockDim.x) {
-        const unsigned long long key = keys[i];
+      const unsigned long long tau = prefix;
+      for (int i = tid; i < m; i += T) {
+        const unsigned long long key = key_at(i);
         if (key >= tau) {
           const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
-          const uint32_t w = atomicAdd(&sh_nwin, 1u);
+          const uint32_t w = atomicAdd(&ss.nwin, 1u);
           if (w < kFinSmemCand) wins[w] = j;
           else atomicOr(p.bitmap + static_cast<size_t>(u) * p.bitmap_words + (j >> 5), 1u << (j & 31));
           fix_winner(i, j);
@@ -1032,28 +1065,26 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     }
   }
   __syncthreads();
-  const uint32_t nwin = min(sh_nwin, static_cast<uint32_t>(kFinSmemCand));
-  if (nwin < sh_nwin) __threadfence_block();   // overflowed winners went to the global bitmap
-
+  const uint32_t nwin_all = ss.nwin;
+  const uint32_t nwin = min(nwin_all, static_cast<uint32_t>(kFinSmemCand));
+  if (nwin < nwin_all) __threadfence_block();   // overflowed winners went to the global bitmap
 
   // ---- compaction of the selection bitmap into ascending positions ----
   const int nw = (N + 31) / 32;
   uint32_t running = 0;
   for (int w0 = 0; w0 < nw; w0 += kFinChunkWords) {
-    if (w0 > 0 || sh_nwin > kFinSmemCand) {
+    if (w0 > 0 || nwin < nwin_all) {   // later passes, or winners that went to the global bitmap
 #pragma unroll
       for (int e = 0; e < kFinWordsPerThread; ++e) {
         const int wi = w0 + kFinWordsPerThread * tid + e;
-        words[e] = wi < nw ? bm[wi] : 0u;
+        words[e] = wi < p.bitmap_words ? __ldcg(bm + wi) : 0u;
       }
     }
 #pragma unroll
-    for (int e = 0; e < kFinWordsPerThread; ++e) {
-      const int wi = w0 + kFinWordsPerThread * tid + e;
-      bmc[kFinWordsPerThread * tid + e] = wi < nw ? words[e] : 0u;
-    }
+    for (int e = 0; e < kFinWordsPerThread; ++e)
+      bmc[kFinWordsPerThread * tid + e] = (w0 + kFinWordsPerThread * tid + e < nw) ? words[e] : 0u;
     __syncthreads();
-    for (uint32_t i = tid; i < nwin; i += blockDim.x) {
+    for (uint32_t i = tid; i < nwin; i += T) {
       const uint32_t j = wins[i];
       const int w = static_cast<int>(j >> 5) - w0;
       if (w >= 0 && w < kFinChunkWords) atomicOr(&bmc[w], 1u << (j & 31));
@@ -1067,7 +1098,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     }
     uint32_t tot;
     {
-      uint32_t o = block_excl_scan(pc, warp_tot, tot);
+      uint32_t o = block_excl_scan(pc, ss.scan_tot, tot);
 #pragma unroll
       for (int e = 0; e < kFinWordsPerThread; ++e) {
         woff[kFinWordsPerThread * tid + e] = o;
@@ -1076,9 +1107,9 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
     }
     __syncthreads();
     // Output entry i of this pass: the word holding it by binary search over the word
-    // offsets, then its bit; every thread writes about tot / 1024 entries whatever the
+    // offsets, then its bit; every thread writes about tot / T entries whatever the
     // positions of the selected tokens.
-    for (uint32_t i = tid; i < tot; i += kFinThreads) {
+    for (uint32_t i = tid; i < tot; i += T) {
       int lo_w = 0, hi_w = kFinChunkWords - 1;   // largest word with woff <= i
       while (lo_w < hi_w) {
         const int mid = (lo_w + hi_w + 1) >> 1;
@@ -1093,7 +1124,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
         // the token's KV-pool row, so the exact attend reads it in one step
         const int pos = s0 + j;
         const int pi = pos / p.page_size;
-        int page = pi < p.max_pages ? (pi < nbt ? bt_s[pi] : bt_row[pi]) : -1;
+        int page = pi < nbt ? bt_s[pi] : (pi < p.max_pages ? bt_row[pi] : -1);
         if (page < 0 || page >= p.num_pages) {
           record_error(p.err, HSA_DEVERR_PAGE);
           page = 0;
@@ -1113,6 +1144,194 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(SelectParams p) {
   // the exact attend and the background of this unit may start (selection rows and
   // the winners' weight fix-up are written)
   publish_flag(&p.units[u].ready);
+}
+
+// Work split over the units' chunks, planned cooperatively by the CTA (one pass over the
+// units per mode, thread t taking units t, t + T, ...). With at least as many CTAs as
+// units that have chunks, every CTA takes one part of exactly one unit (1 + a share of
+// the spare CTAs in proportion to the unit's chunks), so no CTA pays a second unit's
+// set-up; a few CTAs may be left idle. Otherwise every CTA takes a balanced range of the
+// concatenated chunks, which may span several units. The parts land in ss.pu/pc0/pc1;
+// ss.nparts = -1 when a range spans more than kMaxParts units (then walk_parts is used).
+__device__ void plan_parts(const StepParams& p, SelShared& ss) {
+  const int U = p.B * p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long grid = gridDim.x, me = blockIdx.x;
+  long long tot = 0;
+  int act = 0;
+  int n_first = 0;   // chunks of unit tid (reused by the first pass below)
+  for (int u = tid; u < U; u += kScanThreads) {
+    const int n = unit_chunks(p, u);
+    if (u == tid) n_first = n;
+    tot += n;
+    act += n > 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    act += __shfl_xor_sync(0xffffffffu, act, o);
+  }
+  if (lane == 0) {
+    ss.red[warp] = tot;
+    ss.scan_tot[warp] = static_cast<uint32_t>(act);
+  }
+  if (tid == 0) ss.nparts = 0;
+  __syncthreads();
+  if (tid == 0) {
+    long long t = 0;
+    int a = 0;
+    for (int w = 0; w < kScanWarps; ++w) {
+      t += ss.red[w];
+      a += static_cast<int>(ss.scan_tot[w]);
+    }
+    ss.total = t;
+    ss.active = a;
+  }
+  __syncthreads();
+  const long long total = ss.total;
+  const int active = ss.active;
+  if (active == 0) return;
+  const bool per_unit = active <= grid;
+  const long long spare = grid - active;
+  const long long start = total * me / grid, end = total * (me + 1) / grid;
+  long long run = 0;   // items (or CTAs) of the units before this pass
+  for (int u0 = 0; u0 < U; u0 += kScanThreads) {
+    const int u = u0 + tid;
+    const int n = u0 == 0 ? n_first : (u < U ? unit_chunks(p, u) : 0);
+    const int w = per_unit ? (n > 0 ? 1 + static_cast<int>(spare * n / total) : 0) : n;
+    uint32_t pass_tot;
+    const long long base = run + block_excl_scan(static_cast<uint32_t>(w), ss.scan_tot, pass_tot);
+    int i0 = 0, i1 = 0;
+    if (per_unit) {
+      if (n > 0 && me >= base && me < base + w) {
+        const long long kk = me - base;
+        i0 = static_cast<int>(n * kk / w);
+        i1 = static_cast<int>(n * (kk + 1) / w);
+      }
+    } else if (n > 0 && start < base + n && end > base) {
+      i0 = static_cast<int>(max(start - base, 0LL));
+      i1 = static_cast<int>(min(end - base, static_cast<long long>(n)));
+    }
+    if (i1 > i0) {
+      const int at = atomicAdd(&ss.nparts, 1);
+      if (at < kMaxParts) {
+        ss.pu[at] = u;
+        ss.pc0[at] = i0;
+        ss.pc1[at] = i1;
+      }
+    }
+    run += pass_tot;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (ss.nparts > kMaxParts) {
+      ss.nparts = -1;
+    } else {   // unit order (the atomic appends may interleave within a pass)
+      for (int i = 1; i < ss.nparts; ++i)
+        for (int j = i; j > 0 && ss.pu[j - 1] > ss.pu[j]; --j) {
+          int t = ss.pu[j]; ss.pu[j] = ss.pu[j - 1]; ss.pu[j - 1] = t;
+          t = ss.pc0[j]; ss.pc0[j] = ss.pc0[j - 1]; ss.pc0[j - 1] = t;
+          t = ss.pc1[j]; ss.pc1[j] = ss.pc1[j - 1]; ss.pc1[j - 1] = t;
+        }
+    }
+  }
+  __syncthreads();
+}
+
+// The balanced-range split of plan_parts walked unit by unit (for a CTA whose range spans
+// more than kMaxParts units). Calls f(u, i0, i1) in unit order.
+template <typename F>
+__device__ void walk_parts(const StepParams& p, long long total, F&& f) {
+  const long long grid = gridDim.x;
+  const long long start = total * blockIdx.x / grid;
+  const long long end = total * (blockIdx.x + 1) / grid;
+  long long acc = 0;
+  for (int u = 0; u < p.B * p.Hkv && acc < end; ++u) {
+    const int n = unit_chunks(p, u);
+    if (n > 0 && start < acc + n && end > acc) {
+      const int j0 = static_cast<int>(max(start - acc, 0LL));
+      const int j1 = static_cast<int>(min(end - acc, static_cast<long long>(n)));
+      f(u, j0, j1);
+    }
+    acc += n;
+  }
+}
+
+template <int G, int D>
+__global__ void __launch_bounds__(kScanThreads, 1) scan_select_kernel(StepParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float sh_bounds[2 * G];
+  __shared__ SelShared ss;
+  const int lane = threadIdx.x & 31;
+  const uint32_t l7 = lane & 7;
+  // Per-lane subspace skew: lookup i reads subspace s = i ^ (lane & 7), so the 8
+  // lanes of a quarter-warp hit 8 different 16-byte bank groups.
+  uint32_t ysoff[8], sel[4];
+#pragma unroll
+  for (int k2 = 0; k2 < 8; ++k2) {
+    const uint32_t s_lo = ((2 * k2) ^ l7) & 15, s_hi = ((2 * k2 + 1) ^ l7) & 15;
+    ysoff[k2] = (s_lo * 16u) | ((s_hi * 16u) << 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t bi = (i ^ l7) & 3;              // byte of the (swapped) word holding code s
+    sel[i] = (4u + 2u * (i & 1)) | (bi << 4) | (5u << 8) | (5u << 12);
+  }
+  const bool swap_words = (l7 >> 2) & 1;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ScanSmem<G>::tables(p.C) +
+                                              static_cast<size_t>(kScanWarps) * D * kRingSlotBytes);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  // The work split reads only the index lists and lengths, which predate the tables kernel
+  // (it started only once every earlier kernel had completed): plan while the tables finish.
+  plan_parts(p, ss);
+  pdl_wait();
+  pdl_launch_dependents();
+  const int nparts = ss.nparts;
+  const long long total = ss.total;
+  uint32_t phase = 0;
+  int tables_unit = -1;
+  // ---- phase 1: scan ----
+  auto scan = [&](int u, int c0, int c1) {
+    scan_segment<G, D>(p, u, c0, c1, smem, bar, phase, sh_bounds, ysoff, sel, swap_words);
+    tables_unit = u;
+    ++phase;
+  };
+  if (nparts >= 0) {
+    for (int i = 0; i < nparts; ++i) scan(ss.pu[i], ss.pc0[i], ss.pc1[i]);
+  } else {
+    walk_parts(p, total, scan);
+  }
+  // ---- phase 2: selection per unit; phase 3: resolution by the unit's last CTA, after
+  // all of this CTA's filter parts, so that no unit's filter waits behind a resolution ----
+  int nres = 0;
+  auto filt = [&](int u, int c0, int c1) {
+    if (filter_part<G>(p, u, c0, c1, tables_unit == u ? smem : nullptr, smem, ss)) {
+      if (nres < kMaxParts) {
+        if (threadIdx.x == 0) ss.res[nres] = u;
+        ++nres;
+      } else {   // more units to resolve than the list holds: resolve this one now
+        __threadfence();
+        resolve_unit<G>(p, u, smem, ss);
+        tables_unit = -1;
+      }
+    }
+  };
+  if (nparts >= 0) {
+    for (int i = 0; i < nparts; ++i) filt(ss.pu[i], ss.pc0[i], ss.pc1[i]);
+  } else {
+    walk_parts(p, total, filt);
+  }
+  if (nres > 0) {
+    __threadfence();   // acquire: the unit's other CTAs published before counting in
+    __syncthreads();
+    for (int i = 0; i < min(nres, kMaxParts); ++i) resolve_unit<G>(p, ss.res[i], smem, ss);
+  }
+  // units without chunks (nothing indexed) are published by CTA u mod grid
+  for (int u = blockIdx.x; u < p.B * p.Hkv; u += gridDim.x)
+    if (unit_chunks(p, u) == 0) resolve_unit<G>(p, u, smem, ss);
 }
 
 template <typename Kern, typename P>
@@ -1169,15 +1388,15 @@ cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, boo
 }
 
 template <int G, int D>
-cudaError_t launch_scan_t(const ScanParams& p, int grid, cudaStream_t stream, bool pdl) {
+cudaError_t launch_scan_t(const StepParams& p, int grid, cudaStream_t stream, bool pdl) {
   const size_t smem = ScanSmem<G>::bytes(p.C, D);
-  cudaError_t e = ensure_dyn_smem<scan_kernel<G, D>>(smem);
+  cudaError_t e = ensure_dyn_smem<scan_select_kernel<G, D>>(smem);
   if (e != cudaSuccess) return e;
-  return launch_ex(scan_kernel<G, D>, dim3(grid), dim3(scan_threads_of<G>()), smem, stream, pdl, p);
+  return launch_ex(scan_select_kernel<G, D>, dim3(grid), dim3(kScanThreads), smem, stream, pdl, p);
 }
 
 template <int G>
-cudaError_t launch_scan_g(const ScanParams& p, int grid, cudaStream_t stream, bool pdl) {
+cudaError_t launch_scan_g(const StepParams& p, int grid, cudaStream_t stream, bool pdl) {
   switch (p.ring_depth) {
     case 8: return launch_scan_t<G, 8>(p, grid, stream, pdl);
     case 4: return launch_scan_t<G, 4>(p, grid, stream, pdl);
@@ -1186,7 +1405,7 @@ cudaError_t launch_scan_g(const ScanParams& p, int grid, cudaStream_t stream, bo
   }
 }
 
-cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t stream, bool pdl) {
+cudaError_t launch_scan_select(int G, const StepParams& p, int grid, cudaStream_t stream, bool pdl) {
   switch (G) {
     case 1: return launch_scan_g<1>(p, grid, stream, pdl);
     case 2: return launch_scan_g<2>(p, grid, stream, pdl);
@@ -1194,24 +1413,6 @@ cudaError_t launch_scan(int G, const ScanParams& p, int grid, cudaStream_t strea
     case 8: return launch_scan_g<8>(p, grid, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_filter(int G, const SelectParams& p, int grid, cudaStream_t stream, bool pdl) {
-#define CALL(GG) return launch_ex(filter_kernel<GG>, dim3(grid), dim3(kFilterThreads), 0, stream, pdl, p)
-  PQHSA_G_SWITCH(G, CALL)
-#undef CALL
-}
-
-cudaError_t launch_finalize(int G, const SelectParams& p, cudaStream_t stream, bool pdl) {
-  const size_t smem = static_cast<size_t>(fin_bt_cached(p.max_pages)) * sizeof(int32_t);
-#define CALL(GG)                                                                                     \
-  {                                                                                                  \
-    cudaError_t e = ensure_dyn_smem<finalize_kernel<GG>>(smem);                                      \
-    if (e != cudaSuccess) return e;                                                                  \
-    return launch_ex(finalize_kernel<GG>, dim3(p.B * p.Hkv), dim3(kFinThreads), smem, stream, pdl, p); \
-  }
-  PQHSA_G_SWITCH(G, CALL)
-#undef CALL
 }
 
 }  // namespace pqhsa

@@ -9,8 +9,6 @@
 // pacc[U][S][G][128] floats, S = number of split-K chunks.
 #include <cuda.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
-#include <dlfcn.h>
 #include <stdint.h>
 
 #include <algorithm>
@@ -58,49 +56,14 @@ cudaError_t scratch_for_current_device(void** ptr, int* sms) {
   return cudaSuccess;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess && f)
-      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    if (void* h = dlopen("libcuda.so.1", RTLD_NOW | RTLD_LOCAL))
-      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(dlsym(h, "cuTensorMapEncodeTiled"));
-    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
-  }();
-  return fn;
-}
-
-bool kv_tensor_map(CUtensorMap* map, const void* base, const hsa_kv_cache* kv, int box_rows) {
-  auto fn = tensor_map_encoder();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD),
-                        static_cast<cuuint64_t>(kv->num_pages) * kv->Hkv * kv->page_size};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
-  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1u, 1u};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The KV-cache view is validated exactly as dense_decode validates it.
 hsa_status validate(const hsa_kv_cache* kv, const float* q, const float* out) {
-  if (!kv || !kv->k_cache || !kv->v_cache || !kv->block_table || !kv->seq_lens || !kv->seq_lens_host || !q || !out)
-    return HSA_ERR_INVALID_ARG;
-  if (kv->B < 1 || kv->Hkv < 1 || kv->Hq < 1 || kv->max_pages < 1 || kv->num_pages < 1 || kv->Hq % kv->Hkv)
-    return HSA_ERR_INVALID_ARG;
-  const int G = kv->Hq / kv->Hkv;
-  if ((G != 1 && G != 2 && G != 4 && G != 8) || kv->D != kD) return HSA_ERR_UNSUPPORTED;
-  if (kv->page_size < 1 || kv->page_size > 128 || (kv->page_size & (kv->page_size - 1))) return HSA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(kv->num_pages) * kv->Hkv * kv->page_size >= (1LL << 31)) return HSA_ERR_UNSUPPORTED;
-  if (!is_aligned(kv->k_cache, 256) || !is_aligned(kv->v_cache, 256) || !is_aligned(q, 16) || !is_aligned(out, 16))
-    return HSA_ERR_ALIGNMENT;
-  const long long tmax = static_cast<long long>(kv->max_pages) * kv->page_size;
-  for (int b = 0; b < kv->B; ++b)
-    if (kv->seq_lens_host[b] < 0 || kv->seq_lens_host[b] > tmax) return HSA_ERR_CAPACITY;
+  const hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  if (!q || !out) return HSA_ERR_INVALID_ARG;
+  if (!is_aligned(q, 16) || !is_aligned(out, 16)) return HSA_ERR_ALIGNMENT;
   return HSA_OK;
 }
 
@@ -140,7 +103,7 @@ extern "C" hsa_status dense_decode_static(const hsa_kv_cache* kv, const float* q
   const bool rows = kv->page_size < 8;
   CUtensorMap tk = {}, tv = {};
   const int box_rows = std::min(kv->page_size, kTile);
-  if (!rows && (!kv_tensor_map(&tk, kv->k_cache, kv, box_rows) || !kv_tensor_map(&tv, kv->v_cache, kv, box_rows)))
+  if (!rows && (!make_kv_tmap(&tk, kv->k_cache, kv, box_rows) || !make_kv_tmap(&tv, kv->v_cache, kv, box_rows)))
     return HSA_ERR_CUDA;
 
   AttendParams p = {};

@@ -198,3 +198,19 @@ def test_binding_rejects_host_tensors_for_device_arrays():
     ix = P.PQIndex.allocate(B, Hkv, 4, 32, 4, "cpu")
     with pytest.raises(ValueError):
         ix.struct()
+
+
+def test_static_dense_decode_validates_like_dense_decode(lib):
+    """dense_decode_static checks the KV-cache view with the same validation as dense_decode:
+    a misaligned block table or length array is refused on the host, before any launch."""
+    fn = lib.dense_decode_static
+    fn.argtypes = [ctypes.POINTER(P._KV), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    lens = np.full(1, 100, dtype=np.int32)
+    for bt, sl in ((FAKE + 2, FAKE), (FAKE, FAKE + 2)):
+        kv = P._KV(FAKE, FAKE, bt, sl, lens.ctypes.data, 1, 4, 1, 128, 16, 8, 8)
+        assert fn(ctypes.byref(kv), FAKE, FAKE, ctypes.c_float(1.0), None) == 4
+    kv, _ = _kv(Hq=12, Hkv=1)
+    assert fn(ctypes.byref(kv), FAKE, FAKE, ctypes.c_float(1.0), None) == 2
+    kv, _ = _kv()
+    assert fn(ctypes.byref(kv), FAKE + 4, FAKE, ctypes.c_float(1.0), None) == 4

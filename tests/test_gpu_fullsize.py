@@ -37,7 +37,7 @@ def _decode_and_check(w, bt, codes, ids, units, dev):
         N = int(bt.n_indexed[b])
         rows = slice(h * w.G, (h + 1) * w.G)
         assert compare_logits(approx[b, rows, :N], r["s_hat"]) <= LOGIT_RTOL
-        assert nsel[b, h] == r["k"] == P.decode_k(w.budget, N)
+        assert nsel[b, h] == r["k"] == O.decode_k(w.budget, N)
         assert_sorted_positions(sel[b, h, :r["k"]])
         compare_selection(sel[b, h, :r["k"]], r, w.n_sink)
         assert float(np.abs(out[b, rows] - r["out"]).max()) <= OUT_TOL * vmax
@@ -45,7 +45,7 @@ def _decode_and_check(w, bt, codes, ids, units, dev):
     assert np.isfinite(out).all()
     for b in range(w.B):
         for h in range(w.Hkv):
-            k = P.decode_k(w.budget, int(bt.n_indexed[b]))
+            k = O.decode_k(w.budget, int(bt.n_indexed[b]))
             assert nsel[b, h] == k
             s = sel[b, h, :k]
             assert_sorted_positions(s)
@@ -54,6 +54,8 @@ def _decode_and_check(w, bt, codes, ids, units, dev):
 
 
 @pytest.mark.parametrize("name,units", [
+    ("llama8b_8k", [(0, 0), (0, 7)]),        # context sweep: exact tail (1024 rows) larger than k
+    ("llama8b_32k", [(0, 2), (0, 6)]),
     ("llama8b_128k", [(0, 0), (0, 5)]),
     ("llama8b_512k", [(0, 3)]),
     ("batch32_32k", [(0, 0), (13, 7), (31, 2)]),
