@@ -348,6 +348,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(base + L.off_cand);
   float* cand_w = reinterpret_cast<float*>(base + L.off_candw);
   int32_t* cand_c = reinterpret_cast<int32_t*>(base + L.off_candc);
+  int32_t* cand_row = reinterpret_cast<int32_t*>(base + L.off_candr);
   int32_t* sel = reinterpret_cast<int32_t*>(base + L.off_sel);
   float* pm = reinterpret_cast<float*>(base + L.off_pm);
   float* pl = reinterpret_cast<float*>(base + L.off_pl);
@@ -398,6 +399,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   sc.cand = cand;
   sc.cand_w = cand_w;
   sc.cand_c = cand_c;
+  sc.cand_row = cand_row;
   sc.units = units;
   sc.sel = sel;
   sc.block_table = kv->block_table;

@@ -70,10 +70,10 @@ template <bool kRows>
 __device__ __forceinline__ uint32_t v_area() { return kRows ? kTile * kRowPitch : 2 * kHalfBytes; }
 
 
-// Row v of a unit's exact list: the sink [0, s0), then the R tail rows [s0+N, T), then
-// the k selected tokens (ascending position). Sink and tail rows come first because they
-// do not depend on the selection: their copies and math run while the selection kernels
-// are still finishing. The selection stores selected tokens as KV-pool rows.
+// Position of row v of a unit's sink + tail list: the sink [0, s0), then the R tail rows
+// [s0+N, T). Each split takes these rows first, because they do not depend on the
+// selection: their copies and math run while the selection is still finishing. The
+// selection hands over its k tokens as KV-pool rows (in no particular order).
 __device__ __forceinline__ int exact_tail_pos(int v, int s0, int N) { return v < s0 ? v : s0 + N + (v - s0); }
 
 template <int G, bool kExact, bool kRows>
@@ -127,11 +127,30 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
     R = T - s0 - N;
     E = s0 + R + decode_k(p.budget, p.k_override, N);
   }
-  const int r0 = split * p.chunk;
-  const int r1 = min(E, r0 + p.chunk);
-  const int ntiles = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
-  // first tile holding a selected row (rows >= s0 + R); ntiles or more if none
-  const int first_sel_tile = kExact ? max(0, s0 + R - r0) / kTile : 0;
+  // Dense: rows [r0, r1) of the T tokens. Exact: the split's share of the sink and tail rows
+  // (the first ta tiles, rows [a0, a1) of the sink + tail list) and then its share of the
+  // selected rows (tb tiles, entries [e0, e1) of the selection), so every split has some of
+  // each: the tiles before the selection is published are spread over all splits, and so
+  // are the ones after.
+  int r0 = 0, r1 = 0, ta = 0, e0 = 0, e1 = 0;
+  if (kExact) {
+    const int A = s0 + R, K = E - A;
+    const int ca = (A + p.nsplit - 1) / p.nsplit, ce = (K + p.nsplit - 1) / p.nsplit;
+    r0 = min(A, split * ca);
+    r1 = min(A, r0 + ca);
+    e0 = min(K, split * ce);
+    e1 = min(K, e0 + ce);
+    ta = (r1 - r0 + kTile - 1) / kTile;
+  } else {
+    r0 = split * p.chunk;
+    r1 = min(E, r0 + p.chunk);
+    ta = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
+  }
+  const int ntiles = ta + (e1 - e0 + kTile - 1) / kTile;
+  const int first_sel_tile = ta;   // first tile of selected rows (ntiles if none)
+  // rows of tile t: first row (of the sink + tail list, or of the selection) and count
+  auto tile_first = [&](int t) { return t < ta ? r0 + t * kTile : e0 + (t - ta) * kTile; };
+  auto tile_rows = [&](int t) { return t < ta ? min(kTile, r1 - (r0 + t * kTile)) : min(kTile, e1 - (e0 + (t - ta) * kTile)); };
   const int32_t* sel_u = kExact ? p.sel + static_cast<size_t>(u) * p.cap : nullptr;
   const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
 
@@ -188,15 +207,15 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
         ys[i] = -1;
         const int t = t0 + i;
         if (t >= t1) continue;
-        const int row0 = r0 + t * kTile;
-        const int nvalid = min(kTile, r1 - row0);
+        const int row0 = tile_first(t);
+        const int nvalid = tile_rows(t);
         const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
         if (lane < nbox) {
           const int v = row0 + lane;
-          if (kExact && v >= s0 + R) {
+          if (kExact && t >= ta) {
             // already a KV-pool row (checked by the selection); an entry the selection did
             // not write cannot become an out-of-range read
-            int y = sel_u[v - s0 - R];
+            int y = sel_u[v];
             if (y < 0 || y >= p.num_pages * p.Hkv * p.page_size) {
               record_error(p.err, HSA_DEVERR_SELECT);
               y = 0;
@@ -222,8 +241,7 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
           ok = mbar_wait_warp(&empty[s], ((t / kStages) - 1) & 1, p.err);
           if (!ok) break;
         }
-        const int row0 = r0 + t * kTile;
-        const int nvalid = min(kTile, r1 - row0);
+        const int nvalid = tile_rows(t);
         uint8_t* st = stage_base + static_cast<size_t>(s) * kStageBytes;
         const int nbox = kRows ? nvalid : (nvalid + box_rows - 1) / box_rows;
         if (kRows) {
@@ -298,7 +316,7 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
   for (int t = warp; t < ntiles; t += kConsumerWarps) {
     const int s = t % kStages;
     if (!mbar_wait_warp(&full[s], (t / kStages) & 1, p.err)) break;   // converged before ldmatrix/mma
-    const int nvalid = min(kTile, r1 - (r0 + t * kTile));
+    const int nvalid = tile_rows(t);
     uint8_t* st = stage_base + static_cast<size_t>(s) * kStageBytes;
     const uint32_t sa = smem_addr(st);
     if (nvalid < kTile) {

@@ -289,21 +289,25 @@ __host__ __device__ inline long long list_slots_needed(int cap, int C) {
 
 // Workspace layout of hsa_decode (computed identically on host and device).
 // ---------------------------------------------------------------------------
-// Per unit bookkeeping of the scan and selection (zeroed by the tables). Each unit's state
-// takes its own 128-byte lines, and its ready flag (polled by the attention CTAs while the
-// selection runs) a line of its own, so polling never slows the counters' atomics.
+// Per unit bookkeeping of the scan and selection (zeroed by the tables). Every counter
+// that CTAs poll while others update it sits on a 128-byte line of its own (the attention
+// CTAs poll the ready flag, the selection's parts poll the phase counters), so polling
+// never slows the atomics on the other lines.
 struct alignas(128) UnitState {
   int32_t bstar;            // threshold bin
   int32_t above;            // tokens in bins above bstar
   int32_t ncand;            // tokens in bin bstar (candidates)
-  int32_t nsel;             // selected count written by the resolution
+  int32_t ndef;             // tokens above the threshold bin whose rows are written (definite)
+  int32_t pad0[28];
   int32_t scan_done;        // chunks of the unit scanned (histogram, weights and scores written)
-  int32_t filt_done;        // chunks of the unit whose selections and candidates are written
-  int32_t pad0[26];
-  int32_t ready;            // set (release) once the unit's selection and weight fix-up are final
   int32_t pad1[31];
+  int32_t filt_done;        // chunks of the unit whose selections and candidates are written
+  int32_t pad2[31];
+  int32_t pad3[32];
+  int32_t ready;            // set (release) once the unit's selection and weight fix-up are final
+  int32_t pad4[31];
 };
-static_assert(sizeof(UnitState) == 256, "two 128-byte lines per unit");
+static_assert(sizeof(UnitState) == 640, "five 128-byte lines per unit");
 
 // Publish a per-unit flag after this CTA's writes: call from every thread of the CTA.
 __device__ __forceinline__ void publish_flag(int32_t* flag) {
@@ -356,7 +360,7 @@ struct DecodeLayout {
   // byte offsets from the workspace base
   size_t off_units, off_bounds, off_fbounds, off_lut, off_qc, off_w, off_hist, off_sigma, off_cmax, off_bitmap,
       off_cand,
-      off_candw, off_candc, off_sel, off_pm, off_pl, off_pacc, total;
+      off_candw, off_candc, off_candr, off_sel, off_pm, off_pl, off_pacc, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -394,6 +398,7 @@ __host__ __device__ inline DecodeLayout make_decode_layout(int U, int G, int C, 
   L.off_cand = take(u * cap * sizeof(uint64_t));
   L.off_candw = take(u * kCandWeights * G * sizeof(float));
   L.off_candc = take(u * kCandWeights * sizeof(int32_t));
+  L.off_candr = take(u * cap * sizeof(int32_t));   // KV-pool row of each candidate
   L.off_sel = take(u * cap * sizeof(int32_t));
   const size_t parts = u * (nsplit_max + L.nbg) * G;
   L.off_pm = take(parts * sizeof(float));

@@ -148,6 +148,7 @@ struct StepParams {
   unsigned long long* cand;      // [U][cap] threshold-bin candidates (score key, slot)
   float* cand_w;                 // [U][kCandWeights][G] e^{shat_g - ub_g} of the first candidates
   int32_t* cand_c;               // [U][kCandWeights] their clusters
+  int32_t* cand_row;             // [U][cap] KV-pool row of each candidate
   UnitState* units;
   int32_t* sel;                  // [U][cap] KV-pool row of each selected token, ascending position
   const int32_t* block_table;    // [B][max_pages]

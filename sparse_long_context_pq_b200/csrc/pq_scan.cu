@@ -123,7 +123,9 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
       p.hist[static_cast<size_t>(u) * kNB + i] = 0u;
     for (int i = part * blockDim.x + tid; i < p.bitmap_words; i += kLutParts * blockDim.x)
       p.bitmap[static_cast<size_t>(u) * p.bitmap_words + i] = 0u;
-    if (part == 0 && tid < static_cast<int>(sizeof(UnitState) / 4)) reinterpret_cast<int32_t*>(p.units + u)[tid] = 0;
+    if (part == 0)
+      for (int i = tid; i < static_cast<int>(sizeof(UnitState) / 4); i += blockDim.x)
+        reinterpret_cast<int32_t*>(p.units + u)[i] = 0;
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < kSubPerPart; ++i) {
@@ -297,7 +299,7 @@ static_assert(kCandWeights <= kFinSmemCand, "stored candidate weights are resolv
 
 constexpr int kMaxParts = 24;   // (unit, chunk range) parts one CTA plans in shared memory
 #ifndef PQHSA_SCAN_PAIR
-#define PQHSA_SCAN_PAIR 1
+#define PQHSA_SCAN_PAIR 0
 #endif
 constexpr bool kScanPair = PQHSA_SCAN_PAIR != 0;   // phase 1 scores two chunks per warp step
 
@@ -312,6 +314,7 @@ struct SelShared {
   uint32_t nwin;
   int bin;
   uint32_t fin_above;
+  unsigned long long tau;        // the unit's threshold key: candidates with keys >= tau are selected
   int res[kMaxParts];            // units this CTA resolves after its filter parts
   // this CTA's parts
   int nparts;                    // -1: more than kMaxParts, walk the units instead
@@ -326,6 +329,18 @@ __device__ __forceinline__ int unit_chunks(const StepParams& p, int u) {
   const int n = p.list_meta[static_cast<size_t>(u) * (2 + 2 * static_cast<size_t>(p.C))];
   const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
   return N == 0 ? 0 : max(0, min(n, p.list_slots / 32));
+}
+
+// KV-pool row of position pos of KV head h through one block-table row; an entry outside
+// the pool is recorded and replaced by page 0.
+__device__ __forceinline__ int32_t kv_row(const StepParams& p, const int32_t* bt_row, int h, int pos) {
+  const int pi = pos / p.page_size;
+  int page = pi < p.max_pages ? bt_row[pi] : -1;
+  if (page < 0 || page >= p.num_pages) {
+    record_error(p.err, HSA_DEVERR_PAGE);
+    page = 0;
+  }
+  return (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
 }
 
 template <int G>
@@ -611,10 +626,13 @@ __device__ __forceinline__ void scan_segment(const StepParams& p, int u, int ch0
     const uint32_t v = hist_s[i];
     if (v) atomicAdd(hg + i, v);
   }
-  // publish this range: scores, chunk maxima, weights and histogram before the count
-  __threadfence();
+  // publish this range: scores, chunk maxima, weights and histogram before the count (the
+  // barrier orders the CTA's writes before thread 0's fence, which is cumulative)
   __syncthreads();
-  if (tid == 0) atomicAdd(&p.units[u].scan_done, nch);
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(&p.units[u].scan_done, nch);
+  }
 }
 
 // Head weights e^{shat_g - ub_g} of one indexed token (cluster id, code words cw) from the
@@ -656,16 +674,13 @@ __device__ __forceinline__ void remove_weights(const StepParams& p, int u, uint3
   for (int g = 0; g < G; ++g) atomicAdd(&Wu[g * p.C + id], -e[g]);
 }
 
-template <int G>
-__device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* fsm, SelShared& ss);
-
 // Phase 2 for chunks [c0, c1) of unit u (after every CTA of the unit has scanned): the
 // threshold bin, then only the chunks whose maximum reaches it (the bin is monotone in the
-// score). Tokens above the bin are selected (bitmap); the bin's tokens are candidates.
-// Definite selections' weights leave their clusters' sums here, from the tables in shared
-// memory when this CTA holds the unit's (`tables`), else from the global copy; the first
-// candidates' weights are stored for the resolution. Returns true if this CTA was the
-// unit's last to finish (it then resolves the unit, after its other filter parts).
+// score). Tokens above the bin are selected: their KV-pool rows join the unit's rows and
+// their weights leave their clusters' sums here (from the tables in shared memory when this
+// CTA holds the unit's, `tables`, else from the global copy). The bin's tokens are
+// candidates; the first ones' weights are stored for the resolution. Returns true in the
+// part that completes the unit's filter count (it then resolves the unit).
 template <int G>
 __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const uint8_t* tables, uint8_t* smem,
                             SelShared& ss) {
@@ -755,6 +770,10 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
     const uint4* lcodes = reinterpret_cast<const uint4*>(p.list_codes) + static_cast<size_t>(u) * p.list_slots;
     const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * max_chunks;
     uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
+    int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
+    const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
+    const int h = u % p.Hkv;
+    const int s0 = min(p.n_sink, max(0, p.seq_lens[b]));
 
     for (int cb = c0; cb < c1; cb += kCmPass) {
       if (cb != c0) {
@@ -800,13 +819,33 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
           const bool valid = j >= 0 && j < N;
           const int bin = valid ? score_bin(sv[r], lo, inv) : -1;
           const bool definite = bin > bstar;
-          if (definite) atomicOr(bm + (j >> 5), 1u << (j & 31));
+          {   // a definite selection's KV-pool row joins the unit's rows (one atomic per warp)
+            const uint32_t dm = __ballot_sync(0xffffffffu, definite);
+            if (dm) {
+              const uint32_t leader = __ffs(dm) - 1;
+              int at = 0;
+              if (lane == leader) at = atomicAdd(&p.units[u].ndef, __popc(dm));
+              at = __shfl_sync(0xffffffffu, at, leader);
+              if (definite) {
+                const int o = at + __popc(dm & ((1u << lane) - 1u));
+                if (o < p.cap) sel_u[o] = kv_row(p, bt_row, h, s0 + j);
+                if (p.dbg_selected) atomicOr(bm + (j >> 5), 1u << (j & 31));   // for the ascending positions
+              }
+            }
+          }
           int slot = -1;
-          if (bin == bstar) {
-            slot = atomicAdd(&p.units[u].ncand, 1);
-            if (slot < p.cap)
-              p.cand[static_cast<size_t>(u) * p.cap + slot] =
-                  (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+          const uint32_t cm_ = __ballot_sync(0xffffffffu, bin == bstar);
+          if (cm_) {   // one atomic per warp for its candidates
+            const uint32_t leader = __ffs(cm_) - 1;
+            int at = 0;
+            if (lane == leader) at = atomicAdd(&p.units[u].ncand, __popc(cm_));
+            at = __shfl_sync(0xffffffffu, at, leader);
+            if (bin == bstar) slot = at + __popc(cm_ & ((1u << lane) - 1u));
+          }
+          if (bin == bstar && slot < p.cap) {
+            p.cand[static_cast<size_t>(u) * p.cap + slot] =
+                (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+            p.cand_row[static_cast<size_t>(u) * p.cap + slot] = kv_row(p, bt_row, h, s0 + j);
           }
           if (fix) {
             // queue the list slot: a definite selection's weight leaves its cluster's sums
@@ -854,10 +893,11 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
       __syncthreads();   // this pass is done with act[] and n_act
     }
   }
-  // publish this range's selections, candidates and fix-ups, then count it in
-  __threadfence();
+  // publish this range's selections, candidates and fix-ups, then count it in; the part
+  // that completes the count resolves the unit
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const int n = c1 - c0;
     const int old = atomicAdd(&p.units[u].filt_done, n);
     ss.flag = (old < total && old + n >= total) ? 1 : 0;
@@ -896,101 +936,76 @@ __device__ void find_threshold_desc(const uint32_t* cnt, int nbins, uint32_t nee
   }
 }
 
-// Phase 3 for unit u, by the CTA that finished its filter last (or, for a unit with no
-// chunks, by CTA u mod grid): resolve the threshold bin's candidates exactly (score desc,
-// position asc), compact the selection bitmap into ascending positions written as KV-pool
-// rows, take the winners' weights out of the cluster sums, and publish the unit. Every
-// input (lengths, counters, candidate keys and stored weights, the first bitmap pass, the
-// block table) is fetched in one round trip. `fsm` holds kFinScratch bytes (over the
-// tables: the CTA's filter parts are done).
+// Phase 3 for unit u, in the part that completed its filter count: the threshold bin's
+// candidates are resolved exactly (the r largest keys, score desc then position asc, with
+// r = k - tokens above the bin); the winners' KV-pool rows follow the definite selections'
+// rows in key order, their weights leave their clusters' sums, and the unit is published.
+// The rows are in no particular position order (the attention does not need one); only
+// the debug positions are written in ascending order, after the unit is published.
+// `fsm` holds kFinScratch bytes (over the tables: this CTA's filter parts are done).
 template <int G>
-__device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* fsm, SelShared& ss) {
+__device__ void resolve_unit(const StepParams& p, int u, uint8_t* fsm, SelShared& ss) {
   constexpr int GP = (G + 3) / 4;
   constexpr int T = kScanThreads;
   constexpr int kKeysPer = kFinSmemCand / T;   // candidate keys fetched per thread
-  constexpr int kBtPer = kFinBt / T;           // block-table entries fetched per thread
   unsigned long long* ck = reinterpret_cast<unsigned long long*>(fsm);   // [kFinSmemCand]
   uint32_t* bmc = reinterpret_cast<uint32_t*>(ck + kFinSmemCand);         // [kFinChunkWords]
   uint32_t* woff = bmc + kFinChunkWords;                                  // [kFinChunkWords]
-  uint32_t* wins = woff + kFinChunkWords;                                 // [kFinSmemCand]
-  uint32_t* dig = wins + kFinSmemCand;                                    // [256]
-  int32_t* bt_s = reinterpret_cast<int32_t*>(dig + 256);                 // [kFinBt]
+  uint32_t* dig = woff + kFinChunkWords;                                  // [256]
   const int b = u / p.Hkv;
   const int h = u % p.Hkv;
   const int tid = threadIdx.x;
   const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
   const unsigned long long* cg = p.cand + static_cast<size_t>(u) * p.cap;
-  const uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
-  const int nbt = min(p.max_pages, kFinBt);
-  __syncthreads();   // the scratch overlays the tables and the filter's queues
+  int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
+  const int T_len = max(0, p.seq_lens[b]);
+  const int s0 = min(p.n_sink, T_len);
+  const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
+  const int k = decode_k(p.budget, p.k_override, N);
+  const bool fix = p.background && N > k;
+  __syncthreads();   // the scratch overlays the tables and the filter queues
 
-  // ---- one round trip: every load below is independent of the others ----
-  const int T_raw = p.seq_lens[b];
-  const int n_raw = p.n_indexed[b];
+  // ---- one round trip ----
   const int ncand = __ldcg(&p.units[u].ncand);
   const int above = __ldcg(&p.units[u].above);
+  const int ndef = __ldcg(&p.units[u].ndef);
   unsigned long long kr[kKeysPer];   // candidate keys of slots tid + r T (speculative: any count)
 #pragma unroll
   for (int r = 0; r < kKeysPer; ++r) {
     const int i = tid + r * T;
     kr[r] = i < p.cap ? __ldcg(cg + i) : 0ull;
   }
+  const int32_t* crow = p.cand_row + static_cast<size_t>(u) * p.cap;
+  const int32_t rowr = tid < p.cap ? __ldcg(crow + tid) : 0;   // KV-pool row of candidate slot tid
   float cwr[G];                      // stored weights of candidate slot tid
   int32_t ccr = 0;
-  if (p.background) {
+  if (fix) {
     const float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + tid) * G;
 #pragma unroll
     for (int g = 0; g < G; ++g) cwr[g] = tid < kCandWeights ? __ldcg(cw + g) : 0.f;
     ccr = tid < kCandWeights ? __ldcg(p.cand_c + static_cast<size_t>(u) * kCandWeights + tid) : 0;
   }
-  uint32_t words[kFinWordsPerThread];   // first bitmap pass
+  float ub2[G];
 #pragma unroll
-  for (int e = 0; e < kFinWordsPerThread; ++e) {
-    const int wi = kFinWordsPerThread * tid + e;
-    words[e] = wi < p.bitmap_words ? __ldcg(bm + wi) : 0u;
-  }
-  int32_t btv[kBtPer];
-#pragma unroll
-  for (int e = 0; e < kBtPer; ++e) btv[e] = tid + e * T < nbt ? bt_row[tid + e * T] : 0;
+  for (int g = 0; g < G; ++g) ub2[g] = __ldcg(p.fbounds + (static_cast<size_t>(u) * 2 + 0) * G + g) * kLog2e;
 
-  const int T_len = max(0, T_raw);
-  const int s0 = min(p.n_sink, T_len);
-  const int N = min(max(0, min(n_raw, T_len - s0)), p.cap);
-  const int k = decode_k(p.budget, p.k_override, N);
-  const bool fix = p.background && N > k;
-  int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
-  if (k == 0) {
-    if (tid == 0) {
-      p.units[u].nsel = 0;
-      if (p.dbg_nselected) p.dbg_nselected[u] = 0;
-    }
-    publish_flag(&p.units[u].ready);
-    return;
-  }
-  const int m = min(ncand, p.cap);
+  const int m = k > 0 ? min(ncand, p.cap) : 0;
   const int r = k - above;
-  const bool ok = r >= 1 && r <= m;
-  if (!ok && tid == 0) record_error(p.err, HSA_DEVERR_SELECT);
+  const bool ok = k == 0 || (r >= 1 && r <= m);
   const bool in_smem = m <= kFinSmemCand;
 #pragma unroll
   for (int rr = 0; rr < kKeysPer; ++rr)
     if (tid + rr * T < min(m, kFinSmemCand)) ck[tid + rr * T] = kr[rr];
-#pragma unroll
-  for (int e = 0; e < kBtPer; ++e)
-    if (tid + e * T < nbt) bt_s[tid + e * T] = btv[e];
-  if (tid == 0) ss.nwin = 0;
+  if (tid == 0) {
+    ss.tau = ~0ull;
+    ss.nwin = 0;
+  }
   __syncthreads();
   auto key_at = [&](int i) -> unsigned long long { return in_smem ? ck[i] : __ldcg(cg + i); };
-  float ub2[G];
-  {
-    float ub[G], lb[G];
-    final_bounds<G>(p.fbounds, u, ub, lb);
-#pragma unroll
-    for (int g = 0; g < G; ++g) ub2[g] = ub[g] * kLog2e;
-  }
-  // A winner's weights leave its cluster's sums: from registers (candidate slot tid), from
-  // the filter's store (slot < kCandWeights), else recomputed from the global tables.
-  auto fix_winner = [&](int i, uint32_t j) {
+  // A winner: its row after the definite rows (at `o`), its weights out of its cluster's sums.
+  auto take_winner = [&](int i, unsigned long long key, int o) {
+    const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
+    if (ndef + o < p.cap) sel_u[ndef + o] = i == tid ? rowr : __ldcg(crow + i);
     if (!fix) return;
     float e[G];
     uint32_t id;
@@ -1016,17 +1031,15 @@ __device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* f
   };
 
   // ---- winners: the r largest candidate keys (keys are distinct) ----
-  if (ok) {
+  if (k > 0 && ok) {
     if (m <= T) {
-      if (tid < m) {
+      if (tid < m) {   // rank = place in descending key order; the r first win, in rank order
         const unsigned long long key = key_at(tid);
         int rank = 0;
+#pragma unroll 8
         for (int j = 0; j < m; ++j) rank += key_at(j) > key;
-        if (rank < r) {
-          const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
-          wins[atomicAdd(&ss.nwin, 1u)] = j;
-          fix_winner(tid, j);
-        }
+        if (rank < r) take_winner(tid, key, rank);
+        if (rank == r - 1) ss.tau = key;
       }
     } else {
       unsigned long long prefix = 0, mask = 0;
@@ -1051,46 +1064,46 @@ __device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* f
         mask |= 255ull << shift;
         __syncthreads();
       }
-      const unsigned long long tau = prefix;
+      if (tid == 0) ss.tau = prefix;
       for (int i = tid; i < m; i += T) {
         const unsigned long long key = key_at(i);
-        if (key >= tau) {
-          const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
-          const uint32_t w = atomicAdd(&ss.nwin, 1u);
-          if (w < kFinSmemCand) wins[w] = j;
-          else atomicOr(p.bitmap + static_cast<size_t>(u) * p.bitmap_words + (j >> 5), 1u << (j & 31));
-          fix_winner(i, j);
-        }
+        if (key >= prefix) take_winner(i, key, static_cast<int>(atomicAdd(&ss.nwin, 1u)));
       }
     }
   }
+  // publish: the rows and the winners' fix-ups are written
   __syncthreads();
-  const uint32_t nwin_all = ss.nwin;
-  const uint32_t nwin = min(nwin_all, static_cast<uint32_t>(kFinSmemCand));
-  if (nwin < nwin_all) __threadfence_block();   // overflowed winners went to the global bitmap
+  const int nsel = ndef + ((k > 0 && ok) ? r : 0);
+  if (tid == 0) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(&p.units[u].ready), "r"(1) : "memory");
+    if (!ok || nsel != k) record_error(p.err, HSA_DEVERR_SELECT);
+    if (p.dbg_nselected) p.dbg_nselected[u] = nsel;
+  }
+  if (!p.dbg_selected || k == 0) return;
 
-  // ---- compaction of the selection bitmap into ascending positions ----
+  // ---- debug: the selected positions in ascending order (definite bits and winners) ----
+  const uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
+  const unsigned long long tau = ss.tau;
   const int nw = (N + 31) / 32;
   uint32_t running = 0;
   for (int w0 = 0; w0 < nw; w0 += kFinChunkWords) {
-    if (w0 > 0 || nwin < nwin_all) {   // later passes, or winners that went to the global bitmap
+    const int we = min(nw, w0 + kFinChunkWords);
 #pragma unroll
-      for (int e = 0; e < kFinWordsPerThread; ++e) {
-        const int wi = w0 + kFinWordsPerThread * tid + e;
-        words[e] = wi < p.bitmap_words ? __ldcg(bm + wi) : 0u;
-      }
+    for (int e = 0; e < kFinWordsPerThread; ++e) {
+      const int wi = w0 + kFinWordsPerThread * tid + e;
+      bmc[kFinWordsPerThread * tid + e] = wi < we ? __ldcg(bm + wi) : 0u;
     }
-#pragma unroll
-    for (int e = 0; e < kFinWordsPerThread; ++e)
-      bmc[kFinWordsPerThread * tid + e] = (w0 + kFinWordsPerThread * tid + e < nw) ? words[e] : 0u;
     __syncthreads();
-    for (uint32_t i = tid; i < nwin; i += T) {
-      const uint32_t j = wins[i];
+    for (int i = tid; i < m; i += T) {
+      const unsigned long long key = key_at(i);
+      if (key < tau) continue;
+      const uint32_t j = 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
       const int w = static_cast<int>(j >> 5) - w0;
-      if (w >= 0 && w < kFinChunkWords) atomicOr(&bmc[w], 1u << (j & 31));
+      if (w >= 0 && w < we - w0) atomicOr(&bmc[w], 1u << (j & 31));
     }
     __syncthreads();
-    uint32_t pc = 0;
+    uint32_t words[kFinWordsPerThread], pc = 0;
 #pragma unroll
     for (int e = 0; e < kFinWordsPerThread; ++e) {
       words[e] = bmc[kFinWordsPerThread * tid + e];
@@ -1106,9 +1119,6 @@ __device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* f
       }
     }
     __syncthreads();
-    // Output entry i of this pass: the word holding it by binary search over the word
-    // offsets, then its bit; every thread writes about tot / T entries whatever the
-    // positions of the selected tokens.
     for (uint32_t i = tid; i < tot; i += T) {
       int lo_w = 0, hi_w = kFinChunkWords - 1;   // largest word with woff <= i
       while (lo_w < hi_w) {
@@ -1118,32 +1128,23 @@ __device__ __noinline__ void resolve_unit(const StepParams& p, int u, uint8_t* f
       }
       uint32_t wv = bmc[lo_w];
       for (uint32_t c = i - woff[lo_w]; c > 0; --c) wv &= wv - 1;
-      const int j = (w0 + lo_w) * 32 + (__ffs(wv) - 1);
       const uint32_t off = running + i;
-      if (off < static_cast<uint32_t>(p.cap)) {
-        // the token's KV-pool row, so the exact attend reads it in one step
-        const int pos = s0 + j;
-        const int pi = pos / p.page_size;
-        int page = pi < nbt ? bt_s[pi] : (pi < p.max_pages ? bt_row[pi] : -1);
-        if (page < 0 || page >= p.num_pages) {
-          record_error(p.err, HSA_DEVERR_PAGE);
-          page = 0;
-        }
-        sel_u[off] = (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
-        if (p.dbg_selected) p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = pos;
-      }
+      if (off < static_cast<uint32_t>(p.cap))
+        p.dbg_selected[static_cast<size_t>(u) * p.cap + off] = s0 + (w0 + lo_w) * 32 + (__ffs(wv) - 1);
     }
     running += tot;
     __syncthreads();   // woff / bmc are rewritten by the next pass
   }
-  if (tid == 0) {
-    p.units[u].nsel = static_cast<int32_t>(running);
-    if (running != static_cast<uint32_t>(k)) record_error(p.err, HSA_DEVERR_SELECT);
-    if (p.dbg_nselected) p.dbg_nselected[u] = static_cast<int32_t>(running);
+}
+
+// A unit with no chunks to scan (nothing indexed): nothing is selected; publish it.
+__device__ void publish_empty_unit(const StepParams& p, int u) {
+  if (threadIdx.x == 0) {
+    const int N = unit_n(p.seq_lens, p.n_indexed, u / p.Hkv, p.n_sink, p.cap);
+    if (decode_k(p.budget, p.k_override, N) != 0) record_error(p.err, HSA_DEVERR_SELECT);
+    if (p.dbg_nselected) p.dbg_nselected[u] = 0;
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(&p.units[u].ready), "r"(1) : "memory");
   }
-  // the exact attend and the background of this unit may start (selection rows and
-  // the winners' weight fix-up are written)
-  publish_flag(&p.units[u].ready);
 }
 
 // Work split over the units' chunks, planned cooperatively by the CTA (one pass over the
@@ -1204,9 +1205,9 @@ __device__ void plan_parts(const StepParams& p, SelShared& ss) {
     int i0 = 0, i1 = 0;
     if (per_unit) {
       if (n > 0 && me >= base && me < base + w) {
-        const long long kk = me - base;
-        i0 = static_cast<int>(n * kk / w);
-        i1 = static_cast<int>(n * (kk + 1) / w);
+        const int kk = static_cast<int>(me - base);
+        i0 = static_cast<int>(static_cast<long long>(n) * kk / w);
+        i1 = static_cast<int>(static_cast<long long>(n) * (kk + 1) / w);
       }
     } else if (n > 0 && start < base + n && end > base) {
       i0 = static_cast<int>(max(start - base, 0LL));
@@ -1304,8 +1305,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_select_kernel(StepParams
   } else {
     walk_parts(p, total, scan);
   }
-  // ---- phase 2: selection per unit; phase 3: resolution by the unit's last CTA, after
-  // all of this CTA's filter parts, so that no unit's filter waits behind a resolution ----
+  // ---- phase 2: selection per unit; phase 3: the part that completes a unit's filter
+  // resolves it, after all of this CTA's filter parts (no unit's filter waits behind it) ----
   int nres = 0;
   auto filt = [&](int u, int c0, int c1) {
     if (filter_part<G>(p, u, c0, c1, tables_unit == u ? smem : nullptr, smem, ss)) {
@@ -1325,13 +1326,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_select_kernel(StepParams
     walk_parts(p, total, filt);
   }
   if (nres > 0) {
-    __threadfence();   // acquire: the unit's other CTAs published before counting in
+    __threadfence();   // acquire: the unit's other parts published before counting in
     __syncthreads();
     for (int i = 0; i < min(nres, kMaxParts); ++i) resolve_unit<G>(p, ss.res[i], smem, ss);
   }
   // units without chunks (nothing indexed) are published by CTA u mod grid
   for (int u = blockIdx.x; u < p.B * p.Hkv; u += gridDim.x)
-    if (unit_chunks(p, u) == 0) resolve_unit<G>(p, u, smem, ss);
+    if (unit_chunks(p, u) == 0) publish_empty_unit(p, u);
 }
 
 template <typename Kern, typename P>
