@@ -20,6 +20,17 @@ def lib():
     return P.load_library()
 
 
+@pytest.fixture(scope="module")
+def host_only(lib):
+    """Tests that pass fake device pointers expect the call to refuse on the host before any
+    launch; they run only where no GPU is visible, so a validation regression can never
+    launch a kernel on addresses that are not device memory."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-validation test with fake device pointers: CPU-only")
+    return lib
+
+
 def _declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -93,7 +104,8 @@ def _decode(lib, kv, ix, ws_bytes=1 << 30, q=FAKE):
     (dict(seq=1000), 3),               # longer than the block table
     (dict(aligned=False), 4),          # cache pointer not 256-byte aligned
 ])
-def test_decode_rejects_bad_cache(lib, mutate, status):
+def test_decode_rejects_bad_cache(host_only, mutate, status):
+    lib = host_only
     kv, lens = _kv(**mutate)
     ix, nh = _ix()
     assert _decode(lib, kv, ix) == status
@@ -109,13 +121,15 @@ def test_decode_rejects_bad_cache(lib, mutate, status):
     (dict(list_slot=FAKE + 4), 4),     # list slots are streamed by 16-byte async copies
     (dict(chunk_cluster=FAKE + 2), 4), # cluster ids are fetched as aligned 4-byte words
 ])
-def test_decode_rejects_bad_index(lib, mutate, status):
+def test_decode_rejects_bad_index(host_only, mutate, status):
+    lib = host_only
     kv, lens = _kv()
     ix, nh = _ix(**mutate)
     assert _decode(lib, kv, ix) == status
 
 
-def test_decode_rejects_small_workspace_and_null_q(lib):
+def test_decode_rejects_small_workspace_and_null_q(host_only):
+    lib = host_only
     kv, lens = _kv()
     ix, nh = _ix()
     assert _decode(lib, kv, ix, ws_bytes=16) == 5
@@ -124,7 +138,8 @@ def test_decode_rejects_small_workspace_and_null_q(lib):
     assert need > 0 and need % 256 == 0
 
 
-def test_append_checks_capacity(lib):
+def test_append_checks_capacity(host_only):
+    lib = host_only
     kv, lens = _kv(seq=100)
     ix, nh = _ix(n_idx=50, n_sink=4, cap=60)
     big = 1 << 30
@@ -135,7 +150,8 @@ def test_append_checks_capacity(lib):
     assert nh2[0] == 50                                                                           # untouched
 
 
-def test_append_workspace(lib):
+def test_append_workspace(host_only):
+    lib = host_only
     kv, lens = _kv(seq=100)
     ix, nh = _ix(n_idx=40, n_sink=4, cap=128, C=16)
     q = lambda k, i, n: lib.hsa_index_workspace_bytes(ctypes.byref(k), ctypes.byref(i), n)
@@ -147,7 +163,8 @@ def test_append_workspace(lib):
     assert q(kv4, ix, 20) == 256                                # 4-row pages: CUDA-core encoding
 
 
-def test_dense_rejects_bad_args(lib):
+def test_dense_rejects_bad_args(host_only):
+    lib = host_only
     kv, lens = _kv()
     assert lib.dense_decode(ctypes.byref(kv), FAKE + 4, FAKE, ctypes.c_float(1.0), FAKE, 1 << 30, None) == 4
     assert lib.dense_decode(ctypes.byref(kv), FAKE, FAKE, ctypes.c_float(1.0), FAKE, 8, None) == 5
@@ -168,13 +185,15 @@ def _train(lib, kv, ix, n_train=40, coarse=2, pq=2, ws_bytes=1 << 30, init=FAKE,
     (dict(assign_out=FAKE + 2), 4),
     (dict(ws_bytes=64), 5),
 ])
-def test_train_rejects_bad_args(lib, kw, status):
+def test_train_rejects_bad_args(host_only, kw, status):
+    lib = host_only
     kv, lens = _kv()
     ix, nh = _ix()
     assert _train(lib, kv, ix, **kw) == status
 
 
-def test_train_rejects_unsupported_index(lib):
+def test_train_rejects_unsupported_index(host_only):
+    lib = host_only
     kv, lens = _kv(seq=2 << 20, max_pages=(2 << 20) // 16, num_pages=(2 << 20) // 16)
     ix, nh = _ix(cap=2 << 20)
     assert _train(lib, kv, ix, n_train=65535 * 32 + 1) == 2   # beyond the longest training set
@@ -200,9 +219,10 @@ def test_binding_rejects_host_tensors_for_device_arrays():
         ix.struct()
 
 
-def test_static_dense_decode_validates_like_dense_decode(lib):
+def test_static_dense_decode_validates_like_dense_decode(host_only):
     """dense_decode_static checks the KV-cache view with the same validation as dense_decode:
     a misaligned block table or length array is refused on the host, before any launch."""
+    lib = host_only
     fn = lib.dense_decode_static
     fn.argtypes = [ctypes.POINTER(P._KV), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
     fn.restype = ctypes.c_int
@@ -214,3 +234,21 @@ def test_static_dense_decode_validates_like_dense_decode(lib):
     assert fn(ctypes.byref(kv), FAKE, FAKE, ctypes.c_float(1.0), None) == 2
     kv, _ = _kv()
     assert fn(ctypes.byref(kv), FAKE + 4, FAKE, ctypes.c_float(1.0), None) == 4
+
+
+def test_static_dense_decode_rejects_shapes_beyond_its_array(host_only):
+    """The split-K partials of one chunk need B * Hkv * G * 520 bytes plus 768 of alignment
+    slack in the 8 MiB array (after a 256-byte header): B * Hkv * G <= 16129 fits, 16130 does
+    not. Refused shapes return HSA_ERR_WORKSPACE before any CUDA call (the pointers here are
+    never dereferenced: only refused shapes are passed)."""
+    lib = host_only
+    fn = lib.dense_decode_static
+    fn.argtypes = [ctypes.POINTER(P._KV), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    limit = ((8 << 20) - 256 - 768) // 520
+    assert limit == 16129
+    for B, Hq, Hkv in ((4096, 64, 8), (253, 64, 8), (16130, 1, 1)):
+        assert B * Hq >= limit + 1                    # B * Hkv * G = B * Hq
+        lens = np.full(B, 64, dtype=np.int32)
+        kv = P._KV(FAKE, FAKE, FAKE, FAKE, lens.ctypes.data, B, Hq, Hkv, 128, 16, 4, 4096)
+        assert fn(ctypes.byref(kv), FAKE, FAKE, ctypes.c_float(1.0), None) == 5

@@ -91,13 +91,3 @@ def test_static_scratch_at_its_largest_shape(cuda_device):
         assert float(np.abs(got[b, h * w.G:(h + 1) * w.G] - r).max()) <= tol
     ws_out = P.dense_decode(kv, q, scale=scale).cpu().numpy()
     assert float(np.abs(got - ws_out).max()) <= tol
-
-
-def test_static_scratch_rejects_shapes_beyond_its_limit(cuda_device):
-    lens = np.full(4096, 64, dtype=np.int32)
-    fake = 1 << 20
-    kvs = P._KV(fake, fake, fake, fake, lens.ctypes.data, 4096, 64, 8, 128, 16, 4, 4096)  # B*Hkv*G = 262144
-    assert _entry()(ctypes.byref(kvs), fake, fake, ctypes.c_float(1.0), None) == 5
-    lens = np.full(252, 64, dtype=np.int32)
-    kvs = P._KV(fake, fake, fake, fake, lens.ctypes.data, 252, 64, 8, 128, 16, 4, 4096)     # 16128: just over
-    assert _entry()(ctypes.byref(kvs), fake, fake, ctypes.c_float(1.0), None) == 5
