@@ -241,9 +241,10 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
 // scores them against the unit's tables in shared memory: approximate logits, the
 // selection score sigma, per-cluster exp-weight sums, a histogram of sigma and each
 // chunk's largest sigma. Phase 2 (filter), per unit, once every CTA of the unit has
-// scanned its chunks: the threshold bin from the unit's histogram, the definite
-// selections (bitmap), the threshold-bin candidates and the weight fix-ups of this
-// CTA's chunks. Phase 3 (resolution), by the unit's last CTA to finish phase 2: the
+// scanned its chunks: the threshold bin from the unit's histogram, then, over this CTA's
+// share of the unit's chunks (spread over the whole list), the definite selections' rows,
+// the threshold-bin candidates and the weight fix-ups. Phase 3 (resolution), by the
+// unit's last CTA to finish phase 2: the
 // exact order of the candidates (score desc, position asc), the selected tokens as
 // KV-pool rows in ascending position order, the winners' weight fix-ups, the ready flag.
 //
@@ -284,8 +285,7 @@ struct ScanSmem {
 constexpr int kCmPerThread = 4;                                  // chunk maxima per thread per pass
 constexpr int kCmPass = kCmPerThread * kScanThreads;             // chunks examined per pass
 constexpr int kActPerWarp = 2;                                   // active chunks per warp per round
-constexpr int kFixCap = kActPerWarp * kScanThreads;              // queued tokens per round
-constexpr size_t kFilterScratch = (kCmPass + 2 * kFixCap) * 4;
+constexpr size_t kFilterScratch = kCmPass * 4;
 constexpr int kFinWordsPerThread = 8;
 constexpr int kFinChunkWords = kFinWordsPerThread * kScanThreads;   // 131072 slots per pass
 constexpr int kFinSmemCand = 1024;                                  // candidates resolved in shared memory
@@ -309,7 +309,6 @@ struct SelShared {
   int bstar;
   uint32_t above;
   int n_act;
-  uint32_t fix_n;
   int flag;
   uint32_t nwin;
   int bin;
@@ -319,6 +318,7 @@ struct SelShared {
   // this CTA's parts
   int nparts;                    // -1: more than kMaxParts, walk the units instead
   int pu[kMaxParts], pc0[kMaxParts], pc1[kMaxParts];
+  uint32_t pst[kMaxParts];       // phase-2 chunk permutation stride of the part's unit
   long long total;
   int active;
 };
@@ -674,18 +674,50 @@ __device__ __forceinline__ void remove_weights(const StepParams& p, int u, uint3
   for (int g = 0; g < G; ++g) atomicAdd(&Wu[g * p.C + id], -e[g]);
 }
 
-// Phase 2 for chunks [c0, c1) of unit u (after every CTA of the unit has scanned): the
-// threshold bin, then only the chunks whose maximum reaches it (the bin is monotone in the
-// score). Tokens above the bin are selected: their KV-pool rows join the unit's rows and
-// their weights leave their clusters' sums here (from the tables in shared memory when this
-// CTA holds the unit's, `tables`, else from the global copy). The bin's tokens are
-// candidates; the first ones' weights are stored for the resolution. Returns true in the
-// part that completes the unit's filter count (it then resolves the unit).
+// Stride of the chunk permutation c -> (c * stride) mod n of phase 2: about n / golden
+// ratio and coprime with n, so the map is a bijection of [0, n) and any run of consecutive
+// chunks (a high-scoring cluster's) is spread evenly over every range of c. Every CTA of a
+// unit derives the same stride from n alone. Terminates: n - 1 is coprime with n.
+__device__ __forceinline__ uint32_t gcd_u32(uint32_t a, uint32_t b) {   // binary gcd, a, b > 0
+  const int sh = __ffs(a | b) - 1;
+  a >>= __ffs(a) - 1;
+  do {
+    b >>= __ffs(b) - 1;
+    if (a > b) {
+      const uint32_t t = a;
+      a = b;
+      b = t;
+    }
+    b -= a;
+  } while (b);
+  return a << sh;
+}
+__device__ __forceinline__ uint32_t scatter_stride(uint32_t n) {
+  if (n <= 2) return 1u;
+  uint32_t s = static_cast<uint32_t>((static_cast<unsigned long long>(n) * 2654435769ull) >> 32);
+  if (s == 0) s = 1;
+  while (gcd_u32(n, s) != 1u) ++s;
+  return s;
+}
+
+// Phase 2 for part [c0, c1) of unit u (after every CTA of the unit has scanned): the
+// threshold bin, then the part's chunks, c -> (c * stride) mod total with
+// stride = scatter_stride(total), whose maximum reaches
+// it (the bin is monotone in the score). The permutation only decides which part handles
+// a chunk (parts still partition the unit's chunks); it keeps the chunks of high-scoring
+// clusters, which are consecutive in list order, from piling up in one part. Tokens above
+// the bin are selected: their KV-pool rows join the unit's rows and their weights leave
+// their clusters' sums here (from the tables in shared memory when this CTA holds the
+// unit's, `tables`, else from the global copy). The bin's tokens are candidates; the
+// first ones' weights are stored for the resolution. Every lane handles its own slot, so
+// a warp's chunks need no block-wide step. Returns true in the part that completes the
+// unit's filter count (it then resolves the unit).
 template <int G>
-__device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const uint8_t* tables, uint8_t* smem,
-                            SelShared& ss) {
+__device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t stride, const uint8_t* tables,
+                            uint8_t* smem, SelShared& ss) {
   constexpr int GP = (G + 3) / 4;
   constexpr int NW = kScanWarps;
+  constexpr int T = kScanThreads;
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane = tid & 31;
   const int b = u / p.Hkv;
@@ -693,21 +725,21 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
   const int k = decode_k(p.budget, p.k_override, N);
   const int max_chunks = p.list_slots / 32;
   const int total = unit_chunks(p, u);
-  uint8_t* scratch = smem + ScanSmem<G>::hist_off(p.C);
-  int32_t* act = reinterpret_cast<int32_t*>(scratch);                    // active chunks of the pass
-  uint32_t* fix_list = reinterpret_cast<uint32_t*>(act + kCmPass);       // list slots
-  int32_t* fix_cand = reinterpret_cast<int32_t*>(fix_list + kFixCap);    // candidate slot, -1 = definite
+  int32_t* act = reinterpret_cast<int32_t*>(smem + ScanSmem<G>::hist_off(p.C));   // active chunks of the pass
   const float4* lut4 = tables ? reinterpret_cast<const float4*>(tables)
                               : reinterpret_cast<const float4*>(p.lut) + static_cast<size_t>(u) * GP * kNcode * kM;
   const float4* qc4 = tables ? reinterpret_cast<const float4*>(tables) + GP * kNcode * kM
                              : reinterpret_cast<const float4*>(p.qc) + static_cast<size_t>(u) * GP * p.C;
+  // chunk of local index c0 + tid, and the step to local index + T (both mod total)
+  const uint32_t nt = static_cast<uint32_t>(max(total, 1));   // parts exist only for units with chunks
+  const uint32_t step = static_cast<uint32_t>((static_cast<unsigned long long>(T) * stride) % nt);
+  uint32_t pc = static_cast<uint32_t>((static_cast<unsigned long long>(c0 + tid) * stride) % nt);
 
   __syncthreads();   // shared state of the previous part is no longer read
   if (tid == 0) {
     wait_count(&p.units[u].scan_done, total, p.err);   // every CTA of the unit has scanned
     ss.bstar = kNB;   // k == 0: nothing selected
     ss.above = 0;
-    ss.fix_n = 0;
   }
   __syncthreads();
   // one round trip: this thread's histogram bins, the first pass of chunk maxima, the bounds
@@ -716,10 +748,18 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
                           (kNB / 4 - 1 - tid));
   const float* cmax = p.chunk_max + static_cast<size_t>(u) * max_chunks;
   float cm[kCmPerThread];
+  int32_t cc[kCmPerThread];
+  auto next_chunk = [&]() {   // chunk of this thread's next local index, then advance
+    const int32_t c = static_cast<int32_t>(pc);
+    pc += step;
+    if (pc >= nt) pc -= nt;
+    return c;
+  };
 #pragma unroll
   for (int e = 0; e < kCmPerThread; ++e) {
-    const int c = c0 + tid + e * kScanThreads;
-    cm[e] = c < c1 ? __ldcg(cmax + c) : -INFINITY;
+    const int c = c0 + tid + e * T;
+    cc[e] = next_chunk();
+    cm[e] = c < c1 ? __ldcg(cmax + cc[e]) : -INFINITY;
   }
   float ub[G], lb[G];
 #pragma unroll
@@ -771,6 +811,10 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
     const uint16_t* ccl = p.chunk_cluster + static_cast<size_t>(u) * max_chunks;
     uint32_t* bm = p.bitmap + static_cast<size_t>(u) * p.bitmap_words;
     int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
+    unsigned long long* cand_u = p.cand + static_cast<size_t>(u) * p.cap;
+    int32_t* cand_row_u = p.cand_row + static_cast<size_t>(u) * p.cap;
+    // low word: candidates, high word: definite selections (neither count exceeds N < 2^31)
+    unsigned long long* counts = reinterpret_cast<unsigned long long*>(&p.units[u].ncand);
     const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
     const int h = u % p.Hkv;
     const int s0 = min(p.n_sink, max(0, p.seq_lens[b]));
@@ -779,8 +823,9 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
       if (cb != c0) {
 #pragma unroll
         for (int e = 0; e < kCmPerThread; ++e) {
-          const int c = cb + tid + e * kScanThreads;
-          cm[e] = c < c1 ? __ldcg(cmax + c) : -INFINITY;
+          const int c = cb + tid + e * T;
+          cc[e] = next_chunk();
+          cm[e] = c < c1 ? __ldcg(cmax + cc[e]) : -INFINITY;
         }
       }
       if (tid == 0) ss.n_act = 0;
@@ -788,7 +833,7 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
       // chunks whose maximum reaches the threshold bin, compacted warp by warp
 #pragma unroll
       for (int e = 0; e < kCmPerThread; ++e) {
-        const int c = cb + tid + e * kScanThreads;
+        const int c = cb + tid + e * T;
         const bool active = c < c1 && score_bin(cm[e], lo, inv) >= bstar;
         const uint32_t m = __ballot_sync(0xffffffffu, active);
         if (m) {
@@ -796,98 +841,96 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, const ui
           int at = 0;
           if (lane == leader) at = atomicAdd(&ss.n_act, __popc(m));
           at = __shfl_sync(0xffffffffu, at, leader);
-          if (active) act[at + __popc(m & ((1u << lane) - 1u))] = c;
+          if (active) act[at + __popc(m & ((1u << lane) - 1u))] = cc[e];
         }
       }
       __syncthreads();
       const int na = ss.n_act;
-      for (int a0 = 0; a0 < na; a0 += NW * kActPerWarp) {
-        // each warp reads up to kActPerWarp active chunks at once; lane = slot of the chunk
+      for (int a0 = warp * kActPerWarp; a0 < na; a0 += NW * kActPerWarp) {
+        // up to kActPerWarp active chunks of this warp, every load in one round trip;
+        // lane = slot of the chunk
         float sv[kActPerWarp];
         int32_t jv[kActPerWarp];
-        int chv[kActPerWarp];
+        uint4 cwv[kActPerWarp];
+        uint32_t idv[kActPerWarp];
 #pragma unroll
         for (int r = 0; r < kActPerWarp; ++r) {
-          const int a = a0 + warp + NW * r;
-          chv[r] = a < na ? act[a] : -1;
-          sv[r] = chv[r] >= 0 ? __ldcg(sig + static_cast<size_t>(chv[r]) * 32 + lane) : -INFINITY;
-          jv[r] = chv[r] >= 0 ? lslot[static_cast<size_t>(chv[r]) * 32 + lane] : -1;
+          const int ch = a0 + r < na ? act[a0 + r] : -1;
+          const size_t ls = static_cast<size_t>(max(ch, 0)) * 32 + lane;
+          sv[r] = ch >= 0 ? __ldcg(sig + ls) : -INFINITY;
+          jv[r] = ch >= 0 ? __ldg(lslot + ls) : -1;
+          cwv[r] = (ch >= 0 && fix) ? __ldg(lcodes + ls) : make_uint4(0u, 0u, 0u, 0u);
+          idv[r] = (ch >= 0 && fix) ? static_cast<uint32_t>(__ldg(ccl + ch)) : 0u;
         }
+        // classify both chunks, then one atomic per warp for all their selections and
+        // candidates; the block-table reads go out before the counts come back
+        bool defv[kActPerWarp], candv[kActPerWarp];
+        uint32_t dmv[kActPerWarp], cmv[kActPerWarp];
+        int32_t rowv[kActPerWarp];
+        uint32_t ndm = 0, ncm = 0;
 #pragma unroll
         for (int r = 0; r < kActPerWarp; ++r) {
           const int j = jv[r];            // index slot of this list slot
           const bool valid = j >= 0 && j < N;
           const int bin = valid ? score_bin(sv[r], lo, inv) : -1;
-          const bool definite = bin > bstar;
-          {   // a definite selection's KV-pool row joins the unit's rows (one atomic per warp)
-            const uint32_t dm = __ballot_sync(0xffffffffu, definite);
-            if (dm) {
-              const uint32_t leader = __ffs(dm) - 1;
-              int at = 0;
-              if (lane == leader) at = atomicAdd(&p.units[u].ndef, __popc(dm));
-              at = __shfl_sync(0xffffffffu, at, leader);
-              if (definite) {
-                const int o = at + __popc(dm & ((1u << lane) - 1u));
-                if (o < p.cap) sel_u[o] = kv_row(p, bt_row, h, s0 + j);
-                if (p.dbg_selected) atomicOr(bm + (j >> 5), 1u << (j & 31));   // for the ascending positions
-              }
-            }
-          }
-          int slot = -1;
-          const uint32_t cm_ = __ballot_sync(0xffffffffu, bin == bstar);
-          if (cm_) {   // one atomic per warp for its candidates
-            const uint32_t leader = __ffs(cm_) - 1;
-            int at = 0;
-            if (lane == leader) at = atomicAdd(&p.units[u].ncand, __popc(cm_));
-            at = __shfl_sync(0xffffffffu, at, leader);
-            if (bin == bstar) slot = at + __popc(cm_ & ((1u << lane) - 1u));
-          }
-          if (bin == bstar && slot < p.cap) {
-            p.cand[static_cast<size_t>(u) * p.cap + slot] =
-                (static_cast<unsigned long long>(float_key(sv[r])) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
-            p.cand_row[static_cast<size_t>(u) * p.cap + slot] = kv_row(p, bt_row, h, s0 + j);
-          }
-          if (fix) {
-            // queue the list slot: a definite selection's weight leaves its cluster's sums
-            // below; a candidate's weights are stored for the resolution's winners
-            const bool queued = definite || (slot >= 0 && slot < kCandWeights);
-            const uint32_t m = __ballot_sync(0xffffffffu, queued);
-            if (m) {
-              const uint32_t leader = __ffs(m) - 1;
-              uint32_t at = 0;
-              if (lane == leader) at = atomicAdd(&ss.fix_n, static_cast<uint32_t>(__popc(m)));
-              at = __shfl_sync(0xffffffffu, at, leader);
-              if (queued) {
-                at += __popc(m & ((1u << lane) - 1u));
-                fix_list[at] = static_cast<uint32_t>(chv[r]) * 32 + lane;
-                fix_cand[at] = definite ? -1 : slot;
-              }
-            }
-          }
+          defv[r] = bin > bstar;
+          candv[r] = bin == bstar;
+          dmv[r] = __ballot_sync(0xffffffffu, defv[r]);
+          cmv[r] = __ballot_sync(0xffffffffu, candv[r]);
+          rowv[r] = (defv[r] || candv[r]) ? kv_row(p, bt_row, h, s0 + j) : 0;
+          ndm += __popc(dmv[r]);
+          ncm += __popc(cmv[r]);
         }
-        if (fix) {
-          // queued tokens of this round: one per thread, every look-up of a token in flight together
-          __syncthreads();
-          const uint32_t n = ss.fix_n;
-          for (uint32_t i = tid; i < n; i += kScanThreads) {
-            const uint32_t ls = fix_list[i];
-            const int cs = fix_cand[i];
-            uint32_t id = ccl[ls >> 5];
+        if ((ndm | ncm) == 0u) continue;   // warp-uniform
+        unsigned long long old = 0ull;
+        if (lane == 0) old = atomicAdd(counts, (static_cast<unsigned long long>(ndm) << 32) | ncm);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        uint32_t dbase = static_cast<uint32_t>(old >> 32), cbase = static_cast<uint32_t>(old & 0xffffffffull);
+        const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+        for (int r = 0; r < kActPerWarp; ++r) {
+          const int j = jv[r];
+          int slot = -1;
+          if (defv[r]) {
+            const uint32_t o = dbase + __popc(dmv[r] & below);
+            if (o < static_cast<uint32_t>(p.cap)) sel_u[o] = rowv[r];
+            if (p.dbg_selected) atomicOr(bm + (j >> 5), 1u << (j & 31));   // for the ascending positions
+          } else if (candv[r]) {
+            slot = static_cast<int>(cbase + __popc(cmv[r] & below));
+            if (slot < p.cap) {
+              cand_u[slot] = (static_cast<unsigned long long>(float_key(sv[r])) << 32) |
+                             (0xffffffffu - static_cast<uint32_t>(j));
+              cand_row_u[slot] = rowv[r];
+            }
+          }
+          dbase += __popc(dmv[r]);
+          cbase += __popc(cmv[r]);
+          // the definite selections' weights leave their cluster's sums (a chunk holds one
+          // cluster: the warp adds them up and sends one atomic per head); a candidate's
+          // weights are stored for the resolution's winners
+          const bool keep = candv[r] && slot >= 0 && slot < kCandWeights;
+          if (fix && (dmv[r] != 0u || __any_sync(0xffffffffu, keep))) {   // warp-uniform
+            uint32_t id = idv[r];
             if (id >= static_cast<uint32_t>(p.C)) id = 0;
             float e[G];
-            token_weights<G>(lut4, qc4, p.C, id, lcodes[ls], ub2, e);
-            if (cs < 0) {
-              remove_weights<G>(p, u, id, e);
-            } else {
-              float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + cs) * G;
+#pragma unroll
+            for (int g = 0; g < G; ++g) e[g] = 0.f;
+            // only the lanes that need them look their weights up (the look-ups of one
+            // subspace by many lanes would share a bank group)
+            if (defv[r] || keep) token_weights<G>(lut4, qc4, p.C, id, cwv[r], ub2, e);
+            if (keep) {
+              float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + slot) * G;
 #pragma unroll
               for (int g = 0; g < G; ++g) cw[g] = e[g];
-              p.cand_c[static_cast<size_t>(u) * kCandWeights + cs] = static_cast<int32_t>(id);
+              p.cand_c[static_cast<size_t>(u) * kCandWeights + slot] = static_cast<int32_t>(id);
+            }
+            if (dmv[r] != 0u) {
+              float neg[G];
+#pragma unroll
+              for (int g = 0; g < G; ++g) neg[g] = defv[r] ? -e[g] : 0.f;   // candidates add nothing
+              flush_weights<G>(neg, p.W + static_cast<size_t>(u) * G * p.C, p.C, id);
             }
           }
-          __syncthreads();
-          if (tid == 0) ss.fix_n = 0;
-          __syncthreads();
         }
       }
       __syncthreads();   // this pass is done with act[] and n_act
@@ -953,9 +996,7 @@ __device__ void resolve_unit(const StepParams& p, int u, uint8_t* fsm, SelShared
   uint32_t* woff = bmc + kFinChunkWords;                                  // [kFinChunkWords]
   uint32_t* dig = woff + kFinChunkWords;                                  // [256]
   const int b = u / p.Hkv;
-  const int h = u % p.Hkv;
   const int tid = threadIdx.x;
-  const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
   const unsigned long long* cg = p.cand + static_cast<size_t>(u) * p.cap;
   int32_t* sel_u = p.sel + static_cast<size_t>(u) * p.cap;
   const int T_len = max(0, p.seq_lens[b]);
@@ -1219,6 +1260,7 @@ __device__ void plan_parts(const StepParams& p, SelShared& ss) {
         ss.pu[at] = u;
         ss.pc0[at] = i0;
         ss.pc1[at] = i1;
+        ss.pst[at] = scatter_stride(static_cast<uint32_t>(n));
       }
     }
     run += pass_tot;
@@ -1233,6 +1275,7 @@ __device__ void plan_parts(const StepParams& p, SelShared& ss) {
           int t = ss.pu[j]; ss.pu[j] = ss.pu[j - 1]; ss.pu[j - 1] = t;
           t = ss.pc0[j]; ss.pc0[j] = ss.pc0[j - 1]; ss.pc0[j - 1] = t;
           t = ss.pc1[j]; ss.pc1[j] = ss.pc1[j - 1]; ss.pc1[j - 1] = t;
+          const uint32_t st = ss.pst[j]; ss.pst[j] = ss.pst[j - 1]; ss.pst[j - 1] = st;
         }
     }
   }
@@ -1308,8 +1351,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_select_kernel(StepParams
   // ---- phase 2: selection per unit; phase 3: the part that completes a unit's filter
   // resolves it, after all of this CTA's filter parts (no unit's filter waits behind it) ----
   int nres = 0;
-  auto filt = [&](int u, int c0, int c1) {
-    if (filter_part<G>(p, u, c0, c1, tables_unit == u ? smem : nullptr, smem, ss)) {
+  auto filt = [&](int u, int c0, int c1, uint32_t stride) {
+    if (filter_part<G>(p, u, c0, c1, stride, tables_unit == u ? smem : nullptr, smem, ss)) {
       if (nres < kMaxParts) {
         if (threadIdx.x == 0) ss.res[nres] = u;
         ++nres;
@@ -1321,9 +1364,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_select_kernel(StepParams
     }
   };
   if (nparts >= 0) {
-    for (int i = 0; i < nparts; ++i) filt(ss.pu[i], ss.pc0[i], ss.pc1[i]);
+    for (int i = 0; i < nparts; ++i) filt(ss.pu[i], ss.pc0[i], ss.pc1[i], ss.pst[i]);
   } else {
-    walk_parts(p, total, filt);
+    walk_parts(p, total, [&](int u, int c0, int c1) {
+      filt(u, c0, c1, scatter_stride(static_cast<uint32_t>(unit_chunks(p, u))));
+    });
   }
   if (nres > 0) {
     __threadfence();   // acquire: the unit's other parts published before counting in
