@@ -22,7 +22,8 @@ __all__ = [
     "PagedKV", "PQIndex", "HSAError", "load_library", "hsa_decode", "dense_decode",
     "hsa_build_from_codes", "hsa_append_encode", "hsa_decode_workspace_bytes",
     "dense_decode_workspace_bytes", "hsa_index_workspace_bytes", "hsa_read_error", "hsa_strerror",
-    "selected_counts", "HSA_DEVERR_PAGE", "HSA_DEVERR_CLUSTER", "HSA_DEVERR_TIMEOUT", "HSA_DEVERR_SELECT",
+    "selected_counts", "DecodeStep", "HSA_DEVERR_PAGE", "HSA_DEVERR_CLUSTER", "HSA_DEVERR_TIMEOUT",
+    "HSA_DEVERR_SELECT",
 ]
 
 HSA_DEVERR_PAGE, HSA_DEVERR_CLUSTER, HSA_DEVERR_TIMEOUT, HSA_DEVERR_SELECT = 1, 2, 4, 8
@@ -300,6 +301,47 @@ def hsa_decode(kv: PagedKV, index: PQIndex, q: torch.Tensor, out: Optional[torch
                         ctypes.byref(dbg), workspace_buf.data_ptr(), workspace_buf.numel(), _stream(stream))
     _check("hsa_decode", st)
     return out
+
+
+class DecodeStep:
+    """hsa_decode prepared for one cache, index and workspace, for a decode loop: the C-ABI
+    views of the cache and the index, the parameters and the workspace are checked and
+    marshalled once here, and each call passes only q, out and the stream (the library still
+    validates every call, lengths included). The tensors must keep their storage while the
+    step is in use; their contents (lengths, appended tokens, lists) may change between calls.
+    """
+
+    def __init__(self, kv: PagedKV, index: PQIndex, *, scale: float, budget: float = 0.01, k_override: int = -1,
+                 background: bool = True, workspace_buf: Optional[torch.Tensor] = None):
+        self.kv, self.index = kv, index          # keep the tensors behind the views alive
+        self._kvs, self._ixs = kv.struct(), index.struct()
+        if workspace_buf is None:
+            workspace_buf = workspace(hsa_decode_workspace_bytes(kv, index), kv.k_cache.device)
+        _on_gpu(workspace_buf)
+        self.workspace_buf = workspace_buf
+        self._prm = _Params(float(scale), float(budget), int(k_override), 1 if background else 0)
+        self._shape = (kv.B, kv.Hq, kv.k_cache.shape[3])
+        self._device = kv.k_cache.device
+        self._fn = load_library().hsa_decode
+        self._kv_ref, self._ix_ref = ctypes.byref(self._kvs), ctypes.byref(self._ixs)
+        self._prm_ref = ctypes.byref(self._prm)
+        self._ws_ptr, self._ws_len = workspace_buf.data_ptr(), workspace_buf.numel()
+
+    def _check_io(self, t: torch.Tensor, name: str) -> None:
+        if (t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != self._shape
+                or t.device != self._device):
+            raise ValueError(f"{name}: expected a contiguous fp32 tensor {list(self._shape)} on {self._device}")
+
+    def __call__(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        self._check_io(q, "q")
+        if out is None:
+            out = torch.empty_like(q)
+        else:
+            self._check_io(out, "out")
+        st = self._fn(self._kv_ref, self._ix_ref, q.data_ptr(), out.data_ptr(), self._prm_ref, None, self._ws_ptr,
+                      self._ws_len, _stream(stream))
+        _check("hsa_decode", st)
+        return out
 
 
 def selected_counts(kv: PagedKV, index: PQIndex, q: torch.Tensor, *, scale: float, budget: float = 0.01,

@@ -217,6 +217,8 @@ def test_binding_rejects_host_tensors_for_device_arrays():
     ix = P.PQIndex.allocate(B, Hkv, 4, 32, 4, "cpu")
     with pytest.raises(ValueError):
         ix.struct()
+    with pytest.raises(ValueError):     # the prepared step marshals the same views, once
+        P.DecodeStep(kv, ix, scale=0.1)
 
 
 def test_static_dense_decode_validates_like_dense_decode(host_only):

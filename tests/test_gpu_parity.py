@@ -158,3 +158,28 @@ def test_no_index_and_no_sink(cuda_device):
                                             n_indexed=np.array([0, 1500]), n_sink=0)
     res = _run_hsa(w, bt, codes, ids, kv, ix, dev, budget=0.02)
     _check_all(w, bt, res, ids=ids)
+
+
+def test_prepared_step_matches_hsa_decode(cuda_device):
+    """DecodeStep (the cache and index views marshalled once) gives hsa_decode's output, and
+    still does after the lengths change in place behind its views. Two decode calls agree to
+    rounding, not bit for bit: the cluster-weight sums are fp32 atomics in arrival order."""
+    w, bt, codes, ids, kv, ix, dev = _setup(CASES["qwen_g8_8k"])
+    ws_idx = P.workspace(P.hsa_index_workspace_bytes(kv, ix), dev)
+    P.hsa_build_from_codes(kv, ix, workspace_buf=ws_idx)
+    scale = scale_for(w.D)
+    q = torch.from_numpy(bt.q).to(dev)
+    step = P.DecodeStep(kv, ix, scale=scale, budget=w.budget)
+    for _ in range(2):
+        ref = P.hsa_decode(kv, ix, q, scale=scale, budget=w.budget)
+        got = step(q)
+        out = torch.full_like(q, float("nan"))
+        assert step(q, out) is out
+        torch.cuda.synchronize()
+        tol = 1e-6 * float(ref.abs().max()) + 1e-7
+        assert float((got - ref).abs().max()) <= tol and float((out - ref).abs().max()) <= tol
+        assert P.hsa_read_error(step.workspace_buf) == 0
+        kv.seq_lens.sub_(100)                  # a shorter tail, same storage
+        kv.seq_lens_host.sub_(100)
+    with pytest.raises(ValueError):
+        step(q[:, :1].contiguous())
