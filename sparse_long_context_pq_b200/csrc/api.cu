@@ -257,9 +257,9 @@ hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, floa
   if (!dev) return HSA_ERR_CUDA;
   long long Tmax = 0;
   for (int b = 0; b < kv->B; ++b) Tmax = std::max<long long>(Tmax, kv->seq_lens_host[b]);
-  const Split sp = plan_splits(Tmax, U, 0, dev->sms * attend_slots_per_sm());
   // Page tiles by tensor TMA need boxes of >= 8 rows (1024-byte aligned in shared memory).
   const bool rows = kv->page_size < 8;
+  const Split sp = plan_splits(Tmax, U, 0, dev->sms * attend_slots_per_sm(G, false, rows));
   CUtensorMap tk = {}, tv = {};
   const int box_rows = std::min(kv->page_size, kTile);
   if (!rows && (!make_kv_tmap(&tk, kv->k_cache, kv, box_rows) || !make_kv_tmap(&tv, kv->v_cache, kv, box_rows)))
@@ -295,7 +295,7 @@ hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, floa
   p.S_tot = sp.nsplit;
   p.qscale = scale * kLog2e;
   p.k_override = -1;
-  RET_CUDA(launch_attend(G, false, rows, tk, tv, p, U * sp.nsplit, stream, use_pdl()));
+  RET_CUDA(launch_attend(G, false, rows, tk, tv, p, U * sp.nsplit, false, stream, use_pdl()));
   MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, sp.nsplit};
   RET_CUDA(launch_merge(G, mp, stream, use_pdl()));
   return HSA_OK;
@@ -328,7 +328,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
     const int k = decode_k(prm->budget, prm->k_override, N);
     Emax = std::max<long long>(Emax, static_cast<long long>(s0) + k + (T - s0 - N));
   }
-  const Split sp = plan_splits(Emax, U, L.nbg, dev->sms * attend_slots_per_sm());
+  const Split sp = plan_splits(Emax, U, L.nbg, dev->sms * attend_slots_per_sm(G, true, true));
   CUtensorMap tk = {}, tv = {};   // unused: gathered rows are copied by the producer lanes
   cudaEvent_t* ev = dbg ? dbg->stage_events : nullptr;
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], stream) : cudaSuccess; };
@@ -462,7 +462,8 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   p.budget = prm->budget;
   p.qscale = prm->scale * kLog2e;
   RET_CUDA(mark(2));
-  RET_CUDA(launch_attend(G, true, true, tk, tv, p, U * (sp.nsplit + L.nbg), stream, use_pdl()));
+  const int attend_grid = U * (sp.nsplit + L.nbg);
+  RET_CUDA(launch_attend(G, true, true, tk, tv, p, attend_grid, attend_grid > 2 * dev->sms, stream, use_pdl()));
   MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, S_tot};
   RET_CUDA(mark(3));
   RET_CUDA(launch_merge(G, mp, stream, use_pdl()));

@@ -57,7 +57,9 @@ struct AttendSmem {
   static constexpr size_t qs = kD * GP * 16;
   static constexpr size_t pbuf = Pipe<kRows>::CW * 2 * 8 * kTile * 2;   // P hi/lo bf16 [8 heads][32 tokens]
   static constexpr size_t bars = 2 * Pipe<kRows>::S * 8;
-  static constexpr size_t total = 1024 /*alignment slack*/ + stages + qs + pbuf + bars + 64;
+  // swizzled TMA boxes need 1024-byte aligned stages; gathered rows only 16-byte ones
+  static constexpr size_t align = kRows ? 128 : 1024;
+  static constexpr size_t total = align /*alignment slack*/ + stages + qs + pbuf + bars + 64;
 };
 
 // Byte offset of 16-byte chunk c (0..15) of row r inside the K (or V) area of a stage.
@@ -76,8 +78,11 @@ __device__ __forceinline__ uint32_t v_area() { return kRows ? kTile * kRowPitch 
 // selection hands over its k tokens as KV-pool rows (in no particular order).
 __device__ __forceinline__ int exact_tail_pos(int v, int s0, int N) { return v < s0 ? v : s0 + N + (v - s0); }
 
-template <int G, bool kExact, bool kRows>
-__global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
+// kMinB resident CTAs per SM: 2, or 3 for the exact part of G <= 4 when its grid holds more
+// CTAs than two per SM (128 registers and 76 KB of shared memory each: more gathered rows in
+// flight; with at most two CTAs per SM the wider register budget is faster).
+template <int G, bool kExact, bool kRows, int kMinB>
+__global__ void __launch_bounds__(Pipe<kRows>::threads, kMinB)
     attend_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                   AttendParams p) {
   static_assert(kRows || !kExact, "gathered rows use bulk row copies");
@@ -86,7 +91,8 @@ __global__ void __launch_bounds__(Pipe<kRows>::threads, 2)
   constexpr int kStageBytes = Pipe<kRows>::stage_bytes;
   constexpr int GP = (G + 3) / 4;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uintptr_t kAlign = AttendSmem<G, kRows>::align;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + kAlign - 1) & ~(kAlign - 1));
   uint8_t* stage_base = smem;
   float4* qs = reinterpret_cast<float4*>(smem + AttendSmem<G, kRows>::stages);               // [kD][GP]
   uint8_t* pbuf = reinterpret_cast<uint8_t*>(qs + kD * GP);                            // [warps] P buffers
@@ -638,12 +644,13 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams p) {
   }
 }
 
-template <int G, bool kExact, bool kRows>
+template <int G, bool kExact, bool kRows, int kMinB = 2>
 cudaError_t launch_attend_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttendParams& p, int grid,
                             cudaStream_t stream, bool pdl) {
-  auto kern = attend_kernel<G, kExact, kRows>;
+  static_assert(kMinB == 2 || (kMinB == 3 && kExact && G <= 4), "three CTAs per SM only fit the exact G <= 4 part");
+  auto kern = attend_kernel<G, kExact, kRows, kMinB>;
   const size_t smem = AttendSmem<G, kRows>::total;
-  cudaError_t e = ensure_dyn_smem<attend_kernel<G, kExact, kRows>>(smem);
+  cudaError_t e = ensure_dyn_smem<attend_kernel<G, kExact, kRows, kMinB>>(smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -675,22 +682,30 @@ cudaError_t launch_merge_t(const MergeParams& p, cudaStream_t stream, bool pdl) 
 
 }  // namespace
 
-int attend_slots_per_sm() { return 2; }
-size_t attend_smem_bytes(int G) {
-  switch (G) {
-    case 1: return AttendSmem<1, true>::total;
-    case 2: return AttendSmem<2, true>::total;
-    case 4: return AttendSmem<4, true>::total;
-    default: return AttendSmem<8, true>::total;
+// CTAs per SM the split planner sizes its waves with (measured on B200, L2 flushed before
+// every step): for G <= 4 two, as for dense decode (counting a third resident CTA gave more,
+// shorter splits that were slower at 128K); for G = 8, which holds two, three (finer splits
+// of each unit's rows were about 4 % faster per step at the Qwen shape).
+int attend_slots_per_sm(int G, bool exact, bool rows) {
+  (void)rows;
+  return (exact && G >= 8) ? 3 : 2;
+}
+
+template <int G>
+cudaError_t launch_exact_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttendParams& p, int grid,
+                           bool wide, cudaStream_t stream, bool pdl) {
+  if constexpr (G <= 4) {
+    if (wide) return launch_attend_t<G, true, true, 3>(tk, tv, p, grid, stream, pdl);
   }
+  return launch_attend_t<G, true, true, 2>(tk, tv, p, grid, stream, pdl);
 }
 
 cudaError_t launch_attend(int G, bool exact, bool rows, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const AttendParams& p, int grid, cudaStream_t stream, bool pdl) {
-#define PQHSA_ATT(GG)                                                                  \
-  case GG:                                                                             \
-    if (exact) return launch_attend_t<GG, true, true>(tk, tv, p, grid, stream, pdl);   \
-    if (rows) return launch_attend_t<GG, false, true>(tk, tv, p, grid, stream, pdl);   \
+                          const AttendParams& p, int grid, bool wide, cudaStream_t stream, bool pdl) {
+#define PQHSA_ATT(GG)                                                                   \
+  case GG:                                                                              \
+    if (exact) return launch_exact_t<GG>(tk, tv, p, grid, wide, stream, pdl);           \
+    if (rows) return launch_attend_t<GG, false, true>(tk, tv, p, grid, stream, pdl);    \
     return launch_attend_t<GG, false, false>(tk, tv, p, grid, stream, pdl);
   switch (G) {
     PQHSA_ATT(1)

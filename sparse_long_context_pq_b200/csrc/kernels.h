@@ -96,12 +96,12 @@ hsa_status check_kv(const hsa_kv_cache* kv);   // shapes, alignment and lengths 
 // Tensor map over a paged cache viewed as rows of D bf16, box = 64 columns x box_rows rows.
 bool make_kv_tmap(CUtensorMap* map, const void* base, const hsa_kv_cache* kv, int box_rows);
 
-int attend_slots_per_sm();
-size_t attend_smem_bytes(int G);
+int attend_slots_per_sm(int G, bool exact, bool rows);   // resident attend CTAs per SM
 // Row sources: kExact = sink + selected + tail list of hsa_decode, else every token.
 // Loading: page tiles by tensor TMA (dense, page_size >= 8) or 16-byte async copies per row.
+// wide: the grid holds more CTAs than two per SM (the exact part of G <= 4 then runs three).
 cudaError_t launch_attend(int G, bool exact, bool rows, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const AttendParams& p, int grid, cudaStream_t stream, bool pdl);
+                          const AttendParams& p, int grid, bool wide, cudaStream_t stream, bool pdl);
 cudaError_t launch_merge(int G, const MergeParams& p, cudaStream_t stream, bool pdl);
 
 // ---- PQ tables, scan, top-k ------------------------------------------------

@@ -666,6 +666,41 @@ __device__ __forceinline__ void token_weights(const float4* lut4, const float4* 
   }
 }
 
+// token_weights for many lanes at once (the filter's selections): lane l visits subspace
+// s = i ^ (l & 7) at step i, so the 8 lanes of a quarter-warp read 8 different 16-byte bank
+// groups of the shared-memory tables instead of one (same sums up to rounding order).
+template <int G>
+__device__ __forceinline__ void token_weights_skewed(const float4* lut4, const float4* qc4, int C, uint32_t id,
+                                                     const uint4 cw, const float* ub2, float* e) {
+  constexpr int GP = (G + 3) / 4;
+  const uint32_t l7 = threadIdx.x & 7;
+  const uint32_t wlo[2] = {(l7 & 4) ? cw.y : cw.x, (l7 & 4) ? cw.x : cw.y};   // words i>>2 = 0, 1 after the skew
+  const uint32_t whi[2] = {(l7 & 4) ? cw.w : cw.z, (l7 & 4) ? cw.z : cw.w};   // words i>>2 = 2, 3
+  float4 acc[GP];
+#pragma unroll
+  for (int gp = 0; gp < GP; ++gp) acc[gp] = qc4[gp * C + id];
+#pragma unroll
+  for (int i = 0; i < kM; ++i) {
+    const uint32_t s = static_cast<uint32_t>(i) ^ l7;
+    const uint32_t wd = (i < 4) ? wlo[0] : (i < 8) ? wlo[1] : (i < 12) ? whi[0] : whi[1];
+    const uint32_t code = (wd >> (8u * (s & 3u))) & 255u;
+#pragma unroll
+    for (int gp = 0; gp < GP; ++gp) {
+      const float4 v = lut4[(gp * kNcode + code) * kM + s];
+      acc[gp].x = __fadd_rn(acc[gp].x, v.x);
+      acc[gp].y = __fadd_rn(acc[gp].y, v.y);
+      acc[gp].z = __fadd_rn(acc[gp].z, v.z);
+      acc[gp].w = __fadd_rn(acc[gp].w, v.w);
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float4 a = acc[g / 4];
+    const float sh = (g % 4 == 0) ? a.x : (g % 4 == 1) ? a.y : (g % 4 == 2) ? a.z : a.w;
+    e[g] = fast_exp2(fmaf(sh, kLog2e, -ub2[g]));
+  }
+}
+
 // Take a selected token's head weights out of its cluster's sums.
 template <int G>
 __device__ __forceinline__ void remove_weights(const StepParams& p, int u, uint32_t id, const float* e) {
@@ -915,9 +950,8 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
             float e[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) e[g] = 0.f;
-            // only the lanes that need them look their weights up (the look-ups of one
-            // subspace by many lanes would share a bank group)
-            if (defv[r] || keep) token_weights<G>(lut4, qc4, p.C, id, cwv[r], ub2, e);
+            // only the lanes that need them look their weights up
+            if (defv[r] || keep) token_weights_skewed<G>(lut4, qc4, p.C, id, cwv[r], ub2, e);
             if (keep) {
               float* cw = p.cand_w + (static_cast<size_t>(u) * kCandWeights + slot) * G;
 #pragma unroll

@@ -128,7 +128,7 @@ extern "C" hsa_status dense_decode_static(const hsa_kv_cache* kv, const float* q
   p.S_tot = ns;
   p.qscale = scale * kLog2e;
   p.k_override = -1;
-  if (launch_attend(G, false, rows, tk, tv, p, U * ns, stream, false) != cudaSuccess) return HSA_ERR_CUDA;
+  if (launch_attend(G, false, rows, tk, tv, p, U * ns, false, stream, false) != cudaSuccess) return HSA_ERR_CUDA;
   MergeParams mp = {pm, pl, pacc, out, kv->B, kv->Hq, kv->Hkv, ns};
   if (launch_merge(G, mp, stream, false) != cudaSuccess) return HSA_ERR_CUDA;
   return HSA_OK;
