@@ -35,10 +35,32 @@ __device__ __forceinline__ int unit_n(const int32_t* seq_lens, const int32_t* n_
 }
 
 
-__device__ __forceinline__ float warp_min(float v) {
+// Warp sum of G per-lane values, scattered: after log2(G) halving exchanges each lane
+// holds a partial of one value, then plain butterflies finish it. Returns the total of
+// value (lane >> (5 - log2 G)) in every lane of that group (lane (32/G)*g holds head g).
+template <int G>
+__device__ __forceinline__ float warp_sum_scatter(float* v) {
+  const int lane = threadIdx.x & 31;
+  int n = G;
+  int o = 16;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+  for (int step = 0; (1 << step) < G; ++step) {
+    const bool up = (lane & o) != 0;
+    const int half = n >> 1;
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) {
+      if (i < half) {
+        const float send = up ? v[i] : v[i + half];
+        const float keep = up ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    n = half;
+    o >>= 1;
+  }
+  float t = v[0];
+  for (; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  return t;
 }
 
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
@@ -147,8 +169,8 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
       }
 #pragma unroll
       for (int g = 0; g < G4; ++g) {
-        const float a = warp_max(val[g]);
-        const float c = warp_min(val[g]);
+        const float a = warp_max_f32(val[g]);
+        const float c = warp_min_f32(val[g]);
         if (lane == 0) {
           wred[0][warp][i][g] = a;
           wred[1][warp][i][g] = c;
@@ -184,12 +206,11 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
         p.W[(static_cast<size_t>(u) * G + i / nc) * p.C + cs + (i % nc)] = 0.f;
     }
     __syncthreads();
-    float mx[G4], mn[G4];
-#pragma unroll
-    for (int g = 0; g < G4; ++g) {
-      mx[g] = -INFINITY;
-      mn[g] = INFINITY;
-    }
+    // The G4 dot products of a cluster are reduced together (scattered halving): head g's
+    // total ends in the lanes of group g = lane / (32 / G4), which keep its extremes.
+    constexpr int kGroup = 32 / G4;
+    const int hg = lane / kGroup;
+    float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
     for (int i = 0; i < kQcPerWarp; ++i) {
       const int c = c0 + i;
@@ -200,29 +221,21 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
         v = fmaf(qsh[g][lane * 4 + 1], cv[i].y, v);
         v = fmaf(qsh[g][lane * 4 + 2], cv[i].z, v);
         v = fmaf(qsh[g][lane * 4 + 3], cv[i].w, v);
-        val[g] = warp_sum(v);
+        val[g] = v;
       }
+      const float tot = warp_sum_scatter<G4>(val);
       if (c < p.C) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          mx[g] = fmaxf(mx[g], val[g]);
-          mn[g] = fminf(mn[g], val[g]);
+        if (hg < G) {
+          mx = fmaxf(mx, tot);
+          mn = fminf(mn, tot);
         }
-#pragma unroll
-        for (int gp = 0; gp < GP; ++gp) {
-          if (lane == gp) {
-            float4* dst = reinterpret_cast<float4*>(p.qc) + (static_cast<size_t>(u) * GP + gp) * p.C + c;
-            *dst = make_float4(val[gp * 4 + 0], val[gp * 4 + 1], val[gp * 4 + 2], val[gp * 4 + 3]);
-          }
-        }
+        if ((lane & (kGroup - 1)) == 0)   // component hg % 4 of float4 [hg / 4][c]
+          reinterpret_cast<float*>(p.qc)[((static_cast<size_t>(u) * GP + hg / 4) * p.C + c) * 4 + (hg % 4)] = tot;
       }
     }
-    if (lane == 0) {
-#pragma unroll
-      for (int g = 0; g < G4; ++g) {
-        wred[0][warp][0][g] = mx[g];
-        wred[1][warp][0][g] = mn[g];
-      }
+    if ((lane & (kGroup - 1)) == 0) {
+      wred[0][warp][0][hg] = mx;
+      wred[1][warp][0][hg] = mn;
     }
     __syncthreads();
     if (tid < 2 * G4) {
@@ -383,34 +396,6 @@ __device__ __forceinline__ void score_token(const uint4& code, uint32_t id, cons
     if (gp * 4 + 2 < G) sh[gp * 4 + 2] = lo_f(zw);
     if (gp * 4 + 3 < G) sh[gp * 4 + 3] = hi_f(zw);
   }
-}
-
-// Warp sum of G per-lane values, scattered: after log2(G) halving exchanges each lane
-// holds a partial of one value, then plain butterflies finish it. Returns the total of
-// value (lane >> (5 - log2 G)) in every lane of that group (lane (32/G)*g holds head g).
-template <int G>
-__device__ __forceinline__ float warp_sum_scatter(float* v) {
-  const int lane = threadIdx.x & 31;
-  int n = G;
-  int o = 16;
-#pragma unroll
-  for (int step = 0; (1 << step) < G; ++step) {
-    const bool up = (lane & o) != 0;
-    const int half = n >> 1;
-#pragma unroll
-    for (int i = 0; i < G / 2; ++i) {
-      if (i < half) {
-        const float send = up ? v[i] : v[i + half];
-        const float keep = up ? v[i + half] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
-    n = half;
-    o >>= 1;
-  }
-  float t = v[0];
-  for (; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-  return t;
 }
 
 // Add the warp's per-lane weight sums of one cluster run to the cluster's sums.
