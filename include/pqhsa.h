@@ -145,6 +145,26 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* index, const floa
                       const hsa_decode_params* params, const hsa_debug* debug,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Workspace bytes hsa_decode_host needs: hsa_decode's (first, 256-byte aligned), then
+   device room for q and for out (fp32 [B][Hq][D] each, 256-byte aligned). 0 on invalid
+   arguments. */
+size_t hsa_decode_host_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* index);
+
+/*
+ * hsa_decode with q and out in host memory, for callers whose query and result live
+ * on the host. On `stream`: q_host is copied into the workspace, the decode step runs
+ * (as hsa_decode, without debug outputs), and the result is copied to out_host, one
+ * cudaMemcpyAsync each way (page-locked host buffers keep both copies asynchronous).
+ * q_host, out_host: fp32 [B][Hq][D] host memory, caller-owned. Returns once all of it
+ * is queued; out_host holds the result when `stream` reaches the end of this call
+ * (synchronise the stream or an event recorded after it before reading). Arguments
+ * are checked before anything is queued; status, workspace and error word otherwise
+ * as for hsa_decode.
+ */
+hsa_status hsa_decode_host(const hsa_kv_cache* kv, const hsa_index* index, const float* q_host, float* out_host,
+                           const hsa_decode_params* params, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
 /* Workspace bytes dense_decode needs. */
 size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv);
 

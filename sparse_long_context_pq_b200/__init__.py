@@ -19,8 +19,8 @@ import torch
 from . import build as _build
 
 __all__ = [
-    "PagedKV", "PQIndex", "HSAError", "load_library", "hsa_decode", "dense_decode",
-    "hsa_build_from_codes", "hsa_append_encode", "hsa_decode_workspace_bytes",
+    "PagedKV", "PQIndex", "HSAError", "load_library", "hsa_decode", "hsa_decode_host", "dense_decode",
+    "hsa_build_from_codes", "hsa_append_encode", "hsa_decode_workspace_bytes", "hsa_decode_host_workspace_bytes",
     "dense_decode_workspace_bytes", "hsa_index_workspace_bytes", "hsa_read_error", "hsa_strerror",
     "selected_counts", "DecodeStep", "HSA_DEVERR_PAGE", "HSA_DEVERR_CLUSTER", "HSA_DEVERR_TIMEOUT",
     "HSA_DEVERR_SELECT",
@@ -69,8 +69,9 @@ NUM_STAGES = 4
 STAGE_NAMES = ("tables", "scan_select", "attend", "merge")
 
 
-EXPORTS = ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode", "hsa_index_list_slots",
-           "hsa_decode_workspace_bytes", "dense_decode_workspace_bytes", "hsa_index_workspace_bytes",
+EXPORTS = ("hsa_decode", "hsa_decode_host", "dense_decode", "hsa_build_from_codes", "hsa_append_encode",
+           "hsa_index_list_slots", "hsa_decode_workspace_bytes", "hsa_decode_host_workspace_bytes",
+           "dense_decode_workspace_bytes", "hsa_index_workspace_bytes",
            "hsa_read_error", "hsa_strerror", "hsa_abi_sizes")
 
 _lib = None
@@ -95,6 +96,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     P = ctypes.POINTER
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     lib.hsa_decode.argtypes = [P(_KV), P(_Index), vp, vp, P(_Params), P(_Debug), vp, sz, vp]
+    lib.hsa_decode_host.argtypes = [P(_KV), P(_Index), vp, vp, P(_Params), vp, sz, vp]
+    lib.hsa_decode_host_workspace_bytes.argtypes = [P(_KV), P(_Index)]
     lib.dense_decode.argtypes = [P(_KV), vp, vp, ctypes.c_float, vp, sz, vp]
     lib.hsa_build_from_codes.argtypes = [P(_KV), P(_Index), vp, sz, vp]
     lib.hsa_append_encode.argtypes = [P(_KV), P(_Index), i32, vp, sz, vp]
@@ -106,11 +109,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.hsa_read_error.argtypes = [vp, P(i32), vp]
     lib.hsa_strerror.argtypes = [ctypes.c_int]
     lib.hsa_abi_sizes.argtypes = [P(ctypes.c_int64)] * 4
-    for f in ("hsa_decode", "dense_decode", "hsa_build_from_codes", "hsa_append_encode", "hsa_read_error",
-              "hsa_train_index"):
+    for f in ("hsa_decode", "hsa_decode_host", "dense_decode", "hsa_build_from_codes", "hsa_append_encode",
+              "hsa_read_error", "hsa_train_index"):
         getattr(lib, f).restype = ctypes.c_int
-    for f in ("hsa_decode_workspace_bytes", "dense_decode_workspace_bytes", "hsa_index_workspace_bytes",
-              "hsa_train_workspace_bytes"):
+    for f in ("hsa_decode_workspace_bytes", "hsa_decode_host_workspace_bytes", "dense_decode_workspace_bytes",
+              "hsa_index_workspace_bytes", "hsa_train_workspace_bytes"):
         getattr(lib, f).restype = sz
     lib.hsa_strerror.restype = ctypes.c_char_p
     lib.hsa_abi_sizes.restype = None
@@ -257,6 +260,21 @@ def hsa_decode_workspace_bytes(kv: PagedKV, index: PQIndex) -> int:
     return int(n)
 
 
+def hsa_decode_host_workspace_bytes(kv: PagedKV, index: PQIndex) -> int:
+    kvs, ixs = kv.struct(), index.struct()
+    n = load_library().hsa_decode_host_workspace_bytes(ctypes.byref(kvs), ctypes.byref(ixs))
+    if n == 0:
+        raise HSAError("hsa_decode_host_workspace_bytes", 1)
+    return int(n)
+
+
+def _check_host_io(t: torch.Tensor, shape, name: str) -> None:
+    """hsa_decode_host reads and writes these on the host (pinned memory keeps the copies
+    asynchronous)."""
+    if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected a contiguous fp32 host tensor {list(shape)}")
+
+
 def dense_decode_workspace_bytes(kv: PagedKV) -> int:
     kvs = kv.struct()
     n = load_library().dense_decode_workspace_bytes(ctypes.byref(kvs))
@@ -309,6 +327,8 @@ class DecodeStep:
     marshalled once here, and each call passes only q, out and the stream (the library still
     validates every call, lengths included). The tensors must keep their storage while the
     step is in use; their contents (lengths, appended tokens, lists) may change between calls.
+    Calling the step runs hsa_decode on device q / out; .host() runs hsa_decode_host on host
+    q / out (the workspace is sized for both).
     """
 
     def __init__(self, kv: PagedKV, index: PQIndex, *, scale: float, budget: float = 0.01, k_override: int = -1,
@@ -316,13 +336,14 @@ class DecodeStep:
         self.kv, self.index = kv, index          # keep the tensors behind the views alive
         self._kvs, self._ixs = kv.struct(), index.struct()
         if workspace_buf is None:
-            workspace_buf = workspace(hsa_decode_workspace_bytes(kv, index), kv.k_cache.device)
+            workspace_buf = workspace(hsa_decode_host_workspace_bytes(kv, index), kv.k_cache.device)
         _on_gpu(workspace_buf)
         self.workspace_buf = workspace_buf
         self._prm = _Params(float(scale), float(budget), int(k_override), 1 if background else 0)
         self._shape = (kv.B, kv.Hq, kv.k_cache.shape[3])
         self._device = kv.k_cache.device
         self._fn = load_library().hsa_decode
+        self._fn_host = load_library().hsa_decode_host
         self._kv_ref, self._ix_ref = ctypes.byref(self._kvs), ctypes.byref(self._ixs)
         self._prm_ref = ctypes.byref(self._prm)
         self._ws_ptr, self._ws_len = workspace_buf.data_ptr(), workspace_buf.numel()
@@ -342,6 +363,35 @@ class DecodeStep:
                       self._ws_len, _stream(stream))
         _check("hsa_decode", st)
         return out
+
+    def host(self, q_host: torch.Tensor, out_host: torch.Tensor, stream=None) -> torch.Tensor:
+        """hsa_decode_host: q in from and out back to host memory, queued on the stream."""
+        _check_host_io(q_host, self._shape, "q_host")
+        _check_host_io(out_host, self._shape, "out_host")
+        st = self._fn_host(self._kv_ref, self._ix_ref, q_host.data_ptr(), out_host.data_ptr(), self._prm_ref,
+                           self._ws_ptr, self._ws_len, _stream(stream))
+        _check("hsa_decode_host", st)
+        return out_host
+
+
+def hsa_decode_host(kv: PagedKV, index: PQIndex, q_host: torch.Tensor, out_host: torch.Tensor, *, scale: float,
+                    budget: float = 0.01, k_override: int = -1, background: bool = True,
+                    workspace_buf: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """hsa_decode with q and out in host memory (see hsa_decode_host in include/pqhsa.h).
+    Queued on the stream: out_host holds the result once the stream has reached it."""
+    shape = (kv.B, kv.Hq, kv.k_cache.shape[3])
+    _check_host_io(q_host, shape, "q_host")
+    _check_host_io(out_host, shape, "out_host")
+    kvs, ixs = kv.struct(), index.struct()
+    if workspace_buf is None:
+        workspace_buf = workspace(hsa_decode_host_workspace_bytes(kv, index), kv.k_cache.device)
+    _on_gpu(workspace_buf)
+    prm = _Params(float(scale), float(budget), int(k_override), 1 if background else 0)
+    st = load_library().hsa_decode_host(ctypes.byref(kvs), ctypes.byref(ixs), q_host.data_ptr(), out_host.data_ptr(),
+                                        ctypes.byref(prm), workspace_buf.data_ptr(), workspace_buf.numel(),
+                                        _stream(stream))
+    _check("hsa_decode_host", st)
+    return out_host
 
 
 def selected_counts(kv: PagedKV, index: PQIndex, q: torch.Tensor, *, scale: float, budget: float = 0.01,

@@ -180,6 +180,11 @@ Split plan_splits(long long E_max, int U, int nbg, int slots) {
   return best;
 }
 
+// Device room for q (or out) of hsa_decode_host at the end of its workspace.
+size_t host_io_bytes(const hsa_kv_cache* kv) {
+  return align_up(static_cast<size_t>(kv->B) * kv->Hq * kD * sizeof(float), 256);
+}
+
 size_t dense_layout_bytes(int U, int G) {
   const size_t parts = static_cast<size_t>(U) * kMaxSplits * G;
   size_t o = align_up(sizeof(WsHeader), 256);
@@ -223,6 +228,12 @@ size_t hsa_decode_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix) {
   const DecodeLayout L =
       make_decode_layout(kv->B * kv->Hkv, kv->Hq / kv->Hkv, ix->C, ix->cap, ix->list_slots, kMaxSplits);
   return L.total;
+}
+
+size_t hsa_decode_host_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix) {
+  const size_t base = hsa_decode_workspace_bytes(kv, ix);
+  if (base == 0) return 0;
+  return align_up(base, 256) + 2 * host_io_bytes(kv);
 }
 
 size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv) {
@@ -535,6 +546,27 @@ static EncodeLayout encode_layout(int U, int C, int n_new) {
 
 // Encoding runs on the tensor cores when the cache has pages of at least 8 rows.
 static bool mma_encode(const hsa_kv_cache* kv, int n_new) { return kv->page_size >= 8 && n_new > 0; }
+
+hsa_status hsa_decode_host(const hsa_kv_cache* kv, const hsa_index* ix, const float* q_host, float* out_host,
+                           const hsa_decode_params* prm, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  st = check_index(kv, ix, true);
+  if (st != HSA_OK) return st;
+  if (!q_host || !out_host || !prm) return HSA_ERR_INVALID_ARG;
+  const size_t base = align_up(hsa_decode_workspace_bytes(kv, ix), 256);
+  const size_t io = host_io_bytes(kv);
+  if (!ws || !aligned(ws, 256) || ws_bytes < base + 2 * io) return HSA_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* q_dev = reinterpret_cast<float*>(w + base);
+  float* out_dev = reinterpret_cast<float*>(w + base + io);
+  const size_t bytes = static_cast<size_t>(kv->B) * kv->Hq * kD * sizeof(float);
+  RET_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));
+  st = hsa_decode(kv, ix, q_dev, out_dev, prm, nullptr, ws, base, stream);
+  if (st != HSA_OK) return st;
+  RET_CUDA(cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, stream));
+  return HSA_OK;
+}
 
 size_t hsa_index_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix, int32_t n_new) {
   if (!kv || !ix || kv->B < 1 || kv->Hkv < 1 || ix->C < 1 || n_new < 0) return sizeof(WsHeader);

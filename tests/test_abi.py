@@ -138,6 +138,33 @@ def test_decode_rejects_small_workspace_and_null_q(host_only):
     assert need > 0 and need % 256 == 0
 
 
+def test_decode_host_validates_before_queuing(host_only):
+    """hsa_decode_host checks everything before its first copy: a bad cache, a null host
+    pointer or a workspace without room for q and out is refused (fake device pointers
+    are never touched). Its workspace is hsa_decode's plus two 256-byte aligned q/out areas."""
+    lib = host_only
+    kv, lens = _kv()
+    ix, nh = _ix()
+    q = np.zeros((1, 4, 128), dtype=np.float32)
+    out = np.zeros_like(q)
+    prm = P._Params(0.088, 0.01, -1, 1)
+    need = lib.hsa_decode_workspace_bytes(ctypes.byref(kv), ctypes.byref(ix))
+    need_host = lib.hsa_decode_host_workspace_bytes(ctypes.byref(kv), ctypes.byref(ix))
+    assert need_host == need + 2 * 2048   # 1 x 4 x 128 fp32 = 2048 bytes each
+
+    def call(kv_, ix_, qp, op, ws_bytes):
+        return lib.hsa_decode_host(ctypes.byref(kv_), ctypes.byref(ix_), qp, op, ctypes.byref(prm), FAKE, ws_bytes,
+                                   None)
+
+    assert call(kv, ix, None, out.ctypes.data, need_host) == 1
+    assert call(kv, ix, q.ctypes.data, None, need_host) == 1
+    assert call(kv, ix, q.ctypes.data, out.ctypes.data, need) == 5      # no room for q and out
+    bad_kv, _ = _kv(D=64)
+    assert call(bad_kv, ix, q.ctypes.data, out.ctypes.data, need_host) == 2
+    bad_ix, _ = _ix(n_idx=200)
+    assert call(kv, bad_ix, q.ctypes.data, out.ctypes.data, need_host) == 3
+
+
 def test_append_checks_capacity(host_only):
     lib = host_only
     kv, lens = _kv(seq=100)

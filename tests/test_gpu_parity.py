@@ -161,9 +161,10 @@ def test_no_index_and_no_sink(cuda_device):
 
 
 def test_prepared_step_matches_hsa_decode(cuda_device):
-    """DecodeStep (the cache and index views marshalled once) gives hsa_decode's output, and
-    still does after the lengths change in place behind its views. Two decode calls agree to
-    rounding, not bit for bit: the cluster-weight sums are fp32 atomics in arrival order."""
+    """DecodeStep (the cache and index views marshalled once) gives hsa_decode's output, on
+    device and on host buffers (hsa_decode_host), and still does after the lengths change in
+    place behind its views. Two decode calls agree to rounding, not bit for bit: the
+    cluster-weight sums are fp32 atomics in arrival order."""
     w, bt, codes, ids, kv, ix, dev = _setup(CASES["qwen_g8_8k"])
     ws_idx = P.workspace(P.hsa_index_workspace_bytes(kv, ix), dev)
     P.hsa_build_from_codes(kv, ix, workspace_buf=ws_idx)
@@ -178,6 +179,15 @@ def test_prepared_step_matches_hsa_decode(cuda_device):
         torch.cuda.synchronize()
         tol = 1e-6 * float(ref.abs().max()) + 1e-7
         assert float((got - ref).abs().max()) <= tol and float((out - ref).abs().max()) <= tol
+        # the host-buffer entry: q in from and out back to pinned host memory
+        q_h = q.cpu().pin_memory()
+        out_h = torch.full(q.shape, float("nan")).pin_memory()
+        step.host(q_h, out_h)
+        out_h2 = torch.full(q.shape, float("nan")).pin_memory()
+        P.hsa_decode_host(kv, ix, q_h, out_h2, scale=scale, budget=w.budget)
+        torch.cuda.synchronize()
+        ref_h = ref.cpu()
+        assert float((out_h - ref_h).abs().max()) <= tol and float((out_h2 - ref_h).abs().max()) <= tol
         assert P.hsa_read_error(step.workspace_buf) == 0
         kv.seq_lens.sub_(100)                  # a shorter tail, same storage
         kv.seq_lens_host.sub_(100)
