@@ -383,11 +383,11 @@ def run_ours(args):
 
     def e2e_steps(steps, use_prepared=True):
         """End to end through the public API, per step, by the host's wall clock, from pinned
-        host memory to pinned host memory: the prepared step's hsa_decode_host (one C-ABI call
-        that queues the copy of q in, the decode and the copy of out back), or, for comparison,
-        hsa_decode marshalling every argument anew between torch copies in and out; then the
-        wait for the result. The library validates, plans and launches on every call. L2 is
-        flushed, and the flush finished, before each step."""
+        host memory to pinned host memory: the prepared step (hsa_decode_step_run: the library
+        validates and plans, then replays the recorded host-buffer step as one graph launch), or,
+        for comparison, hsa_decode marshalling every argument anew between torch copies in and
+        out; then the wait for the result. L2 is flushed, and the flush finished, before each
+        step."""
         t_wall, t_dev = [], []
         for _ in range(steps):
             flush.zero_()
@@ -533,10 +533,11 @@ def run_ours(args):
                      "duration_us": round(stage_ms[dom] * 1e3, 3)},
         "e2e": {"value": round(ms_e2e * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": q.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 4,
-                "how": "host wall clock per step, pinned host q to pinned host out: one C-ABI hsa_decode_host "
-                       "call through the prepared DecodeStep (cudaMemcpyAsync of q in, validation, planning, "
-                       "the launches, cudaMemcpyAsync of out back; the binding's views marshalled once), then "
-                       "the wait",
+                "how": "host wall clock per step, page-locked host q to page-locked host out: one C-ABI "
+                       "hsa_decode_step_run call through the prepared DecodeStep (validation and split plan "
+                       "every call, then one CUDA-graph launch of the host-buffer step: q staged by a copy "
+                       "kernel, the four decode kernels, out written to host memory by the merge), then the "
+                       "wait",
                 "device_us": round(ms_e2e_dev * 1e3, 3),
                 "hsa_decode_call_us": round(ms_e2e_call * 1e3, 3),   # torch copies + per-call marshalling
                 "graph_staged_us": round(mean(t_staged) * 1e3, 3) if t_staged else None},

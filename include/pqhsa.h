@@ -152,9 +152,10 @@ size_t hsa_decode_host_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* 
 
 /*
  * hsa_decode with q and out in host memory, for callers whose query and result live
- * on the host. On `stream`: q_host is copied into the workspace, the decode step runs
- * (as hsa_decode, without debug outputs), and the result is copied to out_host, one
- * cudaMemcpyAsync each way (page-locked host buffers keep both copies asynchronous).
+ * on the host. On `stream`: q_host is brought into the workspace, the decode step runs
+ * (as hsa_decode, without debug outputs), and the result goes to out_host. Page-locked
+ * (device-addressable) buffers are read by a copy kernel and written by the last kernel
+ * of the step directly; pageable ones take one cudaMemcpyAsync each way.
  * q_host, out_host: fp32 [B][Hq][D] host memory, caller-owned. Returns once all of it
  * is queued; out_host holds the result when `stream` reaches the end of this call
  * (synchronise the stream or an event recorded after it before reading). Arguments
@@ -164,6 +165,39 @@ size_t hsa_decode_host_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* 
 hsa_status hsa_decode_host(const hsa_kv_cache* kv, const hsa_index* index, const float* q_host, float* out_host,
                            const hsa_decode_params* params, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
+
+/* ---- prepared decode step (graph replay) --------------------------------- */
+
+/* A decode step prepared for one cache, index, parameter set and workspace (opaque). */
+typedef struct hsa_decode_step hsa_decode_step;
+
+/*
+ * Prepare hsa_decode_host for a decode loop. Copies the cache and index views and the
+ * parameters, not the arrays they point to: those stay caller-owned, must outlive the
+ * step, and may change in place between runs (lengths, appends, lists). The workspace
+ * must hold hsa_decode_host_workspace_bytes. Validates as hsa_decode_host does and makes
+ * no CUDA call. *step receives the handle, or NULL on error (HSA_ERR_CUDA also when the
+ * step's host memory cannot be allocated).
+ */
+hsa_status hsa_decode_step_create(const hsa_kv_cache* kv, const hsa_index* index, const hsa_decode_params* params,
+                                  void* workspace, size_t workspace_bytes, hsa_decode_step** step);
+
+/*
+ * One decode step on host buffers, as hsa_decode_host, queued on `stream` as one CUDA
+ * graph launch. Every run validates the views and the current lengths again and
+ * recomputes the split-K plan of the exact part (the only launch shape that depends on
+ * host-side values). While that plan, q_host and out_host are those of the previous run,
+ * the run replays the previous run's graph; otherwise (the first run, lengths that moved
+ * the plan, other buffers) it records the host-buffer step on a private stream of the
+ * step and updates the graph. q_host and out_host must be page-locked host memory
+ * (HSA_ERR_INVALID_ARG otherwise). Result and error word as for hsa_decode_host. One
+ * thread at a time per step; runs of steps that share a workspace must not overlap.
+ */
+hsa_status hsa_decode_step_run(hsa_decode_step* step, const float* q_host, float* out_host, cudaStream_t stream);
+
+/* Release a step (its graph and private stream). NULL is ignored. It does not wait:
+   let the step's queued work finish before the arrays it reads are freed. */
+void hsa_decode_step_destroy(hsa_decode_step* step);
 
 /* Workspace bytes dense_decode needs. */
 size_t dense_decode_workspace_bytes(const hsa_kv_cache* kv);

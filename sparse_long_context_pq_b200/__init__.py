@@ -69,7 +69,8 @@ NUM_STAGES = 4
 STAGE_NAMES = ("tables", "scan_select", "attend", "merge")
 
 
-EXPORTS = ("hsa_decode", "hsa_decode_host", "dense_decode", "hsa_build_from_codes", "hsa_append_encode",
+EXPORTS = ("hsa_decode", "hsa_decode_host", "hsa_decode_step_create", "hsa_decode_step_run",
+           "hsa_decode_step_destroy", "dense_decode", "hsa_build_from_codes", "hsa_append_encode",
            "hsa_index_list_slots", "hsa_decode_workspace_bytes", "hsa_decode_host_workspace_bytes",
            "dense_decode_workspace_bytes", "hsa_index_workspace_bytes",
            "hsa_read_error", "hsa_strerror", "hsa_abi_sizes")
@@ -98,6 +99,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.hsa_decode.argtypes = [P(_KV), P(_Index), vp, vp, P(_Params), P(_Debug), vp, sz, vp]
     lib.hsa_decode_host.argtypes = [P(_KV), P(_Index), vp, vp, P(_Params), vp, sz, vp]
     lib.hsa_decode_host_workspace_bytes.argtypes = [P(_KV), P(_Index)]
+    lib.hsa_decode_step_create.argtypes = [P(_KV), P(_Index), P(_Params), vp, sz, P(vp)]
+    lib.hsa_decode_step_run.argtypes = [vp, vp, vp, vp]
+    lib.hsa_decode_step_destroy.argtypes = [vp]
+    lib.hsa_decode_step_destroy.restype = None
     lib.dense_decode.argtypes = [P(_KV), vp, vp, ctypes.c_float, vp, sz, vp]
     lib.hsa_build_from_codes.argtypes = [P(_KV), P(_Index), vp, sz, vp]
     lib.hsa_append_encode.argtypes = [P(_KV), P(_Index), i32, vp, sz, vp]
@@ -109,8 +114,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.hsa_read_error.argtypes = [vp, P(i32), vp]
     lib.hsa_strerror.argtypes = [ctypes.c_int]
     lib.hsa_abi_sizes.argtypes = [P(ctypes.c_int64)] * 4
-    for f in ("hsa_decode", "hsa_decode_host", "dense_decode", "hsa_build_from_codes", "hsa_append_encode",
-              "hsa_read_error", "hsa_train_index"):
+    for f in ("hsa_decode", "hsa_decode_host", "hsa_decode_step_create", "hsa_decode_step_run", "dense_decode",
+              "hsa_build_from_codes", "hsa_append_encode", "hsa_read_error", "hsa_train_index"):
         getattr(lib, f).restype = ctypes.c_int
     for f in ("hsa_decode_workspace_bytes", "hsa_decode_host_workspace_bytes", "dense_decode_workspace_bytes",
               "hsa_index_workspace_bytes", "hsa_train_workspace_bytes"):
@@ -327,8 +332,10 @@ class DecodeStep:
     marshalled once here, and each call passes only q, out and the stream (the library still
     validates every call, lengths included). The tensors must keep their storage while the
     step is in use; their contents (lengths, appended tokens, lists) may change between calls.
-    Calling the step runs hsa_decode on device q / out; .host() runs hsa_decode_host on host
-    q / out (the workspace is sized for both).
+    Calling the step runs hsa_decode on device q / out; .host() runs the step on host q / out
+    (page-locked): by default as the library's prepared step (hsa_decode_step_run, one CUDA
+    graph launch per call while the split plan and buffers stay the same), or with
+    graph=False as one hsa_decode_host call. The workspace is sized for both.
     """
 
     def __init__(self, kv: PagedKV, index: PQIndex, *, scale: float, budget: float = 0.01, k_override: int = -1,
@@ -347,6 +354,8 @@ class DecodeStep:
         self._kv_ref, self._ix_ref = ctypes.byref(self._kvs), ctypes.byref(self._ixs)
         self._prm_ref = ctypes.byref(self._prm)
         self._ws_ptr, self._ws_len = workspace_buf.data_ptr(), workspace_buf.numel()
+        self._lib = load_library()
+        self._handle = ctypes.c_void_p(None)
 
     def _check_io(self, t: torch.Tensor, name: str) -> None:
         if (t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != self._shape
@@ -364,14 +373,35 @@ class DecodeStep:
         _check("hsa_decode", st)
         return out
 
-    def host(self, q_host: torch.Tensor, out_host: torch.Tensor, stream=None) -> torch.Tensor:
-        """hsa_decode_host: q in from and out back to host memory, queued on the stream."""
+    def host(self, q_host: torch.Tensor, out_host: torch.Tensor, stream=None, graph: bool = True) -> torch.Tensor:
+        """q in from and out back to host memory, queued on the stream (out_host holds the result
+        once the stream has reached it)."""
         _check_host_io(q_host, self._shape, "q_host")
         _check_host_io(out_host, self._shape, "out_host")
-        st = self._fn_host(self._kv_ref, self._ix_ref, q_host.data_ptr(), out_host.data_ptr(), self._prm_ref,
-                           self._ws_ptr, self._ws_len, _stream(stream))
-        _check("hsa_decode_host", st)
+        if not graph:
+            st = self._fn_host(self._kv_ref, self._ix_ref, q_host.data_ptr(), out_host.data_ptr(), self._prm_ref,
+                               self._ws_ptr, self._ws_len, _stream(stream))
+            _check("hsa_decode_host", st)
+            return out_host
+        if not self._handle.value:
+            _check("hsa_decode_step_create",
+                   self._lib.hsa_decode_step_create(self._kv_ref, self._ix_ref, self._prm_ref, self._ws_ptr,
+                                                    self._ws_len, ctypes.byref(self._handle)))
+        _check("hsa_decode_step_run", self._lib.hsa_decode_step_run(self._handle, q_host.data_ptr(),
+                                                                    out_host.data_ptr(), _stream(stream)))
         return out_host
+
+    def close(self) -> None:
+        """Release the library's prepared step (after its queued work has finished)."""
+        if getattr(self, "_handle", None) is not None and self._handle.value:
+            self._lib.hsa_decode_step_destroy(self._handle)
+            self._handle = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def hsa_decode_host(kv: PagedKV, index: PQIndex, q_host: torch.Tensor, out_host: torch.Tensor, *, scale: float,

@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cmath>
 #include <mutex>
+#include <new>
 
 #include "../../include/pqhsa.h"
 #include "common.cuh"
@@ -180,6 +181,41 @@ Split plan_splits(long long E_max, int U, int nbg, int slots) {
   return best;
 }
 
+// Split-K plan of hsa_decode's exact part for the current lengths: the longest unit's
+// sink + selected + tail rows over the units' splits (the only launch shape that depends
+// on host-side values).
+Split decode_split_plan(const hsa_kv_cache* kv, const hsa_index* ix, const hsa_decode_params* prm, int nbg,
+                        int sms) {
+  long long Emax = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    const int T = std::max(0, kv->seq_lens_host[b]);
+    const int s0 = std::min(ix->n_sink, T);
+    const int N = host_unit_n(kv, ix, b);
+    const int k = decode_k(prm->budget, prm->k_override, N);
+    Emax = std::max<long long>(Emax, static_cast<long long>(s0) + k + (T - s0 - N));
+  }
+  const int G = kv->Hq / kv->Hkv;
+  return plan_splits(Emax, kv->B * kv->Hkv, nbg, sms * attend_slots_per_sm(G, true, true));
+}
+
+// q of hsa_decode_host from page-locked host memory (device-addressable) into the
+// workspace: one 16-byte load and store per thread, so the step's many CTAs read q from
+// device memory rather than each across the host link.
+__global__ void __launch_bounds__(256) stage_q_kernel(const float4* __restrict__ src, float4* __restrict__ dst,
+                                                      int n4) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) dst[i] = src[i];
+}
+
+// Device address of page-locked host memory (nullptr for pageable memory).
+void* mapped_host_pointer(const void* p) {
+  cudaPointerAttributes a = {};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 // Device room for q (or out) of hsa_decode_host at the end of its workspace.
 size_t host_io_bytes(const hsa_kv_cache* kv) {
   return align_up(static_cast<size_t>(kv->B) * kv->Hq * kD * sizeof(float), 256);
@@ -331,15 +367,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   if (!dev) return HSA_ERR_CUDA;
 
   // ---- plan the exact split-K over sink + selected + tail rows ----
-  long long Emax = 0;
-  for (int b = 0; b < kv->B; ++b) {
-    const int T = std::max(0, kv->seq_lens_host[b]);
-    const int s0 = std::min(ix->n_sink, T);
-    const int N = host_unit_n(kv, ix, b);
-    const int k = decode_k(prm->budget, prm->k_override, N);
-    Emax = std::max<long long>(Emax, static_cast<long long>(s0) + k + (T - s0 - N));
-  }
-  const Split sp = plan_splits(Emax, U, L.nbg, dev->sms * attend_slots_per_sm(G, true, true));
+  const Split sp = decode_split_plan(kv, ix, prm, L.nbg, dev->sms);
   CUtensorMap tk = {}, tv = {};   // unused: gathered rows are copied by the producer lanes
   cudaEvent_t* ev = dbg ? dbg->stage_events : nullptr;
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], stream) : cudaSuccess; };
@@ -561,11 +589,135 @@ hsa_status hsa_decode_host(const hsa_kv_cache* kv, const hsa_index* ix, const fl
   float* q_dev = reinterpret_cast<float*>(w + base);
   float* out_dev = reinterpret_cast<float*>(w + base + io);
   const size_t bytes = static_cast<size_t>(kv->B) * kv->Hq * kD * sizeof(float);
+  // Page-locked buffers are device-addressable: q is staged by a kernel and the merge writes
+  // out across the host link itself (no copy-engine round trips). Pageable ones are copied.
+  const void* q_map = mapped_host_pointer(q_host);
+  void* out_map = mapped_host_pointer(out_host);
+  if (q_map && out_map && aligned(q_map, 16) && aligned(out_map, 16)) {
+    const int n4 = static_cast<int>(bytes / 16);
+    stage_q_kernel<<<std::min(64, (n4 + 255) / 256), 256, 0, stream>>>(static_cast<const float4*>(q_map),
+                                                                       reinterpret_cast<float4*>(q_dev), n4);
+    RET_CUDA(cudaGetLastError());
+    return hsa_decode(kv, ix, q_dev, static_cast<float*>(out_map), prm, nullptr, ws, base, stream);
+  }
   RET_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));
   st = hsa_decode(kv, ix, q_dev, out_dev, prm, nullptr, ws, base, stream);
   if (st != HSA_OK) return st;
   RET_CUDA(cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, stream));
   return HSA_OK;
+}
+
+}  // extern "C"
+
+struct hsa_decode_step {
+  hsa_kv_cache kv;
+  hsa_index ix;
+  hsa_decode_params prm;
+  void* ws;
+  size_t ws_bytes;
+  int device;                   // device current at the first capture
+  cudaStream_t cap;             // private capture stream (created at the first capture)
+  cudaGraphExec_t exec;         // the last recorded step
+  int key_nsplit, key_chunk;    // its split-K plan
+  const float* key_q;
+  float* key_out;
+};
+
+namespace {
+hsa_status check_step_args(const hsa_kv_cache* kv, const hsa_index* ix, const hsa_decode_params* prm, void* ws,
+                           size_t ws_bytes) {
+  hsa_status st = check_kv(kv);
+  if (st != HSA_OK) return st;
+  st = check_index(kv, ix, true);
+  if (st != HSA_OK) return st;
+  if (!prm || !(prm->budget >= 0.0) || !std::isfinite(prm->scale)) return HSA_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < hsa_decode_host_workspace_bytes(kv, ix)) return HSA_ERR_WORKSPACE;
+  return HSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+hsa_status hsa_decode_step_create(const hsa_kv_cache* kv, const hsa_index* ix, const hsa_decode_params* prm,
+                                  void* ws, size_t ws_bytes, hsa_decode_step** step) {
+  if (!step) return HSA_ERR_INVALID_ARG;
+  *step = nullptr;
+  const hsa_status st = check_step_args(kv, ix, prm, ws, ws_bytes);
+  if (st != HSA_OK) return st;
+  hsa_decode_step* s = new (std::nothrow) hsa_decode_step();
+  if (!s) return HSA_ERR_CUDA;
+  s->kv = *kv;
+  s->ix = *ix;
+  s->prm = *prm;
+  s->ws = ws;
+  s->ws_bytes = ws_bytes;
+  s->device = -1;
+  s->cap = nullptr;
+  s->exec = nullptr;
+  *step = s;
+  return HSA_OK;
+}
+
+hsa_status hsa_decode_step_run(hsa_decode_step* s, const float* q_host, float* out_host, cudaStream_t stream) {
+  if (!s) return HSA_ERR_INVALID_ARG;
+  hsa_status st = check_step_args(&s->kv, &s->ix, &s->prm, s->ws, s->ws_bytes);
+  if (st != HSA_OK) return st;
+  if (!q_host || !out_host) return HSA_ERR_INVALID_ARG;
+  const DeviceInfo* dev = device_info();
+  if (!dev) return HSA_ERR_CUDA;
+  const int G = s->kv.Hq / s->kv.Hkv;
+  const DecodeLayout L = make_decode_layout(s->kv.B * s->kv.Hkv, G, s->ix.C, s->ix.cap, s->ix.list_slots, kMaxSplits);
+  const Split sp = decode_split_plan(&s->kv, &s->ix, &s->prm, L.nbg, dev->sms);
+  const bool same = s->exec && sp.nsplit == s->key_nsplit && sp.chunk == s->key_chunk && q_host == s->key_q &&
+                    out_host == s->key_out;
+  if (!same) {
+    // a graph cannot copy pageable host memory: the buffers must be page-locked
+    if (!mapped_host_pointer(q_host) || !mapped_host_pointer(out_host)) return HSA_ERR_INVALID_ARG;
+    int cur = 0;
+    RET_CUDA(cudaGetDevice(&cur));
+    if (s->cap && cur != s->device) return HSA_ERR_INVALID_ARG;   // a step stays on its first device
+    if (!s->cap) {
+      RET_CUDA(cudaStreamCreateWithFlags(&s->cap, cudaStreamNonBlocking));
+      s->device = cur;
+    }
+    // record the host-buffer step (nothing runs while the stream captures)
+    RET_CUDA(cudaStreamBeginCapture(s->cap, cudaStreamCaptureModeThreadLocal));
+    st = hsa_decode_host(&s->kv, &s->ix, q_host, out_host, &s->prm, s->ws, s->ws_bytes, s->cap);
+    cudaGraph_t g = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(s->cap, &g);
+    if (st != HSA_OK || ce != cudaSuccess || !g) {
+      if (g) cudaGraphDestroy(g);
+      (void)cudaGetLastError();   // an invalidated capture (e.g. pageable host memory) is not sticky
+      return st != HSA_OK ? st : HSA_ERR_CUDA;
+    }
+    if (s->exec) {
+      cudaGraphExecUpdateResultInfo info;
+      if (cudaGraphExecUpdate(s->exec, g, &info) != cudaSuccess) {
+        (void)cudaGetLastError();   // the failed update is not sticky; instantiate afresh
+        cudaGraphExecDestroy(s->exec);
+        s->exec = nullptr;
+      }
+    }
+    if (!s->exec && cudaGraphInstantiate(&s->exec, g, 0) != cudaSuccess) {
+      s->exec = nullptr;
+      cudaGraphDestroy(g);
+      return HSA_ERR_CUDA;
+    }
+    cudaGraphDestroy(g);
+    s->key_nsplit = sp.nsplit;
+    s->key_chunk = sp.chunk;
+    s->key_q = q_host;
+    s->key_out = out_host;
+  }
+  RET_CUDA(cudaGraphLaunch(s->exec, stream));
+  return HSA_OK;
+}
+
+void hsa_decode_step_destroy(hsa_decode_step* s) {
+  if (!s) return;
+  if (s->exec) cudaGraphExecDestroy(s->exec);
+  if (s->cap) cudaStreamDestroy(s->cap);
+  delete s;
 }
 
 size_t hsa_index_workspace_bytes(const hsa_kv_cache* kv, const hsa_index* ix, int32_t n_new) {

@@ -165,6 +165,34 @@ def test_decode_host_validates_before_queuing(host_only):
     assert call(kv, bad_ix, q.ctypes.data, out.ctypes.data, need_host) == 3
 
 
+def test_decode_step_validates_without_cuda(host_only):
+    """hsa_decode_step_create checks its arguments and makes no CUDA call; every run checks
+    the views and the current lengths again before anything is recorded or launched."""
+    lib = host_only
+    kv, lens = _kv()
+    ix, nh = _ix()
+    prm = P._Params(0.088, 0.01, -1, 1)
+    need_host = lib.hsa_decode_host_workspace_bytes(ctypes.byref(kv), ctypes.byref(ix))
+    h = ctypes.c_void_p()
+    assert lib.hsa_decode_step_create(ctypes.byref(kv), ctypes.byref(ix), ctypes.byref(prm), FAKE, need_host - 256,
+                                      ctypes.byref(h)) == 5 and not h.value
+    bad_kv, _ = _kv(D=64)
+    assert lib.hsa_decode_step_create(ctypes.byref(bad_kv), ctypes.byref(ix), ctypes.byref(prm), FAKE, need_host,
+                                      ctypes.byref(h)) == 2 and not h.value
+    assert lib.hsa_decode_step_create(ctypes.byref(kv), ctypes.byref(ix), ctypes.byref(prm), FAKE, need_host,
+                                      None) == 1
+    assert lib.hsa_decode_step_create(ctypes.byref(kv), ctypes.byref(ix), ctypes.byref(prm), FAKE, need_host,
+                                      ctypes.byref(h)) == 0 and h.value
+    q = np.zeros((1, 4, 128), dtype=np.float32)
+    out = np.zeros_like(q)
+    assert lib.hsa_decode_step_run(h, None, out.ctypes.data, None) == 1
+    assert lib.hsa_decode_step_run(None, q.ctypes.data, out.ctypes.data, None) == 1
+    lens[0] = 1000                    # grown past the block table after the step was made
+    assert lib.hsa_decode_step_run(h, q.ctypes.data, out.ctypes.data, None) == 3
+    lib.hsa_decode_step_destroy(h)
+    lib.hsa_decode_step_destroy(None)
+
+
 def test_append_checks_capacity(host_only):
     lib = host_only
     kv, lens = _kv(seq=100)

@@ -181,15 +181,30 @@ def test_prepared_step_matches_hsa_decode(cuda_device):
         assert float((got - ref).abs().max()) <= tol and float((out - ref).abs().max()) <= tol
         # the host-buffer entry: q in from and out back to pinned host memory
         q_h = q.cpu().pin_memory()
-        out_h = torch.full(q.shape, float("nan")).pin_memory()
-        step.host(q_h, out_h)
-        out_h2 = torch.full(q.shape, float("nan")).pin_memory()
-        P.hsa_decode_host(kv, ix, q_h, out_h2, scale=scale, budget=w.budget)
+        outs = [torch.full(q.shape, float("nan")).pin_memory() for _ in range(4)]
+        step.host(q_h, outs[0])                 # prepared step: records its graph
+        step.host(q_h, outs[1])                 # replays it
+        step.host(q_h, outs[2], graph=False)    # one hsa_decode_host call
+        P.hsa_decode_host(kv, ix, q_h, outs[3], scale=scale, budget=w.budget)
+        q_pageable = q.cpu()                    # not page-locked: copied by cudaMemcpyAsync
+        out_pageable = torch.full(q.shape, float("nan"))
+        P.hsa_decode_host(kv, ix, q_pageable, out_pageable, scale=scale, budget=w.budget)
         torch.cuda.synchronize()
         ref_h = ref.cpu()
-        assert float((out_h - ref_h).abs().max()) <= tol and float((out_h2 - ref_h).abs().max()) <= tol
+        for o in outs + [out_pageable]:
+            assert float((o - ref_h).abs().max()) <= tol
+        with pytest.raises(P.HSAError):         # the graph-replayed step needs page-locked buffers
+            step.host(q_pageable, out_pageable)
+        # a replay reads the host buffer's current contents
+        q2 = (q * 0.5).contiguous()
+        ref2 = P.hsa_decode(kv, ix, q2, scale=scale, budget=w.budget)
+        q_h.copy_(q2.cpu())
+        step.host(q_h, outs[0])
+        torch.cuda.synchronize()
+        assert float((outs[0] - ref2.cpu()).abs().max()) <= 1e-6 * float(ref2.abs().max()) + 1e-7
         assert P.hsa_read_error(step.workspace_buf) == 0
-        kv.seq_lens.sub_(100)                  # a shorter tail, same storage
-        kv.seq_lens_host.sub_(100)
+        kv.seq_lens.sub_(700)                  # a shorter tail (and another split plan), same storage
+        kv.seq_lens_host.sub_(700)
     with pytest.raises(ValueError):
         step(q[:, :1].contiguous())
+    step.close()
