@@ -297,7 +297,7 @@ struct ScanSmem {
 // scratch (from the start of dynamic shared memory, over the tables).
 constexpr int kCmPerThread = 4;                                  // chunk maxima per thread per pass
 constexpr int kCmPass = kCmPerThread * kScanThreads;             // chunks examined per pass
-constexpr int kActPerWarp = 2;                                   // active chunks per warp per round
+constexpr int kActPerWarp = 1;                                   // active chunks per warp per round
 constexpr size_t kFilterScratch = kCmPass * 4;
 constexpr int kFinWordsPerThread = 8;
 constexpr int kFinChunkWords = kFinWordsPerThread * kScanThreads;   // 131072 slots per pass
@@ -768,18 +768,18 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
                           (kNB / 4 - 1 - tid));
   const float* cmax = p.chunk_max + static_cast<size_t>(u) * max_chunks;
   float cm[kCmPerThread];
-  int32_t cc[kCmPerThread];
   auto next_chunk = [&]() {   // chunk of this thread's next local index, then advance
     const int32_t c = static_cast<int32_t>(pc);
     pc += step;
     if (pc >= nt) pc -= nt;
     return c;
   };
+  uint32_t pc_pass = pc;      // the pass's first chunk; the compaction replays the sequence
 #pragma unroll
   for (int e = 0; e < kCmPerThread; ++e) {
     const int c = c0 + tid + e * T;
-    cc[e] = next_chunk();
-    cm[e] = c < c1 ? __ldcg(cmax + cc[e]) : -INFINITY;
+    const int32_t ch = next_chunk();
+    cm[e] = c < c1 ? __ldcg(cmax + ch) : -INFINITY;
   }
   float ub[G], lb[G];
 #pragma unroll
@@ -841,19 +841,24 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
 
     for (int cb = c0; cb < c1; cb += kCmPass) {
       if (cb != c0) {
+        pc_pass = pc;
 #pragma unroll
         for (int e = 0; e < kCmPerThread; ++e) {
           const int c = cb + tid + e * T;
-          cc[e] = next_chunk();
-          cm[e] = c < c1 ? __ldcg(cmax + cc[e]) : -INFINITY;
+          const int32_t ch = next_chunk();
+          cm[e] = c < c1 ? __ldcg(cmax + ch) : -INFINITY;
         }
       }
       if (tid == 0) ss.n_act = 0;
       __syncthreads();
       // chunks whose maximum reaches the threshold bin, compacted warp by warp
+      uint32_t pr = pc_pass;
 #pragma unroll
       for (int e = 0; e < kCmPerThread; ++e) {
         const int c = cb + tid + e * T;
+        const int32_t ch = static_cast<int32_t>(pr);
+        pr += step;
+        if (pr >= nt) pr -= nt;
         const bool active = c < c1 && score_bin(cm[e], lo, inv) >= bstar;
         const uint32_t m = __ballot_sync(0xffffffffu, active);
         if (m) {
@@ -861,7 +866,7 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
           int at = 0;
           if (lane == leader) at = atomicAdd(&ss.n_act, __popc(m));
           at = __shfl_sync(0xffffffffu, at, leader);
-          if (active) act[at + __popc(m & ((1u << lane) - 1u))] = cc[e];
+          if (active) act[at + __popc(m & ((1u << lane) - 1u))] = ch;
         }
       }
       __syncthreads();
