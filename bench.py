@@ -125,6 +125,13 @@ def step_bytes(w, n_idx: int, k: int):
     return U * per_unit, U * ids, U * dense, kernels
 
 
+def scan_wavefronts(G: int, chunks: int) -> int:
+    """Shared-memory wavefronts of the scan's LUT gathers (its on-chip algorithmic work): per
+    32-slot chunk 16 subspace look-ups, each a 128-bit load per lane per 4 heads (4 wavefronts
+    for the 32 lanes of a warp when conflict-free)."""
+    return chunks * 16 * 4 * ((G + 3) // 4)
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -327,6 +334,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     # selected tokens per unit as the library counts them (the byte model's k)
     n_sel = P.selected_counts(kv, ix, q, scale=scale, budget=budget, workspace_buf=ws)
+    n_chunks = int(ix.list_meta.view(w.B * w.Hkv, -1)[:, 0].sum())   # 32-slot chunks the scan streams
     k = int(n_sel.max())
     assert int(n_sel.min()) == k, "every unit of the workload selects the same count"
 
@@ -493,6 +501,18 @@ def run_ours(args):
     dense_gbs = dense_b / (ms_dense * 1e-3) / 1e9
     traffic = dram_traffic(dom_name + "_kernel", w.name)
     U = w.B * w.Hkv
+    clk_sum = clk.summary()
+    onchip = None
+    if dom_name == "scan_select":
+        # the same launch against its on-chip ceiling: one shared-memory wavefront per clock per SM
+        wav = scan_wavefronts(w.G, n_chunks)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        mhz = clk_sum["sm_mhz"] or clk_sum["sm_max_mhz"] or 1965.0
+        ceil_g = sms * mhz * 1e6 / 1e9
+        ach_g = wav / (stage_ms[dom] * 1e-3) / 1e9
+        onchip = {"bound": "shared-memory wavefronts (LUT gathers)", "algorithmic": wav,
+                  "achieved": round(ach_g, 1), "peak": round(ceil_g, 1), "unit": "G wavefronts/s",
+                  "frac": round(ach_g / ceil_g, 4), "peak_basis": f"{sms} SMs x 1 wavefront/clock x {mhz:.0f} MHz"}
 
     res = {
         "metric": METRIC,
@@ -530,7 +550,7 @@ def run_ours(args):
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": traffic, "algorithmic_bytes": dom_bytes,
                      "traffic_over_algorithmic": round(traffic / dom_bytes, 3) if traffic else None,
-                     "duration_us": round(stage_ms[dom] * 1e3, 3)},
+                     "duration_us": round(stage_ms[dom] * 1e3, 3), "onchip": onchip},
         "e2e": {"value": round(ms_e2e * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": q.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 4,
                 "how": "host wall clock per step, page-locked host q to page-locked host out: one C-ABI "
@@ -546,7 +566,7 @@ def run_ours(args):
         # graph steps (4, + 2 warm)
         "gpu_launches": args.steps * (4 * P.NUM_STAGES + 2) + (
             (args.steps + 2) * P.NUM_STAGES if t_staged is not None else 0),
-        "clocks": clk.summary(),
+        "clocks": clk_sum,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         us, steps, workers, el = oracle_sample(bt, w, budget, args.cpu_seconds)

@@ -37,3 +37,12 @@ def test_step_bytes(name, hsa_mb, dense_mb):
     # the same figures, rounded, as tabulated for the decode workloads (MB = 1e6 bytes)
     assert abs(hsa / 1e6 - hsa_mb) <= 0.05 * max(1.0, hsa_mb / 10)
     assert abs(dense / 1e6 - dense_mb) <= 0.05 * max(1.0, dense_mb / 10)
+
+
+def test_scan_wavefronts_closed_form():
+    """LUT gathers of the scan: 16 look-ups per 32-slot chunk, each 4 wavefronts per 4 heads
+    (a conflict-free 128-bit load by 32 lanes is 512 bytes = 4 x 128-byte wavefronts)."""
+    assert bench.scan_wavefronts(4, 1) == 64
+    assert bench.scan_wavefronts(8, 1) == 128
+    assert bench.scan_wavefronts(1, 1) == bench.scan_wavefronts(4, 1)   # heads padded to 4
+    assert bench.scan_wavefronts(4, 36374) == 36374 * 64
