@@ -346,14 +346,21 @@ __device__ __forceinline__ int unit_chunks(const StepParams& p, int u) {
 
 // KV-pool row of position pos of KV head h through one block-table row; an entry outside
 // the pool is recorded and replaced by page 0.
-__device__ __forceinline__ int32_t kv_row(const StepParams& p, const int32_t* bt_row, int h, int pos) {
+// Split in two so that the block-table read can go out before other round trips: the
+// raw entry of position pos, then the row (an entry outside the pool recorded, page 0).
+__device__ __forceinline__ int32_t kv_page_entry(const StepParams& p, const int32_t* bt_row, int pos) {
   const int pi = pos / p.page_size;
-  int page = pi < p.max_pages ? bt_row[pi] : -1;
+  return pi < p.max_pages ? bt_row[pi] : -1;
+}
+__device__ __forceinline__ int32_t kv_row_of(const StepParams& p, int32_t page, int h, int pos) {
   if (page < 0 || page >= p.num_pages) {
     record_error(p.err, HSA_DEVERR_PAGE);
     page = 0;
   }
   return (page * p.Hkv + h) * p.page_size + (pos % p.page_size);
+}
+__device__ __forceinline__ int32_t kv_row(const StepParams& p, const int32_t* bt_row, int h, int pos) {
+  return kv_row_of(p, kv_page_entry(p, bt_row, pos), h, pos);
 }
 
 template <int G>
@@ -612,12 +619,11 @@ __device__ __forceinline__ void scan_segment(const StepParams& p, int u, int ch0
     if (v) atomicAdd(hg + i, v);
   }
   // publish this range: scores, chunk maxima, weights and histogram before the count (the
-  // barrier orders the CTA's writes before thread 0's fence, which is cumulative)
+  // barrier orders the CTA's writes before thread 0's release, which is cumulative; the
+  // waiters read the count with acquire loads)
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    atomicAdd(&p.units[u].scan_done, nch);
-  }
+  if (tid == 0)
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&p.units[u].scan_done), "r"(nch) : "memory");
 }
 
 // Head weights e^{shat_g - ub_g} of one indexed token (cluster id, code words cw) from the
@@ -742,6 +748,9 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
   const uint32_t lane = tid & 31;
   const int b = u / p.Hkv;
   const int N = unit_n(p.seq_lens, p.n_indexed, b, p.n_sink, p.cap);
+  // read with N, before this part's first global store (which the compiler cannot rule
+  // out as aliasing it, so a later read would be another round trip)
+  const int s0 = min(p.n_sink, max(0, p.seq_lens[b]));
   const int k = decode_k(p.budget, p.k_override, N);
   const int max_chunks = p.list_slots / 32;
   const int total = unit_chunks(p, u);
@@ -837,7 +846,6 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
     unsigned long long* counts = reinterpret_cast<unsigned long long*>(&p.units[u].ncand);
     const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
     const int h = u % p.Hkv;
-    const int s0 = min(p.n_sink, max(0, p.seq_lens[b]));
 
     for (int cb = c0; cb < c1; cb += kCmPass) {
       if (cb != c0) {
@@ -891,7 +899,7 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
         // candidates; the block-table reads go out before the counts come back
         bool defv[kActPerWarp], candv[kActPerWarp];
         uint32_t dmv[kActPerWarp], cmv[kActPerWarp];
-        int32_t rowv[kActPerWarp];
+        int32_t pagev[kActPerWarp];
         uint32_t ndm = 0, ncm = 0;
 #pragma unroll
         for (int r = 0; r < kActPerWarp; ++r) {
@@ -902,7 +910,7 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
           candv[r] = bin == bstar;
           dmv[r] = __ballot_sync(0xffffffffu, defv[r]);
           cmv[r] = __ballot_sync(0xffffffffu, candv[r]);
-          rowv[r] = (defv[r] || candv[r]) ? kv_row(p, bt_row, h, s0 + j) : 0;
+          pagev[r] = (defv[r] || candv[r]) ? kv_page_entry(p, bt_row, s0 + j) : 0;
           ndm += __popc(dmv[r]);
           ncm += __popc(cmv[r]);
         }
@@ -916,16 +924,17 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
         for (int r = 0; r < kActPerWarp; ++r) {
           const int j = jv[r];
           int slot = -1;
+          const int32_t row = (defv[r] || candv[r]) ? kv_row_of(p, pagev[r], h, s0 + j) : 0;
           if (defv[r]) {
             const uint32_t o = dbase + __popc(dmv[r] & below);
-            if (o < static_cast<uint32_t>(p.cap)) sel_u[o] = rowv[r];
+            if (o < static_cast<uint32_t>(p.cap)) sel_u[o] = row;
             if (p.dbg_selected) atomicOr(bm + (j >> 5), 1u << (j & 31));   // for the ascending positions
           } else if (candv[r]) {
             slot = static_cast<int>(cbase + __popc(cmv[r] & below));
             if (slot < p.cap) {
               cand_u[slot] = (static_cast<unsigned long long>(float_key(sv[r])) << 32) |
                              (0xffffffffu - static_cast<uint32_t>(j));
-              cand_row_u[slot] = rowv[r];
+              cand_row_u[slot] = row;
             }
           }
           dbase += __popc(dmv[r]);
@@ -962,11 +971,14 @@ __device__ bool filter_part(const StepParams& p, int u, int c0, int c1, uint32_t
   }
   // publish this range's selections, candidates and fix-ups, then count it in; the part
   // that completes the count resolves the unit
+  // (the barrier orders the CTA's writes before thread 0's release, which is cumulative;
+  // the acquire half lets the part that completes the count read every other part's writes)
   __syncthreads();
   if (tid == 0) {
-    __threadfence();
     const int n = c1 - c0;
-    const int old = atomicAdd(&p.units[u].filt_done, n);
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(&p.units[u].filt_done), "r"(n)
+                 : "memory");
     ss.flag = (old < total && old + n >= total) ? 1 : 0;
   }
   __syncthreads();
@@ -1139,8 +1151,7 @@ __device__ void resolve_unit(const StepParams& p, int u, uint8_t* fsm, SelShared
   // publish: the rows and the winners' fix-ups are written
   __syncthreads();
   const int nsel = ndef + ((k > 0 && ok) ? r : 0);
-  if (tid == 0) {
-    __threadfence();
+  if (tid == 0) {   // release after the barrier: cumulative over the CTA's writes
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(&p.units[u].ready), "r"(1) : "memory");
     if (!ok || nsel != k) record_error(p.err, HSA_DEVERR_SELECT);
     if (p.dbg_nselected) p.dbg_nselected[u] = nsel;
@@ -1395,8 +1406,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_select_kernel(StepParams
     });
   }
   if (nres > 0) {
-    __threadfence();   // acquire: the unit's other parts published before counting in
-    __syncthreads();
+    __syncthreads();   // thread 0's acquiring count orders the other parts' writes before the reads
     for (int i = 0; i < min(nres, kMaxParts); ++i) resolve_unit<G>(p, ss.res[i], smem, ss);
   }
   // units without chunks (nothing indexed) are published by CTA u mod grid
