@@ -315,15 +315,6 @@ struct alignas(128) UnitState {
 };
 static_assert(sizeof(UnitState) == 640, "five 128-byte lines per unit");
 
-// Publish a per-unit flag after this CTA's writes: call from every thread of the CTA.
-__device__ __forceinline__ void publish_flag(int32_t* flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
-  }
-}
-
 // Bounded wait (acquire) for a flag another running grid publishes; a timeout is
 // recorded and returns false. Callers only wait on CTAs that are already resident.
 // Call it from one thread and share the outcome through a barrier (the flag's line is
