@@ -311,10 +311,6 @@ static_assert(kFinScratch <= 128 * 1024, "resolution scratch fits in the scan's 
 static_assert(kCandWeights <= kFinSmemCand, "stored candidate weights are resolved in shared memory");
 
 constexpr int kMaxParts = 24;   // (unit, chunk range) parts one CTA plans in shared memory
-#ifndef PQHSA_SCAN_PAIR
-#define PQHSA_SCAN_PAIR 0
-#endif
-constexpr bool kScanPair = PQHSA_SCAN_PAIR != 0;   // phase 1 scores two chunks per warp step
 
 struct SelShared {
   uint32_t scan_tot[33];
@@ -568,46 +564,18 @@ __device__ __forceinline__ void scan_segment(const StepParams& p, int u, int ch0
     for (int g = 0; g < G; ++g) wacc[g] += valid ? fast_exp2(fmaf(sh[g], kLog2e, -ub2[g])) : 0.f;
     if (valid) atomicAdd(&hist_s[score_bin(sg, lo, inv)], 1u);
   };
-  if (kScanPair) {
-    // two chunks per step: their look-up chains are independent, so each warp keeps twice
-    // as many shared-memory gathers in flight between its synchronisations
-    for (int i = 0; i < cnt; i += 2) {
-      const bool two = i + 1 < cnt;
-      cp_async_wait<D - 2>();            // this lane's copies of chunks i and i + 1 have landed
-      __syncwarp();                      // ... and lane 0's cluster words
-      uint4 code0, code1;
-      uint32_t id0, id1;
-      int fill0, fill1;
-      chunk_in(i, code0, id0, fill0);
-      if (two) chunk_in(i + 1, code1, id1, fill1);
-      else {
-        code1 = code0;
-        id1 = id0;
-        fill1 = 0;
-      }
-      float sh0[G], sh1[G];
-      score_token<G>(code0, id0, lut_b, qc_s, C, ysoff, sel, swap_words, sh0);
-      score_token<G>(code1, id1, lut_b, qc_s, C, ysoff, sel, swap_words, sh1);
-      chunk_out(i, id0, fill0, sh0);
-      if (two) chunk_out(i + 1, id1, fill1, sh1);
-      __syncwarp();                      // every lane has read both slots
-      issue(i + D);                      // refill them with the chunks D ahead
-      issue(i + 1 + D);
-    }
-  } else {
-    for (int i = 0; i < cnt; ++i) {
-      cp_async_wait<D - 1>();            // this lane's copies of chunk i have landed
-      __syncwarp();                      // ... and lane 0's cluster word
-      uint4 code;
-      uint32_t id;
-      int fill;
-      chunk_in(i, code, id, fill);
-      float sh[G];
-      score_token<G>(code, id, lut_b, qc_s, C, ysoff, sel, swap_words, sh);
-      chunk_out(i, id, fill, sh);
-      __syncwarp();                      // every lane has read the slot
-      issue(i + D);                      // refill it with the chunk D ahead
-    }
+  for (int i = 0; i < cnt; ++i) {
+    cp_async_wait<D - 1>();            // this lane's copies of chunk i have landed
+    __syncwarp();                      // ... and lane 0's cluster word
+    uint4 code;
+    uint32_t id;
+    int fill;
+    chunk_in(i, code, id, fill);
+    float sh[G];
+    score_token<G>(code, id, lut_b, qc_s, C, ysoff, sel, swap_words, sh);
+    chunk_out(i, id, fill, sh);
+    __syncwarp();                      // every lane has read the slot
+    issue(i + D);                      // refill it with the chunk D ahead
   }
   if (cur != 0xffffffffu) flush_weights<G>(wacc, Wu, C, cur);
   cp_async_wait<0>();
