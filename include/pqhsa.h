@@ -14,9 +14,12 @@
  * decode (dense_decode), the in-library baseline.
  *
  * Conventions shared by every entry point
- * - Pointers are DEVICE pointers unless their name ends in _host. The caller
- *   owns all memory; the library allocates nothing, keeps no state between
- *   calls, and touches only the buffers it is given.
+ * - Pointers are DEVICE pointers unless their name ends in _host (host memory).
+ *   The caller owns all memory; the library allocates no device memory, keeps
+ *   no state between calls, and touches only the buffers it is given - except
+ *   where an entry point says otherwise: dense_decode_static's static scratch
+ *   array, and a prepared decode step (hsa_decode_step_*), which holds a small
+ *   host object, a private stream and a CUDA graph until it is destroyed.
  * - Every call validates its arguments on the host (from the *_host arrays)
  *   before any launch and returns a status; on an error nothing is launched.
  *   HSA_ERR_CUDA means a launch failed (the CUDA error is left pending).
