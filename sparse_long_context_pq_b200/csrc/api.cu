@@ -203,6 +203,7 @@ Split decode_split_plan(const hsa_kv_cache* kv, const hsa_index* ix, const hsa_d
 // device memory rather than each across the host link.
 __global__ void __launch_bounds__(256) stage_q_kernel(const float4* __restrict__ src, float4* __restrict__ dst,
                                                       int n4) {
+  pdl_launch_dependents();   // the tables kernel may start its index loads meanwhile
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) dst[i] = src[i];
 }
 
@@ -348,9 +349,14 @@ hsa_status dense_decode(const hsa_kv_cache* kv, const float* q, float* out, floa
   return HSA_OK;
 }
 
-hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* q, float* out,
-                      const hsa_decode_params* prm, const hsa_debug* dbg, void* ws, size_t ws_bytes,
-                      cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+// hsa_decode; q_staged: the previous kernel on the stream is hsa_decode_host's q staging
+// (the tables kernel may then read the index before its dependency wait).
+hsa_status decode_impl(const hsa_kv_cache* kv, const hsa_index* ix, const float* q, float* out,
+                       const hsa_decode_params* prm, const hsa_debug* dbg, void* ws, size_t ws_bytes,
+                       cudaStream_t stream, bool q_staged) {
   hsa_status st = check_kv(kv);
   if (st != HSA_OK) return st;
   st = check_index(kv, ix, true);
@@ -413,6 +419,7 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   tp.nq = L.nq;
   tp.bitmap_words = L.bitmap_words;
   tp.scale = prm->scale;
+  tp.index_early = (q_staged && use_pdl()) ? 1 : 0;
   RET_CUDA(mark(0));
   RET_CUDA(launch_tables(G, tp, stream, use_pdl()));
 
@@ -509,6 +516,15 @@ hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* 
   RET_CUDA(mark(4));
   return HSA_OK;
 }
+}  // namespace
+
+extern "C" {
+
+hsa_status hsa_decode(const hsa_kv_cache* kv, const hsa_index* ix, const float* q, float* out,
+                      const hsa_decode_params* prm, const hsa_debug* dbg, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  return decode_impl(kv, ix, q, out, prm, dbg, ws, ws_bytes, stream, false);
+}
 
 // Longest training set: the fallback assignment launches one grid row per 32 keys (at most 65535).
 constexpr int32_t kMaxTrain = 65535 * 32;
@@ -598,7 +614,7 @@ hsa_status hsa_decode_host(const hsa_kv_cache* kv, const hsa_index* ix, const fl
     stage_q_kernel<<<std::min(64, (n4 + 255) / 256), 256, 0, stream>>>(static_cast<const float4*>(q_map),
                                                                        reinterpret_cast<float4*>(q_dev), n4);
     RET_CUDA(cudaGetLastError());
-    return hsa_decode(kv, ix, q_dev, static_cast<float*>(out_map), prm, nullptr, ws, base, stream);
+    return decode_impl(kv, ix, q_dev, static_cast<float*>(out_map), prm, nullptr, ws, base, stream, true);
   }
   RET_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));
   st = hsa_decode(kv, ix, q_dev, out_dev, prm, nullptr, ws, base, stream);

@@ -118,6 +118,9 @@ struct TablesParams {
   UnitState* units;          // zeroed here
   int B, Hq, Hkv, C, nq, bitmap_words;
   float scale;
+  // 1: the codebooks and centroids may be read before the dependency wait (the previous
+  // kernel is the q staging of a host-buffer step, which itself follows every earlier one)
+  int index_early;
 };
 cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, bool pdl);
 

@@ -124,8 +124,12 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
   const int part = blockIdx.y;
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  pdl_wait();
-  pdl_launch_dependents();
+  // the dependency wait: first thing, or (index_early) once this CTA's codebook or
+  // centroid loads are on their way
+  if (!p.index_early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
   float* bnd = p.bounds + static_cast<size_t>(u) * (kLutParts + p.nq) * 2 * G4;
 
   if (part < kLutParts) {
@@ -138,6 +142,10 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
           p.codebooks + ((static_cast<size_t>(u) * kM + part * kSubPerPart + i) * kNcode + m) * kDsub);
       cw[i][0] = src[0];
       cw[i][1] = src[1];
+    }
+    if (p.index_early) {
+      pdl_wait();
+      pdl_launch_dependents();
     }
     stage_q<G4, G>(p, b, h, tid, qsh);
     // zero this unit's selection state (spread over the LUT CTAs)
@@ -198,6 +206,10 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
       const int c = c0 + i;
       cv[i] = c < p.C ? *reinterpret_cast<const float4*>(p.centroids + (static_cast<size_t>(u) * p.C + c) * kD + lane * 4)
                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (p.index_early) {
+      pdl_wait();
+      pdl_launch_dependents();
     }
     stage_q<G4, G>(p, b, h, tid, qsh);
     {   // zero this slice's cluster weights
