@@ -171,7 +171,9 @@ hsa_status hsa_decode_host(const hsa_kv_cache* kv, const hsa_index* index, const
 
 /* ---- prepared decode step (graph replay) --------------------------------- */
 
-/* A decode step prepared for one cache, index, parameter set and workspace (opaque). */
+/* A decode step prepared for one cache, index, parameter set and workspace (opaque), for
+   decode loops: each run replays a recorded CUDA graph of the step while its launch shape
+   and buffers stay the same. */
 typedef struct hsa_decode_step hsa_decode_step;
 
 /*
@@ -186,17 +188,18 @@ hsa_status hsa_decode_step_create(const hsa_kv_cache* kv, const hsa_index* index
                                   void* workspace, size_t workspace_bytes, hsa_decode_step** step);
 
 /*
- * One decode step on host buffers, as hsa_decode_host, queued on `stream` as one CUDA
- * graph launch. Every run validates the views and the current lengths again and
+ * One decode step, queued on `stream` as one CUDA graph launch. q, out: fp32 [B][Hq][D],
+ * both page-locked host memory (the step is hsa_decode_host's) or both device memory
+ * (hsa_decode's, 16-B aligned); anything else, pageable host memory included, is
+ * HSA_ERR_INVALID_ARG. Every run validates the views and the current lengths again and
  * recomputes the split-K plan of the exact part (the only launch shape that depends on
- * host-side values). While that plan, q_host and out_host are those of the previous run,
- * the run replays the previous run's graph; otherwise (the first run, lengths that moved
- * the plan, other buffers) it records the host-buffer step on a private stream of the
- * step and updates the graph. q_host and out_host must be page-locked host memory
- * (HSA_ERR_INVALID_ARG otherwise). Result and error word as for hsa_decode_host. One
- * thread at a time per step; runs of steps that share a workspace must not overlap.
+ * host-side values). While that plan, q and out are those of the previous run, the run
+ * replays the previous run's graph; otherwise (the first run, lengths that moved the plan,
+ * other buffers) it records the step on a private stream of the step and updates the
+ * graph. Result and error word as for hsa_decode_host / hsa_decode. One thread at a time
+ * per step; runs of steps that share a workspace must not overlap.
  */
-hsa_status hsa_decode_step_run(hsa_decode_step* step, const float* q_host, float* out_host, cudaStream_t stream);
+hsa_status hsa_decode_step_run(hsa_decode_step* step, const float* q, float* out, cudaStream_t stream);
 
 /* Release a step (its graph and private stream). NULL is ignored. It does not wait:
    let the step's queued work finish before the arrays it reads are freed. */

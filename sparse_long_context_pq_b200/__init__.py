@@ -332,10 +332,12 @@ class DecodeStep:
     marshalled once here, and each call passes only q, out and the stream (the library still
     validates every call, lengths included). The tensors must keep their storage while the
     step is in use; their contents (lengths, appended tokens, lists) may change between calls.
-    Calling the step runs hsa_decode on device q / out; .host() runs the step on host q / out
-    (page-locked): by default as the library's prepared step (hsa_decode_step_run, one CUDA
-    graph launch per call while the split plan and buffers stay the same), or with
-    graph=False as one hsa_decode_host call. The workspace is sized for both.
+    Calling the step runs it on device q / out: by default as one hsa_decode call, or with
+    graph=True as the library's prepared step (hsa_decode_step_run: one CUDA graph launch per
+    call while the split plan and the buffers stay the same - worth it when a loop reuses
+    the same q and out tensors). .host() runs it on page-locked host q / out: by default as
+    the prepared step, or with graph=False as one hsa_decode_host call. The workspace is
+    sized for all of them.
     """
 
     def __init__(self, kv: PagedKV, index: PQIndex, *, scale: float, budget: float = 0.01, k_override: int = -1,
@@ -363,16 +365,28 @@ class DecodeStep:
                 or t.device != self._device):
             raise ValueError(f"{name}: expected a contiguous fp32 tensor {list(self._shape)} on {self._device}")
 
-    def __call__(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    def __call__(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None,
+                 graph: bool = False) -> torch.Tensor:
         self._check_io(q, "q")
         if out is None:
             out = torch.empty_like(q)
         else:
             self._check_io(out, "out")
+        if graph:
+            self._run_step(q, out, stream)
+            return out
         st = self._fn(self._kv_ref, self._ix_ref, q.data_ptr(), out.data_ptr(), self._prm_ref, None, self._ws_ptr,
                       self._ws_len, _stream(stream))
         _check("hsa_decode", st)
         return out
+
+    def _run_step(self, q: torch.Tensor, out: torch.Tensor, stream) -> None:
+        if not self._handle.value:
+            _check("hsa_decode_step_create",
+                   self._lib.hsa_decode_step_create(self._kv_ref, self._ix_ref, self._prm_ref, self._ws_ptr,
+                                                    self._ws_len, ctypes.byref(self._handle)))
+        _check("hsa_decode_step_run",
+               self._lib.hsa_decode_step_run(self._handle, q.data_ptr(), out.data_ptr(), _stream(stream)))
 
     def host(self, q_host: torch.Tensor, out_host: torch.Tensor, stream=None, graph: bool = True) -> torch.Tensor:
         """q in from and out back to host memory, queued on the stream (out_host holds the result
@@ -389,12 +403,7 @@ class DecodeStep:
                                self._ws_ptr, self._ws_len, _stream(stream))
             _check("hsa_decode_host", st)
             return out_host
-        if not self._handle.value:
-            _check("hsa_decode_step_create",
-                   self._lib.hsa_decode_step_create(self._kv_ref, self._ix_ref, self._prm_ref, self._ws_ptr,
-                                                    self._ws_len, ctypes.byref(self._handle)))
-        _check("hsa_decode_step_run", self._lib.hsa_decode_step_run(self._handle, q_host.data_ptr(),
-                                                                    out_host.data_ptr(), _stream(stream)))
+        self._run_step(q_host, out_host, stream)
         return out_host
 
     def close(self) -> None:

@@ -207,6 +207,18 @@ __global__ void __launch_bounds__(256) stage_q_kernel(const float4* __restrict__
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) dst[i] = src[i];
 }
 
+// Where a buffer of the prepared step lives: 1 page-locked host memory, 2 device (or
+// managed) memory, 0 anything else (pageable host memory, an unknown pointer).
+int buffer_kind(const void* p) {
+  cudaPointerAttributes a = {};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  if (a.type == cudaMemoryTypeHost) return a.devicePointer ? 1 : 0;
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) ? 2 : 0;
+}
+
 // Device address of page-locked host memory (nullptr for pageable memory).
 void* mapped_host_pointer(const void* p) {
   cudaPointerAttributes a = {};
@@ -674,21 +686,23 @@ hsa_status hsa_decode_step_create(const hsa_kv_cache* kv, const hsa_index* ix, c
   return HSA_OK;
 }
 
-hsa_status hsa_decode_step_run(hsa_decode_step* s, const float* q_host, float* out_host, cudaStream_t stream) {
+hsa_status hsa_decode_step_run(hsa_decode_step* s, const float* q, float* out, cudaStream_t stream) {
   if (!s) return HSA_ERR_INVALID_ARG;
   hsa_status st = check_step_args(&s->kv, &s->ix, &s->prm, s->ws, s->ws_bytes);
   if (st != HSA_OK) return st;
-  if (!q_host || !out_host) return HSA_ERR_INVALID_ARG;
+  if (!q || !out) return HSA_ERR_INVALID_ARG;
   const DeviceInfo* dev = device_info();
   if (!dev) return HSA_ERR_CUDA;
   const int G = s->kv.Hq / s->kv.Hkv;
   const DecodeLayout L = make_decode_layout(s->kv.B * s->kv.Hkv, G, s->ix.C, s->ix.cap, s->ix.list_slots, kMaxSplits);
   const Split sp = decode_split_plan(&s->kv, &s->ix, &s->prm, L.nbg, dev->sms);
-  const bool same = s->exec && sp.nsplit == s->key_nsplit && sp.chunk == s->key_chunk && q_host == s->key_q &&
-                    out_host == s->key_out;
+  const bool same = s->exec && sp.nsplit == s->key_nsplit && sp.chunk == s->key_chunk && q == s->key_q &&
+                    out == s->key_out;
   if (!same) {
-    // a graph cannot copy pageable host memory: the buffers must be page-locked
-    if (!mapped_host_pointer(q_host) || !mapped_host_pointer(out_host)) return HSA_ERR_INVALID_ARG;
+    // both page-locked host memory (the host-buffer step) or both device memory (hsa_decode);
+    // a graph cannot copy pageable host memory
+    const int kind = buffer_kind(q);
+    if (kind == 0 || buffer_kind(out) != kind) return HSA_ERR_INVALID_ARG;
     int cur = 0;
     RET_CUDA(cudaGetDevice(&cur));
     if (s->cap && cur != s->device) return HSA_ERR_INVALID_ARG;   // a step stays on its first device
@@ -696,9 +710,10 @@ hsa_status hsa_decode_step_run(hsa_decode_step* s, const float* q_host, float* o
       RET_CUDA(cudaStreamCreateWithFlags(&s->cap, cudaStreamNonBlocking));
       s->device = cur;
     }
-    // record the host-buffer step (nothing runs while the stream captures)
+    // record the step (nothing runs while the stream captures)
     RET_CUDA(cudaStreamBeginCapture(s->cap, cudaStreamCaptureModeThreadLocal));
-    st = hsa_decode_host(&s->kv, &s->ix, q_host, out_host, &s->prm, s->ws, s->ws_bytes, s->cap);
+    st = kind == 1 ? hsa_decode_host(&s->kv, &s->ix, q, out, &s->prm, s->ws, s->ws_bytes, s->cap)
+                   : hsa_decode(&s->kv, &s->ix, q, out, &s->prm, nullptr, s->ws, s->ws_bytes, s->cap);
     cudaGraph_t g = nullptr;
     const cudaError_t ce = cudaStreamEndCapture(s->cap, &g);
     if (st != HSA_OK || ce != cudaSuccess || !g) {
@@ -722,8 +737,8 @@ hsa_status hsa_decode_step_run(hsa_decode_step* s, const float* q_host, float* o
     cudaGraphDestroy(g);
     s->key_nsplit = sp.nsplit;
     s->key_chunk = sp.chunk;
-    s->key_q = q_host;
-    s->key_out = out_host;
+    s->key_q = q;
+    s->key_out = out;
   }
   RET_CUDA(cudaGraphLaunch(s->exec, stream));
   return HSA_OK;

@@ -162,8 +162,8 @@ def test_no_index_and_no_sink(cuda_device):
 
 def test_prepared_step_matches_hsa_decode(cuda_device):
     """DecodeStep (the cache and index views marshalled once) gives hsa_decode's output, on
-    device and on host buffers (hsa_decode_host), and still does after the lengths change in
-    place behind its views. Two decode calls agree to rounding, not bit for bit: the
+    device and on host buffers (hsa_decode_host), eagerly and as the graph-replayed prepared
+    step, and still does after the lengths change in place behind its views. Two decode calls agree to rounding, not bit for bit: the
     cluster-weight sums are fp32 atomics in arrival order."""
     w, bt, codes, ids, kv, ix, dev = _setup(CASES["qwen_g8_8k"])
     ws_idx = P.workspace(P.hsa_index_workspace_bytes(kv, ix), dev)
@@ -176,9 +176,13 @@ def test_prepared_step_matches_hsa_decode(cuda_device):
         got = step(q)
         out = torch.full_like(q, float("nan"))
         assert step(q, out) is out
+        out_g = torch.full_like(q, float("nan"))
+        step(q, out_g, graph=True)              # prepared step on device buffers: records, then replays
+        step(q, out_g, graph=True)
         torch.cuda.synchronize()
         tol = 1e-6 * float(ref.abs().max()) + 1e-7
-        assert float((got - ref).abs().max()) <= tol and float((out - ref).abs().max()) <= tol
+        for o in (got, out, out_g):
+            assert float((o - ref).abs().max()) <= tol
         # the host-buffer entry: q in from and out back to pinned host memory
         q_h = q.cpu().pin_memory()
         outs = [torch.full(q.shape, float("nan")).pin_memory() for _ in range(4)]
