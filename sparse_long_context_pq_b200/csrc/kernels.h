@@ -125,10 +125,10 @@ struct TablesParams {
 cudaError_t launch_tables(int G, const TablesParams& p, cudaStream_t stream, bool pdl);
 
 // One launch after the tables: the scan of the codes (phase 1), then, per unit, the
-// selection (phase 2: threshold bin from the unit's histogram, definite selections and
-// threshold-bin candidates of this CTA's chunks, weight fix-ups) and its resolution by
-// the unit's last CTA (phase 3: exact order of the candidates, ascending write-out of
-// the selected rows, ready flag).
+// selection (phase 2: threshold bin from the unit's histogram; over this CTA's share of
+// the unit's chunks, the definite selections' rows, the threshold-bin candidates and the
+// weight fix-ups) and its resolution by the part that completes the unit's count (phase
+// 3: exact order of the candidates, the winners' rows and fix-ups, ready flag).
 struct StepParams {
   const uint8_t* list_codes;     // [U][list_slots][16] cluster-ordered codes
   const int32_t* list_slot;      // [U][list_slots] index slot of each list slot (-1 empty)

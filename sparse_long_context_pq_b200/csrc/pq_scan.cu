@@ -5,10 +5,11 @@
 //                 indexed token, the selection score sigma = max over the group's heads,
 //                 per-cluster exp-weight sums, a histogram of sigma, each chunk's largest
 //                 sigma); then, per unit, the tokens above the threshold histogram bin
-//                 (selected) and in it (candidates), the selected tokens' weights taken
-//                 out of the cluster sums; then the unit's last CTA resolves the
-//                 candidates exactly (score desc, position asc), writes the selected
-//                 tokens as KV-pool rows in ascending position order and publishes the unit.
+//                 (selected, their KV-pool rows written at once) and in it (candidates),
+//                 the selected tokens' weights taken out of the cluster sums; then the
+//                 part that completes the unit's count resolves the candidates exactly
+//                 (score desc, position asc), writes the winners' rows after the others
+//                 (in no particular position order) and publishes the unit.
 //
 // Source: rit.work "pq-hsa-long-context-attention", section
 // "Как приблизительные оценки возвращают отброшенный контекст" (an approximate
@@ -268,10 +269,11 @@ __global__ void __launch_bounds__(256) tables_kernel(TablesParams p) {
 // chunk's largest sigma. Phase 2 (filter), per unit, once every CTA of the unit has
 // scanned its chunks: the threshold bin from the unit's histogram, then, over this CTA's
 // share of the unit's chunks (spread over the whole list), the definite selections' rows,
-// the threshold-bin candidates and the weight fix-ups. Phase 3 (resolution), by the
-// unit's last CTA to finish phase 2: the
-// exact order of the candidates (score desc, position asc), the selected tokens as
-// KV-pool rows in ascending position order, the winners' weight fix-ups, the ready flag.
+// the threshold-bin candidates and the weight fix-ups. Phase 3 (resolution), by the part
+// that completes the unit's filter count: the exact order of the candidates (score desc,
+// position asc), the winners' KV-pool rows after the others and their weight fix-ups, the
+// ready flag. The attention needs the rows in no particular order; only the debug output
+// of the selected positions is written in ascending order.
 //
 // The per-unit wait of phase 2 only waits on CTAs of the same grid, which are all
 // resident: the grid has one CTA per SM and each CTA needs a whole SM's registers,
